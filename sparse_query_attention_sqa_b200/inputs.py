@@ -1,0 +1,87 @@
+"""Seeded synthetic inputs for Sparse Query Attention workloads.
+
+This module only draws random tensors and names workload shapes; it holds
+none of the attention arithmetic.  The CUDA path's tests, the benchmark and
+the oracle-side tests all take their inputs from here, so both sides see the
+same bf16 bits.
+
+Recipe: a CPU ``torch.Generator`` seeded with ``seed`` draws standard normal
+fp32 tensors in the order q, k, v, dO; each is multiplied by its standard
+deviation (and K by ``k_scale``) and then rounded to bf16.  Shapes follow the
+SQAT-m model card ("Architecture details": d = 256 split over 16 heads, so
+dh = 16; 8 query groups and 4 key/value groups; message length 1024) and the
+arXiv 2510.01817 abstract (32k-200k token sequences), plus a larger-model
+dh = 128 case.  The pages train on Wikipedia text; attention inputs here are
+synthetic Gaussians instead, since the attention core needs no tokens.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    N: int
+    Hq: int
+    Hkv: int
+    dh: int
+    causal: bool
+    backward: bool
+    std: float = 1.0
+    k_scale: float = 1.0
+    scale: float = 0.0  # <= 0 selects 1/sqrt(dh)
+    note: str = ""
+
+    @property
+    def softmax_scale(self) -> float:
+        return self.scale if self.scale > 0 else self.dh ** -0.5
+
+
+# Workload shapes.  Each is one (B, N, H_q, H_kv, dh) point; sweeps list one
+# entry per head configuration.
+WORKLOADS: dict[str, Workload] = {}
+
+
+def _add(w: Workload):
+    WORKLOADS[w.name] = w
+
+
+# SQAT-m single-layer attention, forward only.
+_add(Workload("sqatm_layer_fwd", 1, 1024, 8, 4, 16, True, False, scale=0.25,
+              note="SQAT-m single layer, B=1 N=1024 dh=16 Hq=8 Hkv=4 causal"))
+# SQAT-m training-step attention (forward + backward) and its same-kernel comparisons.
+for hq, hkv, tag in ((8, 4, "sqa"), (16, 4, "gqa"), (16, 16, "mha"), (16, 1, "mqa")):
+    _add(Workload(f"sqatm_train_{tag}", 32, 1024, hq, hkv, 16, True, True,
+                  note=f"SQAT-m training step, B=32 N=1024 dh=16 Hq={hq} Hkv={hkv} causal"))
+# Long-context encoder attention, N=32768, head sweep.
+for hq, hkv in ((8, 4), (8, 8), (4, 4), (16, 16), (16, 4), (16, 1)):
+    _add(Workload(f"enc32k_{hq}_{hkv}", 1, 32768, hq, hkv, 16, False, False,
+                  note=f"encoder, B=1 N=32768 dh=16 Hq={hq} Hkv={hkv} bidirectional"))
+# Long-context encoder attention at 131072 and 200000 tokens (200000 is not a tile multiple).
+for n in (131072, 200000):
+    for hq, hkv in ((4, 4), (8, 4)):
+        _add(Workload(f"enc{n // 1000}k_{hq}_{hkv}", 1, n, hq, hkv, 16, False, False, std=0.5,
+                      note=f"encoder, B=1 N={n} dh=16 Hq={hq} Hkv={hkv} bidirectional, std 0.5"))
+# Larger-model SQA: d=2048 over 16 heads, dh=128.
+_add(Workload("large_dh128", 2, 65536, 8, 4, 128, True, True, k_scale=0.1,
+              note="larger model, B=2 N=65536 dh=128 Hq=8 Hkv=4 causal, K x 0.1"))
+
+
+def make_inputs(B: int, N: int, Hq: int, Hkv: int, dh: int, seed: int = 0, std: float = 1.0,
+                k_scale: float = 1.0, with_dout: bool = False):
+    """Draw q [B,N,Hq,dh], k, v [B,N,Hkv,dh] (and dO [B,N,Hq,dh]) as CPU bf16 tensors."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    q = (torch.randn(B, N, Hq, dh, generator=g) * std).to(torch.bfloat16)
+    k = (torch.randn(B, N, Hkv, dh, generator=g) * (std * k_scale)).to(torch.bfloat16)
+    v = (torch.randn(B, N, Hkv, dh, generator=g) * std).to(torch.bfloat16)
+    dout = torch.randn(B, N, Hq, dh, generator=g).to(torch.bfloat16) if with_dout else None
+    return q, k, v, dout
+
+
+def workload_inputs(w: Workload, seed: int = 0):
+    return make_inputs(w.B, w.N, w.Hq, w.Hkv, w.dh, seed=seed, std=w.std, k_scale=w.k_scale,
+                       with_dout=w.backward)
