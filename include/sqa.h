@@ -1,0 +1,110 @@
+/*
+ * sqa.h -- C ABI of the B200 (sm_100a) Sparse Query Attention library.
+ *
+ * Sparse Query Attention (arXiv 2510.01817, abstract; SQAT-m model card,
+ * "Architecture details" and "Model size difference") is scaled dot-product
+ * attention with H_q query heads, fewer than the H-way split of the model
+ * width, sharing H_kv key/value heads.  The query heads form H_kv contiguous
+ * groups of g = H_q / H_kv heads and every head of a group reads the same K and
+ * V head (GQA summary, "The idea": one key head and one value head per group;
+ * "The notation": GQA-1 is MQA, GQA-H is MHA).  Score FLOPs therefore scale with
+ * H_q.  For query head h, kv(h) = floor(h / g):
+ *
+ *   S_ij  = scale * <Q[b,i,h,:], K[b,j,kv(h),:]>      (-inf where causal and j > i)
+ *   lse_i = ln sum_j exp(S_ij)
+ *   O_i   = sum_j exp(S_ij - lse_i) V[b,j,kv(h),:]
+ *
+ * Tensor layouts (all contiguous, row-major, no padding):
+ *   q, out, dout, dq : bf16 [B][N][H_q][dh]
+ *   k, v, dk, dv     : bf16 [B][N][H_kv][dh]
+ *   lse              : fp32 [B][H_q][N], natural log of the sum of exp(scaled scores)
+ *
+ * Ownership and execution: the caller owns every buffer (device memory, e.g.
+ * from PyTorch) and the stream.  Calls are asynchronous on `stream`; the library
+ * never synchronises, never allocates device memory and keeps no per-call
+ * state on the device.  Arguments are validated on the host before anything is
+ * launched; a call that returns an error has launched nothing.  The calls are
+ * thread-safe; error text is kept per host thread.
+ */
+#ifndef SQA_H_
+#define SQA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *sqa_stream_t; /* a cudaStream_t; NULL is the legacy default stream */
+
+typedef enum {
+    SQA_OK = 0,
+    SQA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, H_q not a multiple of H_kv, NaN scale */
+    SQA_ERR_UNSUPPORTED = 2, /* head dim not in {16, 32, 64, 128}, g > 128, misaligned pointer, size too large */
+    SQA_ERR_CUDA = 3         /* a CUDA runtime/driver call failed; sqa_last_error() has the text */
+} sqa_status;
+
+typedef struct {
+    int B;    /* batch */
+    int N;    /* sequence length (queries and keys) */
+    int H_q;  /* query heads */
+    int H_kv; /* key/value heads; H_q % H_kv == 0 and H_q / H_kv <= 128 */
+    int dh;   /* head dimension: 16, 32, 64 or 128 */
+} sqa_shape;
+
+/*
+ * Forward pass (the definition above).  q, k, v, out must be 16-byte aligned;
+ * lse 4-byte aligned.  out and lse are fully overwritten.  scale <= 0 selects
+ * 1/sqrt(dh).  causal != 0 masks keys j > i (the diagonal j == i stays visible).
+ */
+sqa_status sqa_fwd(const void *q, const void *k, const void *v, void *out, float *lse, sqa_shape s,
+                   int causal, float scale, sqa_stream_t stream);
+
+/*
+ * Bytes of device scratch that sqa_bwd needs for shape s (fp32 dQ accumulator
+ * plus per-row softmax statistics).  The caller allocates it; 256-byte aligned.
+ */
+size_t sqa_bwd_workspace_bytes(sqa_shape s);
+
+/*
+ * Backward pass of L = sum(dout * out) through the forward above.
+ * Inputs: dout, q, k, v, out (bf16, the forward's output) and lse (fp32, the
+ * forward's).  Outputs: dq (bf16, [B][N][H_q][dh]), dk and dv (bf16,
+ * [B][N][H_kv][dh]); all three are fully overwritten.  dK and dV of a key/value
+ * head sum the contributions of every query head in its group.
+ *   D_i   = <dO_i, O_i>,  P_ij = exp(S_ij - lse_i),  dP_ij = <dO_i, V_j>
+ *   dS_ij = P_ij (dP_ij - D_i)
+ *   dQ_i  = scale sum_j dS_ij K_j;  dK_j = scale sum_{h in group} sum_i dS_ij Q_i;
+ *   dV_j  = sum_{h in group} sum_i P_ij dO_i
+ * workspace must hold sqa_bwd_workspace_bytes(s) bytes and be 256-byte
+ * aligned; its contents on entry do not matter and are clobbered.
+ */
+sqa_status sqa_bwd(const void *dout, const void *q, const void *k, const void *v, const void *out,
+                   const float *lse, void *dq, void *dk, void *dv, void *workspace,
+                   size_t workspace_bytes, sqa_shape s, int causal, float scale,
+                   sqa_stream_t stream);
+
+/* Static text for a status code. */
+const char *sqa_status_string(sqa_status status);
+
+/* Detail of the last error on the calling host thread ("" if none). */
+const char *sqa_last_error(void);
+
+/*
+ * Device-side wait status.  Every wait inside the kernels gives up after about
+ * two seconds, sets a bit in a per-device status word and lets the kernel end,
+ * so a broken pipeline reports an error instead of hanging the GPU.  This call
+ * synchronises the current device, returns the word (0 = no timeout seen) and,
+ * if clear != 0, resets it.  Returns SQA_ERR_CUDA if it could not be read.
+ */
+sqa_status sqa_device_status(unsigned int *word, int clear);
+
+/* Library version as an integer (major * 10000 + minor * 100 + patch). */
+int sqa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQA_H_ */

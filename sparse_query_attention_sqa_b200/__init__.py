@@ -1,0 +1,164 @@
+"""Sparse Query Attention on B200 (sm_100a): Python binding of libsqa.so.
+
+Every step of the attention forward and backward runs in the CUDA kernels of
+``libsqa.so`` (C ABI in ``include/sqa.h``).  This module only checks tensor
+metadata, allocates outputs with PyTorch and passes raw pointers and the
+current stream through ctypes.  There is no CPU fallback: if the library is
+missing or cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "SqaError", "load_library", "library_path", "sqa_fwd", "sqa_bwd", "bwd_workspace_bytes",
+    "device_status", "Shape",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libsqa.so")
+_lib = None
+
+SQA_OK, SQA_ERR_INVALID_ARG, SQA_ERR_UNSUPPORTED, SQA_ERR_CUDA = 0, 1, 2, 3
+
+
+class SqaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"[status {status}] {message}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("N", ctypes.c_int), ("H_q", ctypes.c_int), ("H_kv", ctypes.c_int),
+                ("dh", ctypes.c_int)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libsqa.so (built in-tree by ``build.py``); raises if it is absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"libsqa.so is not built ({_LIB_PATH}); run sparse_query_attention_sqa_b200/build.py")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, fp, c_int, c_float, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.sqa_fwd.argtypes = [vp, vp, vp, vp, fp, Shape, c_int, c_float, vp]
+    lib.sqa_fwd.restype = c_int
+    lib.sqa_bwd_workspace_bytes.argtypes = [Shape]
+    lib.sqa_bwd_workspace_bytes.restype = sz
+    lib.sqa_bwd.argtypes = [vp, vp, vp, vp, vp, fp, vp, vp, vp, vp, sz, Shape, c_int, c_float, vp]
+    lib.sqa_bwd.restype = c_int
+    lib.sqa_status_string.argtypes = [c_int]
+    lib.sqa_status_string.restype = ctypes.c_char_p
+    lib.sqa_last_error.argtypes = []
+    lib.sqa_last_error.restype = ctypes.c_char_p
+    lib.sqa_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), c_int]
+    lib.sqa_device_status.restype = c_int
+    lib.sqa_version.argtypes = []
+    lib.sqa_version.restype = c_int
+    _lib = lib
+    return lib
+
+
+def _check(status: int):
+    if status != SQA_OK:
+        lib = load_library()
+        raise SqaError(status, f"{lib.sqa_status_string(status).decode()}: {lib.sqa_last_error().decode()}")
+
+
+def _stream(stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _need(t, name, shape, dtype):
+    import torch
+
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def shape_of(q, k) -> Shape:
+    B, N, Hq, dh = q.shape
+    Hkv = k.shape[2]
+    return Shape(B, N, Hq, Hkv, dh)
+
+
+def sqa_fwd(q, k, v, out=None, lse=None, causal: bool = False, scale: float = 0.0, stream=None):
+    """Forward.  q [B,N,H_q,dh], k/v [B,N,H_kv,dh] bf16 CUDA tensors.
+    Returns (out [B,N,H_q,dh] bf16, lse [B,H_q,N] fp32).  scale <= 0 means 1/sqrt(dh)."""
+    import torch
+
+    lib = load_library()
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q, k, v must be 4-D [B, N, H, dh]")
+    s = shape_of(q, k)
+    _need(q, "q", (s.B, s.N, s.H_q, s.dh), torch.bfloat16)
+    _need(k, "k", (s.B, s.N, s.H_kv, s.dh), torch.bfloat16)
+    _need(v, "v", (s.B, s.N, s.H_kv, s.dh), torch.bfloat16)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((s.B, s.H_q, s.N), dtype=torch.float32, device=q.device)
+    _need(out, "out", (s.B, s.N, s.H_q, s.dh), torch.bfloat16)
+    _need(lse, "lse", (s.B, s.H_q, s.N), torch.float32)
+    _check(lib.sqa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), s,
+                       int(bool(causal)), float(scale), _stream(stream)))
+    return out, lse
+
+
+def bwd_workspace_bytes(B: int, N: int, H_q: int, H_kv: int, dh: int) -> int:
+    return int(load_library().sqa_bwd_workspace_bytes(Shape(B, N, H_q, H_kv, dh)))
+
+
+def sqa_bwd(dout, q, k, v, out, lse, dq=None, dk=None, dv=None, workspace=None, causal: bool = False,
+            scale: float = 0.0, stream=None):
+    """Backward of sum(dout * out).  Returns (dq, dk, dv) as bf16 CUDA tensors."""
+    import torch
+
+    lib = load_library()
+    s = shape_of(q, k)
+    _need(q, "q", (s.B, s.N, s.H_q, s.dh), torch.bfloat16)
+    _need(k, "k", (s.B, s.N, s.H_kv, s.dh), torch.bfloat16)
+    _need(v, "v", (s.B, s.N, s.H_kv, s.dh), torch.bfloat16)
+    _need(dout, "dout", (s.B, s.N, s.H_q, s.dh), torch.bfloat16)
+    _need(out, "out", (s.B, s.N, s.H_q, s.dh), torch.bfloat16)
+    _need(lse, "lse", (s.B, s.H_q, s.N), torch.float32)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _need(dq, "dq", (s.B, s.N, s.H_q, s.dh), torch.bfloat16)
+    _need(dk, "dk", (s.B, s.N, s.H_kv, s.dh), torch.bfloat16)
+    _need(dv, "dv", (s.B, s.N, s.H_kv, s.dh), torch.bfloat16)
+    need = int(lib.sqa_bwd_workspace_bytes(s))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    _check(lib.sqa_bwd(dout.data_ptr(), q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                       lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                       workspace.numel() * workspace.element_size(), s, int(bool(causal)), float(scale),
+                       _stream(stream)))
+    return dq, dk, dv
+
+
+def device_status(clear: bool = True) -> int:
+    """Synchronise and return the device wait-status word (0 = no wait gave up)."""
+    lib = load_library()
+    w = ctypes.c_uint(0)
+    _check(lib.sqa_device_status(ctypes.byref(w), int(bool(clear))))
+    return int(w.value)

@@ -1,0 +1,214 @@
+// sqa_api.cu -- host side of the C ABI declared in include/sqa.h: argument
+// validation, TMA tensor-map encoding and kernel launches on the caller's
+// stream.  This is the only translation unit of libsqa.so.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "sqa.h"
+#include "sqa_bwd.cuh"
+#include "sqa_fwd.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+sqa_status fail(sqa_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+sqa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(SQA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Tensor map over a contiguous bf16 tensor [B][N][H][dh], seen by TMA as the
+// 4-D array {dh, H, N, B} (innermost first), with a box {panel, box_h, box_n, 1}.
+sqa_status make_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int dh, int panel,
+                    int box_h, int box_n) {
+  auto fn = encode_fn();
+  if (!fn) return fail(SQA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[4] = {(cuuint64_t)dh, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)dh * 2, (cuuint64_t)H * dh * 2, (cuuint64_t)N * H * dh * 2};
+  const cuuint32_t box[4] = {(cuuint32_t)panel, (cuuint32_t)box_h, (cuuint32_t)box_n, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUtensorMapSwizzle swz = panel * 2 == 32   ? CU_TENSOR_MAP_SWIZZLE_32B
+                                 : panel * 2 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                   : CU_TENSOR_MAP_SWIZZLE_128B;
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SQA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  return SQA_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+sqa_status check_shape(const sqa_shape& s) {
+  if (s.B < 1 || s.N < 1 || s.H_q < 1 || s.H_kv < 1 || s.dh < 1)
+    return fail(SQA_ERR_INVALID_ARG, "sizes must be positive (B=%d N=%d H_q=%d H_kv=%d dh=%d)", s.B, s.N,
+                s.H_q, s.H_kv, s.dh);
+  if (s.H_q % s.H_kv != 0)
+    return fail(SQA_ERR_INVALID_ARG, "H_q=%d is not a multiple of H_kv=%d", s.H_q, s.H_kv);
+  if (s.dh != 16 && s.dh != 32 && s.dh != 64 && s.dh != 128)
+    return fail(SQA_ERR_UNSUPPORTED, "head dim %d not supported (16, 32, 64 or 128)", s.dh);
+  if (s.H_q / s.H_kv > 128)
+    return fail(SQA_ERR_UNSUPPORTED, "group size H_q/H_kv=%d exceeds 128", s.H_q / s.H_kv);
+  if (s.B > 65535 || s.H_q > 65535)
+    return fail(SQA_ERR_UNSUPPORTED, "B and H_q must be at most 65535");
+  return SQA_OK;
+}
+
+sqa_status resolve_scale(float scale, int dh, float* out) {
+  if (std::isnan(scale) || std::isinf(scale)) return fail(SQA_ERR_INVALID_ARG, "scale is not finite");
+  *out = scale > 0.f ? scale : 1.f / std::sqrt(static_cast<float>(dh));
+  return SQA_OK;
+}
+
+template <typename Kernel>
+sqa_status set_smem(Kernel k, int bytes) {
+  // The attribute is per device; setting it on every call costs little.
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  return SQA_OK;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int DH>
+sqa_status launch_fwd(const void* q, const void* k, const void* v, void* out, float* lse, const sqa_shape& s,
+                      int causal, float scale, cudaStream_t stream) {
+  using Tr = sqa::FwdTraits<DH>;
+  sqa::FwdParams p{};
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.N = s.N;
+  p.Hq = s.H_q;
+  p.Hkv = s.H_kv;
+  p.g = s.H_q / s.H_kv;
+  p.T = Tr::BM / p.g;
+  p.rows = p.T * p.g;
+  p.n_qtiles = (s.N + p.T - 1) / p.T;
+  p.n_pairs = (p.n_qtiles + 1) / 2;
+  p.n_bh = s.B * s.H_kv;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * kLog2e;
+  const long long grid = static_cast<long long>(p.n_pairs) * p.n_bh;
+  if (grid > 0x7fffffffLL) return fail(SQA_ERR_UNSUPPORTED, "problem too large for one launch");
+
+  CUtensorMap mq, mk, mv;
+  sqa_status st;
+  if ((st = make_map(&mq, q, s.B, s.N, s.H_q, DH, Tr::PANEL, p.g, p.T)) != SQA_OK) return st;
+  if ((st = make_map(&mk, k, s.B, s.N, s.H_kv, DH, Tr::PANEL, 1, Tr::NK)) != SQA_OK) return st;
+  if ((st = make_map(&mv, v, s.B, s.N, s.H_kv, DH, Tr::PANEL, 1, Tr::NK)) != SQA_OK) return st;
+  if ((st = set_smem(sqa::sqa_fwd_kernel<DH>, Tr::SMEM_BYTES)) != SQA_OK) return st;
+  sqa::sqa_fwd_kernel<DH><<<static_cast<unsigned>(grid), Tr::THREADS, Tr::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "sqa_fwd launch");
+  return SQA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sqa_status sqa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, sqa_shape s, int causal,
+                   float scale, sqa_stream_t stream) {
+  g_last_error.clear();
+  if (!q || !k || !v || !out || !lse) return fail(SQA_ERR_INVALID_ARG, "null pointer argument");
+  sqa_status st = check_shape(s);
+  if (st != SQA_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4))
+    return fail(SQA_ERR_UNSUPPORTED, "q, k, v, out must be 16-byte aligned and lse 4-byte aligned");
+  float sc;
+  if ((st = resolve_scale(scale, s.dh, &sc)) != SQA_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  switch (s.dh) {
+    case 16: return launch_fwd<16>(q, k, v, out, lse, s, causal, sc, cs);
+    case 32: return launch_fwd<32>(q, k, v, out, lse, s, causal, sc, cs);
+    case 64: return launch_fwd<64>(q, k, v, out, lse, s, causal, sc, cs);
+    default: return launch_fwd<128>(q, k, v, out, lse, s, causal, sc, cs);
+  }
+}
+
+size_t sqa_bwd_workspace_bytes(sqa_shape s) {
+  if (check_shape(s) != SQA_OK) return 0;
+  return sqa::bwd_workspace_bytes(s.B, s.N, s.H_q, s.H_kv, s.dh);
+}
+
+sqa_status sqa_bwd(const void* dout, const void* q, const void* k, const void* v, const void* out, const float* lse,
+                   void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, sqa_shape s, int causal,
+                   float scale, sqa_stream_t stream) {
+  g_last_error.clear();
+  if (!dout || !q || !k || !v || !out || !lse || !dq || !dk || !dv || !workspace)
+    return fail(SQA_ERR_INVALID_ARG, "null pointer argument");
+  sqa_status st = check_shape(s);
+  if (st != SQA_OK) return st;
+  const void* bf[] = {dout, q, k, v, out, dq, dk, dv};
+  for (const void* ptr : bf)
+    if (!aligned(ptr, 16)) return fail(SQA_ERR_UNSUPPORTED, "bf16 tensors must be 16-byte aligned");
+  if (!aligned(lse, 4)) return fail(SQA_ERR_UNSUPPORTED, "lse must be 4-byte aligned");
+  if (!aligned(workspace, 256)) return fail(SQA_ERR_UNSUPPORTED, "workspace must be 256-byte aligned");
+  const size_t need = sqa::bwd_workspace_bytes(s.B, s.N, s.H_q, s.H_kv, s.dh);
+  if (workspace_bytes < need)
+    return fail(SQA_ERR_INVALID_ARG, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
+  float sc;
+  if ((st = resolve_scale(scale, s.dh, &sc)) != SQA_OK) return st;
+  return sqa::launch_bwd(dout, q, k, v, out, lse, dq, dk, dv, workspace, s.B, s.N, s.H_q, s.H_kv, s.dh,
+                         causal ? 1 : 0, sc, reinterpret_cast<cudaStream_t>(stream), encode_fn(), &g_last_error);
+}
+
+const char* sqa_status_string(sqa_status status) {
+  switch (status) {
+    case SQA_OK: return "ok";
+    case SQA_ERR_INVALID_ARG: return "invalid argument";
+    case SQA_ERR_UNSUPPORTED: return "unsupported";
+    case SQA_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+const char* sqa_last_error(void) { return g_last_error.c_str(); }
+
+sqa_status sqa_device_status(unsigned int* word, int clear) {
+  g_last_error.clear();
+  if (!word) return fail(SQA_ERR_INVALID_ARG, "null pointer argument");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  e = cudaMemcpyFromSymbol(word, sqa::g_wait_status, sizeof(unsigned int));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+  if (clear) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(sqa::g_wait_status, &zero, sizeof(unsigned int));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
+    e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  }
+  return SQA_OK;
+}
+
+int sqa_version(void) { return 100; }
+
+}  // extern "C"

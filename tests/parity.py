@@ -1,0 +1,42 @@
+"""Shared comparison helpers for the GPU parity tests.
+
+Tolerances (bf16 inputs, fp32 accumulation, bf16 outputs): max-abs error
+<= 2e-2 and relative Frobenius error <= 5e-3 for O, dQ, dK and dV; max-abs
+<= 1e-3 for lse (natural log, fp32 output).
+"""
+import numpy as np
+
+MAX_ABS = 2e-2
+REL_FRO = 5e-3
+LSE_ABS = 1e-3
+
+
+def to_np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def errors(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    diff = got - ref
+    max_abs = float(np.max(np.abs(diff))) if diff.size else 0.0
+    denom = float(np.linalg.norm(ref))
+    rel = float(np.linalg.norm(diff) / denom) if denom > 0 else float(np.linalg.norm(diff))
+    return max_abs, rel
+
+
+def assert_close(name, got, ref, max_abs=MAX_ABS, rel_fro=REL_FRO):
+    got = np.asarray(got, dtype=np.float64)
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    ma, rf = errors(got, ref)
+    assert ma <= max_abs and rf <= rel_fro, f"{name}: max-abs {ma:.3e} (<= {max_abs}), rel-Frobenius {rf:.3e} (<= {rel_fro})"
+    return ma, rf
+
+
+def assert_lse_close(name, got, ref, tol=LSE_ABS):
+    got = np.asarray(got, dtype=np.float64)
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    ma = float(np.max(np.abs(got - ref))) if got.size else 0.0
+    assert ma <= tol, f"{name}: lse max-abs {ma:.3e} (<= {tol})"
+    return ma

@@ -1,0 +1,107 @@
+"""The C ABI library on a machine without a GPU: it builds, loads, exports every
+symbol that include/sqa.h declares, and rejects bad arguments on the host
+before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_query_attention_sqa_b200 as sqa
+from sparse_query_attention_sqa_b200 import build as sqa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    sqa_build.build()
+    return sqa.load_library()
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(sqa_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert {"sqa_fwd", "sqa_bwd", "sqa_bwd_workspace_bytes", "sqa_last_error"} <= set(names)
+    for name in names:
+        assert hasattr(lib, name), f"{name} is declared but not exported"
+
+
+def test_library_is_in_tree_and_built_for_sm100a():
+    assert os.path.dirname(sqa.library_path()) == os.path.join(ROOT, "sparse_query_attention_sqa_b200")
+    with open(os.path.join(ROOT, "sparse_query_attention_sqa_b200", "build.py")) as f:
+        assert "arch=compute_100a,code=sm_100a" in f.read()
+
+
+def test_status_strings(lib):
+    assert lib.sqa_status_string(0) == b"ok"
+    assert lib.sqa_status_string(1) == b"invalid argument"
+    assert lib.sqa_version() >= 100
+
+
+def _fwd(lib, ptrs, shape, scale=0.0):
+    return lib.sqa_fwd(*ptrs, sqa.Shape(*shape), 1, ctypes.c_float(scale), None)
+
+
+GOOD = [0x10000, 0x20000, 0x30000, 0x40000, 0x50000]
+
+
+@pytest.mark.parametrize("shape,code", [
+    ((1, 8, 6, 4, 16), 1),     # H_q not a multiple of H_kv
+    ((0, 8, 8, 4, 16), 1),     # empty batch
+    ((1, 0, 8, 4, 16), 1),     # empty sequence
+    ((1, 8, 8, 0, 16), 1),     # no KV heads
+    ((1, 8, 8, 4, 48), 2),     # unsupported head dim
+    ((1, 8, 8, 4, 8), 2),      # unsupported head dim
+    ((1, 8, 256, 1, 16), 2),   # group larger than 128
+])
+def test_fwd_rejects_bad_shapes_before_launch(lib, shape, code):
+    assert _fwd(lib, GOOD, shape) == code
+    assert lib.sqa_last_error() != b""
+
+
+def test_fwd_rejects_null_and_misaligned_pointers(lib):
+    for i in range(5):
+        ptrs = list(GOOD)
+        ptrs[i] = 0
+        assert _fwd(lib, ptrs, (1, 8, 8, 4, 16)) == 1
+    ptrs = list(GOOD)
+    ptrs[0] += 8  # q not 16-byte aligned
+    assert _fwd(lib, ptrs, (1, 8, 8, 4, 16)) == 2
+    assert _fwd(lib, GOOD, (1, 8, 8, 4, 16), scale=float("nan")) == 1
+
+
+def test_bwd_rejects_bad_arguments_before_launch(lib):
+    s = sqa.Shape(1, 64, 8, 4, 16)
+    need = lib.sqa_bwd_workspace_bytes(s)
+    assert need > 0
+    p = [0x10000 * (i + 1) for i in range(10)]
+    # workspace too small
+    assert lib.sqa_bwd(*p, need - 1, s, 1, ctypes.c_float(0.0), None) == 1
+    # null pointer
+    q = list(p)
+    q[3] = 0
+    assert lib.sqa_bwd(*q, need, s, 1, ctypes.c_float(0.0), None) == 1
+    # misaligned workspace
+    q = list(p)
+    q[9] += 16
+    assert lib.sqa_bwd(*q, need, s, 1, ctypes.c_float(0.0), None) == 2
+    # bad shape
+    assert lib.sqa_bwd(*p, need, sqa.Shape(1, 64, 6, 4, 16), 1, ctypes.c_float(0.0), None) == 1
+    assert lib.sqa_bwd_workspace_bytes(sqa.Shape(1, 64, 6, 4, 16)) == 0
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(sqa, "_LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(sqa, "_lib", None)
+    with pytest.raises(ImportError):
+        sqa.load_library()

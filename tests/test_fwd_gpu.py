@@ -1,0 +1,105 @@
+"""GPU parity of sqa_fwd against the fp64 oracle, element by element."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_query_attention_sqa_b200.inputs import make_inputs
+from parity import assert_close, assert_lse_close, to_np
+
+pytestmark = pytest.mark.gpu
+
+# (B, N, H_q, H_kv, dh): several 128-row tiles, ragged tails, and every
+# group-size class (g = 1 MHA, 2, 3 and 6 which do not divide 128, 4, 16 MQA).
+SHAPES = [
+    (1, 1, 8, 4, 16),
+    (1, 7, 8, 4, 16),
+    (2, 300, 8, 4, 16),
+    (1, 1024, 8, 4, 16),
+    (2, 257, 16, 16, 16),
+    (2, 200, 16, 1, 16),
+    (1, 333, 12, 4, 16),
+    (1, 513, 6, 1, 16),
+    (2, 129, 16, 4, 16),
+    (1, 390, 8, 4, 32),
+    (1, 390, 8, 4, 64),
+    (2, 300, 8, 4, 128),
+    (1, 129, 4, 4, 128),
+]
+
+
+def run(cuda_lib, B, N, Hq, Hkv, dh, causal, seed=0, std=1.0, k_scale=1.0, scale=0.0):
+    q, k, v, _ = make_inputs(B, N, Hq, Hkv, dh, seed=seed, std=std, k_scale=k_scale)
+    out, lse = cuda_lib.sqa_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert cuda_lib.device_status() == 0
+    ref_out, ref_lse = oracle.sqa_fwd(q, k, v, causal, scale if scale > 0 else None)
+    return to_np(out), to_np(lse), ref_out, ref_lse
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_fwd_matches_oracle(cuda_lib, shape, causal):
+    out, lse, ref_out, ref_lse = run(cuda_lib, *shape, causal)
+    # lse alone checks the QK^T contraction and the softmax statistics;
+    # O additionally checks the PV contraction.
+    assert_lse_close("lse", lse, ref_lse)
+    assert_close("out", out, ref_out)
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+def test_zero_query_gives_prefix_mean(cuda_lib, causal):
+    """All-zero Q exercises the PV contraction independently of QK^T."""
+    B, N, Hq, Hkv, dh = 1, 300, 8, 4, 16
+    _, k, v, _ = make_inputs(B, N, Hq, Hkv, dh, seed=3)
+    q = torch.zeros(B, N, Hq, dh, dtype=torch.bfloat16)
+    out, lse = cuda_lib.sqa_fwd(q.cuda(), k.cuda(), v.cuda(), causal=causal)
+    ref_out, ref_lse = oracle.sqa_fwd(q, k, v, causal)
+    assert_lse_close("lse", to_np(lse), ref_lse)
+    assert_close("out", to_np(out), ref_out)
+
+
+def test_explicit_scale_and_seeds(cuda_lib):
+    for seed in (1, 2):
+        out, lse, ref_out, ref_lse = run(cuda_lib, 2, 300, 8, 4, 16, True, seed=seed, scale=0.25)
+        assert_lse_close("lse", lse, ref_lse)
+        assert_close("out", out, ref_out)
+
+
+def test_wide_score_range_rescales_exactly(cuda_lib):
+    """Large scores force the running maximum up many times along a row."""
+    out, lse, ref_out, ref_lse = run(cuda_lib, 1, 700, 8, 4, 16, False, std=2.0, scale=1.0)
+    assert_lse_close("lse", lse, ref_lse, tol=2e-3)
+    assert_close("out", out, ref_out)
+
+
+def test_outputs_fully_overwritten_and_inputs_untouched(cuda_lib):
+    B, N, Hq, Hkv, dh = 1, 200, 8, 4, 16
+    q, k, v, _ = make_inputs(B, N, Hq, Hkv, dh, seed=4)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    out = torch.full((B, N, Hq, dh), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B, Hq, N), float("nan"), dtype=torch.float32, device="cuda")
+    cuda_lib.sqa_fwd(qd, kd, vd, out=out, lse=lse, causal=True)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+    assert torch.equal(qd.cpu(), q) and torch.equal(kd.cpu(), k) and torch.equal(vd.cpu(), v)
+
+
+def test_deterministic(cuda_lib):
+    q, k, v, _ = make_inputs(2, 333, 8, 4, 16, seed=5)
+    a = cuda_lib.sqa_fwd(q.cuda(), k.cuda(), v.cuda(), causal=True)
+    b = cuda_lib.sqa_fwd(q.cuda(), k.cuda(), v.cuda(), causal=True)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_errors_launch_nothing(cuda_lib):
+    from sparse_query_attention_sqa_b200 import SqaError
+
+    q, k, v, _ = make_inputs(1, 64, 6, 4, 16)
+    with pytest.raises(SqaError) as e:
+        cuda_lib.sqa_fwd(q.cuda(), k.cuda(), v.cuda())
+    assert e.value.status == 1
+    q, k, v, _ = make_inputs(1, 64, 4, 4, 48)
+    with pytest.raises(SqaError) as e:
+        cuda_lib.sqa_fwd(q.cuda(), k.cuda(), v.cuda())
+    assert e.value.status == 2
