@@ -130,6 +130,85 @@ sqa_status launch_fwd(const void* q, const void* k, const void* v, void* out, fl
   return SQA_OK;
 }
 
+int grid_for(long long work, int threads) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long blocks = (work + threads - 1) / threads;
+  const long long cap = static_cast<long long>(sms) * 8;
+  return static_cast<int>(blocks < 1 ? 1 : (blocks > cap ? cap : blocks));
+}
+
+template <int DH>
+sqa_status launch_bwd(const void* dout, const void* q, const void* k, const void* v, const void* out,
+                      const float* lse, void* dq, void* dk, void* dv, void* workspace, const sqa_shape& s,
+                      int causal, float scale, cudaStream_t stream) {
+  using Tr = sqa::BwdTraits<DH>;
+  const sqa::BwdLayout L = sqa::bwd_layout(s.B, s.N, s.H_q, s.H_kv, DH);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* lse2 = reinterpret_cast<float*>(ws);
+  float* Dst = reinterpret_cast<float*>(ws + L.off_D);
+  float* dq_acc = reinterpret_cast<float*>(ws + L.off_dq);
+  const long long grid_main = static_cast<long long>(L.n_kt) * s.B * s.H_kv;
+  if (grid_main > 0x7fffffffLL) return fail(SQA_ERR_UNSUPPORTED, "problem too large for one launch");
+
+  sqa::BwdPrepParams pp{};
+  pp.dout = static_cast<const __nv_bfloat16*>(dout);
+  pp.out = static_cast<const __nv_bfloat16*>(out);
+  pp.lse = lse;
+  pp.lse2 = lse2;
+  pp.D = Dst;
+  pp.dq_acc = dq_acc;
+  pp.N = s.N;
+  pp.Hq = s.H_q;
+  pp.Hkv = s.H_kv;
+  pp.g = L.g;
+  pp.T = L.T;
+  pp.rows = L.rows;
+  pp.n_qt = L.n_qt;
+  pp.n_slots = static_cast<long long>(L.n_slots);
+  pp.dq_vec4 = static_cast<long long>(s.B) * s.N * s.H_q * DH / 4;
+  const long long prep_work = pp.n_slots > pp.dq_vec4 ? pp.n_slots : pp.dq_vec4;
+  sqa::sqa_bwd_prep_kernel<DH><<<grid_for(prep_work, 256), 256, 0, stream>>>(pp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "sqa_bwd prep launch");
+
+  CUtensorMap mq, mdo, mk, mv;
+  sqa_status st;
+  if ((st = make_map(&mq, q, s.B, s.N, s.H_q, DH, Tr::PANEL, L.g, L.T)) != SQA_OK) return st;
+  if ((st = make_map(&mdo, dout, s.B, s.N, s.H_q, DH, Tr::PANEL, L.g, L.T)) != SQA_OK) return st;
+  if ((st = make_map(&mk, k, s.B, s.N, s.H_kv, DH, Tr::PANEL, 1, Tr::NK)) != SQA_OK) return st;
+  if ((st = make_map(&mv, v, s.B, s.N, s.H_kv, DH, Tr::PANEL, 1, Tr::NK)) != SQA_OK) return st;
+  if ((st = set_smem(sqa::sqa_bwd_kernel<DH>, Tr::SMEM_BYTES)) != SQA_OK) return st;
+  sqa::BwdParams p{};
+  p.lse2 = lse2;
+  p.D = Dst;
+  p.dq_acc = dq_acc;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.N = s.N;
+  p.Hq = s.H_q;
+  p.Hkv = s.H_kv;
+  p.g = L.g;
+  p.T = L.T;
+  p.rows = L.rows;
+  p.n_qt = L.n_qt;
+  p.n_bh = s.B * s.H_kv;
+  p.causal = causal;
+  p.scale_log2 = scale * kLog2e;
+  p.scale = scale;
+  sqa::sqa_bwd_kernel<DH><<<static_cast<unsigned>(grid_main), Tr::THREADS, Tr::SMEM_BYTES, stream>>>(mq, mdo, mk,
+                                                                                                     mv, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "sqa_bwd main launch");
+
+  const long long n_vec8 = static_cast<long long>(s.B) * s.N * s.H_q * DH / 8;
+  sqa::sqa_bwd_dq_kernel<<<grid_for(n_vec8, 256), 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq),
+                                                                    n_vec8, scale);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "sqa_bwd dq launch");
+  return SQA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -176,8 +255,14 @@ sqa_status sqa_bwd(const void* dout, const void* q, const void* k, const void* v
     return fail(SQA_ERR_INVALID_ARG, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
   float sc;
   if ((st = resolve_scale(scale, s.dh, &sc)) != SQA_OK) return st;
-  return sqa::launch_bwd(dout, q, k, v, out, lse, dq, dk, dv, workspace, s.B, s.N, s.H_q, s.H_kv, s.dh,
-                         causal ? 1 : 0, sc, reinterpret_cast<cudaStream_t>(stream), encode_fn(), &g_last_error);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const int c = causal ? 1 : 0;
+  switch (s.dh) {
+    case 16: return launch_bwd<16>(dout, q, k, v, out, lse, dq, dk, dv, workspace, s, c, sc, cs);
+    case 32: return launch_bwd<32>(dout, q, k, v, out, lse, dq, dk, dv, workspace, s, c, sc, cs);
+    case 64: return launch_bwd<64>(dout, q, k, v, out, lse, dq, dk, dv, workspace, s, c, sc, cs);
+    default: return launch_bwd<128>(dout, q, k, v, out, lse, dq, dk, dv, workspace, s, c, sc, cs);
+  }
 }
 
 const char* sqa_status_string(sqa_status status) {

@@ -67,8 +67,10 @@ def test_explicit_scale_and_seeds(cuda_lib):
 
 
 def test_wide_score_range_rescales_exactly(cuda_lib):
-    """Large scores force the running maximum up many times along a row."""
-    out, lse, ref_out, ref_lse = run(cuda_lib, 1, 700, 8, 4, 16, False, std=2.0, scale=1.0)
+    """Large scores (scale 3, score std 12) force the running maximum up many
+    times along a row.  V keeps unit variance so that |O| stays where bf16
+    output rounding is below the max-abs bound."""
+    out, lse, ref_out, ref_lse = run(cuda_lib, 1, 700, 8, 4, 16, False, scale=3.0)
     assert_lse_close("lse", lse, ref_lse, tol=2e-3)
     assert_close("out", out, ref_out)
 
