@@ -375,7 +375,10 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     for (int i = 0; i < nq; ++i) {
       const int s = i % QS, qt = qt_first + i;
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full, i & 1, abort_flag, kSiteSoftmax));
+      // The statistics were bulk-copied into this stage; wait on that copy
+      // directly (the stage is not refilled before this tile's ds_ready).
+      ok = __all_sync(0xffffffffu, mbar_wait(qd_full(s), (i / QS) & 1, abort_flag, kSiteSoftmax) &&
+                                       mbar_wait(s_full, i & 1, abort_flag, kSiteSoftmax));
       if (!ok) break;
       tc_fence_after();
       const float* lse2 = reinterpret_cast<const float*>(smem + Tr::OFF_STAT + s * 1024);
