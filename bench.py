@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Benchmark of the Sparse Query Attention hot path on B200.
+
+One step is one pass of the whole path over one batch: sqa_fwd followed by
+sqa_bwd (for forward-only workloads, sqa_fwd alone).  The default workload is
+the SQAT-m training-step attention: B=32, N=1024, dh=16 (d=256 split over 16
+heads), H_q=8 query heads over H_kv=4 key/value heads, causal, forward and
+backward (SQAT-m model card, "Architecture details"; message length 1024).
+
+Throughput counts 4*B*H_q*N^2*dh FLOPs for the forward (halved when causal)
+and 3.5 times that for forward plus backward.  Inputs are seeded synthetic bf16
+Gaussians; several buffer sets whose total exceeds the 126 MB L2 are used in
+rotation, so every step reads its inputs from HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
+
+Under torchrun every rank runs its own copy of the workload (independent
+batches, no collective on the data path): weak scaling.  One JSON line is
+printed by rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 1024 * 1024
+SM_COUNT = 148
+SM_MAX_MHZ = 1965.0
+# Special-function unit: 16 exp2 results per clock per SM (4 per sub-partition).
+SFU_EXP2_PER_CLK_PER_SM = 16
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="sqatm_train_sqa")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="time budget of the CPU-baseline sample")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+def counted_flops(w) -> float:
+    fwd = 4.0 * w.B * w.Hq * w.N * w.N * w.dh
+    if w.causal:
+        fwd /= 2
+    return fwd * (3.5 if w.backward else 1.0)
+
+
+def score_elements(w) -> float:
+    """Unmasked (query row, key) pairs over all query heads: one exp2 each."""
+    per = w.N * (w.N + 1) / 2 if w.causal else float(w.N) * w.N
+    return w.B * w.Hq * per
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def oracle_subproblem(w, seed=0):
+    """One independent slice of the workload: batch entry 0, KV head 0 and its
+    g query heads (the oracle's work on it scales with the counted FLOPs)."""
+    from sparse_query_attention_sqa_b200.inputs import make_inputs
+
+    g = w.Hq // w.Hkv
+    q, k, v, dout = make_inputs(1, w.N, g, 1, w.dh, seed=seed, std=w.std, k_scale=w.k_scale, with_dout=w.backward)
+    sub = type(w)(name=w.name + "_slice", B=1, N=w.N, Hq=g, Hkv=1, dh=w.dh, causal=w.causal, backward=w.backward,
+                  std=w.std, k_scale=w.k_scale, scale=w.scale)
+    return sub, (q, k, v, dout)
+
+
+def run_oracle_step(sub, data):
+    import oracle
+
+    q, k, v, dout = data
+    oracle.sqa_fwd(q, k, v, sub.causal, sub.softmax_scale)
+    if sub.backward:
+        oracle.sqa_bwd(q, k, v, dout, sub.causal, sub.softmax_scale)
+
+
+def omp_threads() -> int:
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def cpu_baseline(w, seconds):
+    sub, data = oracle_subproblem(w)
+    run_oracle_step(sub, data)  # builds the oracle and warms caches
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        run_oracle_step(sub, data)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    rate = counted_flops(sub) * n / el / 1e12
+    return {"value": rate, "unit": "TFLOP/s", "cores": omp_threads(), "kind": "oracle",
+            "sample": f"fp64 oracle fwd{'+bwd' if w.backward else ''} on batch entry 0, KV head 0 and its "
+                      f"{sub.Hq} query heads (N={w.N}, dh={w.dh}), {n} runs in {el:.1f} s"}
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    def __init__(self, enabled, index):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        if not enabled:
+            return
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(index),
+                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[4:8]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- GPU arm
+def alloc_set(w, q, k, v, dout, lib, torch):
+    dev = "cuda"
+    s = {"q": q.to(dev), "k": k.to(dev), "v": v.to(dev)}
+    s["out"] = torch.empty_like(s["q"])
+    s["lse"] = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+    if w.backward:
+        s["dout"] = dout.to(dev)
+        s["dq"] = torch.empty_like(s["q"])
+        s["dk"] = torch.empty_like(s["k"])
+        s["dv"] = torch.empty_like(s["v"])
+        s["ws"] = torch.empty(lib.bwd_workspace_bytes(w.B, w.N, w.Hq, w.Hkv, w.dh), dtype=torch.uint8, device=dev)
+    return s
+
+
+def set_bytes(s) -> int:
+    return sum(t.numel() * t.element_size() for t in s.values())
+
+
+def step(lib, w, s):
+    lib.sqa_fwd(s["q"], s["k"], s["v"], out=s["out"], lse=s["lse"], causal=w.causal, scale=w.scale)
+    if w.backward:
+        lib.sqa_bwd(s["dout"], s["q"], s["k"], s["v"], s["out"], s["lse"], dq=s["dq"], dk=s["dk"], dv=s["dv"],
+                    workspace=s["ws"], causal=w.causal, scale=w.scale)
+
+
+def roofline_for(w, kernel_name, ms, peaks, peak_kind):
+    if w.dh <= 32:
+        # exp-bound: one exp2 per unmasked score element on the special-function unit
+        units = score_elements(w)
+        achieved = units / (ms * 1e-3) / 1e9
+        peak = SM_COUNT * SFU_EXP2_PER_CLK_PER_SM * SM_MAX_MHZ * 1e6 / 1e9
+        return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Gexp2/s", "frac": achieved / peak,
+                "traffic": traffic_for(kernel_name, w), "kernel": kernel_name,
+                "peak_source": "derived: 148 SMs x 16 exp2/clk/SM x 1965 MHz"}
+    flops = 4.0 * w.B * w.Hq * w.N * w.N * w.dh / (2 if w.causal else 1)
+    if kernel_name.startswith("sqa_bwd"):
+        flops *= 2.5
+    achieved = flops / (ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": traffic_for(kernel_name, w), "kernel": kernel_name, "peak_source": f"{peak_kind} bf16_tflops"}
+
+
+def traffic_for(kernel_name, w):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current source."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            table = json.load(f)
+    except Exception:
+        return None
+    h = hashlib.sha256()
+    for fn in ("sqa_device.cuh", "sqa_fwd.cuh", "sqa_bwd.cuh"):
+        with open(os.path.join(ROOT, "sparse_query_attention_sqa_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    for e in table.get("entries", []):
+        if e.get("kernel") == kernel_name and e.get("workload") == w.name and e.get("source_sha256") == h.hexdigest():
+            return e.get("dram_bytes_per_launch")
+    return None
+
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import sparse_query_attention_sqa_b200 as lib
+    from sparse_query_attention_sqa_b200.inputs import workload_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    lib.load_library()
+
+    q, k, v, dout = workload_inputs(w, seed=rank)
+    first = alloc_set(w, q, k, v, dout, lib, torch)
+    n_sets = max(2, math.ceil(2 * L2_BYTES / set_bytes(first)))
+    sets = [first] + [alloc_set(w, q, k, v, dout, lib, torch) for _ in range(n_sets - 1)]
+
+    # Which kernel dominates: time both main kernels once per set during warm-up.
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    kern = {}
+    for i in range(max(args.warmup, 3)):
+        s = sets[i % n_sets]
+        e0, e1, e2, e3 = ev(), ev(), ev(), ev()
+        lib.set_timing_events(0, e0, e1)
+        lib.set_timing_events(1, e2, e3)
+        step(lib, w, s)
+        lib.set_timing_events(0)
+        lib.set_timing_events(1)
+        torch.cuda.synchronize()
+        kern.setdefault("sqa_fwd_kernel", []).append(e0.elapsed_time(e1))
+        if w.backward:
+            kern.setdefault("sqa_bwd_kernel", []).append(e2.elapsed_time(e3))
+    assert lib.device_status() == 0, "a kernel wait gave up during warm-up"
+    dominant = max(kern, key=lambda n: statistics.median(kern[n]))
+    dom_idx = 0 if dominant == "sqa_fwd_kernel" else 1
+
+    # Timed region: K steps, per-step events around the dominant kernel.
+    starts = [ev() for _ in range(args.steps)]
+    stops = [ev() for _ in range(args.steps)]
+    t0, t1 = ev(), ev()
+    clocks = ClockSampler(not args.no_clocks and rank == 0, local)
+    time.sleep(0.2 if clocks.proc else 0)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    t0.record()
+    for i in range(args.steps):
+        lib.set_timing_events(dom_idx, starts[i], stops[i])
+        step(lib, w, sets[i % n_sets])
+    t1.record()
+    lib.set_timing_events(dom_idx)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall = time.perf_counter() - wall0
+    clk = clocks.stop()
+    ms_total = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([ms_total], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    dom_ms = statistics.fmean(a.elapsed_time(b) for a, b in zip(starts, stops))
+    assert lib.device_status() == 0, "a kernel wait gave up during the timed region"
+    ms_step = ms_total / args.steps
+    flops_job = counted_flops(w) * world
+    value = flops_job / (ms_step * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+
+    # End to end through the public API with host buffers: pinned inputs copied
+    # in, the step, outputs copied back, all inside the timed region.
+    host_in = {n: sets[0][n].cpu().pin_memory() for n in ("q", "k", "v", "dout") if n in sets[0]}
+    outs = ("out", "lse", "dq", "dk", "dv") if w.backward else ("out", "lse")
+    host_out = {n: torch.empty(sets[0][n].shape, dtype=sets[0][n].dtype, pin_memory=True) for n in outs}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    e_steps = max(3, min(args.e2e_steps, args.steps))
+
+    def e2e_step(s):
+        for n, t in host_in.items():
+            s[n].copy_(t, non_blocking=True)
+        step(lib, w, s)
+        for n in outs:
+            host_out[n].copy_(s[n], non_blocking=True)
+
+    for i in range(3):
+        e2e_step(sets[i % n_sets])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a, b = ev(), ev()
+    a.record()
+    for i in range(e_steps):
+        e2e_step(sets[i % n_sets])
+    b.record()
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        dist.barrier()
+
+    line = None
+    if rank == 0:
+        line = {
+            "metric": f"SQA attention {'fwd+bwd' if w.backward else 'fwd'} TFLOP/s ({w.note})",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded Gaussian bf16 inputs)",
+            "config": {"workload": w.name, "B": w.B, "N": w.N, "H_q": w.Hq, "H_kv": w.Hkv, "dh": w.dh,
+                       "causal": w.causal, "pass": "fwd+bwd" if w.backward else "fwd",
+                       "parallelism": f"{world} independent replicas" if world > 1 else "single GPU",
+                       "l2": f"{n_sets} rotating buffer sets of {set_bytes(first) / 2**20:.0f} MiB "
+                             f"(> L2 in total), no flush"},
+            "tokens_per_s": w.B * w.N * world / (ms_step * 1e-3),
+            "tensor_frac_of_bf16_peak": value / peaks["bf16_tflops"],
+            "roofline": roofline_for(w, dominant, dom_ms, peaks, peak_kind),
+            "kernel_ms": {n: statistics.median(v) for n, v in kern.items()},
+            "e2e": {"value": flops_job / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": args.steps * (4 if w.backward else 1),
+            "clocks": clk,
+            "wall_s_timed_region": wall,
+        }
+    # CPU baseline: rank 0 at N=1 only, after all GPU work.
+    if world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return line
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return None
+    sub, data = oracle_subproblem(w)
+    # Each step is the oracle's fwd(+bwd) on one batch entry's first KV group.
+    # Cap the executed steps so the whole run stays within a few minutes.
+    run_oracle_step(sub, data)
+    t = time.perf_counter()
+    run_oracle_step(sub, data)
+    one = time.perf_counter() - t
+    budget = 150.0
+    warm = min(args.warmup, max(0, int(0.1 * budget / one)))
+    steps = max(1, min(args.steps, int(0.9 * budget / one)))
+    for _ in range(warm):
+        run_oracle_step(sub, data)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        run_oracle_step(sub, data)
+    el = time.perf_counter() - t0
+    ms = el / steps * 1e3
+    value = counted_flops(sub) / (ms * 1e-3) / 1e12
+    sample = (f"fp64 oracle fwd{'+bwd' if w.backward else ''} on batch entry 0, KV head 0 and its {sub.Hq} "
+              f"query heads (N={w.N}, dh={w.dh}); {steps} of the requested {args.steps} steps run")
+    return {"impl": "reference", "metric": f"SQA attention {'fwd+bwd' if w.backward else 'fwd'} TFLOP/s ({w.note})",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "N": w.N, "H_q": w.Hq, "H_kv": w.Hkv, "dh": w.dh,
+                       "causal": w.causal, "pass": "fwd+bwd" if w.backward else "fwd"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": omp_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    from sparse_query_attention_sqa_b200.inputs import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    line = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

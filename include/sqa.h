@@ -100,6 +100,17 @@ const char *sqa_last_error(void);
  */
 sqa_status sqa_device_status(unsigned int *word, int clear);
 
+/*
+ * Optional timing hook for benchmarks.  While set on the calling host thread,
+ * sqa_fwd (kernel = 0) or sqa_bwd (kernel = 1) records `start` on its stream
+ * just before launching its main attention kernel and `stop` just after it, so
+ * the caller can time that one kernel with cudaEventElapsedTime.  start and
+ * stop are cudaEvent_t handles owned by the caller; pass NULL for both to turn
+ * the hook off.  Returns SQA_ERR_INVALID_ARG for another kernel index or when
+ * only one of the two events is given.
+ */
+sqa_status sqa_set_timing_events(int kernel, void *start, void *stop);
+
 /* Library version as an integer (major * 10000 + minor * 100 + patch). */
 int sqa_version(void);
 

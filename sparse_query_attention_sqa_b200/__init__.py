@@ -13,7 +13,7 @@ import os
 
 __all__ = [
     "SqaError", "load_library", "library_path", "sqa_fwd", "sqa_bwd", "bwd_workspace_bytes",
-    "device_status", "Shape",
+    "device_status", "set_timing_events", "Shape",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -59,6 +59,8 @@ def load_library():
     lib.sqa_last_error.restype = ctypes.c_char_p
     lib.sqa_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), c_int]
     lib.sqa_device_status.restype = c_int
+    lib.sqa_set_timing_events.argtypes = [c_int, vp, vp]
+    lib.sqa_set_timing_events.restype = c_int
     lib.sqa_version.argtypes = []
     lib.sqa_version.restype = c_int
     _lib = lib
@@ -154,6 +156,15 @@ def sqa_bwd(dout, q, k, v, out, lse, dq=None, dk=None, dv=None, workspace=None, 
                        workspace.numel() * workspace.element_size(), s, int(bool(causal)), float(scale),
                        _stream(stream)))
     return dq, dk, dv
+
+
+def set_timing_events(kernel: int, start=None, stop=None):
+    """Record torch.cuda.Event `start`/`stop` around the main kernel of sqa_fwd
+    (kernel=0) or sqa_bwd (kernel=1) on this thread; None turns it off."""
+    lib = load_library()
+    s = ctypes.c_void_p(start.cuda_event if start is not None else None)
+    e = ctypes.c_void_p(stop.cuda_event if stop is not None else None)
+    _check(lib.sqa_set_timing_events(int(kernel), s, e))
 
 
 def device_status(clear: bool = True) -> int:

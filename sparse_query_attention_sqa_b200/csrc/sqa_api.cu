@@ -16,6 +16,9 @@
 namespace {
 
 thread_local std::string g_last_error;
+thread_local cudaEvent_t g_timing[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+
+sqa_status record_timing(int kernel, int which, cudaStream_t stream);
 
 sqa_status fail(sqa_status st, const char* fmt, ...) {
   char buf[512];
@@ -61,6 +64,14 @@ sqa_status make_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int 
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SQA_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  return SQA_OK;
+}
+
+sqa_status record_timing(int kernel, int which, cudaStream_t stream) {
+  cudaEvent_t ev = g_timing[kernel][which];
+  if (!ev) return SQA_OK;
+  cudaError_t e = cudaEventRecord(ev, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord (timing hook)");
   return SQA_OK;
 }
 
@@ -124,10 +135,11 @@ sqa_status launch_fwd(const void* q, const void* k, const void* v, void* out, fl
   if ((st = make_map(&mk, k, s.B, s.N, s.H_kv, DH, Tr::PANEL, 1, Tr::NK)) != SQA_OK) return st;
   if ((st = make_map(&mv, v, s.B, s.N, s.H_kv, DH, Tr::PANEL, 1, Tr::NK)) != SQA_OK) return st;
   if ((st = set_smem(sqa::sqa_fwd_kernel<DH>, Tr::SMEM_BYTES)) != SQA_OK) return st;
+  if ((st = record_timing(0, 0, stream)) != SQA_OK) return st;
   sqa::sqa_fwd_kernel<DH><<<static_cast<unsigned>(grid), Tr::THREADS, Tr::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "sqa_fwd launch");
-  return SQA_OK;
+  return record_timing(0, 1, stream);
 }
 
 int grid_for(long long work, int threads) {
@@ -196,10 +208,12 @@ sqa_status launch_bwd(const void* dout, const void* q, const void* k, const void
   p.causal = causal;
   p.scale_log2 = scale * kLog2e;
   p.scale = scale;
+  if ((st = record_timing(1, 0, stream)) != SQA_OK) return st;
   sqa::sqa_bwd_kernel<DH><<<static_cast<unsigned>(grid_main), Tr::THREADS, Tr::SMEM_BYTES, stream>>>(mq, mdo, mk,
                                                                                                      mv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "sqa_bwd main launch");
+  if ((st = record_timing(1, 1, stream)) != SQA_OK) return st;
 
   const long long n_vec8 = static_cast<long long>(s.B) * s.N * s.H_q * DH / 8;
   sqa::sqa_bwd_dq_kernel<<<grid_for(n_vec8, 256), 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq),
@@ -291,6 +305,15 @@ sqa_status sqa_device_status(unsigned int* word, int clear) {
     e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
   }
+  return SQA_OK;
+}
+
+sqa_status sqa_set_timing_events(int kernel, void* start, void* stop) {
+  g_last_error.clear();
+  if (kernel < 0 || kernel > 1) return fail(SQA_ERR_INVALID_ARG, "kernel index %d is not 0 (fwd) or 1 (bwd)", kernel);
+  if ((start == nullptr) != (stop == nullptr)) return fail(SQA_ERR_INVALID_ARG, "give both events or neither");
+  g_timing[kernel][0] = static_cast<cudaEvent_t>(start);
+  g_timing[kernel][1] = static_cast<cudaEvent_t>(stop);
   return SQA_OK;
 }
 
