@@ -162,8 +162,15 @@ def set_timing_events(kernel: int, start=None, stop=None):
     """Record torch.cuda.Event `start`/`stop` around the main kernel of sqa_fwd
     (kernel=0) or sqa_bwd (kernel=1) on this thread; None turns it off."""
     lib = load_library()
-    s = ctypes.c_void_p(start.cuda_event if start is not None else None)
-    e = ctypes.c_void_p(stop.cuda_event if stop is not None else None)
+
+    def handle(ev):
+        if ev is None:
+            return ctypes.c_void_p(None)
+        if not ev.cuda_event:  # torch creates the CUDA event on its first record
+            ev.record()
+        return ctypes.c_void_p(ev.cuda_event)
+
+    s, e = handle(start), handle(stop)
     _check(lib.sqa_set_timing_events(int(kernel), s, e))
 
 
