@@ -101,6 +101,15 @@ const char *sqa_last_error(void);
 sqa_status sqa_device_status(unsigned int *word, int clear);
 
 /*
+ * Where the first wait that gave up on the current device was: info[0] = 1 if
+ * one did (0 otherwise), info[1] = block index, info[2] = (role << 16) |
+ * barrier index within the kernel's barrier block (roles: 0 producer, 1 MMA
+ * issuer, 2 softmax, 3 epilogue or converter, 4 drain), info[3] = (thread << 8)
+ * | phase parity.  Synchronises the device; clear != 0 resets the record.
+ */
+sqa_status sqa_device_timeout_info(unsigned int info[4], int clear);
+
+/*
  * Optional timing hook for benchmarks.  While set on the calling host thread,
  * sqa_fwd (kernel = 0) or sqa_bwd (kernel = 1) records `start` on its stream
  * just before launching its main attention kernel and `stop` just after it, so

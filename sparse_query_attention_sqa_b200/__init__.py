@@ -13,7 +13,7 @@ import os
 
 __all__ = [
     "SqaError", "load_library", "library_path", "sqa_fwd", "sqa_bwd", "bwd_workspace_bytes",
-    "device_status", "set_timing_events", "Shape",
+    "device_status", "timeout_info", "set_timing_events", "Shape",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -59,6 +59,8 @@ def load_library():
     lib.sqa_last_error.restype = ctypes.c_char_p
     lib.sqa_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), c_int]
     lib.sqa_device_status.restype = c_int
+    lib.sqa_device_timeout_info.argtypes = [ctypes.POINTER(ctypes.c_uint), c_int]
+    lib.sqa_device_timeout_info.restype = c_int
     lib.sqa_set_timing_events.argtypes = [c_int, vp, vp]
     lib.sqa_set_timing_events.restype = c_int
     lib.sqa_version.argtypes = []
@@ -172,6 +174,17 @@ def set_timing_events(kernel: int, start=None, stop=None):
 
     s, e = handle(start), handle(stop)
     _check(lib.sqa_set_timing_events(int(kernel), s, e))
+
+
+def timeout_info(clear: bool = True):
+    """First wait that gave up on this device: None, or a dict (block, role, barrier, thread, parity)."""
+    lib = load_library()
+    info = (ctypes.c_uint * 4)()
+    _check(lib.sqa_device_timeout_info(info, int(bool(clear))))
+    if info[0] == 0:
+        return None
+    return {"block": int(info[1]), "role": int(info[2] >> 16), "barrier": int(info[2] & 0xFFFF),
+            "thread": int(info[3] >> 8), "parity": int(info[3] & 0xFF)}
 
 
 def device_status(clear: bool = True) -> int:

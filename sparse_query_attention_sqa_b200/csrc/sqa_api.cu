@@ -11,6 +11,7 @@
 
 #include "sqa.h"
 #include "sqa_bwd.cuh"
+#include "sqa_bwd_tf32.cuh"
 #include "sqa_fwd.cuh"
 
 namespace {
@@ -190,7 +191,6 @@ sqa_status launch_bwd(const void* dout, const void* q, const void* k, const void
   if ((st = make_map(&mdo, dout, s.B, s.N, s.H_q, DH, Tr::PANEL, L.g, L.T)) != SQA_OK) return st;
   if ((st = make_map(&mk, k, s.B, s.N, s.H_kv, DH, Tr::PANEL, 1, Tr::NK)) != SQA_OK) return st;
   if ((st = make_map(&mv, v, s.B, s.N, s.H_kv, DH, Tr::PANEL, 1, Tr::NK)) != SQA_OK) return st;
-  if ((st = set_smem(sqa::sqa_bwd_kernel<DH>, Tr::SMEM_BYTES)) != SQA_OK) return st;
   sqa::BwdParams p{};
   p.lse2 = lse2;
   p.D = Dst;
@@ -208,9 +208,19 @@ sqa_status launch_bwd(const void* dout, const void* q, const void* k, const void
   p.causal = causal;
   p.scale_log2 = scale * kLog2e;
   p.scale = scale;
-  if ((st = record_timing(1, 0, stream)) != SQA_OK) return st;
-  sqa::sqa_bwd_kernel<DH><<<static_cast<unsigned>(grid_main), Tr::THREADS, Tr::SMEM_BYTES, stream>>>(mq, mdo, mk,
-                                                                                                     mv, p);
+  if constexpr (DH <= 32) {
+    // dh 16 and 32: tf32 gradient contractions, half-tile pipelining
+    using T32 = sqa::BwdTf32Traits<DH>;
+    if ((st = set_smem(sqa::sqa_bwd_tf32_kernel<DH>, T32::SMEM_BYTES)) != SQA_OK) return st;
+    if ((st = record_timing(1, 0, stream)) != SQA_OK) return st;
+    sqa::sqa_bwd_tf32_kernel<DH><<<static_cast<unsigned>(grid_main), T32::THREADS, T32::SMEM_BYTES, stream>>>(
+        mq, mdo, mk, mv, p);
+  } else {
+    if ((st = set_smem(sqa::sqa_bwd_kernel<DH>, Tr::SMEM_BYTES)) != SQA_OK) return st;
+    if ((st = record_timing(1, 0, stream)) != SQA_OK) return st;
+    sqa::sqa_bwd_kernel<DH><<<static_cast<unsigned>(grid_main), Tr::THREADS, Tr::SMEM_BYTES, stream>>>(mq, mdo, mk,
+                                                                                                       mv, p);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "sqa_bwd main launch");
   if ((st = record_timing(1, 1, stream)) != SQA_OK) return st;
@@ -304,6 +314,22 @@ sqa_status sqa_device_status(unsigned int* word, int clear) {
     if (e != cudaSuccess) return cuda_fail(e, "clearing the device status word");
     e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  }
+  return SQA_OK;
+}
+
+sqa_status sqa_device_timeout_info(unsigned int info[4], int clear) {
+  g_last_error.clear();
+  if (!info) return fail(SQA_ERR_INVALID_ARG, "null pointer argument");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  e = cudaMemcpyFromSymbol(info, sqa::g_timeout_info, 4 * sizeof(unsigned int));
+  if (e != cudaSuccess) return cuda_fail(e, "reading the timeout record");
+  if (clear) {
+    const unsigned int zero[4] = {0, 0, 0, 0};
+    e = cudaMemcpyToSymbol(sqa::g_timeout_info, zero, sizeof(zero));
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the timeout record");
   }
   return SQA_OK;
 }

@@ -12,6 +12,10 @@ namespace sqa {
 
 // Per-device status word; a bit is set when a wait inside a kernel gives up.
 static __device__ unsigned int g_wait_status;
+// First wait that gave up on this device: {1, block, (site << 16) | barrier index,
+// (thread << 8) | parity}.  Barrier blocks start 1024-byte aligned, so the low
+// ten bits of a barrier's shared address give its index in the block.
+static __device__ unsigned int g_timeout_info[4];
 
 namespace dev {
 
@@ -79,6 +83,11 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       *abort_flag = 1;
       atomicOr(&g_wait_status, 1u << site);
+      if (atomicCAS(&g_timeout_info[0], 0u, 1u) == 0u) {
+        g_timeout_info[1] = blockIdx.x;
+        g_timeout_info[2] = (site << 16) | ((bar & 0x3FFu) >> 3);
+        g_timeout_info[3] = (threadIdx.x << 8) | parity;
+      }
       return false;
     }
   }
@@ -248,6 +257,41 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Register rebalancing between warpgroups (all four warps of a warpgroup run
+// the same instruction).  The increases must fit in what the decreases free
+// from the launch allocation.
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+// Packed pair arithmetic on the fp32x2 path: (a0,a1)*(b0,b1)+(c0,c1) and (a0,a1)+(b0,b1).
+__device__ __forceinline__ void ffma2(float& r0, float& r1, float a0, float a1, float b0, float b1, float c0,
+                                      float c1) {
+  asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(r0), "=f"(r1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void fadd2(float& r0, float& r1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(r0), "=f"(r1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
 }  // namespace dev

@@ -9,13 +9,17 @@
 // head and one value head; arXiv 2510.01817 abstract: score FLOPs scale with H_q).
 //
 // Roles (384 threads):
-//   warp 0      TMA producer: Q tiles once, then K/V tiles through a ring of stages
-//   warp 1      TMEM allocator and MMA issuer (one thread):
+//   warps 0-3   softmax for Q tile 0; warps 4-7 softmax for Q tile 1 (a warp
+//               reaches TMEM lanes 32*(warp%4) .. +31, so each warpgroup covers
+//               the 128 rows of its tile)
+//   warp 8      TMA producer: Q tiles once, then 64-key K/V tiles through a ring
+//   warp 9      TMEM allocator and MMA issuer (one thread); warps 10-11 idle
 //                 S_t = Q_t K_j^T  (tcgen05, both operands K-major in smem)
 //                 O_t += P_t V_j   (tcgen05, P from TMEM, V MN-major in smem)
-//   warps 4-7   softmax for Q tile 0; warps 8-11 softmax for Q tile 1
-// TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+dh), O_1 [384,384+dh).
-// P_t (bf16) overwrites the first half of S_t's columns in place.
+// TMEM (512 columns): S_t has two 64-column buffers at 128 t + 64 (j % 2), so the
+// tensor core computes S_t for key tile j + 1 while the softmax warps work on
+// tile j; O_t sits at 256 + 128 t.  P_t (bf16 pairs) overwrites the first 32
+// columns of its S buffer.
 //
 // Online softmax (exact): each row keeps a reference maximum m (log2 units) and
 // l = sum 2^(s*scale*log2e - m).  m is raised only when a tile's maximum exceeds
@@ -24,6 +28,7 @@
 #pragma once
 
 #include "sqa_device.cuh"
+#include "sqa_tmem_wide.cuh"
 
 namespace sqa {
 
@@ -43,27 +48,28 @@ struct FwdParams {
 template <int DH>
 struct FwdTraits {
   static constexpr int BM = 128;  // stacked rows per Q tile
-  static constexpr int NK = 128;  // keys per K/V tile
+  static constexpr int NK = 64;   // keys per K/V tile
   static constexpr int PANEL = DH < 64 ? DH : 64;  // elements per swizzled row segment
   static constexpr int NPANEL = DH / PANEL;
   static constexpr int ROWB = PANEL * 2;  // bytes per row segment
   static constexpr uint32_t LAYOUT = ROWB == 32 ? 6u : (ROWB == 64 ? 4u : 2u);
   static constexpr int Q_BYTES = BM * DH * 2;
   static constexpr int KV_BYTES = NK * DH * 2;
-  static constexpr int STAGES = DH <= 32 ? 4 : (DH == 64 ? 3 : 2);
+  static constexpr int STAGES = DH <= 32 ? 8 : (DH == 64 ? 4 : 3);
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
-  static constexpr int N_BARS = 1 + 2 * STAGES + 6 + 1;
+  // q_full | kv_full[S] | kv_empty[S] | s_full[2][2] | p_full[2][2] | o_done[2] | o_final[2] | drain
+  static constexpr int N_BARS = 1 + 2 * STAGES + 4 + 4 + 2 + 2 + 1;
   static constexpr int SMEM_USED = OFF_BAR + N_BARS * 8 + 16;
   // Ask for enough shared memory that only one CTA fits per SM (each CTA holds
   // all 512 TMEM columns), plus slack to align the base to 1024 bytes.
   static constexpr int SMEM_BYTES = (SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024) + 1024;
-  // TMEM column of S_t and O_t
-  __host__ __device__ static constexpr uint32_t tm_s(int t) { return t ? 128u : 0u; }
-  __host__ __device__ static constexpr uint32_t tm_o(int t) { return t ? 384u : 256u; }
+  __host__ __device__ static constexpr uint32_t tm_s(int t, int buf) { return 128u * t + 64u * buf; }
+  __host__ __device__ static constexpr uint32_t tm_o(int t) { return 256u + 128u * t; }
   static constexpr int THREADS = 384;
+  static constexpr int WARP_PRODUCER = 8, WARP_MMA = 9;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   static_assert(DH % 16 == 0 && DH <= 128, "head dim");
 };
@@ -74,7 +80,7 @@ __global__ void __launch_bounds__(384, 1)
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using Tr = FwdTraits<DH>;
   using namespace dev;
-  constexpr int BM = Tr::BM, NK = Tr::NK, ROWB = Tr::ROWB, PANEL = Tr::PANEL;
+  constexpr int BM = Tr::BM, NK = Tr::NK, ROWB = Tr::ROWB, PANEL = Tr::PANEL, ST = Tr::STAGES;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -97,27 +103,33 @@ __global__ void __launch_bounds__(384, 1)
   const int nkv1 = has1 ? kv_tiles(qt0 + 1) : 0;
   const int nkv = max(nkv0, nkv1);
 
-  // Barriers: q_full | kv_full[S] | kv_empty[S] | s_full[2] | p_full[2] | o_final[2] | drain
   const uint32_t bar0 = sbase + Tr::OFF_BAR;
   const uint32_t q_full = bar0;
   auto kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto kv_empty = [&](int s) { return bar0 + 8u * (1 + Tr::STAGES + s); };
-  auto s_full = [&](int t) { return bar0 + 8u * (1 + 2 * Tr::STAGES + t); };
-  auto p_full = [&](int t) { return bar0 + 8u * (3 + 2 * Tr::STAGES + t); };
-  auto o_final = [&](int t) { return bar0 + 8u * (5 + 2 * Tr::STAGES + t); };
-  const uint32_t drain = bar0 + 8u * (7 + 2 * Tr::STAGES);
+  auto kv_empty = [&](int s) { return bar0 + 8u * (1 + ST + s); };
+  auto s_full = [&](int t, int buf) { return bar0 + 8u * (1 + 2 * ST + 2 * t + buf); };
+  // P of key tile j is announced on the barrier of its S buffer (j % 2): with two
+  // S buffers a softmax warpgroup can finish tiles j and j + 1 before the MMA
+  // issuer looks, and one barrier per buffer keeps each at most one phase ahead.
+  auto p_full = [&](int t, int buf) { return bar0 + 8u * (5 + 2 * ST + 2 * t + buf); };
+  auto o_done = [&](int t) { return bar0 + 8u * (9 + 2 * ST + t); };
+  auto o_final = [&](int t) { return bar0 + 8u * (11 + 2 * ST + t); };
+  const uint32_t drain = bar0 + 8u * (13 + 2 * ST);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Tr::OFF_BAR + Tr::N_BARS * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < Tr::STAGES; ++s) {
+    for (int s = 0; s < ST; ++s) {
       mbar_init(kv_full(s), 1);
       mbar_init(kv_empty(s), 1);
     }
     for (int t = 0; t < 2; ++t) {
-      mbar_init(s_full(t), 1);
-      mbar_init(p_full(t), 128);
+      mbar_init(s_full(t, 0), 1);
+      mbar_init(s_full(t, 1), 1);
+      mbar_init(p_full(t, 0), 128);
+      mbar_init(p_full(t, 1), 128);
+      mbar_init(o_done(t), 1);
       mbar_init(o_final(t), 1);
     }
     mbar_init(drain, 1);
@@ -136,7 +148,7 @@ __global__ void __launch_bounds__(384, 1)
       }
     fence_async_smem();
   }
-  if (warp == 1) {
+  if (warp == Tr::WARP_MMA) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -145,7 +157,7 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == Tr::WARP_PRODUCER) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_map(&tmQ);
@@ -159,104 +171,104 @@ __global__ void __launch_bounds__(384, 1)
                       kvh * p.g, (qt0 + t) * p.T, b);
       int issued = 0;
       for (int j = 0; j < nkv; ++j) {
-        const int s = j % Tr::STAGES;
-        if (j >= Tr::STAGES &&
-            !mbar_wait(kv_empty(s), ((j / Tr::STAGES) - 1) & 1, abort_flag, kSiteProducer))
-          break;
+        const int s = j % ST;
+        if (j >= ST && !mbar_wait(kv_empty(s), ((j / ST) - 1) & 1, abort_flag, kSiteProducer)) break;
         mbar_expect_tx(kv_full(s), 2u * Tr::KV_BYTES);
         for (int pn = 0; pn < Tr::NPANEL; ++pn) {
-          tma_load_4d(sbase + Tr::OFF_K + s * Tr::KV_BYTES + pn * NK * ROWB, &tmK, kv_full(s),
-                      pn * PANEL, kvh, j * NK, b);
-          tma_load_4d(sbase + Tr::OFF_V + s * Tr::KV_BYTES + pn * NK * ROWB, &tmV, kv_full(s),
-                      pn * PANEL, kvh, j * NK, b);
+          tma_load_4d(sbase + Tr::OFF_K + s * Tr::KV_BYTES + pn * NK * ROWB, &tmK, kv_full(s), pn * PANEL, kvh,
+                      j * NK, b);
+          tma_load_4d(sbase + Tr::OFF_V + s * Tr::KV_BYTES + pn * NK * ROWB, &tmV, kv_full(s), pn * PANEL, kvh,
+                      j * NK, b);
         }
         issued = j + 1;
       }
       if (*abort_flag) {  // let in-flight copies land before the CTA exits
         mbar_wait_drain(q_full, 0);
-        for (int j = max(0, issued - Tr::STAGES); j < issued; ++j)
-          mbar_wait_drain(kv_full(j % Tr::STAGES), (j / Tr::STAGES) & 1);
+        for (int j = max(0, issued - ST); j < issued; ++j) mbar_wait_drain(kv_full(j % ST), (j / ST) & 1);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == Tr::WARP_MMA) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, NK, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, DH, false, true);
       const uint32_t q_addr = sbase + Tr::OFF_Q, k_addr = sbase + Tr::OFF_K, v_addr = sbase + Tr::OFF_V;
-      auto issue_qk = [&](int t, int s) {
+      auto issue_qk = [&](int t, int j) {
+        const int s = j % ST;
 #pragma unroll
         for (int ks = 0; ks < DH / 16; ++ks) {
           const uint32_t pn = (ks * 16) / PANEL, off = ((ks * 16) % PANEL) * 2;
-          const uint64_t a = smem_desc(q_addr + t * Tr::Q_BYTES + pn * BM * ROWB + off, 16, 8 * ROWB,
-                                       Tr::LAYOUT);
-          const uint64_t bd = smem_desc(k_addr + s * Tr::KV_BYTES + pn * NK * ROWB + off, 16, 8 * ROWB,
-                                        Tr::LAYOUT);
-          mma_ss(tmem + Tr::tm_s(t), a, bd, idesc_qk, ks > 0 ? 1u : 0u);
+          const uint64_t a =
+              smem_desc(q_addr + t * Tr::Q_BYTES + pn * BM * ROWB + off, 16, 8 * ROWB, Tr::LAYOUT);
+          const uint64_t bd =
+              smem_desc(k_addr + s * Tr::KV_BYTES + pn * NK * ROWB + off, 16, 8 * ROWB, Tr::LAYOUT);
+          mma_ss(tmem + Tr::tm_s(t, j & 1), a, bd, idesc_qk, ks > 0 ? 1u : 0u);
         }
+        mma_commit(s_full(t, j & 1));
       };
-      auto issue_pv = [&](int t, int s, bool acc) {
+      auto issue_pv = [&](int t, int j) {
+        const int s = j % ST;
 #pragma unroll
         for (int ks = 0; ks < NK / 16; ++ks) {
-          const uint64_t bd = smem_desc(v_addr + s * Tr::KV_BYTES + ks * 16 * ROWB, NK * ROWB, 8 * ROWB,
-                                        Tr::LAYOUT);
-          mma_ts(tmem + Tr::tm_o(t), tmem + Tr::tm_s(t) + ks * 8, bd, idesc_pv,
-                 (acc || ks > 0) ? 1u : 0u);
+          const uint64_t bd =
+              smem_desc(v_addr + s * Tr::KV_BYTES + ks * 16 * ROWB, NK * ROWB, 8 * ROWB, Tr::LAYOUT);
+          mma_ts(tmem + Tr::tm_o(t), tmem + Tr::tm_s(t, j & 1) + ks * 8, bd, idesc_pv,
+                 (j > 0 || ks > 0) ? 1u : 0u);
         }
+        mma_commit(o_done(t));
       };
-      bool ok = mbar_wait(q_full, 0, abort_flag, kSiteMma) &&
-                mbar_wait(kv_full(0), 0, abort_flag, kSiteMma);
-      if (ok) {
-        tc_fence_after();
-        issue_qk(0, 0);
-        mma_commit(s_full(0));
-        if (has1) {
-          issue_qk(1, 0);
-          mma_commit(s_full(1));
+      const int nkv_t[2] = {nkv0, nkv1};
+      int loaded = 0;  // key tiles whose kv_full phase has been observed
+      auto ensure_loaded = [&](int j) {
+        while (loaded <= j) {
+          if (!mbar_wait(kv_full(loaded % ST), (loaded / ST) & 1, abort_flag, kSiteMma)) return false;
+          ++loaded;
         }
+        tc_fence_after();
+        return true;
+      };
+      bool ok = mbar_wait(q_full, 0, abort_flag, kSiteMma);
+      // Prologue: S for key tiles 0 and 1 of both Q tiles.
+      for (int j = 0; ok && j < 2 && j < nkv; ++j) {
+        ok = ensure_loaded(j);
+        for (int t = 0; ok && t < 2; ++t)
+          if (j < nkv_t[t]) issue_qk(t, j);
       }
       for (int j = 0; ok && j < nkv; ++j) {
-        const int s = j % Tr::STAGES, sn = (j + 1) % Tr::STAGES;
-        bool next_ready = false;
         for (int t = 0; t < 2 && ok; ++t) {
-          const int nkv_t = t ? nkv1 : nkv0;
-          if (j >= nkv_t) continue;
-          if (!mbar_wait(p_full(t), j & 1, abort_flag, kSiteMma)) {
+          if (j >= nkv_t[t]) continue;
+          if (!mbar_wait(p_full(t, j & 1), (j >> 1) & 1, abort_flag, kSiteMma)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          issue_pv(t, s, j > 0);
-          if (j + 1 < nkv_t) {
-            if (!next_ready) {
-              if (!mbar_wait(kv_full(sn), ((j + 1) / Tr::STAGES) & 1, abort_flag, kSiteMma)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              next_ready = true;
+          issue_pv(t, j);
+          if (j + 2 < nkv_t[t]) {
+            // S_t for tile j + 2 reuses this buffer: the PV just issued reads P
+            // from it first (MMAs from one thread execute in order).
+            if (!ensure_loaded(j + 2)) {
+              ok = false;
+              break;
             }
-            issue_qk(t, sn);
-            mma_commit(s_full(t));
-          } else {
-            mma_commit(o_final(t));
+            issue_qk(t, j + 2);
           }
+          if (j + 1 == nkv_t[t]) mma_commit(o_final(t));
         }
-        mma_commit(kv_empty(s));
+        mma_commit(kv_empty(j % ST));
       }
       if (!ok) {  // wait for issued MMAs before TMEM is released
         mma_commit(drain);
         mbar_wait_drain(drain, 0);
       }
     }
-  } else if (warp >= 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax
-    const int t = (warp - 4) >> 2;
+    const int t = warp >> 2;
     const int nkv_t = t ? nkv1 : nkv0;
     const int qt = qt0 + t;
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t tS = lane_addr + Tr::tm_s(t), tO = lane_addr + Tr::tm_o(t);
+    const uint32_t tO = lane_addr + Tr::tm_o(t);
     const int tok = qt * p.T + row / p.g;
     const int head = kvh * p.g + row % p.g;
     const bool row_valid = row < p.rows && tok < p.N;
@@ -266,34 +278,45 @@ __global__ void __launch_bounds__(384, 1)
     for (int j = 0; ok && j < nkv_t; ++j) {
       // Every lane waits; the verdict is made warp-uniform so that the
       // warp-wide TMEM instructions below are never reached divergently.
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full(t), j & 1, abort_flag, kSiteSoftmax));
+      ok = __all_sync(0xffffffffu, mbar_wait(s_full(t, j & 1), (j >> 1) & 1, abort_flag, kSiteSoftmax));
       if (!ok) break;
       tc_fence_after();
+      const uint32_t tS = lane_addr + Tr::tm_s(t, j & 1);
       const int k0 = j * NK;
       const bool masked = (k0 + NK > p.N) || (p.causal && k0 + NK - 1 > qt * p.T);
-      // last visible key of this tile, relative to k0 (may be negative)
-      const int last = masked ? min(p.N - 1, p.causal ? tok : p.N - 1) - k0 : NK - 1;
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < NK / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS + c * 32, r);
-        if (masked) {
+      uint32_t sr[NK];
+      tmem_ld32x2(tS, tS + 32, sr);
+      if (masked) {
+        // last visible key of this tile, relative to k0 (may be negative)
+        const int last = min(p.N - 1, p.causal ? tok : p.N - 1) - k0;
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (c * 32 + i <= last) mx = fmaxf(mx, __uint_as_float(r[i]));
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(r[i]));
-        }
+        for (int i = 0; i < NK; ++i)
+          if (i > last) sr[i] = __float_as_uint(-INFINITY);
       }
+      // Row maximum: eight independent chains of three-input maxima.
+      float acc[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        acc[c] = fmax3(__uint_as_float(sr[c]), __uint_as_float(sr[8 + c]), __uint_as_float(sr[16 + c]));
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        acc[c] = fmax3(acc[c], __uint_as_float(sr[24 + c]), __uint_as_float(sr[32 + c]));
+        acc[c] = fmax3(acc[c], __uint_as_float(sr[40 + c]), __uint_as_float(sr[48 + c]));
+        acc[c] = fmaxf(acc[c], __uint_as_float(sr[56 + c]));
+      }
+      const float mx =
+          fmax3(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], acc[5]), fmaxf(acc[6], acc[7]));
       const float mnew = fmaxf(m, mx * sl2);
       const bool raise = mnew > m + 8.f;
       const float alpha = (raise && m != -INFINITY) ? ex2(m - mnew) : 1.f;
       if (__any_sync(0xffffffffu, alpha != 1.f)) {
-        // O holds P*V of the earlier tiles: the MMA that wrote it completed
-        // before s_full fired for this tile.  Lanes that keep their reference
-        // multiply by 1.
+        // O must hold P*V of every earlier tile before it is rescaled: wait for
+        // the PV of tile j - 1 (o_done is at most one phase behind here).
+        if (j > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(o_done(t), (j - 1) & 1, abort_flag, kSiteSoftmax));
+          if (!ok) break;
+          tc_fence_after();
+        }
 #pragma unroll 1
         for (int c = 0; c < DH; c += 16) {
           uint32_t r[16];
@@ -305,28 +328,27 @@ __global__ void __launch_bounds__(384, 1)
       }
       l *= alpha;
       if (raise) m = mnew;
-      const float mref = m == -INFINITY ? 0.f : m;
-#pragma unroll 1
-      for (int c = 0; c < NK / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS + c * 32, r);
-        uint32_t pk[16];
+      // Masked scores are -inf, so their P is exactly 0 (the scale is positive).
+      const float nref = m == -INFINITY ? 0.f : -m;
+      float sum0[8], sum1[8];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float p0 = ex2(fmaf(__uint_as_float(r[i]), sl2, -mref));
-          float p1 = ex2(fmaf(__uint_as_float(r[i + 1]), sl2, -mref));
-          if (masked) {
-            if (c * 32 + i > last) p0 = 0.f;
-            if (c * 32 + i + 1 > last) p1 = 0.f;
-          }
-          l += p0 + p1;
-          pk[i >> 1] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(tS + c * 16, pk);
+      for (int c = 0; c < 8; ++c) sum0[c] = sum1[c] = 0.f;
+      uint32_t pk[NK / 2];
+#pragma unroll
+      for (int i = 0; i < NK / 2; ++i) {
+        float x0, x1;
+        ffma2(x0, x1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), sl2, sl2, nref, nref);
+        const float p0 = ex2(x0), p1 = ex2(x1);
+        fadd2(sum0[i & 7], sum1[i & 7], sum0[i & 7], sum1[i & 7], p0, p1);
+        pk[i] = pack_bf16x2(p0, p1);
       }
+      tmem_st32(tS, pk);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) fadd2(sum0[c], sum1[c], sum0[c], sum1[c], sum0[c + 4], sum1[c + 4]);
+      l += ((sum0[0] + sum1[0]) + (sum0[1] + sum1[1])) + ((sum0[2] + sum1[2]) + (sum0[3] + sum1[3]));
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full(t));
+      mbar_arrive(p_full(t, j & 1));
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_final(t), 0, abort_flag, kSiteEpilogue));
     if (ok) {
@@ -359,7 +381,7 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 512);
+  if (warp == Tr::WARP_MMA) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace sqa
