@@ -85,6 +85,35 @@ sqa_status sqa_bwd(const void *dout, const void *q, const void *k, const void *v
                    size_t workspace_bytes, sqa_shape s, int causal, float scale,
                    sqa_stream_t stream);
 
+/*
+ * Largest scratch, in bytes, that sqa_bwd_static_scratch can use (64 MiB).
+ */
+#define SQA_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/*
+ * sqa_bwd without a workspace argument, for callers that cannot allocate
+ * device memory: a plugin inside a framework that owns every device
+ * allocation (a cudaMalloc there bypasses the framework's pool and can
+ * synchronise the whole device), or code that must not allocate once a step
+ * has started.  The paper has no counterpart to this entry point.
+ *
+ * Arguments, layouts, results and errors are those of sqa_bwd.  The scratch
+ * that sqa_bwd takes from the caller lives here in one file-scope device array
+ * of SQA_STATIC_SCRATCH_BYTES, which every GPU that loads the library holds
+ * until the process exits; shapes whose sqa_bwd_workspace_bytes() exceeds it
+ * are rejected with SQA_ERR_UNSUPPORTED before anything is launched.  Nothing
+ * is allocated or freed by this call.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current), so make that first call before any stream capture.  All
+ * calls share the one array and it keeps the last call's contents; the
+ * kernels clear what must start at zero.  Calls whose GPU work overlaps (on
+ * different streams, or from different threads) race on the array: order them.
+ */
+sqa_status sqa_bwd_static_scratch(const void *dout, const void *q, const void *k, const void *v,
+                                  const void *out, const float *lse, void *dq, void *dk, void *dv,
+                                  sqa_shape s, int causal, float scale, sqa_stream_t stream);
+
 /* Static text for a status code. */
 const char *sqa_status_string(sqa_status status);
 

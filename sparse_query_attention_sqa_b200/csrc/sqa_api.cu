@@ -233,6 +233,31 @@ sqa_status launch_bwd(const void* dout, const void* q, const void* k, const void
   return SQA_OK;
 }
 
+// Scratch for sqa_bwd_static_scratch: one device array per GPU that loads the
+// library.  In host code the name is only a handle; its device address comes
+// from cudaGetSymbolAddress, looked up once per device and cached.
+static __device__ __align__(256) unsigned char g_static_scratch[SQA_STATIC_SCRATCH_BYTES];
+
+std::mutex g_static_scratch_mu;
+constexpr int kMaxDevices = 128;
+void* g_static_scratch_addr[kMaxDevices] = {};
+
+sqa_status static_scratch_address(void** addr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(SQA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (!g_static_scratch_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress (static scratch)");
+    g_static_scratch_addr[dev] = p;
+  }
+  *addr = g_static_scratch_addr[dev];
+  return SQA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -287,6 +312,21 @@ sqa_status sqa_bwd(const void* dout, const void* q, const void* k, const void* v
     case 64: return launch_bwd<64>(dout, q, k, v, out, lse, dq, dk, dv, workspace, s, c, sc, cs);
     default: return launch_bwd<128>(dout, q, k, v, out, lse, dq, dk, dv, workspace, s, c, sc, cs);
   }
+}
+
+sqa_status sqa_bwd_static_scratch(const void* dout, const void* q, const void* k, const void* v, const void* out,
+                                  const float* lse, void* dq, void* dk, void* dv, sqa_shape s, int causal,
+                                  float scale, sqa_stream_t stream) {
+  g_last_error.clear();
+  sqa_status st = check_shape(s);
+  if (st != SQA_OK) return st;
+  const size_t need = sqa::bwd_workspace_bytes(s.B, s.N, s.H_q, s.H_kv, s.dh);
+  if (need > SQA_STATIC_SCRATCH_BYTES)
+    return fail(SQA_ERR_UNSUPPORTED, "this shape needs %zu bytes of scratch; the static scratch holds %u (use sqa_bwd)",
+                need, SQA_STATIC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  if ((st = static_scratch_address(&scratch)) != SQA_OK) return st;
+  return sqa_bwd(dout, q, k, v, out, lse, dq, dk, dv, scratch, SQA_STATIC_SCRATCH_BYTES, s, causal, scale, stream);
 }
 
 const char* sqa_status_string(sqa_status status) {
