@@ -127,8 +127,15 @@ sqa_status launch_fwd(const void* q, const void* k, const void* v, void* out, fl
   p.n_bh = s.B * s.H_kv;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * kLog2e;
-  const long long grid = static_cast<long long>(p.n_pairs) * p.n_bh;
-  if (grid > 0x7fffffffLL) return fail(SQA_ERR_UNSUPPORTED, "problem too large for one launch");
+  const long long items = static_cast<long long>(p.n_pairs) * p.n_bh;
+  if (items > 0x7fffffffLL) return fail(SQA_ERR_UNSUPPORTED, "problem too large for one launch");
+  p.n_items = static_cast<int>(items);
+  // Persistent kernel: at most one CTA per SM, each walking several work items.
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "querying the SM count");
+  const long long grid = items < sms ? items : sms;
 
   CUtensorMap mq, mk, mv;
   sqa_status st;
@@ -138,7 +145,7 @@ sqa_status launch_fwd(const void* q, const void* k, const void* v, void* out, fl
   if ((st = set_smem(sqa::sqa_fwd_kernel<DH>, Tr::SMEM_BYTES)) != SQA_OK) return st;
   if ((st = record_timing(0, 0, stream)) != SQA_OK) return st;
   sqa::sqa_fwd_kernel<DH><<<static_cast<unsigned>(grid), Tr::THREADS, Tr::SMEM_BYTES, stream>>>(mq, mk, mv, p);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "sqa_fwd launch");
   return record_timing(0, 1, stream);
 }

@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(384, 1)
                         const BwdParams p) {
   using Tr = BwdTf32Traits<DH>;
   using namespace dev;
-  constexpr int BM = Tr::BM, NK = Tr::NK, ROWB = Tr::ROWB, ROWB32 = Tr::ROWB32, QS = Tr::QS;
+  constexpr int BM = Tr::BM, NK = Tr::NK, ROWB = Tr::ROWB, QS = Tr::QS;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);

@@ -67,13 +67,13 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
-// Wait for the phase of `bar` with the given parity.  Gives up when another
+// Wait for the phase of `bar` with the given parity (mbar_wait below is the
+// entry point).  Gives up when another
 // role of the CTA has raised `abort_flag`, or after kWaitLimitNs (then it
 // raises the flag and records `site` in the device status word).  Returns
 // true when the phase completed.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                       unsigned site) {
-  if (mbar_test(bar, parity)) return true;
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                            unsigned site) {
   const unsigned long long t0 = global_timer_ns();
   while (true) {
 #pragma unroll 1
@@ -91,6 +91,12 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
       return false;
     }
   }
+}
+
+// Completed phases cost one test; only real waits take the bounded slow path.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, unsigned site) {
+  if (mbar_test(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort_flag, site);
 }
 
 // Bounded wait used only on the abort path, to let in-flight copies and MMAs

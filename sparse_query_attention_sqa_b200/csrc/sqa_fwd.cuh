@@ -1,6 +1,6 @@
 // sqa_fwd.cuh -- Sparse Query Attention forward on sm_100a.
 //
-// One CTA owns one key/value head of one batch entry and two Q tiles.  A Q tile
+// Work item: one key/value head of one batch entry and two Q tiles.  A Q tile
 // stacks the g = H_q / H_kv query heads that share the key/value head: its 128
 // MMA rows are (token, head) pairs, row r = t * g + head, which is exactly how
 // [B][N][H_q][dh] stores the group's heads side by side, so one TMA box
@@ -8,18 +8,23 @@
 // used by all heads of its group (GQA summary, "The idea": a group shares one key
 // head and one value head; arXiv 2510.01817 abstract: score FLOPs scale with H_q).
 //
+// The kernel is persistent: one CTA per SM walks a list of work items, heaviest
+// first, so the loads and the first QK^T of the next item overlap the end of
+// the current one.  The K/V ring and every barrier phase run on across items.
+//
 // Roles (384 threads):
 //   warps 0-3   softmax for Q tile 0; warps 4-7 softmax for Q tile 1 (a warp
 //               reaches TMEM lanes 32*(warp%4) .. +31, so each warpgroup covers
-//               the 128 rows of its tile)
-//   warp 8      TMA producer: Q tiles once, then 64-key K/V tiles through a ring
-//   warp 9      TMEM allocator and MMA issuer (one thread); warps 10-11 idle
+//               the 128 rows of its tile), plus the O / lse epilogue
+//   warp 8      TMA producer: Q tiles per item, 64-key K/V tiles through a ring
+//   warps 9-10  MMA issuers, one thread each, for Q tiles 0 and 1 (warp 9 also
+//               allocates TMEM); warp 11 idle
 //                 S_t = Q_t K_j^T  (tcgen05, both operands K-major in smem)
 //                 O_t += P_t V_j   (tcgen05, P from TMEM, V MN-major in smem)
-// TMEM (512 columns): S_t has two 64-column buffers at 128 t + 64 (j % 2), so the
-// tensor core computes S_t for key tile j + 1 while the softmax warps work on
-// tile j; O_t sits at 256 + 128 t.  P_t (bf16 pairs) overwrites the first 32
-// columns of its S buffer.
+// TMEM (512 columns): S_t has two 64-column buffers at 128 t + 64 (step % 2), so
+// the tensor core computes S_t for the next key tile while the softmax warps work
+// on the current one; O_t sits at 256 + 128 t.  P_t (bf16 pairs) overwrites the
+// first 32 columns of its S buffer.
 //
 // Online softmax (exact): each row keeps a reference maximum m (log2 units) and
 // l = sum 2^(s*scale*log2e - m).  m is raised only when a tile's maximum exceeds
@@ -41,6 +46,7 @@ struct FwdParams {
   int n_qtiles;  // ceil(N / T) per (batch, kv head)
   int n_pairs;   // ceil(n_qtiles / 2)
   int n_bh;      // B * Hkv
+  int n_items;   // n_pairs * n_bh
   int causal;
   float scale_log2;  // scale * log2(e)
 };
@@ -55,13 +61,15 @@ struct FwdTraits {
   static constexpr uint32_t LAYOUT = ROWB == 32 ? 6u : (ROWB == 64 ? 4u : 2u);
   static constexpr int Q_BYTES = BM * DH * 2;
   static constexpr int KV_BYTES = NK * DH * 2;
+  static constexpr int QBUF = DH <= 64 ? 2 : 1;  // Q-tile pairs in flight
   static constexpr int STAGES = DH <= 32 ? 8 : (DH == 64 ? 4 : 3);
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
+  static constexpr int OFF_K = OFF_Q + QBUF * 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
-  // q_full | kv_full[S] | kv_empty[S] | s_full[2][2] | p_full[2][2] | o_done[2] | o_final[2] | drain
-  static constexpr int N_BARS = 1 + 2 * STAGES + 4 + 4 + 2 + 2 + 1;
+  // q_full[QB] | q_empty[QB] | kv_full[S] | kv_empty[S] | s_full[2][2] | p_full[2][2] |
+  // o_done[2] | o_final[2] | o_free[2] | drain[2]
+  static constexpr int N_BARS = 2 * QBUF + 2 * STAGES + 4 + 4 + 2 + 2 + 2 + 2;
   static constexpr int SMEM_USED = OFF_BAR + N_BARS * 8 + 16;
   // Ask for enough shared memory that only one CTA fits per SM (each CTA holds
   // all 512 TMEM columns), plus slack to align the base to 1024 bytes.
@@ -74,13 +82,43 @@ struct FwdTraits {
   static_assert(DH % 16 == 0 && DH <= 128, "head dim");
 };
 
+// The r-th work item of this CTA in a snake order over the heaviest-first item
+// list (even rounds left to right, odd rounds right to left), which evens out
+// the per-CTA totals; -1 when the CTA has no r-th item.
+__device__ __forceinline__ int fwd_item(int r, int n_items) {
+  const int G = gridDim.x, c = blockIdx.x;
+  const long long item = static_cast<long long>(r) * G + ((r & 1) ? (G - 1 - c) : c);
+  return item < n_items ? static_cast<int>(item) : -1;
+}
+
+struct FwdItem {
+  int b, kvh, qt0, nkv0, nkv1, nkv;
+  bool has1;
+};
+
+__device__ __forceinline__ FwdItem fwd_decode(const FwdParams& p, int item, int NK) {
+  FwdItem it;
+  const int pair = p.n_pairs - 1 - item / p.n_bh;  // latest tokens (heaviest under a causal mask) first
+  const int bh = item % p.n_bh;
+  it.b = bh / p.Hkv;
+  it.kvh = bh % p.Hkv;
+  it.qt0 = 2 * pair;
+  it.has1 = it.qt0 + 1 < p.n_qtiles;
+  const int end0 = p.causal ? min(p.N, (it.qt0 + 1) * p.T) : p.N;
+  const int end1 = p.causal ? min(p.N, (it.qt0 + 2) * p.T) : p.N;
+  it.nkv0 = (end0 + NK - 1) / NK;
+  it.nkv1 = it.has1 ? (end1 + NK - 1) / NK : 0;
+  it.nkv = max(it.nkv0, it.nkv1);
+  return it;
+}
+
 template <int DH>
 __global__ void __launch_bounds__(384, 1)
     sqa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using Tr = FwdTraits<DH>;
   using namespace dev;
-  constexpr int BM = Tr::BM, NK = Tr::NK, ROWB = Tr::ROWB, PANEL = Tr::PANEL, ST = Tr::STAGES;
+  constexpr int BM = Tr::BM, NK = Tr::NK, ROWB = Tr::ROWB, PANEL = Tr::PANEL, ST = Tr::STAGES, QB = Tr::QBUF;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -89,40 +127,31 @@ __global__ void __launch_bounds__(384, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Heaviest Q-tile pairs (the latest tokens, under a causal mask) go first.
-  const int pair = p.n_pairs - 1 - static_cast<int>(blockIdx.x / p.n_bh);
-  const int bh = blockIdx.x % p.n_bh;
-  const int b = bh / p.Hkv, kvh = bh % p.Hkv;
-  const int qt0 = 2 * pair;
-  const bool has1 = qt0 + 1 < p.n_qtiles;
-  auto kv_tiles = [&](int qt) {
-    const int end = p.causal ? min(p.N, (qt + 1) * p.T) : p.N;
-    return (end + NK - 1) / NK;
-  };
-  const int nkv0 = kv_tiles(qt0);
-  const int nkv1 = has1 ? kv_tiles(qt0 + 1) : 0;
-  const int nkv = max(nkv0, nkv1);
-
   const uint32_t bar0 = sbase + Tr::OFF_BAR;
-  const uint32_t q_full = bar0;
-  auto kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto kv_empty = [&](int s) { return bar0 + 8u * (1 + ST + s); };
-  auto s_full = [&](int t, int buf) { return bar0 + 8u * (1 + 2 * ST + 2 * t + buf); };
-  // P of key tile j is announced on the barrier of its S buffer (j % 2): with two
-  // S buffers a softmax warpgroup can finish tiles j and j + 1 before the MMA
-  // issuer looks, and one barrier per buffer keeps each at most one phase ahead.
-  auto p_full = [&](int t, int buf) { return bar0 + 8u * (5 + 2 * ST + 2 * t + buf); };
-  auto o_done = [&](int t) { return bar0 + 8u * (9 + 2 * ST + t); };
-  auto o_final = [&](int t) { return bar0 + 8u * (11 + 2 * ST + t); };
-  const uint32_t drain = bar0 + 8u * (13 + 2 * ST);
+  auto q_full = [&](int qb) { return bar0 + 8u * qb; };
+  auto q_empty = [&](int qb) { return bar0 + 8u * (QB + qb); };
+  auto kv_full = [&](int s) { return bar0 + 8u * (2 * QB + s); };
+  auto kv_empty = [&](int s) { return bar0 + 8u * (2 * QB + ST + s); };
+  auto s_full = [&](int t, int buf) { return bar0 + 8u * (2 * QB + 2 * ST + 2 * t + buf); };
+  // P of S step G is announced on the barrier of its S buffer (G % 2): with two
+  // S buffers a softmax warpgroup can finish two steps before the MMA issuer
+  // looks, and one barrier per buffer keeps each at most one phase ahead.
+  auto p_full = [&](int t, int buf) { return bar0 + 8u * (2 * QB + 2 * ST + 4 + 2 * t + buf); };
+  auto o_done = [&](int t) { return bar0 + 8u * (2 * QB + 2 * ST + 8 + t); };
+  auto o_final = [&](int t) { return bar0 + 8u * (2 * QB + 2 * ST + 10 + t); };
+  auto o_free = [&](int t) { return bar0 + 8u * (2 * QB + 2 * ST + 12 + t); };
+  auto drain = [&](int t) { return bar0 + 8u * (2 * QB + 2 * ST + 14 + t); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Tr::OFF_BAR + Tr::N_BARS * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    for (int qb = 0; qb < QB; ++qb) {
+      mbar_init(q_full(qb), 1);
+      mbar_init(q_empty(qb), 2);  // one release per MMA issuer
+    }
     for (int s = 0; s < ST; ++s) {
       mbar_init(kv_full(s), 1);
-      mbar_init(kv_empty(s), 1);
+      mbar_init(kv_empty(s), 2);  // one release per MMA issuer
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(s_full(t, 0), 1);
@@ -131,8 +160,10 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(p_full(t, 1), 128);
       mbar_init(o_done(t), 1);
       mbar_init(o_final(t), 1);
+      mbar_init(o_free(t), 128);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain(0), 1);
+    mbar_init(drain(1), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -140,7 +171,7 @@ __global__ void __launch_bounds__(384, 1)
   // 128) stay zero, so their scores are finite; they are never stored.
   if (p.rows < BM) {
     const int pad_bytes = (BM - p.rows) * ROWB;
-    for (int t = 0; t < 2; ++t)
+    for (int t = 0; t < 2 * QB; ++t)
       for (int pn = 0; pn < Tr::NPANEL; ++pn) {
         uint8_t* base = smem + Tr::OFF_Q + t * Tr::Q_BYTES + pn * BM * ROWB + p.rows * ROWB;
         for (int i = threadIdx.x * 16; i < pad_bytes; i += Tr::THREADS * 16)
@@ -164,217 +195,262 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_map(&tmK);
       tma_prefetch_map(&tmV);
       const uint32_t q_bytes = static_cast<uint32_t>(p.rows * ROWB * Tr::NPANEL);
-      mbar_expect_tx(q_full, q_bytes * (has1 ? 2u : 1u));
-      for (int t = 0; t < (has1 ? 2 : 1); ++t)
-        for (int pn = 0; pn < Tr::NPANEL; ++pn)
-          tma_load_4d(sbase + Tr::OFF_Q + t * Tr::Q_BYTES + pn * BM * ROWB, &tmQ, q_full, pn * PANEL,
-                      kvh * p.g, (qt0 + t) * p.T, b);
-      int issued = 0;
-      for (int j = 0; j < nkv; ++j) {
-        const int s = j % ST;
-        if (j >= ST && !mbar_wait(kv_empty(s), ((j / ST) - 1) & 1, abort_flag, kSiteProducer)) break;
-        mbar_expect_tx(kv_full(s), 2u * Tr::KV_BYTES);
-        for (int pn = 0; pn < Tr::NPANEL; ++pn) {
-          tma_load_4d(sbase + Tr::OFF_K + s * Tr::KV_BYTES + pn * NK * ROWB, &tmK, kv_full(s), pn * PANEL, kvh,
-                      j * NK, b);
-          tma_load_4d(sbase + Tr::OFF_V + s * Tr::KV_BYTES + pn * NK * ROWB, &tmV, kv_full(s), pn * PANEL, kvh,
-                      j * NK, b);
+      int g = 0;  // K/V tiles issued so far (across items)
+      bool ok = true;
+      for (int r = 0, item; ok && (item = fwd_item(r, p.n_items)) >= 0; ++r) {
+        const FwdItem it = fwd_decode(p, item, NK);
+        const int qb = r % QB;
+        if (r >= QB && !mbar_wait(q_empty(qb), ((r / QB) - 1) & 1, abort_flag, kSiteProducer)) break;
+        mbar_expect_tx(q_full(qb), q_bytes * (it.has1 ? 2u : 1u));
+        for (int t = 0; t < (it.has1 ? 2 : 1); ++t)
+          for (int pn = 0; pn < Tr::NPANEL; ++pn)
+            tma_load_4d(sbase + Tr::OFF_Q + (qb * 2 + t) * Tr::Q_BYTES + pn * BM * ROWB, &tmQ, q_full(qb),
+                        pn * PANEL, it.kvh * p.g, (it.qt0 + t) * p.T, it.b);
+        for (int j = 0; j < it.nkv; ++j, ++g) {
+          const int s = g % ST;
+          if (g >= ST && !mbar_wait(kv_empty(s), ((g / ST) - 1) & 1, abort_flag, kSiteProducer)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(kv_full(s), 2u * Tr::KV_BYTES);
+          for (int pn = 0; pn < Tr::NPANEL; ++pn) {
+            tma_load_4d(sbase + Tr::OFF_K + s * Tr::KV_BYTES + pn * NK * ROWB, &tmK, kv_full(s), pn * PANEL,
+                        it.kvh, j * NK, it.b);
+            tma_load_4d(sbase + Tr::OFF_V + s * Tr::KV_BYTES + pn * NK * ROWB, &tmV, kv_full(s), pn * PANEL,
+                        it.kvh, j * NK, it.b);
+          }
         }
-        issued = j + 1;
       }
       if (*abort_flag) {  // let in-flight copies land before the CTA exits
-        mbar_wait_drain(q_full, 0);
-        for (int j = max(0, issued - ST); j < issued; ++j) mbar_wait_drain(kv_full(j % ST), (j / ST) & 1);
+        for (int j = max(0, g - ST); j < g; ++j) mbar_wait_drain(kv_full(j % ST), (j / ST) & 1);
       }
     }
-  } else if (warp == Tr::WARP_MMA) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == Tr::WARP_MMA || warp == Tr::WARP_MMA + 1) {
+    // ------------------------------------------------------------ MMA issuers, one thread per Q tile
+    // A single issuing thread shares its sub-partition with busy softmax warps and
+    // could not keep two tiles fed; two issuers also let the tiles run apart.
+    const int t = warp - Tr::WARP_MMA;
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, NK, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, DH, false, true);
-      const uint32_t q_addr = sbase + Tr::OFF_Q, k_addr = sbase + Tr::OFF_K, v_addr = sbase + Tr::OFF_V;
-      auto issue_qk = [&](int t, int j) {
-        const int s = j % ST;
+      // Descriptors of Q buffer 0 / stage 0; other buffers, stages and K-steps add
+      // their byte offset (in 16-byte units) to the start-address field.
+      const uint64_t dq0 = smem_desc(sbase + Tr::OFF_Q + t * Tr::Q_BYTES, 16, 8 * ROWB, Tr::LAYOUT);
+      const uint64_t dk0 = smem_desc(sbase + Tr::OFF_K, 16, 8 * ROWB, Tr::LAYOUT);
+      const uint64_t dv0 = smem_desc(sbase + Tr::OFF_V, NK * ROWB, 8 * ROWB, Tr::LAYOUT);
+      const uint32_t tS0 = tmem + Tr::tm_s(t, 0), tO = tmem + Tr::tm_o(t);
+      auto issue_qk = [&](int qb, int s, int buf) {
+        const uint64_t a0 = dq0 + static_cast<uint64_t>((qb * 2 * Tr::Q_BYTES) >> 4);
+        const uint64_t b0 = dk0 + static_cast<uint64_t>((s * Tr::KV_BYTES) >> 4);
 #pragma unroll
         for (int ks = 0; ks < DH / 16; ++ks) {
-          const uint32_t pn = (ks * 16) / PANEL, off = ((ks * 16) % PANEL) * 2;
-          const uint64_t a =
-              smem_desc(q_addr + t * Tr::Q_BYTES + pn * BM * ROWB + off, 16, 8 * ROWB, Tr::LAYOUT);
-          const uint64_t bd =
-              smem_desc(k_addr + s * Tr::KV_BYTES + pn * NK * ROWB + off, 16, 8 * ROWB, Tr::LAYOUT);
-          mma_ss(tmem + Tr::tm_s(t, j & 1), a, bd, idesc_qk, ks > 0 ? 1u : 0u);
+          const uint32_t within = ((ks * 16) % PANEL) * 2, pn = (ks * 16) / PANEL;
+          mma_ss(tS0 + 64u * buf, a0 + ((pn * BM * ROWB + within) >> 4), b0 + ((pn * NK * ROWB + within) >> 4),
+                 idesc_qk, ks > 0 ? 1u : 0u);
         }
-        mma_commit(s_full(t, j & 1));
+        mma_commit(s_full(t, buf));
       };
-      auto issue_pv = [&](int t, int j) {
-        const int s = j % ST;
+      auto issue_pv = [&](int s, int buf, bool acc) {
+        const uint64_t b0 = dv0 + static_cast<uint64_t>((s * Tr::KV_BYTES) >> 4);
 #pragma unroll
-        for (int ks = 0; ks < NK / 16; ++ks) {
-          const uint64_t bd =
-              smem_desc(v_addr + s * Tr::KV_BYTES + ks * 16 * ROWB, NK * ROWB, 8 * ROWB, Tr::LAYOUT);
-          mma_ts(tmem + Tr::tm_o(t), tmem + Tr::tm_s(t, j & 1) + ks * 8, bd, idesc_pv,
-                 (j > 0 || ks > 0) ? 1u : 0u);
-        }
+        for (int ks = 0; ks < NK / 16; ++ks)
+          mma_ts(tO, tS0 + 64u * buf + ks * 8, b0 + ((ks * 16 * ROWB) >> 4), idesc_pv, (acc || ks > 0) ? 1u : 0u);
         mma_commit(o_done(t));
       };
-      const int nkv_t[2] = {nkv0, nkv1};
-      int loaded = 0;  // key tiles whose kv_full phase has been observed
-      auto ensure_loaded = [&](int j) {
-        while (loaded <= j) {
+      int loaded = 0;  // K/V tiles whose kv_full phase this thread has observed
+      auto ensure_loaded = [&](int gj) {
+        while (loaded <= gj) {
           if (!mbar_wait(kv_full(loaded % ST), (loaded / ST) & 1, abort_flag, kSiteMma)) return false;
           ++loaded;
         }
         tc_fence_after();
         return true;
       };
-      bool ok = mbar_wait(q_full, 0, abort_flag, kSiteMma);
-      // Prologue: S for key tiles 0 and 1 of both Q tiles.
-      for (int j = 0; ok && j < 2 && j < nkv; ++j) {
-        ok = ensure_loaded(j);
-        for (int t = 0; ok && t < 2; ++t)
-          if (j < nkv_t[t]) issue_qk(t, j);
-      }
-      for (int j = 0; ok && j < nkv; ++j) {
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (j >= nkv_t[t]) continue;
-          if (!mbar_wait(p_full(t, j & 1), (j >> 1) & 1, abort_flag, kSiteMma)) {
+      int g = 0;   // first K/V tile (global index) of the current item
+      int G = 0;   // S steps of this Q tile so far (across items)
+      int nd = 0;  // items finished by this Q tile
+      bool ok = true;
+      for (int r = 0, item; ok && (item = fwd_item(r, p.n_items)) >= 0; ++r) {
+        const FwdItem it = fwd_decode(p, item, NK);
+        const int nkv_t = t ? it.nkv1 : it.nkv0;
+        const int qb = r % QB;
+        // Both issuers observe this item's Q load before releasing its buffer, so a
+        // release never lands in the phase of an earlier item.
+        if (!mbar_wait(q_full(qb), (r / QB) & 1, abort_flag, kSiteMma)) {
+          ok = false;
+          break;
+        }
+        for (int j = 0; ok && j < 2 && j < nkv_t; ++j) {  // prologue: S for key tiles 0 and 1
+          ok = ensure_loaded(g + j);
+          if (ok) issue_qk(qb, (g + j) % ST, (G + j) & 1);
+        }
+        for (int j = 0; ok && j < nkv_t; ++j) {
+          const int Gt = G + j;
+          if (!mbar_wait(p_full(t, Gt & 1), (Gt >> 1) & 1, abort_flag, kSiteMma)) {
+            ok = false;
+            break;
+          }
+          // O_t still holds the previous item until its epilogue has read it.
+          if (j == 0 && nd > 0 && !mbar_wait(o_free(t), (nd - 1) & 1, abort_flag, kSiteMma)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          issue_pv(t, j);
-          if (j + 2 < nkv_t[t]) {
-            // S_t for tile j + 2 reuses this buffer: the PV just issued reads P
-            // from it first (MMAs from one thread execute in order).
-            if (!ensure_loaded(j + 2)) {
+          issue_pv((g + j) % ST, Gt & 1, j > 0);
+          if (j + 2 < nkv_t) {
+            // The next S in this buffer: the PV just issued reads P from it first
+            // (MMAs from one thread execute in order).
+            if (!ensure_loaded(g + j + 2)) {
               ok = false;
               break;
             }
-            issue_qk(t, j + 2);
+            issue_qk(qb, (g + j + 2) % ST, Gt & 1);
           }
-          if (j + 1 == nkv_t[t]) mma_commit(o_final(t));
+          if (j + 1 == nkv_t) mma_commit(o_final(t));
+          mma_commit(kv_empty((g + j) % ST));
         }
-        mma_commit(kv_empty(j % ST));
+        // K/V tiles of this item that this Q tile does not need (causal: the other
+        // tile reaches one tile further) are released too, once they are loaded.
+        for (int j = nkv_t; ok && j < it.nkv; ++j) {
+          ok = ensure_loaded(g + j);
+          if (ok) mma_commit(kv_empty((g + j) % ST));
+        }
+        if (!ok) break;
+        mma_commit(q_empty(qb));
+        G += nkv_t;
+        nd += nkv_t > 0 ? 1 : 0;
+        g += it.nkv;
       }
       if (!ok) {  // wait for issued MMAs before TMEM is released
-        mma_commit(drain);
-        mbar_wait_drain(drain, 0);
+        mma_commit(drain(t));
+        mbar_wait_drain(drain(t), 0);
       }
     }
   } else if (warp < 8) {
-    // ------------------------------------------------------------ softmax
+    // ------------------------------------------------------------ softmax and epilogue
     const int t = warp >> 2;
-    const int nkv_t = t ? nkv1 : nkv0;
-    const int qt = qt0 + t;
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const uint32_t tO = lane_addr + Tr::tm_o(t);
-    const int tok = qt * p.T + row / p.g;
-    const int head = kvh * p.g + row % p.g;
-    const bool row_valid = row < p.rows && tok < p.N;
     const float sl2 = p.scale_log2;
-    float m = -INFINITY, l = 0.f;
-    bool ok = nkv_t > 0;
-    for (int j = 0; ok && j < nkv_t; ++j) {
-      // Every lane waits; the verdict is made warp-uniform so that the
-      // warp-wide TMEM instructions below are never reached divergently.
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full(t, j & 1), (j >> 1) & 1, abort_flag, kSiteSoftmax));
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t tS = lane_addr + Tr::tm_s(t, j & 1);
-      const int k0 = j * NK;
-      const bool masked = (k0 + NK > p.N) || (p.causal && k0 + NK - 1 > qt * p.T);
-      uint32_t sr[NK];
-      tmem_ld32x2(tS, tS + 32, sr);
-      if (masked) {
-        // last visible key of this tile, relative to k0 (may be negative)
-        const int last = min(p.N - 1, p.causal ? tok : p.N - 1) - k0;
+    int G = 0, nd = 0;
+    bool ok = true;
+    for (int r = 0, item; ok && (item = fwd_item(r, p.n_items)) >= 0; ++r) {
+      const FwdItem it = fwd_decode(p, item, NK);
+      const int nkv_t = t ? it.nkv1 : it.nkv0;
+      if (nkv_t == 0) continue;
+      const int qt = it.qt0 + t;
+      const int tok = qt * p.T + row / p.g;
+      const int head = it.kvh * p.g + row % p.g;
+      const bool row_valid = row < p.rows && tok < p.N;
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < nkv_t; ++j) {
+        const int Gt = G + j;
+        // Every lane waits; the verdict is made warp-uniform so that the
+        // warp-wide TMEM instructions below are never reached divergently.
+        ok = __all_sync(0xffffffffu, mbar_wait(s_full(t, Gt & 1), (Gt >> 1) & 1, abort_flag, kSiteSoftmax));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t tS = lane_addr + Tr::tm_s(t, Gt & 1);
+        const int k0 = j * NK;
+        const bool masked = (k0 + NK > p.N) || (p.causal && k0 + NK - 1 > qt * p.T);
+        uint32_t sr[NK];
+        tmem_ld32x2(tS, tS + 32, sr);
+        if (masked) {
+          // last visible key of this tile, relative to k0 (may be negative)
+          const int last = min(p.N - 1, p.causal ? tok : p.N - 1) - k0;
 #pragma unroll
-        for (int i = 0; i < NK; ++i)
-          if (i > last) sr[i] = __float_as_uint(-INFINITY);
-      }
-      // Row maximum: eight independent chains of three-input maxima.
-      float acc[8];
+          for (int i = 0; i < NK; ++i)
+            if (i > last) sr[i] = __float_as_uint(-INFINITY);
+        }
+        // Row maximum: eight independent chains of three-input maxima.
+        float acc[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        acc[c] = fmax3(__uint_as_float(sr[c]), __uint_as_float(sr[8 + c]), __uint_as_float(sr[16 + c]));
+        for (int c = 0; c < 8; ++c)
+          acc[c] = fmax3(__uint_as_float(sr[c]), __uint_as_float(sr[8 + c]), __uint_as_float(sr[16 + c]));
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        acc[c] = fmax3(acc[c], __uint_as_float(sr[24 + c]), __uint_as_float(sr[32 + c]));
-        acc[c] = fmax3(acc[c], __uint_as_float(sr[40 + c]), __uint_as_float(sr[48 + c]));
-        acc[c] = fmaxf(acc[c], __uint_as_float(sr[56 + c]));
-      }
-      const float mx =
-          fmax3(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], acc[5]), fmaxf(acc[6], acc[7]));
-      const float mnew = fmaxf(m, mx * sl2);
-      const bool raise = mnew > m + 8.f;
-      const float alpha = (raise && m != -INFINITY) ? ex2(m - mnew) : 1.f;
-      if (__any_sync(0xffffffffu, alpha != 1.f)) {
-        // O must hold P*V of every earlier tile before it is rescaled: wait for
-        // the PV of tile j - 1 (o_done is at most one phase behind here).
-        if (j > 0) {
-          ok = __all_sync(0xffffffffu, mbar_wait(o_done(t), (j - 1) & 1, abort_flag, kSiteSoftmax));
+        for (int c = 0; c < 8; ++c) {
+          acc[c] = fmax3(acc[c], __uint_as_float(sr[24 + c]), __uint_as_float(sr[32 + c]));
+          acc[c] = fmax3(acc[c], __uint_as_float(sr[40 + c]), __uint_as_float(sr[48 + c]));
+          acc[c] = fmaxf(acc[c], __uint_as_float(sr[56 + c]));
+        }
+        const float mx =
+            fmax3(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], acc[5]), fmaxf(acc[6], acc[7]));
+        const float mnew = fmaxf(m, mx * sl2);
+        const bool raise = mnew > m + 8.f;
+        const float alpha = (raise && m != -INFINITY) ? ex2(m - mnew) : 1.f;
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+          // O must hold P*V of every earlier step of this item before it is
+          // rescaled: wait for the PV of step Gt - 1 (o_done is at most one phase
+          // behind here; alpha is 1 at an item's first step).
+          ok = __all_sync(0xffffffffu, mbar_wait(o_done(t), (Gt - 1) & 1, abort_flag, kSiteSoftmax));
           if (!ok) break;
           tc_fence_after();
-        }
 #pragma unroll 1
-        for (int c = 0; c < DH; c += 16) {
-          uint32_t r[16];
-          tmem_ld16(tO + c, r);
+          for (int c = 0; c < DH; c += 16) {
+            uint32_t rr[16];
+            tmem_ld16(tO + c, rr);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st16(tO + c, r);
+            for (int i = 0; i < 16; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+            tmem_st16(tO + c, rr);
+          }
         }
+        l *= alpha;
+        if (raise) m = mnew;
+        // Masked scores are -inf, so their P is exactly 0 (the scale is positive).
+        const float nref = m == -INFINITY ? 0.f : -m;
+        float sum0[8], sum1[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) sum0[c] = sum1[c] = 0.f;
+        uint32_t pk[NK / 2];
+#pragma unroll
+        for (int i = 0; i < NK / 2; ++i) {
+          float x0, x1;
+          ffma2(x0, x1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), sl2, sl2, nref, nref);
+          const float p0 = ex2(x0), p1 = ex2(x1);
+          fadd2(sum0[i & 7], sum1[i & 7], sum0[i & 7], sum1[i & 7], p0, p1);
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tS, pk);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) fadd2(sum0[c], sum1[c], sum0[c], sum1[c], sum0[c + 4], sum1[c + 4]);
+        l += ((sum0[0] + sum1[0]) + (sum0[1] + sum1[1])) + ((sum0[2] + sum1[2]) + (sum0[3] + sum1[3]));
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full(t, Gt & 1));
       }
-      l *= alpha;
-      if (raise) m = mnew;
-      // Masked scores are -inf, so their P is exactly 0 (the scale is positive).
-      const float nref = m == -INFINITY ? 0.f : -m;
-      float sum0[8], sum1[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) sum0[c] = sum1[c] = 0.f;
-      uint32_t pk[NK / 2];
-#pragma unroll
-      for (int i = 0; i < NK / 2; ++i) {
-        float x0, x1;
-        ffma2(x0, x1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), sl2, sl2, nref, nref);
-        const float p0 = ex2(x0), p1 = ex2(x1);
-        fadd2(sum0[i & 7], sum1[i & 7], sum0[i & 7], sum1[i & 7], p0, p1);
-        pk[i] = pack_bf16x2(p0, p1);
-      }
-      tmem_st32(tS, pk);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) fadd2(sum0[c], sum1[c], sum0[c], sum1[c], sum0[c + 4], sum1[c + 4]);
-      l += ((sum0[0] + sum1[0]) + (sum0[1] + sum1[1])) + ((sum0[2] + sum1[2]) + (sum0[3] + sum1[3]));
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(p_full(t, j & 1));
-    }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_final(t), 0, abort_flag, kSiteEpilogue));
-    if (ok) {
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(o_final(t), nd & 1, abort_flag, kSiteEpilogue));
+      if (!ok) break;
       tc_fence_after();
       const float inv_l = row_valid ? 1.f / l : 0.f;
-      __nv_bfloat16* dst = p.out + ((static_cast<size_t>(b) * p.N + (row_valid ? tok : 0)) * p.Hq + head) * DH;
+      __nv_bfloat16* dst =
+          p.out + ((static_cast<size_t>(it.b) * p.N + (row_valid ? tok : 0)) * p.Hq + head) * DH;
 #pragma unroll 1
       for (int c = 0; c < DH; c += 16) {
-        uint32_t r[16];
-        tmem_ld16(tO + c, r);  // warp-wide: every lane loads, only valid rows store
+        uint32_t rr[16];
+        tmem_ld16(tO + c, rr);  // warp-wide: every lane loads, only valid rows store
         uint4 lo, hi;
-        lo.x = pack_bf16x2(__uint_as_float(r[0]) * inv_l, __uint_as_float(r[1]) * inv_l);
-        lo.y = pack_bf16x2(__uint_as_float(r[2]) * inv_l, __uint_as_float(r[3]) * inv_l);
-        lo.z = pack_bf16x2(__uint_as_float(r[4]) * inv_l, __uint_as_float(r[5]) * inv_l);
-        lo.w = pack_bf16x2(__uint_as_float(r[6]) * inv_l, __uint_as_float(r[7]) * inv_l);
-        hi.x = pack_bf16x2(__uint_as_float(r[8]) * inv_l, __uint_as_float(r[9]) * inv_l);
-        hi.y = pack_bf16x2(__uint_as_float(r[10]) * inv_l, __uint_as_float(r[11]) * inv_l);
-        hi.z = pack_bf16x2(__uint_as_float(r[12]) * inv_l, __uint_as_float(r[13]) * inv_l);
-        hi.w = pack_bf16x2(__uint_as_float(r[14]) * inv_l, __uint_as_float(r[15]) * inv_l);
+        lo.x = pack_bf16x2(__uint_as_float(rr[0]) * inv_l, __uint_as_float(rr[1]) * inv_l);
+        lo.y = pack_bf16x2(__uint_as_float(rr[2]) * inv_l, __uint_as_float(rr[3]) * inv_l);
+        lo.z = pack_bf16x2(__uint_as_float(rr[4]) * inv_l, __uint_as_float(rr[5]) * inv_l);
+        lo.w = pack_bf16x2(__uint_as_float(rr[6]) * inv_l, __uint_as_float(rr[7]) * inv_l);
+        hi.x = pack_bf16x2(__uint_as_float(rr[8]) * inv_l, __uint_as_float(rr[9]) * inv_l);
+        hi.y = pack_bf16x2(__uint_as_float(rr[10]) * inv_l, __uint_as_float(rr[11]) * inv_l);
+        hi.z = pack_bf16x2(__uint_as_float(rr[12]) * inv_l, __uint_as_float(rr[13]) * inv_l);
+        hi.w = pack_bf16x2(__uint_as_float(rr[14]) * inv_l, __uint_as_float(rr[15]) * inv_l);
         if (row_valid) {
           *reinterpret_cast<uint4*>(dst + c) = lo;
           *reinterpret_cast<uint4*>(dst + c + 8) = hi;
         }
       }
+      // O has been read: the next item's first PV may overwrite it.
+      tc_fence_before();
+      mbar_arrive(o_free(t));
       if (row_valid)
-        p.lse[(static_cast<size_t>(b) * p.Hq + head) * p.N + tok] = (m + __log2f(l)) * 0.69314718055994531f;
+        p.lse[(static_cast<size_t>(it.b) * p.Hq + head) * p.N + tok] = (m + __log2f(l)) * 0.69314718055994531f;
+      G += nkv_t;
+      ++nd;
     }
   }
 
