@@ -231,22 +231,30 @@ def roofline_for(w, kernel_name, ms, peaks, peak_kind):
             "traffic": traffic_for(kernel_name, w), "kernel": kernel_name, "peak_source": f"{peak_kind} bf16_tflops"}
 
 
-def traffic_for(kernel_name, w):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current source."""
+def kernel_source_sha256():
+    """Hash of every CUDA source of the library (a profile is valid only for the code it measured)."""
     import hashlib
 
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_query_attention_sqa_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(fn.encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def traffic_for(kernel_name, w):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current source."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             table = json.load(f)
     except Exception:
         return None
-    h = hashlib.sha256()
-    for fn in ("sqa_device.cuh", "sqa_fwd.cuh", "sqa_bwd.cuh"):
-        with open(os.path.join(ROOT, "sparse_query_attention_sqa_b200", "csrc", fn), "rb") as f:
-            h.update(f.read())
+    digest = kernel_source_sha256()
     for e in table.get("entries", []):
-        if e.get("kernel") == kernel_name and e.get("workload") == w.name and e.get("source_sha256") == h.hexdigest():
+        if e.get("kernel") == kernel_name and e.get("workload") == w.name and e.get("source_sha256") == digest:
             return e.get("dram_bytes_per_launch")
     return None
 
