@@ -1,10 +1,11 @@
 // sqa_bwd.cuh -- Sparse Query Attention backward on sm_100a.
 //
 // Three launches on the caller's stream:
-//   1. prep:  D_i = <dO_i, O_i> and lse_i * log2(e) for every query row, written
-//             in the stacked-tile order the main kernel reads (slots of padding
-//             rows get lse = +inf and D = 0, which makes their P exactly 0), and
-//             the fp32 dQ accumulator zeroed.
+//   1. prep:  -D_i = -<dO_i, O_i> and -lse_i * log2(e) for every query row,
+//             written in the stacked-tile order the main kernel reads (slots of
+//             padding rows get lse = +inf and D = 0, which makes their P exactly
+//             0), the fp32 dQ accumulator zeroed, and for dh <= 32 transposed
+//             fp32 images of the Q and dO tiles (tf32 MMA operands).
 //   2. main:  one CTA per (128-key tile, batch, KV head).  It keeps K and V in
 //             shared memory and walks the Q tiles that see its keys.  A Q tile
 //             stacks the g query heads of the group (row r = t * g + head), so
@@ -37,6 +38,8 @@ struct BwdLayout {
   size_t n_slots;     // B * H_kv * n_qt * 128
   size_t off_D;       // byte offsets inside the workspace
   size_t off_dq;
+  size_t off_q32;     // dh <= 32 only: fp32 transposed images of the stacked Q and dO tiles
+  size_t off_do32;
   size_t bytes;
 };
 
@@ -51,6 +54,12 @@ inline BwdLayout bwd_layout(int B, int N, int Hq, int Hkv, int dh) {
   L.off_D = align256(L.n_slots * sizeof(float));
   L.off_dq = L.off_D + align256(L.n_slots * sizeof(float));
   L.bytes = L.off_dq + align256(static_cast<size_t>(B) * N * Hq * dh * sizeof(float));
+  if (dh <= 32) {
+    const size_t img = align256(L.n_slots * dh * sizeof(float));
+    L.off_q32 = L.bytes;
+    L.off_do32 = L.bytes + img;
+    L.bytes += 2 * img;
+  }
   return L;
 }
 
@@ -63,14 +72,27 @@ inline size_t bwd_workspace_bytes(int B, int N, int Hq, int Hkv, int dh) {
 struct BwdPrepParams {
   const __nv_bfloat16* dout;
   const __nv_bfloat16* out;
+  const __nv_bfloat16* q;
   const float* lse;
   float* lse2;
   float* D;
   float* dq_acc;
+  float* q32;   // null, or the fp32 tile images (see below)
+  float* do32;
   int N, Hq, Hkv, g, T, rows, n_qt;
   long long n_slots;
   long long dq_vec4;  // dq accumulator length / 4
 };
+
+// Offset (in floats) of element (row r, column n) inside the fp32 image of one
+// stacked 128-row tile: the tile transposed to [dh][128] and cut into four
+// panels of 32 rows, each panel dh lines of 128 bytes with the 128-byte swizzle
+// (16-byte chunk c of line n stored at chunk c ^ (n % 8)).  This is the K-major
+// operand layout of a tf32 MMA whose contraction runs over the tile's rows, so
+// the image is copied to shared memory as is.
+__host__ __device__ __forceinline__ int tf32_image_index(int r, int n, int dh) {
+  return (r >> 5) * dh * 32 + n * 32 + ((((r & 31) >> 2) ^ (n & 7)) << 2) + (r & 3);
+}
 
 template <int DH>
 __global__ void __launch_bounds__(256) sqa_bwd_prep_kernel(const BwdPrepParams p) {
@@ -84,7 +106,10 @@ __global__ void __launch_bounds__(256) sqa_bwd_prep_kernel(const BwdPrepParams p
     const int b = static_cast<int>(bkv / p.Hkv), kvh = static_cast<int>(bkv % p.Hkv);
     const int tok = qt * p.T + r / p.g;
     float l2 = INFINITY, d = 0.f;
-    if (r < p.rows && tok < p.N) {
+    const bool live = r < p.rows && tok < p.N;
+    float* qi = p.q32 ? p.q32 + (s - r) * DH : nullptr;
+    float* di = p.q32 ? p.do32 + (s - r) * DH : nullptr;
+    if (live) {
       const int head = kvh * p.g + r % p.g;
       const size_t row = (static_cast<size_t>(b) * p.N + tok) * p.Hq + head;
       const uint4* o = reinterpret_cast<const uint4*>(p.out + row * DH);
@@ -99,12 +124,34 @@ __global__ void __launch_bounds__(256) sqa_bwd_prep_kernel(const BwdPrepParams p
           const float2 fa = __bfloat1622float2(a2[e]), fb = __bfloat1622float2(b2[e]);
           d = fmaf(fa.x, fb.x, d);
           d = fmaf(fa.y, fb.y, d);
+          if (DH <= 32 && di) {
+            di[tf32_image_index(r, 8 * c + 2 * e, DH)] = fb.x;
+            di[tf32_image_index(r, 8 * c + 2 * e + 1, DH)] = fb.y;
+          }
+        }
+      }
+      if (DH <= 32 && qi) {
+        const uint4* qr = reinterpret_cast<const uint4*>(p.q + row * DH);
+#pragma unroll
+        for (int c = 0; c < DH / 8; ++c) {
+          const uint4 a = qr[c];
+          const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 fa = __bfloat1622float2(a2[e]);
+            qi[tf32_image_index(r, 8 * c + 2 * e, DH)] = fa.x;
+            qi[tf32_image_index(r, 8 * c + 2 * e + 1, DH)] = fa.y;
+          }
         }
       }
       l2 = p.lse[(static_cast<size_t>(b) * p.Hq + head) * p.N + tok] * 1.4426950408889634f;
+    } else if (DH <= 32 && qi) {
+#pragma unroll
+      for (int n = 0; n < DH; ++n) qi[tf32_image_index(r, n, DH)] = di[tf32_image_index(r, n, DH)] = 0.f;
     }
-    p.lse2[s] = l2;
-    p.D[s] = d;
+    // Stored negated: the main kernels add them (x = S * scale * log2(e) - lse2, dP - D).
+    p.lse2[s] = -l2;
+    p.D[s] = -d;
   }
   float4* acc = reinterpret_cast<float4*>(p.dq_acc);
   for (long long i = tid; i < p.dq_vec4; i += stride) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -130,9 +177,11 @@ __global__ void __launch_bounds__(256)
 // ---------------------------------------------------------------------------
 // 2. main
 struct BwdParams {
-  const float* lse2;  // stacked [B*H_kv][n_qt][128]
-  const float* D;
+  const float* lse2;  // stacked [B*H_kv][n_qt][128], negated: -lse * log2(e) (-inf on padding rows)
+  const float* D;     // negated: -<dO, O> (0 on padding rows)
   float* dq_acc;      // [B][N][H_q][dh] fp32
+  const float* q32;   // dh <= 32: fp32 images of the stacked Q and dO tiles
+  const float* do32;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int N, Hq, Hkv, g, T, rows, n_qt, n_bh, causal;
@@ -381,8 +430,8 @@ __global__ void __launch_bounds__(384, 1)
                                        mbar_wait(s_full, i & 1, abort_flag, kSiteSoftmax));
       if (!ok) break;
       tc_fence_after();
-      const float* lse2 = reinterpret_cast<const float*>(smem + Tr::OFF_STAT + s * 1024);
-      const float* Dv = lse2 + 128;
+      const float* lse2 = reinterpret_cast<const float*>(smem + Tr::OFF_STAT + s * 1024);  // negated
+      const float* Dv = lse2 + 128;                                                          // negated
       const bool masked = p.causal && (k0 + NK - 1 > qt * p.T);
       const int key_rel = key - qt * p.T;  // visible iff key_rel <= rtok[r]
 #pragma unroll 1
@@ -398,10 +447,10 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int r = col0 + e + u;
-            float pr = ex2(fmaf(__uint_as_float(sr[e + u]), sl2, -lse2[r]));
+            float pr = ex2(fmaf(__uint_as_float(sr[e + u]), sl2, lse2[r]));
             if (!key_ok || (masked && key_rel > rtok[r])) pr = 0.f;
             pv[u] = pr;
-            dv[u] = pr * (__uint_as_float(dr[e + u]) - Dv[r]);
+            dv[u] = pr * (__uint_as_float(dr[e + u]) + Dv[r]);
           }
           pp[e >> 1] = pack_bf16x2(pv[0], pv[1]);
           dd[e >> 1] = pack_bf16x2(dv[0], dv[1]);

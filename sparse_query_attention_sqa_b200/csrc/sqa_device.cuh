@@ -277,6 +277,28 @@ __device__ __forceinline__ void regs_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// 2^x for a pair of values on the FMA pipe instead of the special-function
+// unit, to share the exponentials of a softmax between the two.  Range
+// reduction: n = round(x) by adding and subtracting 1.5 * 2^23 (round to
+// nearest), f = x - n in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose
+// coefficients are a relative-error minimax fit on [-1/2, 1/2] made for this
+// library (Remez exchange; largest relative error 7.5e-5, below a quarter of a
+// bf16 ulp); the exponent n is added to the bits of 2^f.  x is clamped to
+// -126 first so the exponent never underflows (results below 2^-126 come out
+// as about 1.2e-38 instead).
+__device__ __forceinline__ float2 exp2_poly2(float x0, float x1) {
+  const float2 x = make_float2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const float2 shift = make_float2(12582912.f, 12582912.f);
+  const float2 j = __fadd2_rn(x, shift);                                    // bits: n + const
+  const float2 f = __fadd2_rn(x, __fadd2_rn(shift, make_float2(-j.x, -j.y)));  // x - n
+  float2 p = __ffma2_rn(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
+                        make_float2(0.2426111251115799f, 0.2426111251115799f));
+  p = __ffma2_rn(p, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+  p = __ffma2_rn(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(j.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(j.y) << 23)));
+}
+
 // Three-input maximum (one instruction on sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;

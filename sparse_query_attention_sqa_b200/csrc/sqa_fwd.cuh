@@ -112,7 +112,9 @@ __device__ __forceinline__ FwdItem fwd_decode(const FwdParams& p, int item, int 
   return it;
 }
 
-template <int DH>
+// POLY: of every 8 pairs of scores in an unmasked tile, how many take the
+// polynomial exponential (exp2_poly2) instead of the special-function unit.
+template <int DH, int POLY = (DH <= 32 ? 3 : 0)>
 __global__ void __launch_bounds__(384, 1)
     sqa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -403,13 +405,34 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int c = 0; c < 8; ++c) sum0[c] = sum1[c] = 0.f;
         uint32_t pk[NK / 2];
+        if (!masked) {
+          // POLY of every 8 pairs take the FMA-pipe exponential, the rest the
+          // special-function unit, so that neither pipe alone sets the pace.
 #pragma unroll
-        for (int i = 0; i < NK / 2; ++i) {
-          float x0, x1;
-          ffma2(x0, x1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), sl2, sl2, nref, nref);
-          const float p0 = ex2(x0), p1 = ex2(x1);
-          fadd2(sum0[i & 7], sum1[i & 7], sum0[i & 7], sum1[i & 7], p0, p1);
-          pk[i] = pack_bf16x2(p0, p1);
+          for (int i = 0; i < NK / 2; ++i) {
+            float x0, x1, p0, p1;
+            ffma2(x0, x1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), sl2, sl2, nref, nref);
+            if ((i & 7) * POLY % 8 + POLY >= 8) {  // POLY evenly spread indices of 0..7
+              const float2 pp = exp2_poly2(x0, x1);
+              p0 = pp.x;
+              p1 = pp.y;
+            } else {
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
+            fadd2(sum0[i & 7], sum1[i & 7], sum0[i & 7], sum1[i & 7], p0, p1);
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+        } else {
+          // Masked scores are -inf: the special-function unit gives exactly 0 there.
+#pragma unroll
+          for (int i = 0; i < NK / 2; ++i) {
+            float x0, x1;
+            ffma2(x0, x1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), sl2, sl2, nref, nref);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            fadd2(sum0[i & 7], sum1[i & 7], sum0[i & 7], sum1[i & 7], p0, p1);
+            pk[i] = pack_bf16x2(p0, p1);
+          }
         }
         tmem_st32(tS, pk);
 #pragma unroll
