@@ -222,11 +222,15 @@ sqa_status launch_bwd(const void* dout, const void* q, const void* k, const void
   p.scale = scale;
   if constexpr (DH <= 32) {
     // dh 16 and 32: tf32 gradient contractions, half-tile pipelining
+    // Persistent: one CTA per SM walks the items.
     using T32 = sqa::BwdTf32Traits<DH>;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    p.n_items = static_cast<int>(grid_main);
+    const unsigned grid = static_cast<unsigned>(grid_main < sms ? grid_main : sms);
     if ((st = set_smem(sqa::sqa_bwd_tf32_kernel<DH>, T32::SMEM_BYTES)) != SQA_OK) return st;
     if ((st = record_timing(1, 0, stream)) != SQA_OK) return st;
-    sqa::sqa_bwd_tf32_kernel<DH><<<static_cast<unsigned>(grid_main), T32::THREADS, T32::SMEM_BYTES, stream>>>(
-        mq, mdo, mk, mv, p);
+    sqa::sqa_bwd_tf32_kernel<DH><<<grid, T32::THREADS, T32::SMEM_BYTES, stream>>>(mq, mdo, mk, mv, p);
   } else {
     if ((st = set_smem(sqa::sqa_bwd_kernel<DH>, Tr::SMEM_BYTES)) != SQA_OK) return st;
     if ((st = record_timing(1, 0, stream)) != SQA_OK) return st;

@@ -185,6 +185,7 @@ struct BwdParams {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int N, Hq, Hkv, g, T, rows, n_qt, n_bh, causal;
+  int n_items;  // persistent kernels: 128-key tiles x (batch, KV head)
   float scale_log2, scale;
 };
 
@@ -348,66 +349,64 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
-      constexpr uint32_t idesc_kv = idesc_bf16_f32(128, DH, false, true);    // dV, dK (A in TMEM)
-      constexpr uint32_t idesc_q = idesc_bf16_f32(128, DH, true, true);      // dQ (A = dS MN-major)
-      const uint32_t k_addr = sbase + Tr::OFF_K, v_addr = sbase + Tr::OFF_V;
-      const uint32_t ds_addr = sbase + Tr::OFF_DS;
-      bool ok = mbar_wait(kv_full, 0, abort_flag, kSiteMma);
-      for (int i = 0; ok && i < nq; ++i) {
-        const int s = i % QS;
-        const uint32_t q_addr = sbase + Tr::OFF_Q + s * Tr::TILE, do_addr = sbase + Tr::OFF_DO + s * Tr::TILE;
-        if (!mbar_wait(qd_full(s), (i / QS) & 1, abort_flag, kSiteMma)) { ok = false; break; }
-        if (Tr::TM_DQ == Tr::TM_ST && i > 0 && !mbar_wait(dq_empty, (i - 1) & 1, abort_flag, kSiteMma)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // S^T = K Q^T and dP^T = V dO^T: M = 128 keys, N = 128 stacked query rows, K = dh.
+    // ------------------------------------------------------------ MMA issuer (the whole warp; one elected lane issues)
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
+    constexpr uint32_t idesc_kv = idesc_bf16_f32(128, DH, false, true);    // dV, dK (A in TMEM)
+    constexpr uint32_t idesc_q = idesc_bf16_f32(128, DH, true, true);      // dQ (A = dS MN-major)
+    const uint32_t k_addr = sbase + Tr::OFF_K, v_addr = sbase + Tr::OFF_V;
+    const uint32_t ds_addr = sbase + Tr::OFF_DS;
+    bool ok = mbar_wait_warp(kv_full, 0, abort_flag, kSiteMma);
+    for (int i = 0; ok && i < nq; ++i) {
+      const int s = i % QS;
+      const uint32_t q_addr = sbase + Tr::OFF_Q + s * Tr::TILE, do_addr = sbase + Tr::OFF_DO + s * Tr::TILE;
+      if (!mbar_wait_warp(qd_full(s), (i / QS) & 1, abort_flag, kSiteMma)) { ok = false; break; }
+      if (Tr::TM_DQ == Tr::TM_ST && i > 0 && !mbar_wait_warp(dq_empty, (i - 1) & 1, abort_flag, kSiteMma)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // S^T = K Q^T and dP^T = V dO^T: M = 128 keys, N = 128 stacked query rows, K = dh.
 #pragma unroll
-        for (int ks = 0; ks < DH / 16; ++ks) {
-          const uint32_t pn = (ks * 16) / PANEL, off = ((ks * 16) % PANEL) * 2;
-          mma_ss(tmem + Tr::TM_ST, smem_desc(k_addr + pn * NK * ROWB + off, 16, 8 * ROWB, Tr::LAYOUT),
+      for (int ks = 0; ks < DH / 16; ++ks) {
+        const uint32_t pn = (ks * 16) / PANEL, off = ((ks * 16) % PANEL) * 2;
+        mma_ss_w(tmem + Tr::TM_ST, smem_desc(k_addr + pn * NK * ROWB + off, 16, 8 * ROWB, Tr::LAYOUT),
                  smem_desc(q_addr + pn * BM * ROWB + off, 16, 8 * ROWB, Tr::LAYOUT), idesc_s, ks > 0);
-          mma_ss(tmem + Tr::TM_DPT, smem_desc(v_addr + pn * NK * ROWB + off, 16, 8 * ROWB, Tr::LAYOUT),
+        mma_ss_w(tmem + Tr::TM_DPT, smem_desc(v_addr + pn * NK * ROWB + off, 16, 8 * ROWB, Tr::LAYOUT),
                  smem_desc(do_addr + pn * BM * ROWB + off, 16, 8 * ROWB, Tr::LAYOUT), idesc_s, ks > 0);
-        }
-        mma_commit(s_full);
-        if (!mbar_wait(ds_ready, i & 1, abort_flag, kSiteMma)) { ok = false; break; }
-        tc_fence_after();
-        // dV += P^T dO and dK += dS^T Q: K = 128 stacked query rows.  P^T / dS^T sit
-        // in two 32-column halves of packed bf16 pairs at column offsets 0 and 64.
+      }
+      mma_commit_w(s_full);
+      if (!mbar_wait_warp(ds_ready, i & 1, abort_flag, kSiteMma)) { ok = false; break; }
+      tc_fence_after();
+      // dV += P^T dO and dK += dS^T Q: K = 128 stacked query rows.  P^T / dS^T sit
+      // in two 32-column halves of packed bf16 pairs at column offsets 0 and 64.
 #pragma unroll
-        for (int ks = 0; ks < BM / 16; ++ks) {
-          const uint32_t acol = ks < 4 ? 8u * ks : 64u + 8u * (ks - 4);
-          const uint32_t brow = ks * 16 * ROWB;
-          mma_ts(tmem + Tr::TM_DV, tmem + Tr::TM_ST + acol,
+      for (int ks = 0; ks < BM / 16; ++ks) {
+        const uint32_t acol = ks < 4 ? 8u * ks : 64u + 8u * (ks - 4);
+        const uint32_t brow = ks * 16 * ROWB;
+        mma_ts_w(tmem + Tr::TM_DV, tmem + Tr::TM_ST + acol,
                  smem_desc(do_addr + brow, BM * ROWB, 8 * ROWB, Tr::LAYOUT), idesc_kv, (i > 0 || ks > 0));
-          mma_ts(tmem + Tr::TM_DK, tmem + Tr::TM_DPT + acol,
+        mma_ts_w(tmem + Tr::TM_DK, tmem + Tr::TM_DPT + acol,
                  smem_desc(q_addr + brow, BM * ROWB, 8 * ROWB, Tr::LAYOUT), idesc_kv, (i > 0 || ks > 0));
-        }
-        if (Tr::TM_DQ != Tr::TM_ST && i > 0 && !mbar_wait(dq_empty, (i - 1) & 1, abort_flag, kSiteMma)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // dQ = dS K: M = 128 stacked query rows, N = dh, K = 128 keys.  dS is
-        // MN-major (query rows contiguous) with a 128-byte swizzle: two 64-row
-        // panels 16 KB apart, 8-key groups 1 KB apart.
+      }
+      if (Tr::TM_DQ != Tr::TM_ST && i > 0 && !mbar_wait_warp(dq_empty, (i - 1) & 1, abort_flag, kSiteMma)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // dQ = dS K: M = 128 stacked query rows, N = dh, K = 128 keys.  dS is
+      // MN-major (query rows contiguous) with a 128-byte swizzle: two 64-row
+      // panels 16 KB apart, 8-key groups 1 KB apart.
 #pragma unroll
-        for (int ks = 0; ks < NK / 16; ++ks)
-          mma_ss(tmem + Tr::TM_DQ, smem_desc(ds_addr + ks * 2048, 16384, 1024, 2u),
+      for (int ks = 0; ks < NK / 16; ++ks)
+        mma_ss_w(tmem + Tr::TM_DQ, smem_desc(ds_addr + ks * 2048, 16384, 1024, 2u),
                  smem_desc(k_addr + ks * 16 * ROWB, NK * ROWB, 8 * ROWB, Tr::LAYOUT), idesc_q, ks > 0);
-        mma_commit(dq_full);
-        mma_commit(qd_empty(s));
-      }
-      if (ok) mma_commit(dkv_final);
-      else {
-        mma_commit(drain);
-        mbar_wait_drain(drain, 0);
-      }
+      mma_commit_w(dq_full);
+      mma_commit_w(qd_empty(s));
+    }
+    if (ok) mma_commit_w(dkv_final);
+    else {
+      mma_commit_w(drain);
+      mbar_wait_drain(drain, 0);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ P, dS, dQ epilogue, dK/dV epilogue

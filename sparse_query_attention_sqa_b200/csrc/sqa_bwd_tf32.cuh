@@ -1,10 +1,12 @@
 // sqa_bwd_tf32.cuh -- Sparse Query Attention backward, main kernel for head
 // dims 16 and 32 (the SQAT-m shapes).
 //
-// Same decomposition as sqa_bwd_kernel (one CTA per 128-key tile, batch and KV
+// Same decomposition as sqa_bwd_kernel (work item = 128-key tile, batch and KV
 // head; stacked Q tiles of the g query heads of the group, so dK and dV are
 // reduced over the group inside the tensor-core accumulation), organised for
-// small head dims.  There every tensor-core instruction is tiny (N = dh) and
+// small head dims.  The grid is persistent: each CTA walks a snake-ordered,
+// heaviest-first list of items, with K / V double-buffered so the next item's
+// tiles load while the current one finishes.  There every tensor-core instruction is tiny (N = dh) and
 // costs the tensor pipe a fixed number of cycles whatever its size, so the
 // schedule is built around keeping MMAs in flight while the softmax warps work:
 //
@@ -57,6 +59,17 @@ __device__ __forceinline__ void mma_ts_tf32(uint32_t d_tmem, uint32_t a_tmem, ui
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Warp-collective form: every lane calls it, one elected lane issues.
+__device__ __forceinline__ void mma_ts_tf32_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // fp32 bits rounded to the nearest tf32 value (10 mantissa bits; halfway cases
 // away from zero), with integer operations only.
 __device__ __forceinline__ uint32_t round_tf32(float x) {
@@ -75,22 +88,25 @@ struct BwdTf32Traits {
   static constexpr int PANEL32 = DH * 128;
   static constexpr int TILE = 128 * DH * 2;
   static constexpr int TILE32 = 128 * DH * 4;
-  static constexpr int QS = DH == 16 ? 3 : 2;  // Q / dO stages (shared memory bounds dh 32 to two)
+  static constexpr int QS = DH == 16 ? 4 : 2;  // Q / dO stages (shared memory bounds dh 32 to two)
   static constexpr int NBUF = 3;  // S^T / dP^T buffers in TMEM
   static constexpr int DS_BYTES = 128 * 128 * 2;  // bf16 dS, MN-major (query rows contiguous)
   static constexpr int OFF_DS = 0;                 // two buffers: Q tile i uses buffer i % 2
-  static constexpr int OFF_K = OFF_DS + 2 * DS_BYTES;
-  static constexpr int OFF_V = OFF_K + TILE;
-  static constexpr int OFF_Q = OFF_V + TILE;
+  static constexpr int OFF_K = OFF_DS + 2 * DS_BYTES;  // two buffers each (item r uses r % 2)
+  static constexpr int OFF_V = OFF_K + 2 * TILE;
+  static constexpr int OFF_Q = OFF_V + 2 * TILE;
   static constexpr int OFF_DO = OFF_Q + QS * TILE;
   static constexpr int OFF_Q32 = OFF_DO + QS * TILE;
   static constexpr int OFF_DO32 = OFF_Q32 + QS * TILE32;
   static constexpr int OFF_STAT = OFF_DO32 + QS * TILE32;  // per stage: lse2[128], D[128]
   static constexpr int OFF_RTOK = OFF_STAT + QS * 1024;
   static constexpr int OFF_BAR = OFF_RTOK + 512;
-  // kv_full, qd_full[3], qd_empty[3], s_full[3], ds_ready[3], kvmma_done[3], dsq_ready[2],
-  // dq_full[2], dq_empty[2], dkv_final, drain[3]
-  static constexpr int N_BARS = 26;
+  // Barrier slots: kv_full[2], kv_empty[2], qd_full[QS], qd_empty[QS], s_full[3], ds_ready[3],
+  // kvmma_done[3], dsq_ready[2], dq_full[2], dq_empty[2], dkv_final, dkv_free, drain[3].
+  static constexpr int B_QF = 4, B_QE = B_QF + QS, B_SF = B_QE + QS, B_DR = B_SF + NBUF, B_KD = B_DR + NBUF;
+  static constexpr int B_DSQ = B_KD + NBUF, B_DQF = B_DSQ + 2, B_DQE = B_DQF + 2, B_DKV = B_DQE + 2;
+  static constexpr int B_DRAIN = B_DKV + 2;
+  static constexpr int N_BARS = B_DRAIN + 3;
   static constexpr int SMEM_USED = OFF_BAR + N_BARS * 8 + 16;
   // Enough shared memory that only one CTA fits per SM (each holds all 512 TMEM columns).
   static constexpr int SMEM_BYTES = (SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024) + 1024;
@@ -140,6 +156,24 @@ __device__ __forceinline__ void bwd_p_ds(const uint32_t (&sr)[64], const float* 
   }
 }
 
+// One work item of the persistent backward: a 128-key tile of one (batch, KV
+// head).  Items are numbered key tile major, so under a causal mask the first
+// key tiles, which see the most Q tiles, come first.
+struct BwdItem {
+  int b, kvh, bh, k0, qt_first, nq;
+};
+__device__ __forceinline__ BwdItem bwd_decode(const BwdParams& p, int item) {
+  BwdItem it;
+  const int kt = item / p.n_bh;
+  it.bh = item % p.n_bh;
+  it.b = it.bh / p.Hkv;
+  it.kvh = it.bh % p.Hkv;
+  it.k0 = kt * kBwdTile;
+  it.qt_first = p.causal ? it.k0 / p.T : 0;
+  it.nq = p.n_qt - it.qt_first;
+  return it;
+}
+
 template <int DH>
 __global__ void __launch_bounds__(384, 1)
     sqa_bwd_tf32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
@@ -155,33 +189,29 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Under a causal mask the first key tiles see the most query tiles: they go first.
-  const int kt = static_cast<int>(blockIdx.x / p.n_bh);
-  const int bh = blockIdx.x % p.n_bh;
-  const int b = bh / p.Hkv, kvh = bh % p.Hkv;
-  const int k0 = kt * NK;
-  const int qt_first = p.causal ? k0 / p.T : 0;
-  const int nq = p.n_qt - qt_first;
-  const int nh = 2 * nq;  // halves
-
   const uint32_t bar0 = sbase + Tr::OFF_BAR;
-  const uint32_t kv_full = bar0;
-  auto qd_full = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto qd_empty = [&](int s) { return bar0 + 8u * (4 + s); };
-  auto s_full = [&](int x) { return bar0 + 8u * (7 + x); };
-  auto ds_ready = [&](int x) { return bar0 + 8u * (10 + x); };
-  auto kvmma_done = [&](int x) { return bar0 + 8u * (13 + x); };
-  auto dsq_ready = [&](int w) { return bar0 + 8u * (16 + w); };  // warpgroup w wrote its half of dS
-  auto dq_full = [&](int x) { return bar0 + 8u * (18 + x); };    // dQ of tile i in buffer x = i % 2 done
-  auto dq_empty = [&](int x) { return bar0 + 8u * (20 + x); };
-  const uint32_t dkv_final = bar0 + 8u * 22;
-  auto drain = [&](int x) { return bar0 + 8u * (23 + x); };
+  auto kv_full = [&](int kb) { return bar0 + 8u * (0 + kb); };
+  auto kv_empty = [&](int kb) { return bar0 + 8u * (2 + kb); };
+  auto qd_full = [&](int s) { return bar0 + 8u * (Tr::B_QF + s); };
+  auto qd_empty = [&](int s) { return bar0 + 8u * (Tr::B_QE + s); };
+  auto s_full = [&](int x) { return bar0 + 8u * (Tr::B_SF + x); };
+  auto ds_ready = [&](int x) { return bar0 + 8u * (Tr::B_DR + x); };
+  auto kvmma_done = [&](int x) { return bar0 + 8u * (Tr::B_KD + x); };
+  auto dsq_ready = [&](int w) { return bar0 + 8u * (Tr::B_DSQ + w); };  // warpgroup w wrote its columns of dS
+  auto dq_full = [&](int x) { return bar0 + 8u * (Tr::B_DQF + x); };    // dQ of tile G in buffer x = G % 2 done
+  auto dq_empty = [&](int x) { return bar0 + 8u * (Tr::B_DQE + x); };
+  const uint32_t dkv_final = bar0 + 8u * Tr::B_DKV;       // dV / dK of the item complete
+  const uint32_t dkv_free = bar0 + 8u * (Tr::B_DKV + 1);  // the epilogue has read them
+  auto drain = [&](int x) { return bar0 + 8u * (Tr::B_DRAIN + x); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Tr::OFF_BAR + Tr::N_BARS * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* rtok = reinterpret_cast<int*>(smem + Tr::OFF_RTOK);
 
   if (threadIdx.x == 0) {
-    mbar_init(kv_full, 1);
+    for (int kb = 0; kb < 2; ++kb) {
+      mbar_init(kv_full(kb), 1);
+      mbar_init(kv_empty(kb), 1);  // issuer A
+    }
     for (int s = 0; s < QS; ++s) {
       mbar_init(qd_full(s), 1);
       mbar_init(qd_empty(s), 3);  // released by the three MMA issuers
@@ -198,6 +228,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(dq_empty(x), 256);
     }
     mbar_init(dkv_final, 2);
+    mbar_init(dkv_free, 256);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -220,6 +251,8 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // Counters shared by every role: r = this CTA's item round, gt = Q tiles of
+  // earlier items.  Global tile G = gt + i, global half H = 2 G + hh.
   if (warp == Tr::WARP_PRODUCER) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -227,96 +260,122 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_map(&tmDO);
       tma_prefetch_map(&tmK);
       tma_prefetch_map(&tmV);
-      mbar_expect_tx(kv_full, 2u * Tr::TILE);
-      tma_load_4d(sbase + Tr::OFF_K, &tmK, kv_full, 0, kvh, k0, b);
-      tma_load_4d(sbase + Tr::OFF_V, &tmV, kv_full, 0, kvh, k0, b);
       const uint32_t qd_bytes = 2u * p.rows * ROWB + 2u * 512u + 2u * Tr::TILE32;
-      int issued = 0;
-      for (int i = 0; i < nq; ++i) {
-        const int s = i % QS, qt = qt_first + i;
-        if (i >= QS && !mbar_wait(qd_empty(s), ((i / QS) - 1) & 1, abort_flag, kSiteProducer)) break;
-        mbar_expect_tx(qd_full(s), qd_bytes);
-        tma_load_4d(sbase + Tr::OFF_Q + s * Tr::TILE, &tmQ, qd_full(s), 0, kvh * p.g, qt * p.T, b);
-        tma_load_4d(sbase + Tr::OFF_DO + s * Tr::TILE, &tmDO, qd_full(s), 0, kvh * p.g, qt * p.T, b);
-        const size_t slot = (static_cast<size_t>(bh) * p.n_qt + qt) * kBwdTile;
-        bulk_load(sbase + Tr::OFF_STAT + s * 1024, p.lse2 + slot, 512, qd_full(s));
-        bulk_load(sbase + Tr::OFF_STAT + s * 1024 + 512, p.D + slot, 512, qd_full(s));
-        bulk_load(sbase + Tr::OFF_Q32 + s * Tr::TILE32, p.q32 + slot * DH, Tr::TILE32, qd_full(s));
-        bulk_load(sbase + Tr::OFF_DO32 + s * Tr::TILE32, p.do32 + slot * DH, Tr::TILE32, qd_full(s));
-        issued = i + 1;
+      int gt = 0, items_issued = 0, tiles_issued = 0;
+      bool ok = true;
+      for (int r = 0, item; ok && (item = snake_item(r, p.n_items)) >= 0; ++r) {
+        const BwdItem it = bwd_decode(p, item);
+        const int kb = r & 1;
+        if (r >= 2 && !mbar_wait(kv_empty(kb), ((r >> 1) - 1) & 1, abort_flag, kSiteProducer)) break;
+        mbar_expect_tx(kv_full(kb), 2u * Tr::TILE);
+        tma_load_4d(sbase + Tr::OFF_K + kb * Tr::TILE, &tmK, kv_full(kb), 0, it.kvh, it.k0, it.b);
+        tma_load_4d(sbase + Tr::OFF_V + kb * Tr::TILE, &tmV, kv_full(kb), 0, it.kvh, it.k0, it.b);
+        items_issued = r + 1;
+        for (int i = 0; i < it.nq; ++i) {
+          const int G = gt + i, s = G % QS, qt = it.qt_first + i;
+          if (G >= QS && !mbar_wait(qd_empty(s), ((G / QS) - 1) & 1, abort_flag, kSiteProducer)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(qd_full(s), qd_bytes);
+          tma_load_4d(sbase + Tr::OFF_Q + s * Tr::TILE, &tmQ, qd_full(s), 0, it.kvh * p.g, qt * p.T, it.b);
+          tma_load_4d(sbase + Tr::OFF_DO + s * Tr::TILE, &tmDO, qd_full(s), 0, it.kvh * p.g, qt * p.T, it.b);
+          const size_t slot = (static_cast<size_t>(it.bh) * p.n_qt + qt) * kBwdTile;
+          bulk_load(sbase + Tr::OFF_STAT + s * 1024, p.lse2 + slot, 512, qd_full(s));
+          bulk_load(sbase + Tr::OFF_STAT + s * 1024 + 512, p.D + slot, 512, qd_full(s));
+          bulk_load(sbase + Tr::OFF_Q32 + s * Tr::TILE32, p.q32 + slot * DH, Tr::TILE32, qd_full(s));
+          bulk_load(sbase + Tr::OFF_DO32 + s * Tr::TILE32, p.do32 + slot * DH, Tr::TILE32, qd_full(s));
+          tiles_issued = G + 1;
+        }
+        gt += it.nq;
       }
-      if (*abort_flag) {
-        mbar_wait_drain(kv_full, 0);
-        for (int i = max(0, issued - QS); i < issued; ++i) mbar_wait_drain(qd_full(i % QS), (i / QS) & 1);
+      if (*abort_flag) {  // let in-flight copies land before the CTA exits
+        for (int j = max(0, items_issued - 2); j < items_issued; ++j) mbar_wait_drain(kv_full(j & 1), (j >> 1) & 1);
+        for (int G = max(0, tiles_issued - QS); G < tiles_issued; ++G) mbar_wait_drain(qd_full(G % QS), (G / QS) & 1);
       }
     }
   } else if (warp == Tr::WARP_MMA_A) {
     // ------------------------------------------------------------ MMA issuer A: S^T, dP^T, dQ
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);  // S^T, dP^T halves
-      constexpr uint32_t idesc_q = idesc_bf16_f32(128, DH, true, true);    // dQ = dS K (both MN-major)
-      // Descriptors of stage 0 / K-step 0; others add their byte offset / 16.
-      const uint64_t dk = smem_desc(sbase + Tr::OFF_K, 16, 8 * ROWB, Tr::LAYOUT);
-      const uint64_t dv = smem_desc(sbase + Tr::OFF_V, 16, 8 * ROWB, Tr::LAYOUT);
-      const uint64_t dqt = smem_desc(sbase + Tr::OFF_Q, 16, 8 * ROWB, Tr::LAYOUT);
-      const uint64_t ddo = smem_desc(sbase + Tr::OFF_DO, 16, 8 * ROWB, Tr::LAYOUT);
-      const uint64_t dds = smem_desc(sbase + Tr::OFF_DS, 16384, 1024, 2u);
-      const uint64_t dkmn = smem_desc(sbase + Tr::OFF_K, NK * ROWB, 8 * ROWB, Tr::LAYOUT);
-      // S^T and dP^T of half h (query rows 64 (h % 2) .. of Q tile h / 2) into
-      // TMEM buffer h % 3, once its Q / dO tile has landed and DV and DK have
-      // finished reading the half that used the buffer before (h - 3).
-      auto issue_half = [&](int h) -> bool {
-        const int i = h >> 1, s = i % QS, x = h % NBUF;
-        if ((h & 1) == 0 && !mbar_wait(qd_full(s), (i / QS) & 1, abort_flag, kSiteMma)) return false;
-        if (h >= NBUF && !mbar_wait(kvmma_done(x), ((h / NBUF) - 1) & 1, abort_flag, kSiteMma)) return false;
+    // The whole warp runs the loop; one elected lane issues each MMA.
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);  // S^T, dP^T halves
+    constexpr uint32_t idesc_q = idesc_bf16_f32(128, DH, true, true);    // dQ = dS K (both MN-major)
+    // Descriptors of buffer / stage 0 and K-step 0; others add their byte offset / 16.
+    const uint64_t dk0 = smem_desc(sbase + Tr::OFF_K, 16, 8 * ROWB, Tr::LAYOUT);
+    const uint64_t dv0 = smem_desc(sbase + Tr::OFF_V, 16, 8 * ROWB, Tr::LAYOUT);
+    const uint64_t dqt = smem_desc(sbase + Tr::OFF_Q, 16, 8 * ROWB, Tr::LAYOUT);
+    const uint64_t ddo = smem_desc(sbase + Tr::OFF_DO, 16, 8 * ROWB, Tr::LAYOUT);
+    const uint64_t dds = smem_desc(sbase + Tr::OFF_DS, 16384, 1024, 2u);
+    const uint64_t dkmn0 = smem_desc(sbase + Tr::OFF_K, NK * ROWB, 8 * ROWB, Tr::LAYOUT);
+    int gt = 0;
+    bool ok = true;
+    for (int r = 0, item; ok && (item = snake_item(r, p.n_items)) >= 0; ++r) {
+      const BwdItem it = bwd_decode(p, item);
+      const int kb = r & 1, nh = 2 * it.nq;
+      const uint64_t koff = static_cast<uint64_t>((kb * Tr::TILE) >> 4);
+      if (!(ok = mbar_wait_warp(kv_full(kb), (r >> 1) & 1, abort_flag, kSiteMma))) break;
+      // S^T and dP^T of the item's half hl (query rows 64 (hl % 2) .. of its tile
+      // hl / 2) into TMEM buffer H % 3, once the Q / dO tile has landed and DV and
+      // DK have finished reading the half that used the buffer before (H - 3).
+      auto issue_half = [&](int hl) -> bool {
+        const int G = gt + (hl >> 1), H = 2 * gt + hl, s = G % QS, x = H % NBUF;
+        if ((hl & 1) == 0 && !mbar_wait_warp(qd_full(s), (G / QS) & 1, abort_flag, kSiteMma)) return false;
+        if (H >= NBUF && !mbar_wait_warp(kvmma_done(x), ((H / NBUF) - 1) & 1, abort_flag, kSiteMma)) return false;
         tc_fence_after();
-        const uint64_t off = static_cast<uint64_t>((s * Tr::TILE + (h & 1) * 64 * ROWB) >> 4);
+        const uint64_t off = static_cast<uint64_t>((s * Tr::TILE + (hl & 1) * 64 * ROWB) >> 4);
 #pragma unroll
         for (int ks = 0; ks < DH / 16; ++ks) {
-          mma_ss(tmem + Tr::tm_st(x), dk + 2 * ks, dqt + off + 2 * ks, idesc_s, ks > 0);
-          mma_ss(tmem + Tr::tm_dpt(x), dv + 2 * ks, ddo + off + 2 * ks, idesc_s, ks > 0);
+          mma_ss_w(tmem + Tr::tm_st(x), dk0 + koff + 2 * ks, dqt + off + 2 * ks, idesc_s, ks > 0);
+          mma_ss_w(tmem + Tr::tm_dpt(x), dv0 + koff + 2 * ks, ddo + off + 2 * ks, idesc_s, ks > 0);
         }
-        mma_commit(s_full(x));
+        mma_commit_w(s_full(x));
         return true;
       };
-      bool ok = mbar_wait(kv_full, 0, abort_flag, kSiteMma);
-      for (int h = 0; ok && h < NBUF && h < nh; ++h) ok = issue_half(h);
-      for (int i = 0; ok && i < nq; ++i) {
-        // dQ of tile i once both warpgroups wrote their half of dS, into the
-        // dQ buffer the epilogue of tile i - 2 has emptied.
-        if (!mbar_wait(dsq_ready(0), i & 1, abort_flag, kSiteMma) ||
-            !mbar_wait(dsq_ready(1), i & 1, abort_flag, kSiteMma)) { ok = false; break; }
-        if (i >= 2 && !mbar_wait(dq_empty(i & 1), ((i >> 1) - 1) & 1, abort_flag, kSiteMma)) { ok = false; break; }
+      for (int hl = 0; ok && hl < NBUF && hl < nh; ++hl) ok = issue_half(hl);
+      for (int i = 0; ok && i < it.nq; ++i) {
+        const int G = gt + i;
+        // dQ of tile G once both warpgroups wrote their columns of dS, into the
+        // dQ buffer the epilogue of tile G - 2 has emptied.
+        if (!mbar_wait_warp(dsq_ready(0), G & 1, abort_flag, kSiteMma) ||
+            !mbar_wait_warp(dsq_ready(1), G & 1, abort_flag, kSiteMma)) { ok = false; break; }
+        if (G >= 2 && !mbar_wait_warp(dq_empty(G & 1), ((G >> 1) - 1) & 1, abort_flag, kSiteMma)) { ok = false; break; }
         tc_fence_after();
         // dQ = dS K: M = 128 query rows, N = dh, K = 128 keys in steps of 16 (2 KB of dS, 16 K rows).
-        const uint64_t dsb = dds + static_cast<uint64_t>(((i & 1) * Tr::DS_BYTES) >> 4);
+        const uint64_t dsb = dds + static_cast<uint64_t>(((G & 1) * Tr::DS_BYTES) >> 4);
 #pragma unroll
         for (int ks = 0; ks < NK / 16; ++ks)
-          mma_ss(tmem + Tr::tm_dq(i), dsb + 128 * ks, dkmn + ((ks * 16 * ROWB) >> 4), idesc_q, ks > 0);
-        mma_commit(dq_full(i & 1));
-        mma_commit(qd_empty(i % QS));
+          mma_ss_w(tmem + Tr::tm_dq(G), dsb + 128 * ks, dkmn0 + koff + ((ks * 16 * ROWB) >> 4), idesc_q, ks > 0);
+        mma_commit_w(dq_full(G & 1));
+        mma_commit_w(qd_empty(G % QS));
         if (2 * i + 3 < nh && !(ok = issue_half(2 * i + 3))) break;
         if (2 * i + 4 < nh && !(ok = issue_half(2 * i + 4))) break;
       }
-      if (!ok) {
-        mma_commit(drain(0));
-        mbar_wait_drain(drain(0), 0);
-      }
+      if (!ok) break;
+      mma_commit_w(kv_empty(kb));  // every MMA reading this item's K and V has been issued
+      gt += it.nq;
+    }
+    if (!ok) {
+      mma_commit_w(drain(0));
+      mbar_wait_drain(drain(0), 0);
     }
   } else if (warp == Tr::WARP_MMA_DV || warp == Tr::WARP_MMA_DK) {
     // ------------------------------------------------------------ MMA issuers DV (dV += P^T dO) and DK (dK += dS^T Q)
-    if (lane == 0) {
-      const bool is_dv = warp == Tr::WARP_MMA_DV;
-      constexpr uint32_t idesc_g = idesc_tf32_f32(128, DH, false, false);
-      const uint64_t dimg = smem_desc(sbase + (is_dv ? Tr::OFF_DO32 : Tr::OFF_Q32), 16, 1024, 2u);
-      const uint32_t d_acc = tmem + (is_dv ? Tr::TM_DV : Tr::TM_DK);
-      const uint32_t a_col = is_dv ? 0u : 64u;  // P^T or dS^T inside a buffer
-      bool ok = true;
-      for (int h = 0; h < nh; ++h) {
-        const int i = h >> 1, hh = h & 1, s = i % QS, x = h % NBUF;
-        if (!mbar_wait(ds_ready(x), (h / NBUF) & 1, abort_flag, kSiteMma)) { ok = false; break; }
-        // The image arrived with the Q tile (already complete: the warpgroup waited for it).
-        if (hh == 0 && !mbar_wait(qd_full(s), (i / QS) & 1, abort_flag, kSiteMma)) { ok = false; break; }
+    // The whole warp runs the loop; one elected lane issues each MMA.
+    const bool is_dv = warp == Tr::WARP_MMA_DV;
+    constexpr uint32_t idesc_g = idesc_tf32_f32(128, DH, false, false);
+    const uint64_t dimg = smem_desc(sbase + (is_dv ? Tr::OFF_DO32 : Tr::OFF_Q32), 16, 1024, 2u);
+    const uint32_t d_acc = tmem + (is_dv ? Tr::TM_DV : Tr::TM_DK);
+    const uint32_t a_col = is_dv ? 0u : 64u;  // P^T or dS^T inside a buffer
+    int gt = 0;
+    bool ok = true;
+    for (int r = 0, item; ok && (item = snake_item(r, p.n_items)) >= 0; ++r) {
+      const BwdItem it = bwd_decode(p, item);
+      for (int hl = 0; hl < 2 * it.nq; ++hl) {
+        const int G = gt + (hl >> 1), H = 2 * gt + hl, s = G % QS, x = H % NBUF;
+        if (!(ok = mbar_wait_warp(ds_ready(x), (H / NBUF) & 1, abort_flag, kSiteMma))) break;
+        // The accumulators still hold the previous item until its epilogue has read them.
+        if (hl == 0 && r > 0 && !(ok = mbar_wait_warp(dkv_free, (r - 1) & 1, abort_flag, kSiteMma))) break;
+        // The image arrived with the Q tile (already complete: the warpgroups waited for it).
+        if ((hl & 1) == 0 && !(ok = mbar_wait_warp(qd_full(s), (G / QS) & 1, abort_flag, kSiteMma))) break;
         tc_fence_after();
         // K = 8 query rows per tf32 MMA: rows q0..q0+7 are 32 bytes at offset
         // (q0 % 32) * 4 of panel q0 / 32 of the image.
@@ -324,147 +383,153 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t a0 = tmem + Tr::tm_st(x) + a_col;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const int q0 = hh * 64 + ks * 8;
+          const int q0 = (hl & 1) * 64 + ks * 8;
           const uint64_t boff = stage_off + (((q0 >> 5) * Tr::PANEL32 + (q0 & 31) * 4) >> 4);
-          mma_ts_tf32(d_acc, a0 + 8 * ks, dimg + boff, idesc_g, (h > 0 || ks > 0) ? 1u : 0u);
+          mma_ts_tf32_w(d_acc, a0 + 8 * ks, dimg + boff, idesc_g, (hl > 0 || ks > 0) ? 1u : 0u);
         }
-        mma_commit(kvmma_done(x));
-        if (hh == 1) mma_commit(qd_empty(s));
+        mma_commit_w(kvmma_done(x));
+        if (hl & 1) mma_commit_w(qd_empty(s));
       }
-      if (ok) mma_commit(dkv_final);
-      else {
-        const int x = is_dv ? 1 : 2;
-        mma_commit(drain(x));
-        mbar_wait_drain(drain(x), 0);
-      }
+      if (!ok) break;
+      mma_commit_w(dkv_final);
+      gt += it.nq;
+    }
+    if (!ok) {
+      const int x = is_dv ? 1 : 2;
+      mma_commit_w(drain(x));
+      mbar_wait_drain(drain(x), 0);
     }
   } else {
     // ------------------------------------------------------------ P^T, dS^T, dQ and dK/dV epilogues
     const int w = warp >> 2;                  // warpgroup: 32-column slice of each half, dh/2 columns of dQ, dK, dV
     const int kk = (warp & 3) * 32 + lane;    // TMEM lane: key (S^T, dP^T, dK, dV) or query row (dQ)
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const int key = k0 + kk;
-    const bool key_ok = key < p.N;
-    const bool ragged = k0 + NK > p.N;  // the last key tile: rows past N hold zeros
     const float2 sl2 = make_float2(p.scale_log2, p.scale_log2);
     const int qrow_tok = kk < p.rows ? kk / p.g : (1 << 30);
-    const int qrow_head = kvh * p.g + kk % p.g;
+    int gt = 0;
     bool ok = true;
+    for (int r = 0, item; ok && (item = snake_item(r, p.n_items)) >= 0; ++r) {
+      const BwdItem it = bwd_decode(p, item);
+      const int key = it.k0 + kk;
+      const bool key_ok = key < p.N;
+      const bool ragged = it.k0 + NK > p.N;  // the last key tile: rows past N hold zeros
+      const int qrow_head = it.kvh * p.g + kk % p.g;
 
-    // dQ of Q tile i: TMEM -> fp32 accumulator (this warpgroup: dh/2 columns).
-    auto dq_epilogue = [&](int i) {
-      float v[DH / 2];
-      tmem_ld_half<DH>(lane_addr + Tr::tm_dq(i) + w * (DH / 2), v);
-      tc_fence_before();
-      mbar_arrive(dq_empty(i & 1));
-      const int tok = (qt_first + i) * p.T + qrow_tok;
-      if (tok < p.N) {
-        float* dst = p.dq_acc + ((static_cast<size_t>(b) * p.N + tok) * p.Hq + qrow_head) * DH + w * (DH / 2);
+      // dQ of the item's tile i (global G): TMEM -> fp32 accumulator (this warpgroup: dh/2 columns).
+      auto dq_epilogue = [&](int i) {
+        const int G = gt + i;
+        float v[DH / 2];
+        tmem_ld_half<DH>(lane_addr + Tr::tm_dq(G) + w * (DH / 2), v);
+        tc_fence_before();
+        mbar_arrive(dq_empty(G & 1));
+        const int tok = (it.qt_first + i) * p.T + qrow_tok;
+        if (tok < p.N) {
+          float* dst =
+              p.dq_acc + ((static_cast<size_t>(it.b) * p.N + tok) * p.Hq + qrow_head) * DH + w * (DH / 2);
 #pragma unroll
-        for (int c = 0; c < DH / 2; c += 4)
-          atomicAdd(reinterpret_cast<float4*>(dst + c), make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]));
-      }
-    };
+          for (int c = 0; c < DH / 2; c += 4)
+            atomicAdd(reinterpret_cast<float4*>(dst + c), make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]));
+        }
+      };
 
-    for (int i = 0; i < nq; ++i) {
-      const int s = i % QS, qt = qt_first + i;
-      ok = __all_sync(0xffffffffu, mbar_wait(qd_full(s), (i / QS) & 1, abort_flag, kSiteSoftmax));
-      if (!ok) break;
-      const bool masked = p.causal && (k0 + NK - 1 > qt * p.T);
-      // P is zeroed where lim > rtok[row]: keys past N always, keys after the
-      // row's token on the causal diagonal.
-      const int lim = !key_ok ? 0x7fffffff : (masked ? key - qt * p.T : -0x7fffffff);
-      uint8_t* ds_smem = smem + Tr::OFF_DS + (i & 1) * Tr::DS_BYTES;
-#pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
-        // Both warpgroups work on half hh of the tile: this one on its 32
-        // query columns col0 .. col0 + 31.
-        const int h = 2 * i + hh, x = h % NBUF;
-        const int col0 = 64 * hh + 32 * w;
-        ok = __all_sync(0xffffffffu, mbar_wait(s_full(x), (h / NBUF) & 1, abort_flag, kSiteSoftmax));
+      for (int i = 0; i < it.nq; ++i) {
+        const int G = gt + i, s = G % QS, qt = it.qt_first + i;
+        ok = __all_sync(0xffffffffu, mbar_wait(qd_full(s), (G / QS) & 1, abort_flag, kSiteSoftmax));
         if (!ok) break;
-        tc_fence_after();
-        const float* nl2 = reinterpret_cast<const float*>(smem + Tr::OFF_STAT + s * 1024) + col0;
-        uint32_t sr[64];  // [0,32): S^T, [32,64): dP^T
-        tmem_ld32x2(lane_addr + Tr::tm_st(x) + 32 * w, lane_addr + Tr::tm_dpt(x) + 32 * w, sr);
-        uint32_t pt[32], dst[32], dsb[16];
-        if (masked || ragged)
-          bwd_p_ds<true>(sr, nl2, nl2 + 128, rtok + col0, lim, sl2, pt, dst, dsb);
-        else
-          bwd_p_ds<false>(sr, nl2, nl2 + 128, rtok + col0, lim, sl2, pt, dst, dsb);
-        tmem_st32(lane_addr + Tr::tm_st(x) + 32 * w, pt);
-        tmem_st32(lane_addr + Tr::tm_dpt(x) + 32 * w, dst);
-        // dS (bf16) for the dQ MMA: the dQ of Q tile i - 2 read this buffer, so
-        // wait for it before the first write of a tile.
-        if (hh == 0 && i >= 2) {
-          ok = __all_sync(0xffffffffu, mbar_wait(dq_full(i & 1), ((i >> 1) - 1) & 1, abort_flag, kSiteSoftmax));
+        const bool masked = p.causal && (it.k0 + NK - 1 > qt * p.T);
+        // P is zeroed where lim > rtok[row]: keys past N always, keys after the
+        // row's token on the causal diagonal.
+        const int lim = !key_ok ? 0x7fffffff : (masked ? key - qt * p.T : -0x7fffffff);
+        uint8_t* ds_smem = smem + Tr::OFF_DS + (G & 1) * Tr::DS_BYTES;
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          // Both warpgroups work on half hh of the tile: this one on its 32
+          // query columns col0 .. col0 + 31.
+          const int H = 2 * G + hh, x = H % NBUF;
+          const int col0 = 64 * hh + 32 * w;
+          ok = __all_sync(0xffffffffu, mbar_wait(s_full(x), (H / NBUF) & 1, abort_flag, kSiteSoftmax));
+          if (!ok) break;
+          tc_fence_after();
+          const float* nl2 = reinterpret_cast<const float*>(smem + Tr::OFF_STAT + s * 1024) + col0;
+          uint32_t sr[64];  // [0,32): S^T, [32,64): dP^T
+          tmem_ld32x2(lane_addr + Tr::tm_st(x) + 32 * w, lane_addr + Tr::tm_dpt(x) + 32 * w, sr);
+          uint32_t pt[32], dst[32], dsb[16];
+          if (masked || ragged)
+            bwd_p_ds<true>(sr, nl2, nl2 + 128, rtok + col0, lim, sl2, pt, dst, dsb);
+          else
+            bwd_p_ds<false>(sr, nl2, nl2 + 128, rtok + col0, lim, sl2, pt, dst, dsb);
+          tmem_st32(lane_addr + Tr::tm_st(x) + 32 * w, pt);
+          tmem_st32(lane_addr + Tr::tm_dpt(x) + 32 * w, dst);
+          // dS (bf16) for the dQ MMA: the dQ of tile G - 2 read this buffer, so
+          // wait for it before the first write of a tile.
+          if (hh == 0 && G >= 2) {
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(dq_full(G & 1), ((G >> 1) - 1) & 1, abort_flag, kSiteSoftmax));
+            if (!ok) break;
+          }
+          // dS[q][key] for q = col0..col0+31 into the MN-major 128B-swizzled tile:
+          // panel q / 64, key row kk (128 bytes), 16-byte chunk (q % 64) / 8.
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            const int q = col0 + 8 * ch;
+            const int panel = q >> 6, chunk = (q & 63) >> 3;
+            *reinterpret_cast<uint4*>(ds_smem + panel * 16384 + kk * 128 + ((chunk ^ (kk & 7)) << 4)) =
+                make_uint4(dsb[4 * ch], dsb[4 * ch + 1], dsb[4 * ch + 2], dsb[4 * ch + 3]);
+          }
+          tmem_wait_st();
+          fence_async_smem();
+          tc_fence_before();
+          mbar_arrive(ds_ready(x));
+        }
+        if (!ok) break;
+        // dsq_ready(w) is signalled only after the dQ of tile G - 1 completed,
+        // which keeps it at most one phase ahead of issuer A's wait.
+        if (G > 0) {
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(dq_full((G - 1) & 1), ((G - 1) >> 1) & 1, abort_flag, kSiteSoftmax));
           if (!ok) break;
         }
-        // dS[q][key] for q = col0..col0+31 into the MN-major 128B-swizzled tile:
-        // panel q / 64, key row kk (128 bytes), 16-byte chunk (q % 64) / 8.
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const int q = col0 + 8 * ch;
-          const int panel = q >> 6, chunk = (q & 63) >> 3;
-          *reinterpret_cast<uint4*>(ds_smem + panel * 16384 + kk * 128 + ((chunk ^ (kk & 7)) << 4)) =
-              make_uint4(dsb[4 * ch], dsb[4 * ch + 1], dsb[4 * ch + 2], dsb[4 * ch + 3]);
+        mbar_arrive(dsq_ready(w));
+        if (i > 0) {
+          tc_fence_after();
+          dq_epilogue(i - 1);
         }
-        tmem_wait_st();
-        fence_async_smem();
-        tc_fence_before();
-        mbar_arrive(ds_ready(x));
       }
       if (!ok) break;
-      // dsq_ready(w) is signalled only after the dQ of tile i - 1 completed,
-      // which keeps it at most one phase ahead of issuer A's wait.
-      if (i > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(dq_full((i - 1) & 1), ((i - 1) >> 1) & 1, abort_flag, kSiteSoftmax));
+      {
+        const int G = gt + it.nq - 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(dq_full(G & 1), (G >> 1) & 1, abort_flag, kSiteEpilogue));
         if (!ok) break;
-      }
-      mbar_arrive(dsq_ready(w));
-      if (i > 0) {
         tc_fence_after();
-        dq_epilogue(i - 1);
+        dq_epilogue(it.nq - 1);
       }
-    }
-    if (ok && nq > 0) {
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait(dq_full((nq - 1) & 1), ((nq - 1) >> 1) & 1, abort_flag, kSiteEpilogue));
-      if (ok) {
-        tc_fence_after();
-        dq_epilogue(nq - 1);
-      }
-    }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(dkv_final, 0, abort_flag, kSiteEpilogue));
-    if (ok) {
+      ok = __all_sync(0xffffffffu, mbar_wait(dkv_final, r & 1, abort_flag, kSiteEpilogue));
+      if (!ok) break;
       tc_fence_after();
-      const size_t off = ((static_cast<size_t>(b) * p.N + (key_ok ? key : 0)) * p.Hkv + kvh) * DH + w * (DH / 2);
-      float v[DH / 2];
-      tmem_ld_half<DH>(lane_addr + Tr::TM_DV + w * (DH / 2), v);
+      float dv[DH / 2], dk[DH / 2];
+      tmem_ld_half<DH>(lane_addr + Tr::TM_DV + w * (DH / 2), dv);
+      tmem_ld_half<DH>(lane_addr + Tr::TM_DK + w * (DH / 2), dk);
+      tc_fence_before();
+      mbar_arrive(dkv_free);
       if (key_ok) {
-#pragma unroll
-        for (int c = 0; c < DH / 2; c += 8) {
-          uint4 o;
-          o.x = pack_bf16x2(v[c], v[c + 1]);
-          o.y = pack_bf16x2(v[c + 2], v[c + 3]);
-          o.z = pack_bf16x2(v[c + 4], v[c + 5]);
-          o.w = pack_bf16x2(v[c + 6], v[c + 7]);
-          *reinterpret_cast<uint4*>(p.dv + off + c) = o;
-        }
-      }
-      tmem_ld_half<DH>(lane_addr + Tr::TM_DK + w * (DH / 2), v);
-      if (key_ok) {
+        const size_t off = ((static_cast<size_t>(it.b) * p.N + key) * p.Hkv + it.kvh) * DH + w * (DH / 2);
         const float sc = p.scale;
 #pragma unroll
         for (int c = 0; c < DH / 2; c += 8) {
           uint4 o;
-          o.x = pack_bf16x2(v[c] * sc, v[c + 1] * sc);
-          o.y = pack_bf16x2(v[c + 2] * sc, v[c + 3] * sc);
-          o.z = pack_bf16x2(v[c + 4] * sc, v[c + 5] * sc);
-          o.w = pack_bf16x2(v[c + 6] * sc, v[c + 7] * sc);
+          o.x = pack_bf16x2(dv[c], dv[c + 1]);
+          o.y = pack_bf16x2(dv[c + 2], dv[c + 3]);
+          o.z = pack_bf16x2(dv[c + 4], dv[c + 5]);
+          o.w = pack_bf16x2(dv[c + 6], dv[c + 7]);
+          *reinterpret_cast<uint4*>(p.dv + off + c) = o;
+          o.x = pack_bf16x2(dk[c] * sc, dk[c + 1] * sc);
+          o.y = pack_bf16x2(dk[c + 2] * sc, dk[c + 3] * sc);
+          o.z = pack_bf16x2(dk[c + 4] * sc, dk[c + 5] * sc);
+          o.w = pack_bf16x2(dk[c + 6] * sc, dk[c + 7] * sc);
           *reinterpret_cast<uint4*>(p.dk + off + c) = o;
         }
       }
+      gt += it.nq;
     }
   }
 

@@ -67,6 +67,21 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about `hint_ns` pass, instead of spinning on issue slots that
+// the warps sharing its sub-partition need.
+__device__ __forceinline__ bool mbar_test_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return done != 0;
+}
+
 // Wait for the phase of `bar` with the given parity (mbar_wait below is the
 // entry point).  Gives up when another
 // role of the CTA has raised `abort_flag`, or after kWaitLimitNs (then it
@@ -77,8 +92,8 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volat
   const unsigned long long t0 = global_timer_ns();
   while (true) {
 #pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_test(bar, parity)) return true;
+    for (int i = 0; i < 8; ++i)
+      if (mbar_test_sleep(bar, parity, 20000u)) return true;
     if (*abort_flag) return false;
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       *abort_flag = 1;
@@ -97,6 +112,12 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volat
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, unsigned site) {
   if (mbar_test(bar, parity)) return true;
   return mbar_wait_slow(bar, parity, abort_flag, site);
+}
+
+// mbar_wait by every lane of a converged warp, with one verdict for all lanes.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                               unsigned site) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, site));
 }
 
 // Bounded wait used only on the abort path, to let in-flight copies and MMAs
@@ -195,6 +216,38 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");
+}
+
+// Warp-collective forms of the three calls above: every lane of a converged
+// warp calls them with the same arguments and one elected lane issues.  A
+// single thread issuing from inside a lane-divergent branch takes about twice
+// as long per MMA, which matters when the MMAs are small.
+__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit_w(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+      : "memory");
 }
 
 // TMEM -> registers: lane = this thread's row, `N` consecutive 32-bit columns.
@@ -297,6 +350,15 @@ __device__ __forceinline__ float2 exp2_poly2(float x0, float x1) {
   p = __ffma2_rn(p, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
   return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(j.x) << 23)),
                      __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(j.y) << 23)));
+}
+
+// The r-th work item of this CTA of a persistent grid, in a snake order over a
+// heaviest-first item list (even rounds left to right, odd rounds right to
+// left), which evens out the per-CTA totals; -1 when the CTA has no r-th item.
+__device__ __forceinline__ int snake_item(int r, int n_items) {
+  const int G = gridDim.x, c = blockIdx.x;
+  const long long item = static_cast<long long>(r) * G + ((r & 1) ? (G - 1 - c) : c);
+  return item < n_items ? static_cast<int>(item) : -1;
 }
 
 // Three-input maximum (one instruction on sm_100).

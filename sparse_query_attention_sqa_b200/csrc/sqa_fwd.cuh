@@ -82,14 +82,7 @@ struct FwdTraits {
   static_assert(DH % 16 == 0 && DH <= 128, "head dim");
 };
 
-// The r-th work item of this CTA in a snake order over the heaviest-first item
-// list (even rounds left to right, odd rounds right to left), which evens out
-// the per-CTA totals; -1 when the CTA has no r-th item.
-__device__ __forceinline__ int fwd_item(int r, int n_items) {
-  const int G = gridDim.x, c = blockIdx.x;
-  const long long item = static_cast<long long>(r) * G + ((r & 1) ? (G - 1 - c) : c);
-  return item < n_items ? static_cast<int>(item) : -1;
-}
+__device__ __forceinline__ int fwd_item(int r, int n_items) { return dev::snake_item(r, n_items); }
 
 struct FwdItem {
   int b, kvh, qt0, nkv0, nkv1, nkv;
@@ -228,105 +221,104 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
   } else if (warp == Tr::WARP_MMA || warp == Tr::WARP_MMA + 1) {
-    // ------------------------------------------------------------ MMA issuers, one thread per Q tile
-    // A single issuing thread shares its sub-partition with busy softmax warps and
+    // ------------------------------------------------------------ MMA issuers, one warp per Q tile
+    // A single issuing warp shares its sub-partition with busy softmax warps and
     // could not keep two tiles fed; two issuers also let the tiles run apart.
+    // The whole warp runs the loop and one elected lane issues each MMA.
     const int t = warp - Tr::WARP_MMA;
-    if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, NK, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, DH, false, true);
-      // Descriptors of Q buffer 0 / stage 0; other buffers, stages and K-steps add
-      // their byte offset (in 16-byte units) to the start-address field.
-      const uint64_t dq0 = smem_desc(sbase + Tr::OFF_Q + t * Tr::Q_BYTES, 16, 8 * ROWB, Tr::LAYOUT);
-      const uint64_t dk0 = smem_desc(sbase + Tr::OFF_K, 16, 8 * ROWB, Tr::LAYOUT);
-      const uint64_t dv0 = smem_desc(sbase + Tr::OFF_V, NK * ROWB, 8 * ROWB, Tr::LAYOUT);
-      const uint32_t tS0 = tmem + Tr::tm_s(t, 0), tO = tmem + Tr::tm_o(t);
-      auto issue_qk = [&](int qb, int s, int buf) {
-        const uint64_t a0 = dq0 + static_cast<uint64_t>((qb * 2 * Tr::Q_BYTES) >> 4);
-        const uint64_t b0 = dk0 + static_cast<uint64_t>((s * Tr::KV_BYTES) >> 4);
+    constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, NK, false, false);
+    constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, DH, false, true);
+    // Descriptors of Q buffer 0 / stage 0; other buffers, stages and K-steps add
+    // their byte offset (in 16-byte units) to the start-address field.
+    const uint64_t dq0 = smem_desc(sbase + Tr::OFF_Q + t * Tr::Q_BYTES, 16, 8 * ROWB, Tr::LAYOUT);
+    const uint64_t dk0 = smem_desc(sbase + Tr::OFF_K, 16, 8 * ROWB, Tr::LAYOUT);
+    const uint64_t dv0 = smem_desc(sbase + Tr::OFF_V, NK * ROWB, 8 * ROWB, Tr::LAYOUT);
+    const uint32_t tS0 = tmem + Tr::tm_s(t, 0), tO = tmem + Tr::tm_o(t);
+    auto issue_qk = [&](int qb, int s, int buf) {
+      const uint64_t a0 = dq0 + static_cast<uint64_t>((qb * 2 * Tr::Q_BYTES) >> 4);
+      const uint64_t b0 = dk0 + static_cast<uint64_t>((s * Tr::KV_BYTES) >> 4);
 #pragma unroll
-        for (int ks = 0; ks < DH / 16; ++ks) {
-          const uint32_t within = ((ks * 16) % PANEL) * 2, pn = (ks * 16) / PANEL;
-          mma_ss(tS0 + 64u * buf, a0 + ((pn * BM * ROWB + within) >> 4), b0 + ((pn * NK * ROWB + within) >> 4),
+      for (int ks = 0; ks < DH / 16; ++ks) {
+        const uint32_t within = ((ks * 16) % PANEL) * 2, pn = (ks * 16) / PANEL;
+        mma_ss_w(tS0 + 64u * buf, a0 + ((pn * BM * ROWB + within) >> 4), b0 + ((pn * NK * ROWB + within) >> 4),
                  idesc_qk, ks > 0 ? 1u : 0u);
-        }
-        mma_commit(s_full(t, buf));
-      };
-      auto issue_pv = [&](int s, int buf, bool acc) {
-        const uint64_t b0 = dv0 + static_cast<uint64_t>((s * Tr::KV_BYTES) >> 4);
+      }
+      mma_commit_w(s_full(t, buf));
+    };
+    auto issue_pv = [&](int s, int buf, bool acc) {
+      const uint64_t b0 = dv0 + static_cast<uint64_t>((s * Tr::KV_BYTES) >> 4);
 #pragma unroll
-        for (int ks = 0; ks < NK / 16; ++ks)
-          mma_ts(tO, tS0 + 64u * buf + ks * 8, b0 + ((ks * 16 * ROWB) >> 4), idesc_pv, (acc || ks > 0) ? 1u : 0u);
-        mma_commit(o_done(t));
-      };
-      int loaded = 0;  // K/V tiles whose kv_full phase this thread has observed
-      auto ensure_loaded = [&](int gj) {
-        while (loaded <= gj) {
-          if (!mbar_wait(kv_full(loaded % ST), (loaded / ST) & 1, abort_flag, kSiteMma)) return false;
-          ++loaded;
-        }
-        tc_fence_after();
-        return true;
-      };
-      int g = 0;   // first K/V tile (global index) of the current item
-      int G = 0;   // S steps of this Q tile so far (across items)
-      int nd = 0;  // items finished by this Q tile
-      bool ok = true;
-      for (int r = 0, item; ok && (item = fwd_item(r, p.n_items)) >= 0; ++r) {
-        const FwdItem it = fwd_decode(p, item, NK);
-        const int nkv_t = t ? it.nkv1 : it.nkv0;
-        const int qb = r % QB;
-        // Both issuers observe this item's Q load before releasing its buffer, so a
-        // release never lands in the phase of an earlier item.
-        if (!mbar_wait(q_full(qb), (r / QB) & 1, abort_flag, kSiteMma)) {
+      for (int ks = 0; ks < NK / 16; ++ks)
+        mma_ts_w(tO, tS0 + 64u * buf + ks * 8, b0 + ((ks * 16 * ROWB) >> 4), idesc_pv, (acc || ks > 0) ? 1u : 0u);
+      mma_commit_w(o_done(t));
+    };
+    int loaded = 0;  // K/V tiles whose kv_full phase this warp has observed
+    auto ensure_loaded = [&](int gj) {
+      while (loaded <= gj) {
+        if (!mbar_wait_warp(kv_full(loaded % ST), (loaded / ST) & 1, abort_flag, kSiteMma)) return false;
+        ++loaded;
+      }
+      tc_fence_after();
+      return true;
+    };
+    int g = 0;   // first K/V tile (global index) of the current item
+    int G = 0;   // S steps of this Q tile so far (across items)
+    int nd = 0;  // items finished by this Q tile
+    bool ok = true;
+    for (int r = 0, item; ok && (item = fwd_item(r, p.n_items)) >= 0; ++r) {
+      const FwdItem it = fwd_decode(p, item, NK);
+      const int nkv_t = t ? it.nkv1 : it.nkv0;
+      const int qb = r % QB;
+      // Both issuers observe this item's Q load before releasing its buffer, so a
+      // release never lands in the phase of an earlier item.
+      if (!mbar_wait_warp(q_full(qb), (r / QB) & 1, abort_flag, kSiteMma)) {
+        ok = false;
+        break;
+      }
+      for (int j = 0; ok && j < 2 && j < nkv_t; ++j) {  // prologue: S for key tiles 0 and 1
+        ok = ensure_loaded(g + j);
+        if (ok) issue_qk(qb, (g + j) % ST, (G + j) & 1);
+      }
+      for (int j = 0; ok && j < nkv_t; ++j) {
+        const int Gt = G + j;
+        if (!mbar_wait_warp(p_full(t, Gt & 1), (Gt >> 1) & 1, abort_flag, kSiteMma)) {
           ok = false;
           break;
         }
-        for (int j = 0; ok && j < 2 && j < nkv_t; ++j) {  // prologue: S for key tiles 0 and 1
-          ok = ensure_loaded(g + j);
-          if (ok) issue_qk(qb, (g + j) % ST, (G + j) & 1);
+        // O_t still holds the previous item until its epilogue has read it.
+        if (j == 0 && nd > 0 && !mbar_wait_warp(o_free(t), (nd - 1) & 1, abort_flag, kSiteMma)) {
+          ok = false;
+          break;
         }
-        for (int j = 0; ok && j < nkv_t; ++j) {
-          const int Gt = G + j;
-          if (!mbar_wait(p_full(t, Gt & 1), (Gt >> 1) & 1, abort_flag, kSiteMma)) {
+        tc_fence_after();
+        issue_pv((g + j) % ST, Gt & 1, j > 0);
+        if (j + 2 < nkv_t) {
+          // The next S in this buffer: the PV just issued reads P from it first
+          // (MMAs from one issuer execute in order).
+          if (!ensure_loaded(g + j + 2)) {
             ok = false;
             break;
           }
-          // O_t still holds the previous item until its epilogue has read it.
-          if (j == 0 && nd > 0 && !mbar_wait(o_free(t), (nd - 1) & 1, abort_flag, kSiteMma)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_pv((g + j) % ST, Gt & 1, j > 0);
-          if (j + 2 < nkv_t) {
-            // The next S in this buffer: the PV just issued reads P from it first
-            // (MMAs from one thread execute in order).
-            if (!ensure_loaded(g + j + 2)) {
-              ok = false;
-              break;
-            }
-            issue_qk(qb, (g + j + 2) % ST, Gt & 1);
-          }
-          if (j + 1 == nkv_t) mma_commit(o_final(t));
-          mma_commit(kv_empty((g + j) % ST));
+          issue_qk(qb, (g + j + 2) % ST, Gt & 1);
         }
-        // K/V tiles of this item that this Q tile does not need (causal: the other
-        // tile reaches one tile further) are released too, once they are loaded.
-        for (int j = nkv_t; ok && j < it.nkv; ++j) {
-          ok = ensure_loaded(g + j);
-          if (ok) mma_commit(kv_empty((g + j) % ST));
-        }
-        if (!ok) break;
-        mma_commit(q_empty(qb));
-        G += nkv_t;
-        nd += nkv_t > 0 ? 1 : 0;
-        g += it.nkv;
+        if (j + 1 == nkv_t) mma_commit_w(o_final(t));
+        mma_commit_w(kv_empty((g + j) % ST));
       }
-      if (!ok) {  // wait for issued MMAs before TMEM is released
-        mma_commit(drain(t));
-        mbar_wait_drain(drain(t), 0);
+      // K/V tiles of this item that this Q tile does not need (causal: the other
+      // tile reaches one tile further) are released too, once they are loaded.
+      for (int j = nkv_t; ok && j < it.nkv; ++j) {
+        ok = ensure_loaded(g + j);
+        if (ok) mma_commit_w(kv_empty((g + j) % ST));
       }
+      if (!ok) break;
+      mma_commit_w(q_empty(qb));
+      G += nkv_t;
+      nd += nkv_t > 0 ? 1 : 0;
+      g += it.nkv;
+    }
+    if (!ok) {  // wait for issued MMAs before TMEM is released
+      mma_commit_w(drain(t));
+      mbar_wait_drain(drain(t), 0);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax and epilogue
