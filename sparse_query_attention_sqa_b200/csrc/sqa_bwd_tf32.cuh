@@ -70,11 +70,6 @@ __device__ __forceinline__ void mma_ts_tf32_w(uint32_t d_tmem, uint32_t a_tmem, 
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// fp32 bits rounded to the nearest tf32 value (10 mantissa bits; halfway cases
-// away from zero), with integer operations only.
-__device__ __forceinline__ uint32_t round_tf32(float x) {
-  return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u;
-}
 }  // namespace dev
 
 template <int DH>
@@ -120,17 +115,20 @@ struct BwdTf32Traits {
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
-// P^T, tf32-rounded dS^T and bf16 dS for 32 query columns of one key row (the
-// calling thread's TMEM lane).  sr: S^T in [0, 32), dP^T in [32, 64); nl2, nd:
+// P^T, tf32-rounded dS^T and bf16 dS for 16 query columns of one key row (the
+// calling thread's TMEM lane).  sr: S^T in [0, 16), dP^T in [16, 32); nl2, nd:
 // the columns' negated statistics (-lse * log2 e, -D); with MASK, P is zeroed
-// where lim > rtok[column].
+// where lim > rtok[column].  dS is rounded to the nearest tf32 value by
+// Veltkamp splitting (with C = 2^13 + 1, C x - (C x - x) keeps the 11 leading
+// significant bits, rounded to nearest), in packed fp32 pairs.
 template <bool MASK>
-__device__ __forceinline__ void bwd_p_ds(const uint32_t (&sr)[64], const float* nl2, const float* nd,
-                                         const int* rtok, int lim, float2 sl2, uint32_t (&pt)[32],
-                                         uint32_t (&dst)[32], uint32_t (&dsb)[16]) {
+__device__ __forceinline__ void bwd_p_ds16(const uint32_t (&sr)[32], const float* nl2, const float* nd,
+                                           const int* rtok, int lim, float2 sl2, uint32_t (&pt)[16],
+                                           uint32_t (&dst)[16], uint32_t (&dsb)[8]) {
   using namespace dev;
+  const float2 split = make_float2(8193.f, 8193.f), minus1 = make_float2(-1.f, -1.f);
 #pragma unroll
-  for (int e = 0; e < 32; e += 4) {
+  for (int e = 0; e < 16; e += 4) {
     const float4 l4 = *reinterpret_cast<const float4*>(nl2 + e);
     const float4 d4 = *reinterpret_cast<const float4*>(nd + e);
     int4 r4 = make_int4(0, 0, 0, 0);
@@ -145,12 +143,14 @@ __device__ __forceinline__ void bwd_p_ds(const uint32_t (&sr)[64], const float* 
         if (lim > (u == 0 ? r4.x : r4.z)) p0 = 0.f;
         if (lim > (u == 0 ? r4.y : r4.w)) p1 = 0.f;
       }
-      const float2 t = __fadd2_rn(make_float2(__uint_as_float(sr[32 + e + u]), __uint_as_float(sr[32 + e + u + 1])), d);
+      const float2 t = __fadd2_rn(make_float2(__uint_as_float(sr[16 + e + u]), __uint_as_float(sr[16 + e + u + 1])), d);
       const float2 ds = __fmul2_rn(make_float2(p0, p1), t);
+      const float2 cx = __fmul2_rn(ds, split);
+      const float2 hi = __ffma2_rn(__ffma2_rn(ds, minus1, cx), minus1, cx);
       pt[e + u] = __float_as_uint(p0);
       pt[e + u + 1] = __float_as_uint(p1);
-      dst[e + u] = round_tf32(ds.x);
-      dst[e + u + 1] = round_tf32(ds.y);
+      dst[e + u] = __float_as_uint(hi.x);
+      dst[e + u + 1] = __float_as_uint(hi.y);
       dsb[(e + u) >> 1] = pack_bf16x2(ds.x, ds.y);
     }
   }
@@ -451,31 +451,41 @@ __global__ void __launch_bounds__(384, 1)
           if (!ok) break;
           tc_fence_after();
           const float* nl2 = reinterpret_cast<const float*>(smem + Tr::OFF_STAT + s * 1024) + col0;
-          uint32_t sr[64];  // [0,32): S^T, [32,64): dP^T
-          tmem_ld32x2(lane_addr + Tr::tm_st(x) + 32 * w, lane_addr + Tr::tm_dpt(x) + 32 * w, sr);
-          uint32_t pt[32], dst[32], dsb[16];
-          if (masked || ragged)
-            bwd_p_ds<true>(sr, nl2, nl2 + 128, rtok + col0, lim, sl2, pt, dst, dsb);
-          else
-            bwd_p_ds<false>(sr, nl2, nl2 + 128, rtok + col0, lim, sl2, pt, dst, dsb);
-          tmem_st32(lane_addr + Tr::tm_st(x) + 32 * w, pt);
-          tmem_st32(lane_addr + Tr::tm_dpt(x) + 32 * w, dst);
-          // dS (bf16) for the dQ MMA: the dQ of tile G - 2 read this buffer, so
-          // wait for it before the first write of a tile.
-          if (hh == 0 && G >= 2) {
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(dq_full(G & 1), ((G >> 1) - 1) & 1, abort_flag, kSiteSoftmax));
-            if (!ok) break;
-          }
-          // dS[q][key] for q = col0..col0+31 into the MN-major 128B-swizzled tile:
-          // panel q / 64, key row kk (128 bytes), 16-byte chunk (q % 64) / 8.
+          const uint32_t tS = lane_addr + Tr::tm_st(x) + 32 * w, tP = lane_addr + Tr::tm_dpt(x) + 32 * w;
+          // Two chunks of 16 columns: the second one's TMEM load is in flight
+          // while the first one is computed.
+          uint32_t ca[32], cb[32];  // [0,16): S^T, [16,32): dP^T
+          tmem_ld16x2(tS, tP, ca);
+          tmem_ld16x2_nowait(tS + 16, tP + 16, cb);
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            const int q = col0 + 8 * ch;
-            const int panel = q >> 6, chunk = (q & 63) >> 3;
-            *reinterpret_cast<uint4*>(ds_smem + panel * 16384 + kk * 128 + ((chunk ^ (kk & 7)) << 4)) =
-                make_uint4(dsb[4 * ch], dsb[4 * ch + 1], dsb[4 * ch + 2], dsb[4 * ch + 3]);
+          for (int c16 = 0; c16 < 2; ++c16) {
+            if (c16 == 1) tmem_wait_ld32(cb);
+            uint32_t pt[16], dst[16], dsb[8];
+            if (masked || ragged)
+              bwd_p_ds16<true>(c16 ? cb : ca, nl2 + 16 * c16, nl2 + 128 + 16 * c16, rtok + col0 + 16 * c16, lim, sl2,
+                               pt, dst, dsb);
+            else
+              bwd_p_ds16<false>(c16 ? cb : ca, nl2 + 16 * c16, nl2 + 128 + 16 * c16, rtok + col0 + 16 * c16, lim, sl2,
+                                pt, dst, dsb);
+            tmem_st16x2(tS + 16 * c16, tP + 16 * c16, pt, dst);
+            // dS (bf16) for the dQ MMA: the dQ of tile G - 2 read this buffer, so
+            // wait for it before the first write of a tile.
+            if (c16 == 0 && hh == 0 && G >= 2) {
+              ok = __all_sync(0xffffffffu,
+                              mbar_wait(dq_full(G & 1), ((G >> 1) - 1) & 1, abort_flag, kSiteSoftmax));
+              if (!ok) break;
+            }
+            // dS[q][key] for q = col0 + 16 c16 .. + 15 into the MN-major 128B-swizzled
+            // tile: panel q / 64, key row kk (128 bytes), 16-byte chunk (q % 64) / 8.
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+              const int q = col0 + 16 * c16 + 8 * ch;
+              const int panel = q >> 6, chunk = (q & 63) >> 3;
+              *reinterpret_cast<uint4*>(ds_smem + panel * 16384 + kk * 128 + ((chunk ^ (kk & 7)) << 4)) =
+                  make_uint4(dsb[4 * ch], dsb[4 * ch + 1], dsb[4 * ch + 2], dsb[4 * ch + 3]);
+            }
           }
+          if (!ok) break;
           tmem_wait_st();
           fence_async_smem();
           tc_fence_before();
