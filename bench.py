@@ -60,6 +60,23 @@ def counted_flops(w) -> float:
     return fwd * (3.5 if w.backward else 1.0)
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of the ranks' values, returned on every rank (x itself on one rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(w, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the work of every rank's replica over the slowest rank's step time."""
+    return counted_flops(w) * world / (ms_per_step * 1e-3) / 1e12
+
+
 def score_elements(w) -> float:
     """Unmasked (query row, key) pairs over all query heads: one exp2 each."""
     per = w.N * (w.N + 1) / 2 if w.causal else float(w.N) * w.N
@@ -321,16 +338,11 @@ def run_ours(args, w):
         dist.barrier()
     wall = time.perf_counter() - wall0
     clk = clocks.stop()
-    ms_total = t0.elapsed_time(t1)
-    if world > 1:
-        t = torch.tensor([ms_total], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(t0.elapsed_time(t1), world, "cuda")
     dom_ms = statistics.fmean(a.elapsed_time(b) for a, b in zip(starts, stops))
     assert lib.device_status() == 0, "a kernel wait gave up during the timed region"
     ms_step = ms_total / args.steps
-    flops_job = counted_flops(w) * world
-    value = flops_job / (ms_step * 1e-3) / 1e12
+    value = job_tflops(w, world, ms_step)
     peaks, peak_kind = load_peaks()
 
     # End to end through the public API with host buffers: pinned inputs copied
@@ -360,11 +372,8 @@ def run_ours(args, w):
         e2e_step(sets[i % n_sets])
     b.record()
     torch.cuda.synchronize()
-    e2e_ms = a.elapsed_time(b) / e_steps
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / e_steps, world, "cuda")
     if world > 1:
-        t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
         dist.barrier()
 
     line = None
@@ -383,7 +392,7 @@ def run_ours(args, w):
             "tensor_frac_of_bf16_peak": value / peaks["bf16_tflops"],
             "roofline": roofline_for(w, dominant, dom_ms, peaks, peak_kind),
             "kernel_ms": {n: statistics.median(v) for n, v in kern.items()},
-            "e2e": {"value": flops_job / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "e2e": {"value": job_tflops(w, world, e2e_ms), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": args.steps * (4 if w.backward else 1),
             "clocks": clk,

@@ -149,6 +149,21 @@ sqa_status sqa_device_timeout_info(unsigned int info[4], int clear);
  */
 sqa_status sqa_set_timing_events(int kernel, void *start, void *stop);
 
+/*
+ * Self-test hook for the polynomial exponential that sqa_fwd uses for part of
+ * the softmax exponentials at dh <= 32 (3 of every 8 pairs of scores in tiles
+ * without masked keys; the rest use the special-function unit).  It exists so
+ * that tests can compare that function with 2^x; the pages have no
+ * counterpart.  y[i] = the library's 2^x[i] for 0 <= i < n; x and y are device
+ * pointers to fp32 arrays of n elements, 8-byte aligned, owned by the caller.
+ * Method: n = round(x), f = x - n, a degree-3 minimax polynomial in f (largest
+ * relative error 7.5e-5), exponent n added to its bits; x is clamped to -126
+ * first, so results below 2^-126 come out as about 1.2e-38.  Asynchronous on
+ * `stream`; n <= 0 launches nothing.  SQA_ERR_INVALID_ARG for null or
+ * misaligned pointers.
+ */
+sqa_status sqa_selftest_exp2_poly(const float *x, float *y, int n, sqa_stream_t stream);
+
 /* Library version as an integer (major * 10000 + minor * 100 + patch). */
 int sqa_version(void);
 

@@ -150,6 +150,17 @@ sqa_status launch_fwd(const void* q, const void* k, const void* v, void* out, fl
   return record_timing(0, 1, stream);
 }
 
+// y = exp2_poly2(x) elementwise (the forward's polynomial exponential), for tests.
+__global__ void exp2_poly_kernel(const float* x, float* y, int n) {
+  const int pairs = (n + 1) / 2;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < pairs; i += gridDim.x * blockDim.x) {
+    const int j = 2 * i;
+    const float2 r = sqa::dev::exp2_poly2(x[j], j + 1 < n ? x[j + 1] : 0.f);
+    y[j] = r.x;
+    if (j + 1 < n) y[j + 1] = r.y;
+  }
+}
+
 int grid_for(long long work, int threads) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -343,6 +354,18 @@ sqa_status sqa_bwd_static_scratch(const void* dout, const void* q, const void* k
   void* scratch = nullptr;
   if ((st = static_scratch_address(&scratch)) != SQA_OK) return st;
   return sqa_bwd(dout, q, k, v, out, lse, dq, dk, dv, scratch, SQA_STATIC_SCRATCH_BYTES, s, causal, scale, stream);
+}
+
+sqa_status sqa_selftest_exp2_poly(const float* x, float* y, int n, sqa_stream_t stream) {
+  g_last_error.clear();
+  if (n <= 0) return SQA_OK;
+  if (!x || !y) return fail(SQA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(x, 8) || !aligned(y, 8)) return fail(SQA_ERR_INVALID_ARG, "x and y must be 8-byte aligned");
+  const int pairs = (n + 1) / 2;
+  exp2_poly_kernel<<<grid_for(pairs, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "sqa_selftest_exp2_poly launch");
+  return SQA_OK;
 }
 
 const char* sqa_status_string(sqa_status status) {

@@ -105,3 +105,12 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(sqa, "_lib", None)
     with pytest.raises(ImportError):
         sqa.load_library()
+
+
+def test_exp2_selftest_rejects_null_pointers_before_launch(lib):
+    f = lib.sqa_selftest_exp2_poly
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    assert f(None, None, 0, None) == 0  # nothing to do
+    assert f(None, 0x100, 4, None) == 1
+    assert f(0x100, 0x104, 4, None) == 1  # y misaligned
