@@ -151,7 +151,7 @@ sqa_status sqa_set_timing_events(int kernel, void *start, void *stop);
 
 /*
  * Self-test hook for the polynomial exponential that sqa_fwd uses for part of
- * the softmax exponentials at dh <= 32 (3 of every 8 pairs of scores in tiles
+ * the softmax exponentials at dh <= 32 (2 of every 8 pairs of scores in tiles
  * without masked keys; the rest use the special-function unit).  It exists so
  * that tests can compare that function with 2^x; the pages have no
  * counterpart.  y[i] = the library's 2^x[i] for 0 <= i < n; x and y are device

@@ -117,11 +117,10 @@ struct BwdTf32Traits {
 
 // P^T, tf32-rounded dS^T and bf16 dS for 16 query columns of one key row (the
 // calling thread's TMEM lane).  sr: S^T in [0, 16), dP^T in [16, 32); nl2, nd:
-// the columns' negated statistics (-lse * log2 e, -D); with MASK, P is zeroed
-// where lim > rtok[column].  dS is rounded to the nearest tf32 value by
+// the columns' negated statistics (-lse * log2 e, -D); P is zeroed where
+// lim > rtok[column].  dS is rounded to the nearest tf32 value by
 // Veltkamp splitting (with C = 2^13 + 1, C x - (C x - x) keeps the 11 leading
 // significant bits, rounded to nearest), in packed fp32 pairs.
-template <bool MASK>
 __device__ __forceinline__ void bwd_p_ds16(const uint32_t (&sr)[32], const float* nl2, const float* nd,
                                            const int* rtok, int lim, float2 sl2, uint32_t (&pt)[16],
                                            uint32_t (&dst)[16], uint32_t (&dsb)[8]) {
@@ -131,18 +130,15 @@ __device__ __forceinline__ void bwd_p_ds16(const uint32_t (&sr)[32], const float
   for (int e = 0; e < 16; e += 4) {
     const float4 l4 = *reinterpret_cast<const float4*>(nl2 + e);
     const float4 d4 = *reinterpret_cast<const float4*>(nd + e);
-    int4 r4 = make_int4(0, 0, 0, 0);
-    if (MASK) r4 = *reinterpret_cast<const int4*>(rtok + e);
+    const int4 r4 = *reinterpret_cast<const int4*>(rtok + e);
 #pragma unroll
     for (int u = 0; u < 4; u += 2) {
       const float2 l = u == 0 ? make_float2(l4.x, l4.y) : make_float2(l4.z, l4.w);
       const float2 d = u == 0 ? make_float2(d4.x, d4.y) : make_float2(d4.z, d4.w);
       const float2 xx = __ffma2_rn(make_float2(__uint_as_float(sr[e + u]), __uint_as_float(sr[e + u + 1])), sl2, l);
       float p0 = ex2(xx.x), p1 = ex2(xx.y);
-      if (MASK) {
-        if (lim > (u == 0 ? r4.x : r4.z)) p0 = 0.f;
-        if (lim > (u == 0 ? r4.y : r4.w)) p1 = 0.f;
-      }
+      if (lim > (u == 0 ? r4.x : r4.z)) p0 = 0.f;
+      if (lim > (u == 0 ? r4.y : r4.w)) p1 = 0.f;
       const float2 t = __fadd2_rn(make_float2(__uint_as_float(sr[16 + e + u]), __uint_as_float(sr[16 + e + u + 1])), d);
       const float2 ds = __fmul2_rn(make_float2(p0, p1), t);
       const float2 cx = __fmul2_rn(ds, split);
@@ -412,7 +408,6 @@ __global__ void __launch_bounds__(384, 1)
       const BwdItem it = bwd_decode(p, item);
       const int key = it.k0 + kk;
       const bool key_ok = key < p.N;
-      const bool ragged = it.k0 + NK > p.N;  // the last key tile: rows past N hold zeros
       const int qrow_head = it.kvh * p.g + kk % p.g;
 
       // dQ of the item's tile i (global G): TMEM -> fp32 accumulator (this warpgroup: dh/2 columns).
@@ -441,7 +436,12 @@ __global__ void __launch_bounds__(384, 1)
         // row's token on the causal diagonal.
         const int lim = !key_ok ? 0x7fffffff : (masked ? key - qt * p.T : -0x7fffffff);
         uint8_t* ds_smem = smem + Tr::OFF_DS + (G & 1) * Tr::DS_BYTES;
-#pragma unroll 1
+        // dS (bf16) for the dQ MMA goes to this buffer, which the dQ of tile G - 2 read.
+        if (G >= 2) {
+          ok = __all_sync(0xffffffffu, mbar_wait(dq_full(G & 1), ((G >> 1) - 1) & 1, abort_flag, kSiteSoftmax));
+          if (!ok) break;
+        }
+#pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           // Both warpgroups work on half hh of the tile: this one on its 32
           // query columns col0 .. col0 + 31.
@@ -460,21 +460,12 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int c16 = 0; c16 < 2; ++c16) {
             if (c16 == 1) tmem_wait_ld32(cb);
+            // The mask test runs on every tile (lim makes it a no-op off the
+            // diagonal): cheaper than branching between two versions.
             uint32_t pt[16], dst[16], dsb[8];
-            if (masked || ragged)
-              bwd_p_ds16<true>(c16 ? cb : ca, nl2 + 16 * c16, nl2 + 128 + 16 * c16, rtok + col0 + 16 * c16, lim, sl2,
-                               pt, dst, dsb);
-            else
-              bwd_p_ds16<false>(c16 ? cb : ca, nl2 + 16 * c16, nl2 + 128 + 16 * c16, rtok + col0 + 16 * c16, lim, sl2,
-                                pt, dst, dsb);
+            bwd_p_ds16(c16 ? cb : ca, nl2 + 16 * c16, nl2 + 128 + 16 * c16, rtok + col0 + 16 * c16, lim, sl2, pt,
+                             dst, dsb);
             tmem_st16x2(tS + 16 * c16, tP + 16 * c16, pt, dst);
-            // dS (bf16) for the dQ MMA: the dQ of tile G - 2 read this buffer, so
-            // wait for it before the first write of a tile.
-            if (c16 == 0 && hh == 0 && G >= 2) {
-              ok = __all_sync(0xffffffffu,
-                              mbar_wait(dq_full(G & 1), ((G >> 1) - 1) & 1, abort_flag, kSiteSoftmax));
-              if (!ok) break;
-            }
             // dS[q][key] for q = col0 + 16 c16 .. + 15 into the MN-major 128B-swizzled
             // tile: panel q / 64, key row kk (128 bytes), 16-byte chunk (q % 64) / 8.
 #pragma unroll

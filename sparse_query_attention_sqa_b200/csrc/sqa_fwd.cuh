@@ -107,7 +107,7 @@ __device__ __forceinline__ FwdItem fwd_decode(const FwdParams& p, int item, int 
 
 // POLY: of every 8 pairs of scores in an unmasked tile, how many take the
 // polynomial exponential (exp2_poly2) instead of the special-function unit.
-template <int DH, int POLY = (DH <= 32 ? 3 : 0)>
+template <int DH, int POLY = (DH <= 32 ? 2 : 0)>
 __global__ void __launch_bounds__(384, 1)
     sqa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
