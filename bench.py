@@ -164,7 +164,12 @@ def cpu_baseline(w, seconds):
 class ClockSampler:
     def __init__(self, enabled, index):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        # Raw samples go to SQA_BENCH_CLOCKS_DIR (a temporary directory by default);
+        # the JSON line carries their summary.
+        import tempfile
+
+        out_dir = os.environ.get("SQA_BENCH_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"clocks_bench_{os.getpid()}.csv")
         if not enabled:
             return
         try:
