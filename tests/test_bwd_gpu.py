@@ -22,6 +22,10 @@ SHAPES = [
     (1, 390, 8, 4, 64),
     (2, 300, 8, 4, 128),
     (1, 129, 4, 4, 128),
+    # more work items than SMs, so every persistent CTA walks several items
+    # (buffer and barrier phases carried across items), with ragged tails
+    (6, 1000, 8, 4, 16),
+    (26, 300, 8, 2, 32),
 ]
 
 
