@@ -56,7 +56,9 @@ def _load():
         bbase = [dp, dp, dp, dp, i64, i64, i64, i64, i64, ctypes.c_int, ctypes.c_double]
         lib.sqa_oracle_bwd.argtypes = bbase + [dp, dp, dp]
         lib.sqa_oracle_bwd_rows.argtypes = bbase + [ip, i64, dp, ip, i64, dp, dp]
-        for f in (lib.sqa_oracle_fwd, lib.sqa_oracle_fwd_rows, lib.sqa_oracle_bwd, lib.sqa_oracle_bwd_rows):
+        lib.sqa_oracle_decode.argtypes = [dp, dp, dp, ip, i64, i64, i64, i64, i64, ctypes.c_double, dp, dp]
+        for f in (lib.sqa_oracle_fwd, lib.sqa_oracle_fwd_rows, lib.sqa_oracle_bwd, lib.sqa_oracle_bwd_rows,
+                  lib.sqa_oracle_decode):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -140,3 +142,20 @@ def sqa_bwd_rows(q, k, v, dout, qrows, krows, causal: bool, scale: float | None 
                                        qrows.shape[0], _ptr(dq), _ptr(krows, ctypes.c_int64),
                                        krows.shape[0], _ptr(dk), _ptr(dv)))
     return dq, dk, dv
+
+
+def sqa_decode(q, k, v, lens=None, scale: float | None = None):
+    """Decoding step: q [B,Hq,dh] (one token per sequence) against the first
+    lens[b] entries of the cache k/v [B,N,Hkv,dh] (all N when lens is None).
+    Returns (out [B,Hq,dh], lse [B,Hq]) in fp64."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, dh = q.shape
+    Bk, N, Hkv, dhk = k.shape
+    if (Bk, dhk) != (B, dh) or v.shape != k.shape:
+        raise ValueError("q and k/v shapes disagree")
+    lens = np.full(B, N, dtype=np.int64) if lens is None else np.ascontiguousarray(lens, dtype=np.int64)
+    out = np.zeros((B, Hq, dh))
+    lse = np.zeros((B, Hq))
+    _check(_load().sqa_oracle_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(lens, ctypes.c_int64), B, N, Hq, Hkv, dh,
+                                     _scale(scale, dh), _ptr(out), _ptr(lse)))
+    return out, lse

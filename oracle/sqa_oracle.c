@@ -312,3 +312,50 @@ int sqa_oracle_bwd_rows(const double *q, const double *k, const double *v, const
     free(need);
     return 0;
 }
+
+/* Decoding step (one new token per sequence attending to its key/value cache;
+ * the step where SQA's query-head reduction saves nothing, since the cost is
+ * reading the cache: arXiv 2510.01817 abstract).  For every batch entry b and
+ * query head h, the single query q[b][h] attends to the first lens[b] entries
+ * of the cache with no further mask:
+ *   s_j   = scale * sum_d q[b,h,d] K[b,j,kv(h),d],   j < lens[b]
+ *   lse   = m + ln sum_j exp(s_j - m),  m = max_j s_j
+ *   out   = sum_j exp(s_j - lse) V[b,j,kv(h),:]
+ * Layouts: q, out [B][H_q][dh]; k, v [B][N][H_kv][dh] (N = cache capacity);
+ * lse [B][H_q].  lens[b] must lie in [1, N]. */
+int sqa_oracle_decode(const double *q, const double *k, const double *v, const int64_t *lens, int64_t B,
+                      int64_t N, int64_t Hq, int64_t Hkv, int64_t dh, double scale, double *out,
+                      double *lse) {
+    problem p = {q, k, v, NULL, B, N, Hq, Hkv, dh, 0, scale};
+    int rc = check(&p);
+    if (rc) return rc;
+    for (int64_t b = 0; b < B; ++b)
+        if (lens[b] < 1 || lens[b] > N) return 4;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * N);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < B * Hq; ++r) {
+            const int64_t b = r / Hq, h = r % Hq, kvh = kv_head(&p, h), len = lens[b];
+            const double *qh = q + (b * Hq + h) * dh;
+            double m = -INFINITY;
+            for (int64_t j = 0; j < len; ++j) {
+                s[j] = scale * dot(qh, k_row(&p, b, j, kvh), dh);
+                if (s[j] > m) m = s[j];
+            }
+            double sum = 0.0;
+            for (int64_t j = 0; j < len; ++j) sum += exp(s[j] - m);
+            const double l = m + log(sum);
+            lse[r] = l;
+            double *o = out + r * dh;
+            for (int64_t d = 0; d < dh; ++d) o[d] = 0.0;
+            for (int64_t j = 0; j < len; ++j) {
+                const double pj = exp(s[j] - l);
+                const double *vj = v_row(&p, b, j, kvh);
+                for (int64_t d = 0; d < dh; ++d) o[d] += pj * vj[d];
+            }
+        }
+        free(s);
+    }
+    return 0;
+}
