@@ -54,6 +54,8 @@ def parse():
 
 
 def counted_flops(w) -> float:
+    if w.decode:  # one query row per (sequence, head) against N cached positions
+        return 4.0 * w.B * w.Hq * w.N * w.dh
     fwd = 4.0 * w.B * w.Hq * w.N * w.N * w.dh
     if w.causal:
         fwd /= 2
@@ -79,6 +81,8 @@ def job_tflops(w, world: int, ms_per_step: float) -> float:
 
 def score_elements(w) -> float:
     """Unmasked (query row, key) pairs over all query heads: one exp2 each."""
+    if w.decode:
+        return float(w.B) * w.Hq * w.N
     per = w.N * (w.N + 1) / 2 if w.causal else float(w.N) * w.N
     return w.B * w.Hq * per
 
@@ -95,12 +99,17 @@ def load_peaks():
 def oracle_subproblem(w, seed=0):
     """One independent slice of the workload: batch entry 0, KV head 0 and its
     g query heads (the oracle's work on it scales with the counted FLOPs)."""
-    from sparse_query_attention_sqa_b200.inputs import make_inputs
+    from sparse_query_attention_sqa_b200.inputs import make_decode_inputs, make_inputs
 
     g = w.Hq // w.Hkv
-    q, k, v, dout = make_inputs(1, w.N, g, 1, w.dh, seed=seed, std=w.std, k_scale=w.k_scale, with_dout=w.backward)
+    if w.decode:
+        q, k, v = make_decode_inputs(1, w.N, g, 1, w.dh, seed=seed, std=w.std, k_scale=w.k_scale)
+        dout = None
+    else:
+        q, k, v, dout = make_inputs(1, w.N, g, 1, w.dh, seed=seed, std=w.std, k_scale=w.k_scale,
+                                    with_dout=w.backward)
     sub = type(w)(name=w.name + "_slice", B=1, N=w.N, Hq=g, Hkv=1, dh=w.dh, causal=w.causal, backward=w.backward,
-                  std=w.std, k_scale=w.k_scale, scale=w.scale)
+                  std=w.std, k_scale=w.k_scale, scale=w.scale, decode=w.decode)
     return sub, (q, k, v, dout)
 
 
@@ -108,6 +117,9 @@ def run_oracle_step(sub, data):
     import oracle
 
     q, k, v, dout = data
+    if sub.decode:
+        oracle.sqa_decode(q, k, v, None, sub.softmax_scale)
+        return
     oracle.sqa_fwd(q, k, v, sub.causal, sub.softmax_scale)
     if sub.backward:
         oracle.sqa_bwd(q, k, v, dout, sub.causal, sub.softmax_scale)
@@ -142,7 +154,7 @@ def cpu_baseline_rows(w, seconds):
 
 def cpu_baseline(w, seconds):
     g = w.Hq // w.Hkv
-    if g * w.N * w.N * w.dh > 2 ** 34:  # one slice would take minutes
+    if not w.decode and g * w.N * w.N * w.dh > 2 ** 34:  # one slice would take minutes
         return cpu_baseline_rows(w, seconds)
     sub, data = oracle_subproblem(w)
     run_oracle_step(sub, data)  # builds the oracle and warms caches
@@ -214,6 +226,11 @@ def alloc_set(w, q, k, v, dout, lib, torch):
     dev = "cuda"
     s = {"q": q.to(dev), "k": k.to(dev), "v": v.to(dev)}
     s["out"] = torch.empty_like(s["q"])
+    if w.decode:
+        s["lse"] = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+        s["ws"] = torch.empty(lib.decode_workspace_bytes(w.B, w.N, w.Hq, w.Hkv, w.dh), dtype=torch.uint8,
+                              device=dev)
+        return s
     s["lse"] = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
     if w.backward:
         s["dout"] = dout.to(dev)
@@ -229,13 +246,32 @@ def set_bytes(s) -> int:
 
 
 def step(lib, w, s):
+    if w.decode:
+        lib.sqa_decode(s["q"], s["k"], s["v"], out=s["out"], lse=s["lse"], workspace=s["ws"], scale=w.scale)
+        return
     lib.sqa_fwd(s["q"], s["k"], s["v"], out=s["out"], lse=s["lse"], causal=w.causal, scale=w.scale)
     if w.backward:
         lib.sqa_bwd(s["dout"], s["q"], s["k"], s["v"], s["out"], s["lse"], dq=s["dq"], dk=s["dk"], dv=s["dv"],
                     workspace=s["ws"], causal=w.causal, scale=w.scale)
 
 
+def pass_name(w) -> str:
+    return "decode" if w.decode else ("fwd+bwd" if w.backward else "fwd")
+
+
+def decode_bytes(w) -> float:
+    """Algorithmic bytes of one decoding step: the whole K and V caches once,
+    the new queries, the outputs and their lse."""
+    return 2.0 * w.B * w.N * w.Hkv * w.dh * 2 + 2.0 * w.B * w.Hq * w.dh * 2 + 4.0 * w.B * w.Hq
+
+
 def roofline_for(w, kernel_name, ms, peaks, peak_kind):
+    if w.decode:
+        # HBM-bound: stream the caches once
+        achieved = decode_bytes(w) / (ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": traffic_for(kernel_name, w), "kernel": kernel_name, "peak_source": f"{peak_kind} hbm_gbs"}
     if w.dh <= 32:
         # exp-bound: one exp2 per unmasked score element on the special-function unit
         units = score_elements(w)
@@ -306,21 +342,23 @@ def run_ours(args, w):
     # Which kernel dominates: time both main kernels once per set during warm-up.
     ev = lambda: torch.cuda.Event(enable_timing=True)
     kern = {}
+    hooks = (2,) if w.decode else (0, 1)  # library timing-hook indices: fwd, bwd, decode
+    names = {0: "sqa_fwd_kernel", 1: "sqa_bwd_kernel", 2: "sqa_decode_split_kernel"}
     for i in range(max(args.warmup, 3)):
         s = sets[i % n_sets]
-        e0, e1, e2, e3 = ev(), ev(), ev(), ev()
-        lib.set_timing_events(0, e0, e1)
-        lib.set_timing_events(1, e2, e3)
+        evs = {h: (ev(), ev()) for h in hooks}
+        for h, (e0, e1) in evs.items():
+            lib.set_timing_events(h, e0, e1)
         step(lib, w, s)
-        lib.set_timing_events(0)
-        lib.set_timing_events(1)
+        for h in hooks:
+            lib.set_timing_events(h)
         torch.cuda.synchronize()
-        kern.setdefault("sqa_fwd_kernel", []).append(e0.elapsed_time(e1))
-        if w.backward:
-            kern.setdefault("sqa_bwd_kernel", []).append(e2.elapsed_time(e3))
+        for h, (e0, e1) in evs.items():
+            if h != 1 or w.backward:
+                kern.setdefault(names[h], []).append(e0.elapsed_time(e1))
     assert lib.device_status() == 0, "a kernel wait gave up during warm-up"
     dominant = max(kern, key=lambda n: statistics.median(kern[n]))
-    dom_idx = 0 if dominant == "sqa_fwd_kernel" else 1
+    dom_idx = next(h for h, n in names.items() if n == dominant)
 
     # Timed region: K steps, per-step events around the dominant kernel.
     starts = [ev() for _ in range(args.steps)]
@@ -358,7 +396,10 @@ def run_ours(args, w):
     # directions at once) -- the way a caller pipelines a stream of batches.
     n_pipe = min(3, n_sets)
     streams = [torch.cuda.Stream() for _ in range(n_pipe)]
-    host_in = {n: sets[0][n].cpu().pin_memory() for n in ("q", "k", "v", "dout") if n in sets[0]}
+    # (A decoding step's input is the new token's queries; its key/value cache
+    # stays resident on the device, as in serving.)
+    in_names = ("q",) if w.decode else ("q", "k", "v", "dout")
+    host_in = {n: sets[0][n].cpu().pin_memory() for n in in_names if n in sets[0]}
     outs = ("out", "lse", "dq", "dk", "dv") if w.backward else ("out", "lse")
     host_out = [{n: torch.empty(sets[0][n].shape, dtype=sets[0][n].dtype, pin_memory=True) for n in outs}
                 for _ in range(n_pipe)]
@@ -398,23 +439,23 @@ def run_ours(args, w):
     line = None
     if rank == 0:
         line = {
-            "metric": f"SQA attention {'fwd+bwd' if w.backward else 'fwd'} TFLOP/s ({w.note})",
+            "metric": f"SQA attention {pass_name(w)} TFLOP/s ({w.note})",
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic (seeded Gaussian bf16 inputs)",
             "config": {"workload": w.name, "B": w.B, "N": w.N, "H_q": w.Hq, "H_kv": w.Hkv, "dh": w.dh,
-                       "causal": w.causal, "pass": "fwd+bwd" if w.backward else "fwd",
+                       "causal": w.causal, "pass": pass_name(w),
                        "parallelism": f"{world} independent replicas" if world > 1 else "single GPU",
                        "l2": f"{n_sets} rotating buffer sets of {set_bytes(first) / 2**20:.0f} MiB "
                              f"(> L2 in total), no flush"},
-            "tokens_per_s": w.B * w.N * world / (ms_step * 1e-3),
+            "tokens_per_s": (w.B if w.decode else w.B * w.N) * world / (ms_step * 1e-3),
             "tensor_frac_of_bf16_peak": value / peaks["bf16_tflops"],
             "roofline": roofline_for(w, dominant, dom_ms, peaks, peak_kind),
             "kernel_ms": {n: statistics.median(v) for n, v in kern.items()},
             "e2e": {"value": job_tflops(w, world, e2e_ms), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "streams": n_pipe,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": args.steps * (4 if w.backward else 1),
+            "gpu_launches": args.steps * (4 if w.backward else (2 if w.decode else 1)),
             "clocks": clk,
             "wall_s_timed_region": wall,
         }
@@ -432,14 +473,14 @@ def run_reference(args, w):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return None
-    if (w.Hq // w.Hkv) * w.N * w.N * w.dh > 2 ** 34:  # one slice would take minutes: sample rows
+    if not w.decode and (w.Hq // w.Hkv) * w.N * w.N * w.dh > 2 ** 34:  # one slice would take minutes: sample rows
         cb = cpu_baseline_rows(w, 60.0)
-        return {"impl": "reference", "metric": f"SQA attention {'fwd+bwd' if w.backward else 'fwd'} TFLOP/s ({w.note})",
+        return {"impl": "reference", "metric": f"SQA attention {pass_name(w)} TFLOP/s ({w.note})",
                 "value": cb["value"], "unit": "TFLOP/s", "n_gpus": world, "steps": 1, "warmup": 0,
                 "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f64", "data": "synthetic",
                 "config": {"workload": w.name, "B": w.B, "N": w.N, "H_q": w.Hq, "H_kv": w.Hkv, "dh": w.dh,
-                           "causal": w.causal, "pass": "fwd+bwd" if w.backward else "fwd"},
+                           "causal": w.causal, "pass": pass_name(w)},
                 "cpu_baseline": cb, "e2e": {"value": cb["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                                             "d2h_bytes_per_step": 0}}
     sub, data = oracle_subproblem(w)
@@ -462,11 +503,11 @@ def run_reference(args, w):
     value = counted_flops(sub) / (ms * 1e-3) / 1e12
     sample = (f"fp64 oracle fwd{'+bwd' if w.backward else ''} on batch entry 0, KV head 0 and its {sub.Hq} "
               f"query heads (N={w.N}, dh={w.dh}); {steps} of the requested {args.steps} steps run")
-    return {"impl": "reference", "metric": f"SQA attention {'fwd+bwd' if w.backward else 'fwd'} TFLOP/s ({w.note})",
+    return {"impl": "reference", "metric": f"SQA attention {pass_name(w)} TFLOP/s ({w.note})",
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "N": w.N, "H_q": w.Hq, "H_kv": w.Hkv, "dh": w.dh,
-                       "causal": w.causal, "pass": "fwd+bwd" if w.backward else "fwd"},
+                       "causal": w.causal, "pass": pass_name(w)},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": omp_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

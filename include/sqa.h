@@ -140,14 +140,48 @@ sqa_status sqa_device_timeout_info(unsigned int info[4], int clear);
 
 /*
  * Optional timing hook for benchmarks.  While set on the calling host thread,
- * sqa_fwd (kernel = 0) or sqa_bwd (kernel = 1) records `start` on its stream
- * just before launching its main attention kernel and `stop` just after it, so
+ * sqa_fwd (kernel = 0), sqa_bwd (kernel = 1) or sqa_decode (kernel = 2, its
+ * split kernel) records `start` on its stream just before launching its main
+ * attention kernel and `stop` just after it, so
  * the caller can time that one kernel with cudaEventElapsedTime.  start and
  * stop are cudaEvent_t handles owned by the caller; pass NULL for both to turn
  * the hook off.  Returns SQA_ERR_INVALID_ARG for another kernel index or when
  * only one of the two events is given.
  */
 sqa_status sqa_set_timing_events(int kernel, void *start, void *stop);
+
+/*
+ * Bytes of device scratch that sqa_decode needs for shape s, 0 if s is
+ * invalid.  The caller allocates it; 256-byte aligned.
+ */
+size_t sqa_decode_workspace_bytes(sqa_shape s);
+
+/*
+ * Decoding step: one new
+ * query token per sequence attends to the first seq_lens[b] entries of its
+ * key/value cache, with no further mask (arXiv 2510.01817 abstract: SQA
+ * reduces query heads, so this memory-bound step costs what GQA's does; GQA
+ * summary, "The idea": the K/V head count sets the cache size).
+ *
+ *   s_j   = scale * <q[b,h,:], K[b,j,kv(h),:]>,  j < seq_lens[b]
+ *   lse   = ln sum_j exp(s_j),  out[b,h,:] = sum_j exp(s_j - lse) V[b,j,kv(h),:]
+ *
+ * Shapes (s.N is the cache capacity):
+ *   q, out           : bf16 [B][H_q][dh]
+ *   k_cache, v_cache : bf16 [B][N][H_kv][dh], 16-byte aligned
+ *   seq_lens         : int32 [B] on the device, or NULL for all N; values are
+ *                      clamped to [0, N]; a length of 0 gives out = 0 and
+ *                      lse = -inf
+ *   lse              : fp32 [B][H_q]
+ *   workspace        : sqa_decode_workspace_bytes(s) bytes, 256-byte aligned,
+ *                      contents ignored and overwritten
+ * Supported: dh in {16, 32, 64, 128}, H_q / H_kv <= 128, B * H_kv <= 65535.
+ * Two kernels on `stream`, asynchronous, nothing allocated; out and lse are
+ * fully overwritten.  Errors as for sqa_fwd, returned before any launch.
+ */
+sqa_status sqa_decode(const void *q, const void *k_cache, const void *v_cache, const int *seq_lens,
+                      void *out, float *lse, void *workspace, size_t workspace_bytes, sqa_shape s,
+                      float scale, sqa_stream_t stream);
 
 /*
  * Self-test hook for the polynomial exponential that sqa_fwd uses for part of

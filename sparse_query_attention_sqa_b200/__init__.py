@@ -12,7 +12,8 @@ import ctypes
 import os
 
 __all__ = [
-    "SqaError", "load_library", "library_path", "sqa_fwd", "sqa_bwd", "bwd_workspace_bytes",
+    "SqaError", "load_library", "library_path", "sqa_fwd", "sqa_bwd", "bwd_workspace_bytes", "sqa_decode",
+    "decode_workspace_bytes",
     "device_status", "timeout_info", "set_timing_events", "Shape",
 ]
 
@@ -53,6 +54,10 @@ def load_library():
     lib.sqa_bwd_workspace_bytes.restype = sz
     lib.sqa_bwd.argtypes = [vp, vp, vp, vp, vp, fp, vp, vp, vp, vp, sz, Shape, c_int, c_float, vp]
     lib.sqa_bwd.restype = c_int
+    lib.sqa_decode_workspace_bytes.argtypes = [Shape]
+    lib.sqa_decode_workspace_bytes.restype = sz
+    lib.sqa_decode.argtypes = [vp, vp, vp, vp, vp, fp, vp, sz, Shape, c_float, vp]
+    lib.sqa_decode.restype = c_int
     lib.sqa_status_string.argtypes = [c_int]
     lib.sqa_status_string.restype = ctypes.c_char_p
     lib.sqa_last_error.argtypes = []
@@ -124,6 +129,44 @@ def sqa_fwd(q, k, v, out=None, lse=None, causal: bool = False, scale: float = 0.
     _need(lse, "lse", (s.B, s.H_q, s.N), torch.float32)
     _check(lib.sqa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), s,
                        int(bool(causal)), float(scale), _stream(stream)))
+    return out, lse
+
+
+def decode_workspace_bytes(B: int, N: int, H_q: int, H_kv: int, dh: int) -> int:
+    return int(load_library().sqa_decode_workspace_bytes(Shape(B, N, H_q, H_kv, dh)))
+
+
+def sqa_decode(q, k_cache, v_cache, seq_lens=None, out=None, lse=None, workspace=None, scale: float = 0.0,
+               stream=None):
+    """Decoding step.  q [B,H_q,dh] bf16 (one token per sequence), k_cache/v_cache
+    [B,N,H_kv,dh] bf16, seq_lens int32 [B] on the device (None: all N).
+    Returns (out [B,H_q,dh] bf16, lse [B,H_q] fp32)."""
+    import torch
+
+    lib = load_library()
+    if q.dim() != 3 or k_cache.dim() != 4:
+        raise ValueError("q must be [B, H_q, dh] and the caches [B, N, H_kv, dh]")
+    B, Hq, dh = q.shape
+    N, Hkv = k_cache.shape[1], k_cache.shape[2]
+    s = Shape(B, N, Hq, Hkv, dh)
+    _need(q, "q", (B, Hq, dh), torch.bfloat16)
+    _need(k_cache, "k_cache", (B, N, Hkv, dh), torch.bfloat16)
+    _need(v_cache, "v_cache", (B, N, Hkv, dh), torch.bfloat16)
+    if seq_lens is not None:
+        _need(seq_lens, "seq_lens", (B,), torch.int32)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _need(out, "out", (B, Hq, dh), torch.bfloat16)
+    _need(lse, "lse", (B, Hq), torch.float32)
+    need = int(lib.sqa_decode_workspace_bytes(s))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _check(lib.sqa_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                          0 if seq_lens is None else seq_lens.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                          workspace.data_ptr(), workspace.numel() * workspace.element_size(), s, float(scale),
+                          _stream(stream)))
     return out, lse
 
 

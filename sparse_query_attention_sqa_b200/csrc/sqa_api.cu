@@ -12,12 +12,13 @@
 #include "sqa.h"
 #include "sqa_bwd.cuh"
 #include "sqa_bwd_tf32.cuh"
+#include "sqa_decode.cuh"
 #include "sqa_fwd.cuh"
 
 namespace {
 
 thread_local std::string g_last_error;
-thread_local cudaEvent_t g_timing[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+thread_local cudaEvent_t g_timing[3][2] = {{nullptr, nullptr}, {nullptr, nullptr}, {nullptr, nullptr}};
 
 sqa_status record_timing(int kernel, int which, cudaStream_t stream);
 
@@ -148,6 +149,45 @@ sqa_status launch_fwd(const void* q, const void* k, const void* v, void* out, fl
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "sqa_fwd launch");
   return record_timing(0, 1, stream);
+}
+
+size_t decode_workspace(const sqa_shape& s) {
+  const int ch = sqa::decode_chunk(s.dh);
+  const size_t n_split = (static_cast<size_t>(s.N) + ch - 1) / ch;
+  const size_t g = static_cast<size_t>(s.H_q / s.H_kv);
+  return sqa::align256(static_cast<size_t>(s.B) * s.H_kv * n_split * g * (s.dh + 2) * sizeof(float));
+}
+
+template <int DH>
+sqa_status launch_decode(const void* q, const void* k, const void* v, const int* lens, void* out, float* lse,
+                         void* workspace, const sqa_shape& s, float scale, cudaStream_t stream) {
+  sqa::DecodeParams p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.lens = lens;
+  p.part = static_cast<float*>(workspace);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.N = s.N;
+  p.Hq = s.H_q;
+  p.Hkv = s.H_kv;
+  p.g = s.H_q / s.H_kv;
+  p.n_split = (s.N + sqa::decode_chunk(DH) - 1) / sqa::decode_chunk(DH);
+  p.scale_log2 = scale * kLog2e;
+  const int smem = static_cast<int>(sqa::decode_smem_bytes(p.g, DH));
+  sqa_status st;
+  if ((st = set_smem(sqa::sqa_decode_split_kernel<DH>, smem)) != SQA_OK) return st;
+  const dim3 grid(static_cast<unsigned>(p.n_split * s.H_kv), static_cast<unsigned>(s.B));
+  if ((st = record_timing(2, 0, stream)) != SQA_OK) return st;
+  sqa::sqa_decode_split_kernel<DH><<<grid, sqa::kDecodeThreads, smem, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "sqa_decode split launch");
+  if ((st = record_timing(2, 1, stream)) != SQA_OK) return st;
+  sqa::sqa_decode_combine_kernel<DH><<<static_cast<unsigned>(s.B * s.H_q), sqa::kDecodeThreads, 0, stream>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "sqa_decode combine launch");
+  return SQA_OK;
 }
 
 // y = exp2_poly2(x) elementwise (the forward's polynomial exponential), for tests.
@@ -341,6 +381,39 @@ sqa_status sqa_bwd(const void* dout, const void* q, const void* k, const void* v
   }
 }
 
+size_t sqa_decode_workspace_bytes(sqa_shape s) {
+  if (check_shape(s) != SQA_OK || s.B * static_cast<long long>(s.H_kv) > 65535) return 0;
+  return decode_workspace(s);
+}
+
+sqa_status sqa_decode(const void* q, const void* k_cache, const void* v_cache, const int* seq_lens, void* out,
+                      float* lse, void* workspace, size_t workspace_bytes, sqa_shape s, float scale,
+                      sqa_stream_t stream) {
+  g_last_error.clear();
+  if (!q || !k_cache || !v_cache || !out || !lse || !workspace) return fail(SQA_ERR_INVALID_ARG, "null pointer argument");
+  sqa_status st = check_shape(s);
+  if (st != SQA_OK) return st;
+  if (s.B * static_cast<long long>(s.H_kv) > 65535) return fail(SQA_ERR_UNSUPPORTED, "B * H_kv must be at most 65535");
+  if (!aligned(q, 2) || !aligned(out, 2)) return fail(SQA_ERR_UNSUPPORTED, "q and out must be 2-byte aligned");
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16))
+    return fail(SQA_ERR_UNSUPPORTED, "the key/value caches must be 16-byte aligned");
+  if (!aligned(lse, 4) || (seq_lens && !aligned(seq_lens, 4)))
+    return fail(SQA_ERR_UNSUPPORTED, "lse and seq_lens must be 4-byte aligned");
+  if (!aligned(workspace, 256)) return fail(SQA_ERR_UNSUPPORTED, "workspace must be 256-byte aligned");
+  const size_t need = decode_workspace(s);
+  if (workspace_bytes < need)
+    return fail(SQA_ERR_INVALID_ARG, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
+  float sc;
+  if ((st = resolve_scale(scale, s.dh, &sc)) != SQA_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  switch (s.dh) {
+    case 16: return launch_decode<16>(q, k_cache, v_cache, seq_lens, out, lse, workspace, s, sc, cs);
+    case 32: return launch_decode<32>(q, k_cache, v_cache, seq_lens, out, lse, workspace, s, sc, cs);
+    case 64: return launch_decode<64>(q, k_cache, v_cache, seq_lens, out, lse, workspace, s, sc, cs);
+    default: return launch_decode<128>(q, k_cache, v_cache, seq_lens, out, lse, workspace, s, sc, cs);
+  }
+}
+
 sqa_status sqa_bwd_static_scratch(const void* dout, const void* q, const void* k, const void* v, const void* out,
                                   const float* lse, void* dq, void* dk, void* dv, sqa_shape s, int causal,
                                   float scale, sqa_stream_t stream) {
@@ -415,7 +488,8 @@ sqa_status sqa_device_timeout_info(unsigned int info[4], int clear) {
 
 sqa_status sqa_set_timing_events(int kernel, void* start, void* stop) {
   g_last_error.clear();
-  if (kernel < 0 || kernel > 1) return fail(SQA_ERR_INVALID_ARG, "kernel index %d is not 0 (fwd) or 1 (bwd)", kernel);
+  if (kernel < 0 || kernel > 2)
+    return fail(SQA_ERR_INVALID_ARG, "kernel index %d is not 0 (fwd), 1 (bwd) or 2 (decode)", kernel);
   if ((start == nullptr) != (stop == nullptr)) return fail(SQA_ERR_INVALID_ARG, "give both events or neither");
   g_timing[kernel][0] = static_cast<cudaEvent_t>(start);
   g_timing[kernel][1] = static_cast<cudaEvent_t>(stop);

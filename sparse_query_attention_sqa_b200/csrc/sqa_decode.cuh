@@ -1,0 +1,234 @@
+// sqa_decode.cuh -- Sparse Query Attention decoding step on sm_100a: one new
+// query token per sequence attends to the first lens[b] entries of its
+// key/value cache.
+//
+// The cost of this step is reading the cache (H_kv heads of K and V per
+// position), not the scores: reducing the query heads saves nothing here
+// (arXiv 2510.01817 abstract: the gains are in compute-bound settings; the
+// GQA summary, "The idea": the K/V head count sets the cache size).  So the
+// kernels are built to stream the cache from HBM once at full width, on the
+// CUDA cores: with g query heads per K/V head there are only 2 g dh
+// multiply-adds per cached position, far below what tensor cores are for.
+//
+// Two launches, split-K over the cache:
+//   1. split:   one CTA per (chunk of 256 positions (128 at dh >= 64), K/V head,
+//               batch entry), the K/V heads of one chunk adjacent in launch order
+//               so the cache rows they share are read from DRAM once.  It
+//               copies the chunk's K and V rows (bf16, 16-byte loads) and the
+//               group's g queries into shared memory, forms the g x chunk scores
+//               (log2 units), takes each head's chunk maximum m and
+//               l = sum 2^(s - m) with warp shuffles, and writes the unnormalised
+//               o = sum 2^(s - m) V with m and l to the workspace.
+//   2. combine: one CTA per (batch entry, query head) merges the chunks, its
+//               threads spread over (column, chunk) pairs:
+//               M = max m, L = sum l 2^(m - M), out = sum o 2^(m - M) / L (bf16),
+//               lse = ln 2 * (M + log2 L).
+#pragma once
+
+#include "sqa_device.cuh"
+
+namespace sqa {
+
+constexpr int kDecodeThreads = 256;
+// Cache positions per split: 256, or 128 at dh >= 64 so that the chunk, its
+// scores for a group of up to 128 heads and the queries fit in shared memory.
+__host__ __device__ constexpr int decode_chunk(int dh) { return dh <= 32 ? 256 : 128; }
+
+struct DecodeParams {
+  const __nv_bfloat16* q;  // [B][H_q][dh]
+  const __nv_bfloat16* k;  // [B][N][H_kv][dh]
+  const __nv_bfloat16* v;
+  const int* lens;         // [B] positions in use, or null for all N
+  float* part;             // [B * H_kv][n_split][g][dh + 2]: o, then m and l (log2 units)
+  __nv_bfloat16* out;      // [B][H_q][dh]
+  float* lse;              // [B][H_q]
+  int N, Hq, Hkv, g, n_split;
+  float scale_log2;        // scale * log2(e)
+};
+
+// Shared memory of the split kernel, in bytes.
+__host__ __device__ constexpr size_t decode_smem_bytes(int g, int dh) {
+  return static_cast<size_t>(g) * dh * 4 + static_cast<size_t>(g) * decode_chunk(dh) * 4 +
+         2 * static_cast<size_t>(decode_chunk(dh)) * dh * 2 + static_cast<size_t>(g) * 8 + kDecodeThreads * 4;
+}
+
+__device__ __forceinline__ int decode_len(const DecodeParams& p, int b) {
+  const int len = p.lens ? p.lens[b] : p.N;
+  return len < 0 ? 0 : (len > p.N ? p.N : len);
+}
+
+template <int DH>
+__global__ void __launch_bounds__(kDecodeThreads) sqa_decode_split_kernel(const DecodeParams p) {
+  constexpr int CH = decode_chunk(DH), VEC = DH / 8;  // 16-byte vectors per row
+  const int split = blockIdx.x / p.Hkv, kvh = blockIdx.x % p.Hkv, b = blockIdx.y;
+  const int bk = b * p.Hkv + kvh, g = p.g;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int j0 = split * CH;
+  const int len = decode_len(p, b);
+  const int cnt = max(0, min(CH, len - j0));
+  float* part = p.part + (static_cast<size_t>(bk) * p.n_split + split) * g * (DH + 2);
+
+  if (cnt == 0) {  // chunk past this sequence's length: an empty partial
+    for (int i = tid; i < g * (DH + 2); i += kDecodeThreads) {
+      const int c = i % (DH + 2);
+      part[i] = c == DH ? -INFINITY : 0.f;
+    }
+    return;
+  }
+
+  extern __shared__ __align__(16) uint8_t dsm[];
+  float* qs = reinterpret_cast<float*>(dsm);                         // [g][DH]
+  float* ss = qs + g * DH;                                            // [g][CH] scores, then weights
+  __nv_bfloat16* ks = reinterpret_cast<__nv_bfloat16*>(ss + g * CH);  // [CH][DH]
+  __nv_bfloat16* vs = ks + CH * DH;                                   // [CH][DH]
+  float* ml = reinterpret_cast<float*>(vs + CH * DH);                 // [g][2]: m, l
+  float* red = ml + 2 * g;                                            // [kDecodeThreads] partial sums
+
+  // Queries of the group (heads kvh*g .. kvh*g+g-1 are adjacent) and the chunk.
+  const __nv_bfloat16* qg = p.q + (static_cast<size_t>(b) * p.Hq + kvh * g) * DH;
+  for (int i = tid; i < g * DH; i += kDecodeThreads) qs[i] = __bfloat162float(qg[i]);
+  for (int i = tid; i < cnt * VEC; i += kDecodeThreads) {
+    const int j = i / VEC, c = i % VEC;
+    const size_t row = (static_cast<size_t>(b) * p.N + j0 + j) * p.Hkv + kvh;
+    reinterpret_cast<uint4*>(ks)[i] = reinterpret_cast<const uint4*>(p.k + row * DH)[c];
+    reinterpret_cast<uint4*>(vs)[i] = reinterpret_cast<const uint4*>(p.v + row * DH)[c];
+  }
+  __syncthreads();
+
+  // Scores in log2 units; positions past the chunk's end get -inf.
+  for (int i = tid; i < g * CH; i += kDecodeThreads) {
+    const int h = i / CH, j = i % CH;
+    float acc = -INFINITY;
+    if (j < cnt) {
+      const float* qh = qs + h * DH;
+      const uint4* kr = reinterpret_cast<const uint4*>(ks + j * DH);
+      acc = 0.f;
+#pragma unroll
+      for (int c = 0; c < VEC; ++c) {
+        const uint4 u = kr[c];
+        const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 kf = __bfloat1622float2(k2[e]);
+          acc = fmaf(qh[8 * c + 2 * e], kf.x, acc);
+          acc = fmaf(qh[8 * c + 2 * e + 1], kf.y, acc);
+        }
+      }
+      acc *= p.scale_log2;
+    }
+    ss[i] = acc;
+  }
+  __syncthreads();
+
+  // Per head: chunk maximum, weights 2^(s - m) in place, their sum.
+  for (int h = warp; h < g; h += kDecodeThreads / 32) {
+    float* sh = ss + h * CH;
+    float m = -INFINITY;
+    for (int j = lane; j < CH; j += 32) m = fmaxf(m, sh[j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float l = 0.f;
+    for (int j = lane; j < CH; j += 32) {
+      const float w = dev::ex2(sh[j] - m);  // -inf past the end gives 0
+      sh[j] = w;
+      l += w;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) {
+      ml[2 * h] = m;
+      ml[2 * h + 1] = l;
+    }
+  }
+  __syncthreads();
+
+  // Unnormalised output of every head: sum_j w_j V_j.  With fewer outputs
+  // than threads, nsub threads share one output, each over every nsub-th position.
+  const int go = g * DH;
+  if (go >= kDecodeThreads) {
+    for (int i = tid; i < go; i += kDecodeThreads) {
+      const int h = i / DH, d = i % DH;
+      const float* wh = ss + h * CH;
+      float acc = 0.f;
+      for (int j = 0; j < cnt; ++j) acc = fmaf(wh[j], __bfloat162float(vs[j * DH + d]), acc);
+      part[h * (DH + 2) + d] = acc;
+    }
+  } else {
+    const int nsub = kDecodeThreads / go, o = tid % go, sub = tid / go;
+    float acc = 0.f;
+    if (sub < nsub) {
+      const int h = o / DH, d = o % DH;
+      const float* wh = ss + h * CH;
+      for (int j = sub; j < cnt; j += nsub) acc = fmaf(wh[j], __bfloat162float(vs[j * DH + d]), acc);
+    }
+    red[tid] = acc;
+    __syncthreads();
+    if (tid < go) {
+      float sum = red[tid];
+      for (int k = 1; k < nsub; ++k) sum += red[tid + k * go];
+      part[(tid / DH) * (DH + 2) + tid % DH] = sum;
+    }
+  }
+  for (int h = tid; h < g; h += kDecodeThreads) {
+    part[h * (DH + 2) + DH] = ml[2 * h];
+    part[h * (DH + 2) + DH + 1] = ml[2 * h + 1];
+  }
+}
+
+template <int DH>
+__global__ void __launch_bounds__(kDecodeThreads) sqa_decode_combine_kernel(const DecodeParams p) {
+  constexpr int SL = kDecodeThreads / DH;  // chunks handled side by side
+  const int bh = blockIdx.x;               // (batch entry, query head)
+  const int b = bh / p.Hq, h = bh % p.Hq, kvh = h / p.g, hg = h % p.g;
+  const int tid = threadIdx.x, d = tid % DH, sl = tid / DH;
+  const size_t stride = static_cast<size_t>(p.g) * (DH + 2);
+  const float* part =
+      p.part + static_cast<size_t>(b * p.Hkv + kvh) * p.n_split * stride + static_cast<size_t>(hg) * (DH + 2);
+  const int n_used = (decode_len(p, b) + decode_chunk(DH) - 1) / decode_chunk(DH);
+  __shared__ float red[kDecodeThreads];
+  __shared__ float big_m;
+
+  // M = largest chunk maximum.
+  float m = -INFINITY;
+  for (int s = tid; s < n_used; s += kDecodeThreads) m = fmaxf(m, part[s * stride + DH]);
+  red[tid] = m;
+  __syncthreads();
+  for (int o = kDecodeThreads / 2; o > 0; o >>= 1) {
+    if (tid < o) red[tid] = fmaxf(red[tid], red[tid + o]);
+    __syncthreads();
+  }
+  if (tid == 0) big_m = red[0];
+  __syncthreads();
+  const float M = big_m;
+
+  // Column d over the chunks sl, sl + SL, ..., and (column 0's threads) L.
+  float acc = 0.f, L = 0.f;
+  for (int s = sl; s < n_used; s += SL) {
+    const float* ps = part + s * stride;
+    const float w = dev::ex2(ps[DH] - M);
+    acc = fmaf(ps[d], w, acc);
+    L = fmaf(ps[DH + 1], w, L);
+  }
+  __syncthreads();
+  red[tid] = acc;
+  __syncthreads();
+  if (sl == 0) {
+    for (int k = 1; k < SL; ++k) acc += red[k * DH + d];
+  }
+  __syncthreads();
+  red[tid] = L;
+  __syncthreads();
+  if (tid == 0) {
+    for (int k = 1; k < SL; ++k) L += red[k * DH];
+    red[0] = L;
+  }
+  __syncthreads();
+  L = red[0];
+  if (sl == 0) {
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    p.out[static_cast<size_t>(bh) * DH + d] = __float2bfloat16_rn(acc * inv);
+    if (d == 0) p.lse[bh] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+  }
+}
+
+}  // namespace sqa

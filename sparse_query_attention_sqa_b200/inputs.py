@@ -35,6 +35,7 @@ class Workload:
     k_scale: float = 1.0
     scale: float = 0.0  # <= 0 selects 1/sqrt(dh)
     note: str = ""
+    decode: bool = False  # one new query token per sequence against a cache of N positions
 
     @property
     def softmax_scale(self) -> float:
@@ -69,6 +70,12 @@ for n in (131072, 200000):
 # Larger-model SQA: d=2048 over 16 heads, dh=128.
 _add(Workload("large_dh128", 2, 65536, 8, 4, 128, True, True, k_scale=0.1,
               note="larger model, B=2 N=65536 dh=128 Hq=8 Hkv=4 causal, K x 0.1"))
+# Decoding step: a batch of sequences, each adding one token against a full
+# key/value cache (SQAT-m head layout, and the larger-model dh=128 layout).
+_add(Workload("decode_sqatm", 32, 32768, 8, 4, 16, False, False, decode=True,
+              note="decode step, B=32 sequences, cache N=32768, dh=16 Hq=8 Hkv=4"))
+_add(Workload("decode_dh128", 8, 65536, 8, 4, 128, False, False, k_scale=0.1, decode=True,
+              note="decode step, B=8 sequences, cache N=65536, dh=128 Hq=8 Hkv=4, K x 0.1"))
 
 
 def make_inputs(B: int, N: int, Hq: int, Hkv: int, dh: int, seed: int = 0, std: float = 1.0,
@@ -82,6 +89,19 @@ def make_inputs(B: int, N: int, Hq: int, Hkv: int, dh: int, seed: int = 0, std: 
     return q, k, v, dout
 
 
+def make_decode_inputs(B: int, N: int, Hq: int, Hkv: int, dh: int, seed: int = 0, std: float = 1.0,
+                       k_scale: float = 1.0):
+    """Draw the new token's queries q [B,Hq,dh] and the caches k, v [B,N,Hkv,dh] (CPU bf16), in that order."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    q = (torch.randn(B, Hq, dh, generator=g) * std).to(torch.bfloat16)
+    k = (torch.randn(B, N, Hkv, dh, generator=g) * (std * k_scale)).to(torch.bfloat16)
+    v = (torch.randn(B, N, Hkv, dh, generator=g) * std).to(torch.bfloat16)
+    return q, k, v
+
+
 def workload_inputs(w: Workload, seed: int = 0):
+    """(q, k, v, dout); for a decoding workload q is [B,Hq,dh] and dout is None."""
+    if w.decode:
+        return (*make_decode_inputs(w.B, w.N, w.Hq, w.Hkv, w.dh, seed=seed, std=w.std, k_scale=w.k_scale), None)
     return make_inputs(w.B, w.N, w.Hq, w.Hkv, w.dh, seed=seed, std=w.std, k_scale=w.k_scale,
                        with_dout=w.backward)

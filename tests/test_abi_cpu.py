@@ -114,3 +114,20 @@ def test_exp2_selftest_rejects_null_pointers_before_launch(lib):
     assert f(None, None, 0, None) == 0  # nothing to do
     assert f(None, 0x100, 4, None) == 1
     assert f(0x100, 0x104, 4, None) == 1  # y misaligned
+
+
+def test_decode_rejects_bad_arguments_before_launch(lib):
+    f = lib.sqa_decode
+    vp = ctypes.c_void_p
+    f.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, sqa.Shape, ctypes.c_float, vp]
+    f.restype = ctypes.c_int
+    s = sqa.Shape(2, 300, 8, 4, 16)
+    need = lib.sqa_decode_workspace_bytes(s)
+    assert need > 0
+    ok = [0x1000, 0x2000, 0x3000, 0, 0x4000, 0x5000, 0x6000]
+    assert f(*ok[:3], None, *ok[4:], need, sqa.Shape(2, 300, 6, 4, 16), 0.0, None) == 1  # H_q % H_kv
+    assert f(*ok[:3], None, *ok[4:], need, sqa.Shape(2, 300, 8, 4, 48), 0.0, None) == 2  # head dim
+    assert f(None, *ok[1:3], None, *ok[4:], need, s, 0.0, None) == 1  # null q
+    assert f(ok[0], 0x2008, ok[2], None, *ok[4:], need, s, 0.0, None) == 2  # cache not 16-byte aligned
+    assert f(*ok[:3], None, *ok[4:], need - 1, s, 0.0, None) == 1  # workspace too small
+    assert lib.sqa_decode_workspace_bytes(sqa.Shape(0, 300, 8, 4, 16)) == 0
