@@ -152,7 +152,7 @@ sqa_status launch_fwd(const void* q, const void* k, const void* v, void* out, fl
 }
 
 size_t decode_workspace(const sqa_shape& s) {
-  const int ch = sqa::decode_chunk(s.dh);
+  const int ch = sqa::decode_span(s.dh);
   const size_t n_split = (static_cast<size_t>(s.N) + ch - 1) / ch;
   const size_t g = static_cast<size_t>(s.H_q / s.H_kv);
   return sqa::align256(static_cast<size_t>(s.B) * s.H_kv * n_split * g * (s.dh + 2) * sizeof(float));
@@ -173,7 +173,7 @@ sqa_status launch_decode(const void* q, const void* k, const void* v, const int*
   p.Hq = s.H_q;
   p.Hkv = s.H_kv;
   p.g = s.H_q / s.H_kv;
-  p.n_split = (s.N + sqa::decode_chunk(DH) - 1) / sqa::decode_chunk(DH);
+  p.n_split = (s.N + sqa::decode_span(DH) - 1) / sqa::decode_span(DH);
   p.scale_log2 = scale * kLog2e;
   const int smem = static_cast<int>(sqa::decode_smem_bytes(p.g, DH));
   sqa_status st;

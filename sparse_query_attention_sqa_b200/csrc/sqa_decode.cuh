@@ -11,16 +11,17 @@
 // multiply-adds per cached position, far below what tensor cores are for.
 //
 // Two launches, split-K over the cache:
-//   1. split:   one CTA per (chunk of 256 positions (128 at dh >= 64), K/V head,
-//               batch entry), the K/V heads of one chunk adjacent in launch order
-//               so the cache rows they share are read from DRAM once.  It
-//               copies the chunk's K and V rows (bf16, 16-byte loads) and the
-//               group's g queries into shared memory, forms the g x chunk scores
-//               (log2 units), takes each head's chunk maximum m and
-//               l = sum 2^(s - m) with warp shuffles, and writes the unnormalised
-//               o = sum 2^(s - m) V with m and l to the workspace.
-//   2. combine: one CTA per (batch entry, query head) merges the chunks, its
-//               threads spread over (column, chunk) pairs:
+//   1. split:   one CTA per (4 chunks of positions, K/V head, batch entry), the
+//               K/V heads of one range adjacent in launch order so the cache rows
+//               they share are read from DRAM once.  Chunks (256 positions at
+//               dh <= 32, 128 at dh = 64, 64 at dh = 128) are copied into shared
+//               memory with cp.async, double-buffered so the next chunk streams
+//               in while this one is processed: the g x chunk scores (log2
+//               units), each head's running maximum and sum of 2^(s - m) with
+//               warp shuffles, and the running unnormalised o = sum 2^(s - m) V.
+//               The CTA writes o with m and l to the workspace.
+//   2. combine: one CTA per (batch entry, query head) merges the ranges, its
+//               threads spread over (column, range) pairs:
 //               M = max m, L = sum l 2^(m - M), out = sum o 2^(m - M) / L (bf16),
 //               lse = ln 2 * (M + log2 L).
 #pragma once
@@ -30,9 +31,12 @@
 namespace sqa {
 
 constexpr int kDecodeThreads = 256;
-// Cache positions per split: 256, or 128 at dh >= 64 so that the chunk, its
-// scores for a group of up to 128 heads and the queries fit in shared memory.
-__host__ __device__ constexpr int decode_chunk(int dh) { return dh <= 32 ? 256 : 128; }
+constexpr int kDecodeChunksPerCta = 4;
+// Cache positions per chunk: sized so that two chunk buffers, a group of up to
+// 128 heads' scores, queries and running outputs fit in shared memory.
+__host__ __device__ constexpr int decode_chunk(int dh) { return dh <= 32 ? 256 : (dh == 64 ? 128 : 64); }
+// Positions per split-kernel CTA (one partial result each).
+__host__ __device__ constexpr int decode_span(int dh) { return decode_chunk(dh) * kDecodeChunksPerCta; }
 
 struct DecodeParams {
   const __nv_bfloat16* q;  // [B][H_q][dh]
@@ -46,10 +50,12 @@ struct DecodeParams {
   float scale_log2;        // scale * log2(e)
 };
 
-// Shared memory of the split kernel, in bytes.
+// Shared memory of the split kernel, in bytes: queries and running outputs
+// [g][dh] fp32, scores [g][chunk] fp32, two K and two V chunk buffers (bf16),
+// per-head m, l, rescale factor, and one float per thread.
 __host__ __device__ constexpr size_t decode_smem_bytes(int g, int dh) {
-  return static_cast<size_t>(g) * dh * 4 + static_cast<size_t>(g) * decode_chunk(dh) * 4 +
-         2 * static_cast<size_t>(decode_chunk(dh)) * dh * 2 + static_cast<size_t>(g) * 8 + kDecodeThreads * 4;
+  return 2 * static_cast<size_t>(g) * dh * 4 + static_cast<size_t>(g) * decode_chunk(dh) * 4 +
+         4 * static_cast<size_t>(decode_chunk(dh)) * dh * 2 + static_cast<size_t>(g) * 12 + kDecodeThreads * 4;
 }
 
 __device__ __forceinline__ int decode_len(const DecodeParams& p, int b) {
@@ -57,18 +63,28 @@ __device__ __forceinline__ int decode_len(const DecodeParams& p, int b) {
   return len < 0 ? 0 : (len > p.N ? p.N : len);
 }
 
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dev::smem_u32(smem_dst)), "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 template <int DH>
 __global__ void __launch_bounds__(kDecodeThreads) sqa_decode_split_kernel(const DecodeParams p) {
   constexpr int CH = decode_chunk(DH), VEC = DH / 8;  // 16-byte vectors per row
   const int split = blockIdx.x / p.Hkv, kvh = blockIdx.x % p.Hkv, b = blockIdx.y;
-  const int bk = b * p.Hkv + kvh, g = p.g;
+  const int bk = b * p.Hkv + kvh, g = p.g, go = g * DH;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int j0 = split * CH;
   const int len = decode_len(p, b);
-  const int cnt = max(0, min(CH, len - j0));
+  const int c_first = split * kDecodeChunksPerCta;
+  const int n_chunks = max(0, min(kDecodeChunksPerCta, (len + CH - 1) / CH - c_first));
   float* part = p.part + (static_cast<size_t>(bk) * p.n_split + split) * g * (DH + 2);
 
-  if (cnt == 0) {  // chunk past this sequence's length: an empty partial
+  if (n_chunks == 0) {  // range past this sequence's length: an empty partial
     for (int i = tid; i < g * (DH + 2); i += kDecodeThreads) {
       const int c = i % (DH + 2);
       part[i] = c == DH ? -INFINITY : 0.f;
@@ -78,100 +94,134 @@ __global__ void __launch_bounds__(kDecodeThreads) sqa_decode_split_kernel(const 
 
   extern __shared__ __align__(16) uint8_t dsm[];
   float* qs = reinterpret_cast<float*>(dsm);                         // [g][DH]
-  float* ss = qs + g * DH;                                            // [g][CH] scores, then weights
-  __nv_bfloat16* ks = reinterpret_cast<__nv_bfloat16*>(ss + g * CH);  // [CH][DH]
-  __nv_bfloat16* vs = ks + CH * DH;                                   // [CH][DH]
-  float* ml = reinterpret_cast<float*>(vs + CH * DH);                 // [g][2]: m, l
-  float* red = ml + 2 * g;                                            // [kDecodeThreads] partial sums
+  float* os = qs + go;                                                // [g][DH] running output
+  float* ss = os + go;                                                // [g][CH] scores, then weights
+  __nv_bfloat16* kvs = reinterpret_cast<__nv_bfloat16*>(ss + g * CH);  // [2][K, V][CH][DH]
+  float* mrun = reinterpret_cast<float*>(kvs + 4 * CH * DH);           // [g]
+  float* lrun = mrun + g;                                              // [g]
+  float* alpha = lrun + g;                                             // [g]
+  float* red = alpha + g;                                              // [kDecodeThreads]
 
-  // Queries of the group (heads kvh*g .. kvh*g+g-1 are adjacent) and the chunk.
+  auto chunk_rows = [&](int c) { return min(CH, len - (c_first + c) * CH); };
+  auto load_chunk = [&](int c) {  // cp.async of chunk c into buffer c % 2
+    const int j0 = (c_first + c) * CH, cnt = chunk_rows(c);
+    __nv_bfloat16* kb = kvs + (c & 1) * 2 * CH * DH;
+    __nv_bfloat16* vb = kb + CH * DH;
+    for (int i = tid; i < cnt * VEC; i += kDecodeThreads) {
+      const int j = i / VEC, cc = i % VEC;
+      const size_t row = (static_cast<size_t>(b) * p.N + j0 + j) * p.Hkv + kvh;
+      cp_async16(kb + j * DH + cc * 8, p.k + row * DH + cc * 8);
+      cp_async16(vb + j * DH + cc * 8, p.v + row * DH + cc * 8);
+    }
+    cp_async_commit();
+  };
+
+  load_chunk(0);
+  // Queries of the group (heads kvh*g .. kvh*g+g-1 are adjacent); running state.
   const __nv_bfloat16* qg = p.q + (static_cast<size_t>(b) * p.Hq + kvh * g) * DH;
-  for (int i = tid; i < g * DH; i += kDecodeThreads) qs[i] = __bfloat162float(qg[i]);
-  for (int i = tid; i < cnt * VEC; i += kDecodeThreads) {
-    const int j = i / VEC, c = i % VEC;
-    const size_t row = (static_cast<size_t>(b) * p.N + j0 + j) * p.Hkv + kvh;
-    reinterpret_cast<uint4*>(ks)[i] = reinterpret_cast<const uint4*>(p.k + row * DH)[c];
-    reinterpret_cast<uint4*>(vs)[i] = reinterpret_cast<const uint4*>(p.v + row * DH)[c];
-  }
-  __syncthreads();
-
-  // Scores in log2 units; positions past the chunk's end get -inf.
-  for (int i = tid; i < g * CH; i += kDecodeThreads) {
-    const int h = i / CH, j = i % CH;
-    float acc = -INFINITY;
-    if (j < cnt) {
-      const float* qh = qs + h * DH;
-      const uint4* kr = reinterpret_cast<const uint4*>(ks + j * DH);
-      acc = 0.f;
-#pragma unroll
-      for (int c = 0; c < VEC; ++c) {
-        const uint4 u = kr[c];
-        const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 kf = __bfloat1622float2(k2[e]);
-          acc = fmaf(qh[8 * c + 2 * e], kf.x, acc);
-          acc = fmaf(qh[8 * c + 2 * e + 1], kf.y, acc);
-        }
-      }
-      acc *= p.scale_log2;
-    }
-    ss[i] = acc;
-  }
-  __syncthreads();
-
-  // Per head: chunk maximum, weights 2^(s - m) in place, their sum.
-  for (int h = warp; h < g; h += kDecodeThreads / 32) {
-    float* sh = ss + h * CH;
-    float m = -INFINITY;
-    for (int j = lane; j < CH; j += 32) m = fmaxf(m, sh[j]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float l = 0.f;
-    for (int j = lane; j < CH; j += 32) {
-      const float w = dev::ex2(sh[j] - m);  // -inf past the end gives 0
-      sh[j] = w;
-      l += w;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    if (lane == 0) {
-      ml[2 * h] = m;
-      ml[2 * h + 1] = l;
-    }
-  }
-  __syncthreads();
-
-  // Unnormalised output of every head: sum_j w_j V_j.  With fewer outputs
-  // than threads, nsub threads share one output, each over every nsub-th position.
-  const int go = g * DH;
-  if (go >= kDecodeThreads) {
-    for (int i = tid; i < go; i += kDecodeThreads) {
-      const int h = i / DH, d = i % DH;
-      const float* wh = ss + h * CH;
-      float acc = 0.f;
-      for (int j = 0; j < cnt; ++j) acc = fmaf(wh[j], __bfloat162float(vs[j * DH + d]), acc);
-      part[h * (DH + 2) + d] = acc;
-    }
-  } else {
-    const int nsub = kDecodeThreads / go, o = tid % go, sub = tid / go;
-    float acc = 0.f;
-    if (sub < nsub) {
-      const int h = o / DH, d = o % DH;
-      const float* wh = ss + h * CH;
-      for (int j = sub; j < cnt; j += nsub) acc = fmaf(wh[j], __bfloat162float(vs[j * DH + d]), acc);
-    }
-    red[tid] = acc;
-    __syncthreads();
-    if (tid < go) {
-      float sum = red[tid];
-      for (int k = 1; k < nsub; ++k) sum += red[tid + k * go];
-      part[(tid / DH) * (DH + 2) + tid % DH] = sum;
-    }
+  for (int i = tid; i < go; i += kDecodeThreads) {
+    qs[i] = __bfloat162float(qg[i]);
+    os[i] = 0.f;
   }
   for (int h = tid; h < g; h += kDecodeThreads) {
-    part[h * (DH + 2) + DH] = ml[2 * h];
-    part[h * (DH + 2) + DH + 1] = ml[2 * h + 1];
+    mrun[h] = -INFINITY;
+    lrun[h] = 0.f;
+  }
+
+  for (int c = 0; c < n_chunks; ++c) {
+    if (c + 1 < n_chunks) {
+      load_chunk(c + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();  // chunk c (and, at c = 0, the queries) visible to every thread
+    const int cnt = chunk_rows(c);
+    const __nv_bfloat16* kb = kvs + (c & 1) * 2 * CH * DH;
+    const __nv_bfloat16* vb = kb + CH * DH;
+
+    // Scores in log2 units; positions past the chunk's end get -inf.
+    for (int i = tid; i < g * CH; i += kDecodeThreads) {
+      const int h = i / CH, j = i % CH;
+      float acc = -INFINITY;
+      if (j < cnt) {
+        const float* qh = qs + h * DH;
+        const uint4* kr = reinterpret_cast<const uint4*>(kb + j * DH);
+        acc = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < VEC; ++cc) {
+          const uint4 u = kr[cc];
+          const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 kf = __bfloat1622float2(k2[e]);
+            acc = fmaf(qh[8 * cc + 2 * e], kf.x, acc);
+            acc = fmaf(qh[8 * cc + 2 * e + 1], kf.y, acc);
+          }
+        }
+        acc *= p.scale_log2;
+      }
+      ss[i] = acc;
+    }
+    __syncthreads();
+
+    // Per head: new running maximum, weights 2^(s - m) in place, running sum.
+    for (int h = warp; h < g; h += kDecodeThreads / 32) {
+      float* sh = ss + h * CH;
+      float m = mrun[h];
+      for (int j = lane; j < CH; j += 32) m = fmaxf(m, sh[j]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float l = 0.f;
+      for (int j = lane; j < CH; j += 32) {
+        const float w = dev::ex2(sh[j] - m);  // -inf past the end gives 0
+        sh[j] = w;
+        l += w;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+      if (lane == 0) {
+        const float a = mrun[h] == -INFINITY ? 0.f : dev::ex2(mrun[h] - m);
+        alpha[h] = a;
+        lrun[h] = lrun[h] * a + l;
+        mrun[h] = m;
+      }
+    }
+    __syncthreads();
+
+    // Running output: o = o * alpha + sum_j w_j V_j.  With fewer outputs than
+    // threads, nsub threads share one output, each over every nsub-th position.
+    if (go >= kDecodeThreads) {
+      for (int i = tid; i < go; i += kDecodeThreads) {
+        const int h = i / DH, d = i % DH;
+        const float* wh = ss + h * CH;
+        float acc = 0.f;
+        for (int j = 0; j < cnt; ++j) acc = fmaf(wh[j], __bfloat162float(vb[j * DH + d]), acc);
+        os[i] = fmaf(os[i], alpha[h], acc);
+      }
+    } else {
+      const int nsub = kDecodeThreads / go, o = tid % go, sub = tid / go;
+      float acc = 0.f;
+      if (sub < nsub) {
+        const int h = o / DH, d = o % DH;
+        const float* wh = ss + h * CH;
+        for (int j = sub; j < cnt; j += nsub) acc = fmaf(wh[j], __bfloat162float(vb[j * DH + d]), acc);
+      }
+      red[tid] = acc;
+      __syncthreads();
+      if (tid < go) {
+        float sum = red[tid];
+        for (int k = 1; k < nsub; ++k) sum += red[tid + k * go];
+        os[tid] = fmaf(os[tid], alpha[tid / DH], sum);
+      }
+    }
+    __syncthreads();  // buffer c % 2 and the scores are free for the next chunk
+  }
+
+  for (int i = tid; i < go; i += kDecodeThreads) part[(i / DH) * (DH + 2) + i % DH] = os[i];
+  for (int h = tid; h < g; h += kDecodeThreads) {
+    part[h * (DH + 2) + DH] = mrun[h];
+    part[h * (DH + 2) + DH + 1] = lrun[h];
   }
 }
 
@@ -184,7 +234,7 @@ __global__ void __launch_bounds__(kDecodeThreads) sqa_decode_combine_kernel(cons
   const size_t stride = static_cast<size_t>(p.g) * (DH + 2);
   const float* part =
       p.part + static_cast<size_t>(b * p.Hkv + kvh) * p.n_split * stride + static_cast<size_t>(hg) * (DH + 2);
-  const int n_used = (decode_len(p, b) + decode_chunk(DH) - 1) / decode_chunk(DH);
+  const int n_used = (decode_len(p, b) + decode_span(DH) - 1) / decode_span(DH);
   __shared__ float red[kDecodeThreads];
   __shared__ float big_m;
 
