@@ -52,10 +52,12 @@ struct DecodeParams {
 
 // Shared memory of the split kernel, in bytes: queries and running outputs
 // [g][dh] fp32, scores [g][chunk] fp32, two K and two V chunk buffers (bf16),
-// per-head m, l, rescale factor, and one float per thread.
+// per-head m, l and rescale factor, and (for groups with fewer than one output
+// per thread) two partial sums per thread.
 __host__ __device__ constexpr size_t decode_smem_bytes(int g, int dh) {
   return 2 * static_cast<size_t>(g) * dh * 4 + static_cast<size_t>(g) * decode_chunk(dh) * 4 +
-         4 * static_cast<size_t>(decode_chunk(dh)) * dh * 2 + static_cast<size_t>(g) * 12 + kDecodeThreads * 4;
+         4 * static_cast<size_t>(decode_chunk(dh)) * dh * 2 + static_cast<size_t>(g) * 12 +
+         (g * dh < kDecodeThreads ? 2 * kDecodeThreads * 4 : 0);
 }
 
 __device__ __forceinline__ int decode_len(const DecodeParams& p, int b) {
@@ -100,7 +102,7 @@ __global__ void __launch_bounds__(kDecodeThreads) sqa_decode_split_kernel(const 
   float* mrun = reinterpret_cast<float*>(kvs + 4 * CH * DH);           // [g]
   float* lrun = mrun + g;                                              // [g]
   float* alpha = lrun + g;                                             // [g]
-  float* red = alpha + g;                                              // [kDecodeThreads]
+  float* red = alpha + g;  // [2 * kDecodeThreads] partial sums, only when g * DH < kDecodeThreads
 
   auto chunk_rows = [&](int c) { return min(CH, len - (c_first + c) * CH); };
   auto load_chunk = [&](int c) {  // cp.async of chunk c into buffer c % 2
@@ -141,27 +143,59 @@ __global__ void __launch_bounds__(kDecodeThreads) sqa_decode_split_kernel(const 
     const __nv_bfloat16* vb = kb + CH * DH;
 
     // Scores in log2 units; positions past the chunk's end get -inf.
-    for (int i = tid; i < g * CH; i += kDecodeThreads) {
-      const int h = i / CH, j = i % CH;
-      float acc = -INFINITY;
+    if constexpr (CH == kDecodeThreads) {
+      // One position per thread: its key row is read once into registers and
+      // dotted with every query of the group in packed fp32 pairs (the queries
+      // are the same address for the whole warp).
+      const int j = tid;
+      float2 kr[DH / 2];
       if (j < cnt) {
-        const float* qh = qs + h * DH;
-        const uint4* kr = reinterpret_cast<const uint4*>(kb + j * DH);
-        acc = 0.f;
 #pragma unroll
         for (int cc = 0; cc < VEC; ++cc) {
-          const uint4 u = kr[cc];
+          const uint4 u = reinterpret_cast<const uint4*>(kb + j * DH)[cc];
           const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 kf = __bfloat1622float2(k2[e]);
-            acc = fmaf(qh[8 * cc + 2 * e], kf.x, acc);
-            acc = fmaf(qh[8 * cc + 2 * e + 1], kf.y, acc);
-          }
+          for (int e = 0; e < 4; ++e) kr[4 * cc + e] = __bfloat1622float2(k2[e]);
         }
-        acc *= p.scale_log2;
       }
-      ss[i] = acc;
+      for (int h = 0; h < g; ++h) {
+        float acc = -INFINITY;
+        if (j < cnt) {
+          const float4* qh = reinterpret_cast<const float4*>(qs + h * DH);
+          float2 a2 = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int e = 0; e < DH / 4; ++e) {
+            const float4 qv = qh[e];
+            a2 = __ffma2_rn(make_float2(qv.x, qv.y), kr[2 * e], a2);
+            a2 = __ffma2_rn(make_float2(qv.z, qv.w), kr[2 * e + 1], a2);
+          }
+          acc = (a2.x + a2.y) * p.scale_log2;
+        }
+        ss[h * CH + j] = acc;
+      }
+    } else {
+      for (int i = tid; i < g * CH; i += kDecodeThreads) {
+        const int h = i / CH, j = i % CH;
+        float acc = -INFINITY;
+        if (j < cnt) {
+          const float* qh = qs + h * DH;
+          const uint4* kr = reinterpret_cast<const uint4*>(kb + j * DH);
+          acc = 0.f;
+#pragma unroll
+          for (int cc = 0; cc < VEC; ++cc) {
+            const uint4 u = kr[cc];
+            const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 kf = __bfloat1622float2(k2[e]);
+              acc = fmaf(qh[8 * cc + 2 * e], kf.x, acc);
+              acc = fmaf(qh[8 * cc + 2 * e + 1], kf.y, acc);
+            }
+          }
+          acc *= p.scale_log2;
+        }
+        ss[i] = acc;
+      }
     }
     __syncthreads();
 
@@ -200,14 +234,20 @@ __global__ void __launch_bounds__(kDecodeThreads) sqa_decode_split_kernel(const 
         os[i] = fmaf(os[i], alpha[h], acc);
       }
     } else {
-      const int nsub = kDecodeThreads / go, o = tid % go, sub = tid / go;
-      float acc = 0.f;
+      // Outputs in adjacent pairs (one bf16x2 load of V, one packed FMA each).
+      const int gp = go / 2, nsub = kDecodeThreads / gp, o = tid % gp, sub = tid / gp;
+      float2 acc = make_float2(0.f, 0.f);
       if (sub < nsub) {
-        const int h = o / DH, d = o % DH;
+        const int h = (2 * o) / DH, d = (2 * o) % DH;
         const float* wh = ss + h * CH;
-        for (int j = sub; j < cnt; j += nsub) acc = fmaf(wh[j], __bfloat162float(vb[j * DH + d]), acc);
+        const __nv_bfloat162* vcol = reinterpret_cast<const __nv_bfloat162*>(vb + d);
+        for (int j = sub; j < cnt; j += nsub) {
+          const float w = wh[j];
+          acc = __ffma2_rn(make_float2(w, w), __bfloat1622float2(vcol[j * (DH / 2)]), acc);
+        }
       }
-      red[tid] = acc;
+      red[2 * tid] = acc.x;
+      red[2 * tid + 1] = acc.y;
       __syncthreads();
       if (tid < go) {
         float sum = red[tid];
