@@ -289,16 +289,42 @@ def roofline_for(w, kernel_name, ms, peaks, peak_kind):
             "traffic": traffic_for(kernel_name, w), "kernel": kernel_name, "peak_source": f"{peak_kind} bf16_tflops"}
 
 
+def strip_c_comments(text: str) -> str:
+    """C/C++ source with its comments removed (string and character literals kept)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i : j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return "".join(out)
+
+
 def kernel_source_sha256():
-    """Hash of every CUDA source of the library (a profile is valid only for the code it measured)."""
+    """Hash of the code (comments removed, whitespace runs collapsed) of every
+    CUDA source of the library: a profile is valid only for the code it measured."""
     import hashlib
 
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_query_attention_sqa_b200", "csrc")
     for fn in sorted(os.listdir(csrc)):
         if fn.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(fn.encode() + b"\0" + f.read())
+            with open(os.path.join(csrc, fn), encoding="utf-8") as f:
+                code = " ".join(strip_c_comments(f.read()).split())  # layout ignored too
+                h.update(fn.encode() + b"\0" + code.encode())
     return h.hexdigest()
 
 

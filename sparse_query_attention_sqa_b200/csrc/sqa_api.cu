@@ -151,11 +151,52 @@ sqa_status launch_fwd(const void* q, const void* k, const void* v, void* out, fl
   return record_timing(0, 1, stream);
 }
 
+// Ranges per sequence of the decoding split kernel: the general path's fixed
+// span, or (register-resident path) about four waves of resident CTAs over the
+// whole batch, each range at least rows_min_span positions.  The workspace is
+// sized for the most ranges either path can take.
 size_t decode_workspace(const sqa_shape& s) {
-  const int ch = sqa::decode_span(s.dh);
-  const size_t n_split = (static_cast<size_t>(s.N) + ch - 1) / ch;
-  const size_t g = static_cast<size_t>(s.H_q / s.H_kv);
+  const int g = s.H_q / s.H_kv;
+  size_t n_split = (static_cast<size_t>(s.N) + sqa::decode_span(s.dh) - 1) / sqa::decode_span(s.dh);
+  if (sqa::rows_path(g, s.H_kv, s.dh)) {
+    const int ms = sqa::rows_min_span(s.dh, s.H_kv);
+    const size_t n_rows = (static_cast<size_t>(s.N) + ms - 1) / ms;
+    if (n_rows > n_split) n_split = n_rows;
+  }
   return sqa::align256(static_cast<size_t>(s.B) * s.H_kv * n_split * g * (s.dh + 2) * sizeof(float));
+}
+
+int decode_rows_span(const sqa_shape& s, int ctas_per_sm) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long want = (4LL * sms * ctas_per_sm + s.B - 1) / s.B;  // ranges per sequence
+  const int unit = sqa::rows_step(s.dh) / s.H_kv;                     // positions per CTA step
+  long long span = (s.N + want - 1) / want;
+  span = (span + unit - 1) / unit * unit;
+  const int ms = sqa::rows_min_span(s.dh, s.H_kv);
+  return static_cast<int>(span < ms ? ms : span);
+}
+
+template <int DH, int G>
+sqa_status launch_decode_rows(sqa::DecodeParams& p, const sqa_shape& s, cudaStream_t stream) {
+  const int smem = static_cast<int>(sqa::rows_smem_bytes(G, DH));
+  static const int occ = [smem] {
+    int o = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, sqa::sqa_decode_split_kernel<DH, G>, sqa::kDecodeThreads,
+                                                      smem) != cudaSuccess)
+      o = 0;
+    return o > 0 ? o : 1;
+  }();
+  p.span = decode_rows_span(s, occ);
+  p.n_split = (s.N + p.span - 1) / p.span;
+  sqa_status st;
+  if ((st = set_smem(sqa::sqa_decode_split_kernel<DH, G>, smem)) != SQA_OK) return st;
+  if ((st = record_timing(2, 0, stream)) != SQA_OK) return st;
+  sqa::sqa_decode_split_kernel<DH, G>
+      <<<dim3(static_cast<unsigned>(p.n_split), static_cast<unsigned>(s.B)), sqa::kDecodeThreads, smem, stream>>>(p);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "sqa_decode split launch");
+  return SQA_OK;
 }
 
 template <int DH>
@@ -173,19 +214,30 @@ sqa_status launch_decode(const void* q, const void* k, const void* v, const int*
   p.Hq = s.H_q;
   p.Hkv = s.H_kv;
   p.g = s.H_q / s.H_kv;
-  p.n_split = (s.N + sqa::decode_span(DH) - 1) / sqa::decode_span(DH);
   p.scale_log2 = scale * kLog2e;
-  const int smem = static_cast<int>(sqa::decode_smem_bytes(p.g, DH));
   sqa_status st;
-  if ((st = set_smem(sqa::sqa_decode_split_kernel<DH>, smem)) != SQA_OK) return st;
-  const dim3 grid(static_cast<unsigned>(p.n_split * s.H_kv), static_cast<unsigned>(s.B));
-  if ((st = record_timing(2, 0, stream)) != SQA_OK) return st;
-  sqa::sqa_decode_split_kernel<DH><<<grid, sqa::kDecodeThreads, smem, stream>>>(p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "sqa_decode split launch");
+  if (sqa::rows_path(p.g, s.H_kv, DH) && aligned(q, 16)) {
+    switch (p.g) {
+      case 1: st = launch_decode_rows<DH, 1>(p, s, stream); break;
+      case 2: st = launch_decode_rows<DH, 2>(p, s, stream); break;
+      case 3: st = launch_decode_rows<DH, 3>(p, s, stream); break;
+      default: st = launch_decode_rows<DH, 4>(p, s, stream); break;
+    }
+    if (st != SQA_OK) return st;
+  } else {
+    p.span = sqa::decode_span(DH);
+    p.n_split = (s.N + p.span - 1) / p.span;
+    const int smem = static_cast<int>(sqa::decode_smem_bytes(p.g, DH));
+    if ((st = set_smem(sqa::sqa_decode_split_kernel<DH, 0>, smem)) != SQA_OK) return st;
+    const dim3 grid(static_cast<unsigned>(p.n_split * s.H_kv), static_cast<unsigned>(s.B));
+    if ((st = record_timing(2, 0, stream)) != SQA_OK) return st;
+    sqa::sqa_decode_split_kernel<DH, 0><<<grid, sqa::kDecodeThreads, smem, stream>>>(p);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "sqa_decode split launch");
+  }
   if ((st = record_timing(2, 1, stream)) != SQA_OK) return st;
   sqa::sqa_decode_combine_kernel<DH><<<static_cast<unsigned>(s.B * s.H_q), sqa::kDecodeThreads, 0, stream>>>(p);
-  e = cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "sqa_decode combine launch");
   return SQA_OK;
 }

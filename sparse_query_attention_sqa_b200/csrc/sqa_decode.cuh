@@ -11,15 +11,22 @@
 // multiply-adds per cached position, far below what tensor cores are for.
 //
 // Two launches, split-K over the cache:
-//   1. split:   one CTA per (4 chunks of positions, K/V head, batch entry), the
-//               K/V heads of one range adjacent in launch order so the cache rows
-//               they share are read from DRAM once.  Chunks (256 positions at
-//               dh <= 32, 128 at dh = 64, 64 at dh = 128) are copied into shared
-//               memory with cp.async, double-buffered so the next chunk streams
-//               in while this one is processed: the g x chunk scores (log2
-//               units), each head's running maximum and sum of 2^(s - m) with
-//               warp shuffles, and the running unnormalised o = sum 2^(s - m) V.
-//               The CTA writes o with m and l to the workspace.
+//   1. split:   one CTA per (range of positions, batch entry[, K/V head]),
+//               writing per query head the range's unnormalised output o with
+//               its running maximum m and sum l (log2 units) to the workspace.
+//               Two paths:
+//               - register-resident (groups of at most 4 query heads, a
+//                 power-of-two K/V head count): the range's cache rows of all
+//                 K/V heads are one contiguous run; dh / 8 lanes share a row,
+//                 each thread slot keeps its own running softmax state in
+//                 registers with several rows' loads in flight, and the slots
+//                 of each K/V head merge once at the end.  The number of
+//                 ranges makes about four waves of resident CTAs.
+//               - general (any group up to 128 heads): one CTA per (4 chunks
+//                 of positions, K/V head, batch entry); chunks (256 positions
+//                 at dh <= 32, 128 at dh = 64, 64 at dh = 128) are copied into
+//                 shared memory with cp.async, double-buffered, and scored for
+//                 all g heads of the group with block-wide online softmax.
 //   2. combine: one CTA per (batch entry, query head) merges the ranges, its
 //               threads spread over (column, range) pairs:
 //               M = max m, L = sum l 2^(m - M), out = sum o 2^(m - M) / L (bf16),
@@ -47,8 +54,27 @@ struct DecodeParams {
   __nv_bfloat16* out;      // [B][H_q][dh]
   float* lse;              // [B][H_q]
   int N, Hq, Hkv, g, n_split;
+  int span;                // positions per range (one partial each)
   float scale_log2;        // scale * log2(e)
 };
+
+// Register-resident split path, for groups of at most four query heads whose
+// K/V head count is a power of two no larger than the rows a CTA takes per
+// step.  L = dh / 8 lanes share one cache row (16 bytes of K and 16 of V
+// each); a CTA of kDecodeThreads takes rows_step(dh) consecutive rows per step.
+constexpr int kRowsMaxGroup = 4;
+constexpr int kRowsMinSteps = 16;  // the shortest range is this many steps
+__host__ __device__ constexpr int rows_step(int dh) { return kDecodeThreads * 8 / dh; }
+__host__ __device__ constexpr bool rows_path(int g, int hkv, int dh) {
+  return g >= 1 && g <= kRowsMaxGroup && hkv >= 1 && (hkv & (hkv - 1)) == 0 && hkv <= rows_step(dh);
+}
+// Shortest range of positions (kRowsMinSteps steps of the CTA).
+__host__ __device__ constexpr int rows_min_span(int dh, int hkv) { return kRowsMinSteps * rows_step(dh) / hkv; }
+// Shared memory of the register-resident path: one (o, m, l) record per
+// thread slot for the end-of-range merge.
+__host__ __device__ constexpr size_t rows_smem_bytes(int g, int dh) {
+  return static_cast<size_t>(rows_step(dh)) * g * (dh + 2) * 4;
+}
 
 // Shared memory of the split kernel, in bytes: queries and running outputs
 // [g][dh] fp32, scores [g][chunk] fp32, two K and two V chunk buffers (bf16),
@@ -75,8 +101,9 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// General split path: any group size, the range's chunks staged in shared memory.
 template <int DH>
-__global__ void __launch_bounds__(kDecodeThreads) sqa_decode_split_kernel(const DecodeParams p) {
+__device__ __forceinline__ void decode_split_general(const DecodeParams& p) {
   constexpr int CH = decode_chunk(DH), VEC = DH / 8;  // 16-byte vectors per row
   const int split = blockIdx.x / p.Hkv, kvh = blockIdx.x % p.Hkv, b = blockIdx.y;
   const int bk = b * p.Hkv + kvh, g = p.g, go = g * DH;
@@ -265,6 +292,221 @@ __global__ void __launch_bounds__(kDecodeThreads) sqa_decode_split_kernel(const 
   }
 }
 
+__device__ __forceinline__ uint4 ld_stream16(const __nv_bfloat16* ptr) {
+  return __ldg(reinterpret_cast<const uint4*>(ptr));
+}
+
+__device__ __forceinline__ float2 bf2f(uint32_t w) {
+  __nv_bfloat162 h;
+  memcpy(&h, &w, 4);
+  return __bfloat1622float2(h);
+}
+
+// One cache row's step of the online softmax for the G heads a thread slot
+// holds: scores from this lane's 8 columns summed over the L lanes of the row
+// (butterfly, so every lane of the row gets the same sum), then either the
+// plain update (no score above its head's running maximum anywhere in the
+// warp) or the rescaling one.
+template <int G, int L>
+__device__ __forceinline__ void rows_update(const uint4& kc, const uint4& vc, bool valid, const float2 (&q)[G][4],
+                                            float2 (&o)[G][4], float (&m)[G], float (&l)[G]) {
+  const float2 k0 = bf2f(kc.x), k1 = bf2f(kc.y), k2 = bf2f(kc.z), k3 = bf2f(kc.w);
+  float sc[G];
+  bool up = false;
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    float2 a = __fmul2_rn(q[h][0], k0);
+    a = __ffma2_rn(q[h][1], k1, a);
+    a = __ffma2_rn(q[h][2], k2, a);
+    a = __ffma2_rn(q[h][3], k3, a);
+    float t = a.x + a.y;
+#pragma unroll
+    for (int off = 1; off < L; off <<= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+    sc[h] = t;
+    up |= t > m[h];
+  }
+  up = up && valid;
+  const float2 v0 = bf2f(vc.x), v1 = bf2f(vc.y), v2 = bf2f(vc.z), v3 = bf2f(vc.w);
+  if (__any_sync(0xffffffffu, up)) {
+    if (valid) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float mn = fmaxf(m[h], sc[h]);
+        const float a = dev::ex2(m[h] - mn);  // 0 while m is -inf
+        const float w = dev::ex2(sc[h] - mn);
+        l[h] = fmaf(l[h], a, w);
+        const float2 a2 = make_float2(a, a), w2 = make_float2(w, w);
+        o[h][0] = __ffma2_rn(o[h][0], a2, __fmul2_rn(w2, v0));
+        o[h][1] = __ffma2_rn(o[h][1], a2, __fmul2_rn(w2, v1));
+        o[h][2] = __ffma2_rn(o[h][2], a2, __fmul2_rn(w2, v2));
+        o[h][3] = __ffma2_rn(o[h][3], a2, __fmul2_rn(w2, v3));
+        m[h] = mn;
+      }
+    }
+  } else if (valid) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float w = dev::ex2(sc[h] - m[h]);
+      l[h] += w;
+      const float2 w2 = make_float2(w, w);
+      o[h][0] = __ffma2_rn(w2, v0, o[h][0]);
+      o[h][1] = __ffma2_rn(w2, v1, o[h][1]);
+      o[h][2] = __ffma2_rn(w2, v2, o[h][2]);
+      o[h][3] = __ffma2_rn(w2, v3, o[h][3]);
+    }
+  }
+}
+
+// Register-resident split path (rows_path(g, H_kv, dh) holds, G = g).
+//
+// The cache of one sequence is [N][H_kv][dh]: N * H_kv rows of dh elements,
+// and a range of positions is one contiguous run of rows.  L = dh / 8 lanes
+// share a row, so one warp load covers 32 / L whole consecutive rows (full
+// 128-byte lines).  Thread slot t (L lanes) takes rows t, t + STEP, ... of
+// the run; STEP is a multiple of H_kv, so the slot always meets K/V head
+// t mod H_kv.  It keeps that head's G queries (its 8 columns, in log2 units),
+// its own running maxima, sums and outputs in registers, and the loads of the
+// next IN_FLIGHT rows in flight; nothing is shared during the run.  At the end
+// the slots of each head merge (warp butterfly over slots of the same head,
+// then one record per remaining slot in shared memory) into the partial
+// (o, m, l) per head that the general path writes.
+template <int DH, int G>
+__device__ __forceinline__ void decode_split_rows(const DecodeParams& p) {
+  constexpr int L = DH / 8, P = 32 / L, STEP = rows_step(DH), REC = G * (DH + 2);
+  constexpr int IN_FLIGHT = G <= 2 ? 4 : 2;
+  static_assert(STEP == (kDecodeThreads / 32) * P, "a step is one row per thread slot");
+  const int split = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int slot = lane / L, col = (lane % L) * 8;
+  const int t = warp * P + slot;
+  const int Hkv = p.Hkv, kvh = t & (Hkv - 1);
+  const int len = decode_len(p, b);
+  const int j0 = split * p.span, j1 = min(len, j0 + p.span);
+  const long long n_rows = static_cast<long long>(max(j1 - j0, 0)) * Hkv;
+  const size_t first = (static_cast<size_t>(b) * p.N + (j0 < len ? j0 : 0)) * Hkv;
+  const __nv_bfloat16* kr = p.k + first * DH + col;
+  const __nv_bfloat16* vr = p.v + first * DH + col;
+
+  float2 q[G][4], o[G][4];
+  float m[G], l[G];
+  {
+    const __nv_bfloat16* qg = p.q + (static_cast<size_t>(b) * p.Hq + static_cast<size_t>(kvh) * G) * DH + col;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const uint4 u = *reinterpret_cast<const uint4*>(qg + h * DH);
+      const float2 s2 = make_float2(p.scale_log2, p.scale_log2);
+      q[h][0] = __fmul2_rn(bf2f(u.x), s2);
+      q[h][1] = __fmul2_rn(bf2f(u.y), s2);
+      q[h][2] = __fmul2_rn(bf2f(u.z), s2);
+      q[h][3] = __fmul2_rn(bf2f(u.w), s2);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[h][e] = make_float2(0.f, 0.f);
+      m[h] = -INFINITY;
+      l[h] = 0.f;
+    }
+  }
+
+  const int n_steps = static_cast<int>((n_rows + STEP - 1) / STEP);  // the same for every thread
+  uint4 kq[IN_FLIGHT], vq[IN_FLIGHT];
+#pragma unroll
+  for (int i = 0; i < IN_FLIGHT; ++i) {
+    const long long r = t + static_cast<long long>(i) * STEP;
+    kq[i] = make_uint4(0, 0, 0, 0);
+    vq[i] = kq[i];
+    if (r < n_rows) {
+      kq[i] = ld_stream16(kr + r * DH);
+      vq[i] = ld_stream16(vr + r * DH);
+    }
+  }
+  for (int s0 = 0; s0 < n_steps; s0 += IN_FLIGHT) {
+#pragma unroll
+    for (int i = 0; i < IN_FLIGHT; ++i) {
+      const int st = s0 + i;
+      if (st >= n_steps) break;
+      const long long r = t + static_cast<long long>(st) * STEP;
+      const uint4 kc = kq[i], vc = vq[i];
+      const long long rn = r + static_cast<long long>(IN_FLIGHT) * STEP;
+      if (rn < n_rows) {
+        kq[i] = ld_stream16(kr + rn * DH);
+        vq[i] = ld_stream16(vr + rn * DH);
+      }
+      rows_update<G, L>(kc, vc, r < n_rows, q, o, m, l);
+    }
+  }
+
+  // Merge the slots of one head inside the warp: slot offsets that are
+  // multiples of H_kv (a power of two) keep the head and the columns.
+  for (int off = Hkv * L; off < 32; off <<= 1) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float mo = __shfl_xor_sync(0xffffffffu, m[h], off);
+      const float lo = __shfl_xor_sync(0xffffffffu, l[h], off);
+      const float mn = fmaxf(m[h], mo);
+      const float a = m[h] == -INFINITY ? 0.f : dev::ex2(m[h] - mn);
+      const float c = mo == -INFINITY ? 0.f : dev::ex2(mo - mn);
+      l[h] = l[h] * a + lo * c;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float ox = __shfl_xor_sync(0xffffffffu, o[h][e].x, off);
+        const float oy = __shfl_xor_sync(0xffffffffu, o[h][e].y, off);
+        o[h][e] = make_float2(o[h][e].x * a + ox * c, o[h][e].y * a + oy * c);
+      }
+      m[h] = mn;
+    }
+  }
+
+  // One record per slot that still holds a distinct part: slots below
+  // min(H_kv, P) of every warp.
+  extern __shared__ __align__(16) uint8_t dsm[];
+  float* rec = reinterpret_cast<float*>(dsm);  // [STEP][G][DH + 2]
+  const int held = Hkv < P ? Hkv : P;
+  if (slot < held) {
+    float* rt = rec + t * REC;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        rt[h * (DH + 2) + col + 2 * e] = o[h][e].x;
+        rt[h * (DH + 2) + col + 2 * e + 1] = o[h][e].y;
+      }
+      if (col == 0) {
+        rt[h * (DH + 2) + DH] = m[h];
+        rt[h * (DH + 2) + DH + 1] = l[h];
+      }
+    }
+  }
+  __syncthreads();
+
+  // Holders of head kvh: slot kvh of every warp (H_kv <= P), or the slots
+  // kvh, kvh + H_kv, ... (H_kv > P).
+  const int n_hold = Hkv <= P ? kDecodeThreads / 32 : STEP / Hkv;
+  for (int i = tid; i < Hkv * REC; i += kDecodeThreads) {
+    const int hk = i / REC, rem = i % REC, h = rem / (DH + 2), c = rem % (DH + 2);
+    auto holder = [&](int k) { return Hkv <= P ? k * P + hk : hk + k * Hkv; };
+    float M = -INFINITY;
+    for (int k = 0; k < n_hold; ++k) M = fmaxf(M, rec[holder(k) * REC + h * (DH + 2) + DH]);
+    float val = M;
+    if (c != DH) {
+      val = 0.f;
+      for (int k = 0; k < n_hold; ++k) {
+        const float* rk = rec + holder(k) * REC + h * (DH + 2);
+        const float w = rk[DH] == -INFINITY ? 0.f : dev::ex2(rk[DH] - M);
+        val = fmaf(rk[c], w, val);
+      }
+    }
+    p.part[((static_cast<size_t>(b) * Hkv + hk) * p.n_split + split) * REC + rem] = val;
+  }
+}
+
+template <int DH, int G>
+__global__ void __launch_bounds__(kDecodeThreads, G == 0 ? 1 : 2) sqa_decode_split_kernel(const DecodeParams p) {
+  if constexpr (G == 0) {
+    decode_split_general<DH>(p);
+  } else {
+    decode_split_rows<DH, G>(p);
+  }
+}
+
 template <int DH>
 __global__ void __launch_bounds__(kDecodeThreads) sqa_decode_combine_kernel(const DecodeParams p) {
   constexpr int SL = kDecodeThreads / DH;  // chunks handled side by side
@@ -274,7 +516,7 @@ __global__ void __launch_bounds__(kDecodeThreads) sqa_decode_combine_kernel(cons
   const size_t stride = static_cast<size_t>(p.g) * (DH + 2);
   const float* part =
       p.part + static_cast<size_t>(b * p.Hkv + kvh) * p.n_split * stride + static_cast<size_t>(hg) * (DH + 2);
-  const int n_used = (decode_len(p, b) + decode_span(DH) - 1) / decode_span(DH);
+  const int n_used = (decode_len(p, b) + p.span - 1) / p.span;
   __shared__ float red[kDecodeThreads];
   __shared__ float big_m;
 

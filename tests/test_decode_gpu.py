@@ -1,7 +1,10 @@
 """GPU parity of sqa_decode (one new token per sequence against its key/value
 cache) with the fp64 oracle, on seeded inputs; ragged cache lengths, group
-sizes 1-128, every head dim, a one-entry cache, the whole cache, an empty
-sequence, and the full-size decoding workloads."""
+sizes 1-128, every head dim, K/V head counts that are and are not powers of
+two (the register-resident split path takes groups of at most four heads with a
+power-of-two K/V head count, the shared-memory path the rest), a one-entry
+cache, the whole cache, an empty sequence, and the full-size decoding
+workloads."""
 import numpy as np
 import pytest
 import torch
@@ -34,6 +37,10 @@ CASES = [
     ((2, 1, 8, 4, 16), None),
     ((2, 3000, 128, 1, 16), [2999, 3]),
     ((2, 520, 16, 2, 128), [520, 131]),
+    ((1, 400, 32, 8, 64), None),
+    ((2, 300, 16, 16, 128), [300, 17]),
+    ((2, 500, 6, 3, 32), [500, 250]),
+    ((1, 5000, 8, 2, 128), [4999]),
 ]
 
 
