@@ -70,10 +70,17 @@ __host__ __device__ constexpr bool rows_path(int g, int hkv, int dh) {
 }
 // Shortest range of positions (kRowsMinSteps steps of the CTA).
 __host__ __device__ constexpr int rows_min_span(int dh, int hkv) { return kRowsMinSteps * rows_step(dh) / hkv; }
-// Shared memory of the register-resident path: one (o, m, l) record per
+// Rows in flight per thread of the register-resident path, and its ring of
+// shared-memory slots (one more than that, so a refill never targets the slot
+// being read).
+constexpr int kRowsDepth = 10, kRowsSlots = kRowsDepth + 1;
+// Shared memory of the register-resident path: the per-thread ring of K and V
+// row pieces (16 bytes each) during the run, then one (o, m, l) record per
 // thread slot for the end-of-range merge.
 __host__ __device__ constexpr size_t rows_smem_bytes(int g, int dh) {
-  return static_cast<size_t>(rows_step(dh)) * g * (dh + 2) * 4;
+  const size_t ring = static_cast<size_t>(kRowsSlots) * kDecodeThreads * 32;
+  const size_t recs = static_cast<size_t>(rows_step(dh)) * g * (dh + 2) * 4;
+  return ring > recs ? ring : recs;
 }
 
 // Shared memory of the split kernel, in bytes: queries and running outputs
@@ -292,10 +299,6 @@ __device__ __forceinline__ void decode_split_general(const DecodeParams& p) {
   }
 }
 
-__device__ __forceinline__ uint4 ld_stream16(const __nv_bfloat16* ptr) {
-  return __ldg(reinterpret_cast<const uint4*>(ptr));
-}
-
 __device__ __forceinline__ float2 bf2f(uint32_t w) {
   __nv_bfloat162 h;
   memcpy(&h, &w, 4);
@@ -365,15 +368,15 @@ __device__ __forceinline__ void rows_update(const uint4& kc, const uint4& vc, bo
 // 128-byte lines).  Thread slot t (L lanes) takes rows t, t + STEP, ... of
 // the run; STEP is a multiple of H_kv, so the slot always meets K/V head
 // t mod H_kv.  It keeps that head's G queries (its 8 columns, in log2 units),
-// its own running maxima, sums and outputs in registers, and the loads of the
-// next IN_FLIGHT rows in flight; nothing is shared during the run.  At the end
+// its own running maxima, sums and outputs in registers, and the copies of
+// its next kRowsDepth rows in flight through a private ring of shared-memory
+// slots; nothing is shared between threads during the run.  At the end
 // the slots of each head merge (warp butterfly over slots of the same head,
 // then one record per remaining slot in shared memory) into the partial
 // (o, m, l) per head that the general path writes.
 template <int DH, int G>
 __device__ __forceinline__ void decode_split_rows(const DecodeParams& p) {
   constexpr int L = DH / 8, P = 32 / L, STEP = rows_step(DH), REC = G * (DH + 2);
-  constexpr int IN_FLIGHT = G <= 2 ? 4 : 2;
   static_assert(STEP == (kDecodeThreads / 32) * P, "a step is one row per thread slot");
   const int split = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -406,33 +409,33 @@ __device__ __forceinline__ void decode_split_rows(const DecodeParams& p) {
     }
   }
 
+  // Each thread streams its rows through its own ring of shared-memory slots
+  // with cp.async (16 bytes of K and 16 of V per row), kRowsDepth rows ahead;
+  // it reads back only what it copied itself, so no barrier is needed.
+  extern __shared__ __align__(16) uint8_t dsm[];
+  uint4* ring_k = reinterpret_cast<uint4*>(dsm);  // [kRowsSlots][kDecodeThreads]
+  uint4* ring_v = ring_k + kRowsSlots * kDecodeThreads;
   const int n_steps = static_cast<int>((n_rows + STEP - 1) / STEP);  // the same for every thread
-  uint4 kq[IN_FLIGHT], vq[IN_FLIGHT];
-#pragma unroll
-  for (int i = 0; i < IN_FLIGHT; ++i) {
-    const long long r = t + static_cast<long long>(i) * STEP;
-    kq[i] = make_uint4(0, 0, 0, 0);
-    vq[i] = kq[i];
+  auto issue = [&](int st) {
+    const long long r = t + static_cast<long long>(st) * STEP;
     if (r < n_rows) {
-      kq[i] = ld_stream16(kr + r * DH);
-      vq[i] = ld_stream16(vr + r * DH);
+      const int sl = st % kRowsSlots;
+      cp_async16(ring_k + sl * kDecodeThreads + tid, kr + r * DH);
+      cp_async16(ring_v + sl * kDecodeThreads + tid, vr + r * DH);
     }
+    cp_async_commit();  // one group per step, empty past the run
+  };
+#pragma unroll 1
+  for (int i = 0; i < kRowsDepth; ++i) issue(i);
+#pragma unroll 1
+  for (int st = 0; st < n_steps; ++st) {
+    issue(st + kRowsDepth);          // slot (st - 1) mod kRowsSlots, read in the previous step
+    cp_async_wait<kRowsDepth>();     // every group but the newest kRowsDepth: step st has landed
+    const int sl = st % kRowsSlots;
+    const uint4 kc = ring_k[sl * kDecodeThreads + tid], vc = ring_v[sl * kDecodeThreads + tid];
+    rows_update<G, L>(kc, vc, t + static_cast<long long>(st) * STEP < n_rows, q, o, m, l);
   }
-  for (int s0 = 0; s0 < n_steps; s0 += IN_FLIGHT) {
-#pragma unroll
-    for (int i = 0; i < IN_FLIGHT; ++i) {
-      const int st = s0 + i;
-      if (st >= n_steps) break;
-      const long long r = t + static_cast<long long>(st) * STEP;
-      const uint4 kc = kq[i], vc = vq[i];
-      const long long rn = r + static_cast<long long>(IN_FLIGHT) * STEP;
-      if (rn < n_rows) {
-        kq[i] = ld_stream16(kr + rn * DH);
-        vq[i] = ld_stream16(vr + rn * DH);
-      }
-      rows_update<G, L>(kc, vc, r < n_rows, q, o, m, l);
-    }
-  }
+  cp_async_wait<0>();
 
   // Merge the slots of one head inside the warp: slot offsets that are
   // multiples of H_kv (a power of two) keep the head and the columns.
@@ -456,8 +459,8 @@ __device__ __forceinline__ void decode_split_rows(const DecodeParams& p) {
   }
 
   // One record per slot that still holds a distinct part: slots below
-  // min(H_kv, P) of every warp.
-  extern __shared__ __align__(16) uint8_t dsm[];
+  // min(H_kv, P) of every warp.  The records reuse the ring's memory.
+  __syncthreads();
   float* rec = reinterpret_cast<float*>(dsm);  // [STEP][G][DH + 2]
   const int held = Hkv < P ? Hkv : P;
   if (slot < held) {
@@ -509,57 +512,62 @@ __global__ void __launch_bounds__(kDecodeThreads, G == 0 ? 1 : 2) sqa_decode_spl
 
 template <int DH>
 __global__ void __launch_bounds__(kDecodeThreads) sqa_decode_combine_kernel(const DecodeParams p) {
-  constexpr int SL = kDecodeThreads / DH;  // chunks handled side by side
-  const int bh = blockIdx.x;               // (batch entry, query head)
+  constexpr int DP = DH / 2, SL = kDecodeThreads / DP;  // column pairs; ranges handled side by side
+  constexpr int NW = kDecodeThreads / 32;
+  const int bh = blockIdx.x;                              // (batch entry, query head)
   const int b = bh / p.Hq, h = bh % p.Hq, kvh = h / p.g, hg = h % p.g;
-  const int tid = threadIdx.x, d = tid % DH, sl = tid / DH;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, dp = tid % DP, sl = tid / DP;
   const size_t stride = static_cast<size_t>(p.g) * (DH + 2);
   const float* part =
       p.part + static_cast<size_t>(b * p.Hkv + kvh) * p.n_split * stride + static_cast<size_t>(hg) * (DH + 2);
   const int n_used = (decode_len(p, b) + p.span - 1) / p.span;
-  __shared__ float red[kDecodeThreads];
-  __shared__ float big_m;
+  __shared__ float2 red[kDecodeThreads];
+  __shared__ float wred[NW];
 
-  // M = largest chunk maximum.
+  // M = largest range maximum (warp shuffles, then one value per warp).
   float m = -INFINITY;
   for (int s = tid; s < n_used; s += kDecodeThreads) m = fmaxf(m, part[s * stride + DH]);
-  red[tid] = m;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) wred[warp] = m;
   __syncthreads();
-  for (int o = kDecodeThreads / 2; o > 0; o >>= 1) {
-    if (tid < o) red[tid] = fmaxf(red[tid], red[tid + o]);
-    __syncthreads();
-  }
-  if (tid == 0) big_m = red[0];
-  __syncthreads();
-  const float M = big_m;
+  float M = wred[0];
+#pragma unroll
+  for (int w = 1; w < NW; ++w) M = fmaxf(M, wred[w]);
 
-  // Column d over the chunks sl, sl + SL, ..., and (column 0's threads) L.
-  float acc = 0.f, L = 0.f;
+  // Columns 2 dp, 2 dp + 1 over the ranges sl, sl + SL, ..., several loads in
+  // flight; the dp = 0 threads also sum L.
+  float2 acc = make_float2(0.f, 0.f);
+  float L = 0.f;
+#pragma unroll 4
   for (int s = sl; s < n_used; s += SL) {
     const float* ps = part + s * stride;
     const float w = dev::ex2(ps[DH] - M);
-    acc = fmaf(ps[d], w, acc);
-    L = fmaf(ps[DH + 1], w, L);
+    const float2 o2 = *reinterpret_cast<const float2*>(ps + 2 * dp);
+    acc.x = fmaf(o2.x, w, acc.x);
+    acc.y = fmaf(o2.y, w, acc.y);
+    if (dp == 0) L = fmaf(ps[DH + 1], w, L);
   }
-  __syncthreads();
   red[tid] = acc;
   __syncthreads();
   if (sl == 0) {
-    for (int k = 1; k < SL; ++k) acc += red[k * DH + d];
+    for (int k = 1; k < SL; ++k) {
+      const float2 r = red[k * DP + dp];
+      acc.x += r.x;
+      acc.y += r.y;
+    }
   }
   __syncthreads();
-  red[tid] = L;
+  if (dp == 0) red[sl] = make_float2(L, 0.f);
   __syncthreads();
-  if (tid == 0) {
-    for (int k = 1; k < SL; ++k) L += red[k * DH];
-    red[0] = L;
-  }
-  __syncthreads();
-  L = red[0];
   if (sl == 0) {
+    L = red[0].x;
+    for (int k = 1; k < SL; ++k) L += red[k].x;
     const float inv = L > 0.f ? 1.f / L : 0.f;
-    p.out[static_cast<size_t>(bh) * DH + d] = __float2bfloat16_rn(acc * inv);
-    if (d == 0) p.lse[bh] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+    __nv_bfloat16* ob = p.out + static_cast<size_t>(bh) * DH + 2 * dp;  // out may be only 2-byte aligned
+    ob[0] = __float2bfloat16_rn(acc.x * inv);
+    ob[1] = __float2bfloat16_rn(acc.y * inv);
+    if (dp == 0) p.lse[bh] = L > 0.f ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
   }
 }
 

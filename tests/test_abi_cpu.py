@@ -131,3 +131,26 @@ def test_decode_rejects_bad_arguments_before_launch(lib):
     assert f(ok[0], 0x2008, ok[2], None, *ok[4:], need, s, 0.0, None) == 2  # cache not 16-byte aligned
     assert f(*ok[:3], None, *ok[4:], need - 1, s, 0.0, None) == 1  # workspace too small
     assert lib.sqa_decode_workspace_bytes(sqa.Shape(0, 300, 8, 4, 16)) == 0
+
+
+def _decode_ws_expected(B, N, Hq, Hkv, dh):
+    """Workspace rule of sqa_decode: one (o, m, l) record of dh + 2 floats per
+    (sequence, K/V head, range, query head of the group), for the most ranges
+    either split path can take: the shared-memory path's fixed ranges (4 chunks
+    of 256/128/64 positions at dh <= 32/64/128) or the register-resident path's
+    shortest range (16 steps of 2048/dh cache rows, i.e. 16 * 2048 / dh / H_kv
+    positions) when the group has at most 4 heads and H_kv is a power of two
+    no larger than 2048/dh."""
+    g = Hq // Hkv
+    span = 4 * (256 if dh <= 32 else (128 if dh == 64 else 64))
+    n = -(-N // span)
+    step = 2048 // dh
+    if 1 <= g <= 4 and Hkv & (Hkv - 1) == 0 and Hkv <= step:
+        n = max(n, -(-N // (16 * step // Hkv)))
+    return -(-(B * Hkv * n * g * (dh + 2) * 4) // 256) * 256
+
+
+@pytest.mark.parametrize("shape", [(32, 32768, 8, 4, 16), (8, 65536, 8, 4, 128), (2, 3000, 128, 1, 16),
+                                   (2, 500, 6, 3, 32), (2, 300, 16, 16, 128), (2, 300, 32, 32, 128), (1, 1, 4, 1, 64)])
+def test_decode_workspace_covers_both_split_paths(lib, shape):
+    assert lib.sqa_decode_workspace_bytes(sqa.Shape(*shape)) == _decode_ws_expected(*shape)
