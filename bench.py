@@ -168,7 +168,7 @@ def cpu_baseline(w, seconds):
             break
     rate = counted_flops(sub) * n / el / 1e12
     return {"value": rate, "unit": "TFLOP/s", "cores": omp_threads(), "kind": "oracle",
-            "sample": f"fp64 oracle fwd{'+bwd' if w.backward else ''} on batch entry 0, KV head 0 and its "
+            "sample": f"fp64 oracle {pass_name(w)} on batch entry 0, KV head 0 and its "
                       f"{sub.Hq} query heads (N={w.N}, dh={w.dh}), {n} runs in {el:.1f} s"}
 
 
@@ -527,7 +527,7 @@ def run_reference(args, w):
     el = time.perf_counter() - t0
     ms = el / steps * 1e3
     value = counted_flops(sub) / (ms * 1e-3) / 1e12
-    sample = (f"fp64 oracle fwd{'+bwd' if w.backward else ''} on batch entry 0, KV head 0 and its {sub.Hq} "
+    sample = (f"fp64 oracle {pass_name(w)} on batch entry 0, KV head 0 and its {sub.Hq} "
               f"query heads (N={w.N}, dh={w.dh}); {steps} of the requested {args.steps} steps run")
     return {"impl": "reference", "metric": f"SQA attention {pass_name(w)} TFLOP/s ({w.note})",
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": ms,
