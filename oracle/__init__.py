@@ -5,9 +5,11 @@ test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import it.  It shares no code with the CUDA path, and the
 library never calls it.
 
-The arithmetic lives in ``sqa_oracle.c`` (plain loops in fp64, OpenMP over
-rows).  This module only builds that file with gcc and marshals numpy arrays.
-Inputs are converted to fp64 before the call; bf16 values convert exactly.
+The attention arithmetic lives in ``sqa_oracle.c`` (plain loops in fp64,
+OpenMP over rows).  This module only builds that file with gcc and marshals
+numpy arrays.  Inputs are converted to fp64 before the call; bf16 values
+convert exactly.  ``layer.py`` adds the full layer around that core
+(projections and rotary embedding, in numpy fp64).
 
 What is computed follows the SQAT-m model card ("Architecture details": 16
 heads for the dimension split, 8 query groups, 4 key/value groups; "Model size
