@@ -33,13 +33,16 @@ def _rank_main(rank, world, port, out_dir):
 
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
     import bench
-    from sparse_query_attention_sqa_b200.inputs import WORKLOADS, workload_inputs
+    from sparse_query_attention_sqa_b200.inputs import WORKLOADS, make_decode_inputs, workload_inputs
 
     w = WORKLOADS["sqatm_layer_fwd"]
     # Step times that differ by rank: every rank must see the slowest one.
     ms = bench.max_over_ranks(1.0 + 0.25 * rank, world, "cpu")
     q, _, _, _ = workload_inputs(w, seed=rank)
-    torch.save({"ms": ms, "q": q, "value": bench.job_tflops(w, world, ms)}, os.path.join(out_dir, f"r{rank}.pt"))
+    wd = WORKLOADS["decode_sqatm"]
+    qd = make_decode_inputs(2, 64, wd.Hq, wd.Hkv, wd.dh, seed=rank)[0]
+    torch.save({"ms": ms, "q": q, "qd": qd, "value": bench.job_tflops(w, world, ms),
+                "value_decode": bench.job_tflops(wd, world, ms)}, os.path.join(out_dir, f"r{rank}.pt"))
     dist.barrier()
     dist.destroy_process_group()
 
@@ -67,9 +70,31 @@ def test_job_throughput_counts_every_rank(two_ranks):
 
 
 def test_ranks_draw_independent_inputs(two_ranks):
-    a, b = two_ranks[0]["q"], two_ranks[1]["q"]
-    assert a.shape == b.shape and a.dtype == torch.bfloat16
-    assert not torch.equal(a, b)
+    for key in ("q", "qd"):
+        a, b = two_ranks[0][key], two_ranks[1][key]
+        assert a.shape == b.shape and a.dtype == torch.bfloat16
+        assert not torch.equal(a, b)
+
+
+def test_decoding_job_throughput_counts_every_rank(two_ranks):
+    sys.path.insert(0, ROOT)
+    import bench
+    from sparse_query_attention_sqa_b200.inputs import WORKLOADS
+
+    w = WORKLOADS["decode_sqatm"]
+    # one query row per (sequence, head) against the whole cache, on each rank
+    per_rank = 4.0 * w.B * w.Hq * w.N * w.dh / 1.25e-3 / 1e12
+    assert two_ranks[0]["value_decode"] == pytest.approx(2 * per_rank)
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    from sparse_query_attention_sqa_b200.inputs import WORKLOADS
+
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert bench.run_reference(None, WORKLOADS["decode_sqatm"]) is None
 
 
 def test_single_rank_reduction_is_the_identity():
