@@ -270,7 +270,7 @@ def _drop_wait(role_prefix, barrier):
     return drop
 
 
-# Waits whose removal the model must notice.  (Three other waits of the kernel
+# Waits whose removal the model must notice.  (Two other waits of the kernel
 # are implied by the rest of the protocol and the model shows no failure
 # without them: the DV/DK issuers' dkv_free wait, because their next ds_ready
 # wait already follows every warp's dV/dK epilogue, and issuer A's dq_empty
@@ -304,6 +304,25 @@ def test_model_detects_a_dropped_wait(name):
         except AssertionError:
             failures += 1
     assert failures > 0, name
+
+
+def test_model_detects_the_wait_before_the_dq_epilogue_missing():
+    """The warps' wait for the dQ MMA of tile G - 1 (just before they signal
+    their dS of tile G) also guards their read of that dQ from TMEM: without it
+    the read can start before the MMA has written it."""
+    rnd = random.Random(3)
+    failures = 0
+    for trial in range(150):
+        nqs = [rnd.randint(2, 6) for _ in range(rnd.randint(1, 4))]
+        ops = _roles(nqs, 2)[0]["warp0"]
+        before_signal = {ops[i] for i in range(len(ops) - 1)
+                         if ops[i][0] == "wait" and ops[i][1].startswith("dq_full")
+                         and ops[i + 1][0] == "end" and ops[i + 1][1][0] == "stage"}
+        try:
+            run(nqs, 2, trial, drop=lambda r, op: r.startswith("warp") and op in before_signal)
+        except AssertionError:
+            failures += 1
+    assert failures > 0
 
 
 def test_model_detects_the_hoisted_dq_wait_missing():
