@@ -25,6 +25,7 @@ cover the interleavings a GPU may produce.
 import random
 
 import pytest
+import sync_model
 
 NBUF = 3  # S^T / dP^T TMEM buffers
 NWG = 2   # softmax warpgroups
@@ -182,77 +183,13 @@ def _roles(nqs, QS):
     return roles, cnt
 
 
-class _Buffer:
-    """Version and stage of one buffer, and its users."""
-
-    def __init__(self, stages):
-        self.stages = stages
-        self.version, self.stage, self.ended, self.active = None, None, 0, 0
-
-    def begin(self, v, k):
-        n = len(self.stages)
-        if (v, k) == (self.version, self.stage):
-            assert self.ended + self.active < self.stages[k][1], "more users than the stage has"
-        else:
-            if self.version is not None:
-                assert self.active == 0 and self.ended == self.stages[self.stage][1], \
-                    f"hazard: '{self.stages[k][0]}' v{v} starts while '{self.stages[self.stage][0]}' " \
-                    f"v{self.version} has {self.active} active and {self.ended} finished users"
-            nxt = (self.version, self.stage + 1) if self.version is not None and self.stage + 1 < n else None
-            assert (v, k) == nxt or (k == 0 and (self.version is None or (self.stage == n - 1 and v > self.version))), \
-                f"hazard: '{self.stages[k][0]}' v{v} out of order (at v{self.version} stage {self.stage})"
-            self.version, self.stage, self.ended = v, k, 0
-        self.active += 1
-
-    def end(self, v, k):
-        assert (v, k) == (self.version, self.stage) and self.active > 0
-        self.active -= 1
-        self.ended += 1
-
-
 def run(nqs, QS, seed, drop=None):
-    """drop(role, op) -> True removes that op (used only to show that the
-    model notices a missing wait)."""
+    """One random schedule.  drop(role, op) -> True removes that op (used only
+    to show that the model notices a missing wait)."""
     roles, cnt = _roles(nqs, QS)
     if drop is not None:
         roles = {r: [op for op in ops if not drop(r, op)] for r, ops in roles.items()}
-    done = {b: 0 for b in cnt}
-    arrived = {b: 0 for b in cnt}
-    bufs = {}
-    pc = {r: 0 for r in roles}
-    rnd = random.Random(seed)
-    while True:
-        ready = []
-        for r, ops in roles.items():
-            if pc[r] == len(ops):
-                continue
-            op = ops[pc[r]]
-            if op[0] != "wait":
-                ready.append(r)
-            else:
-                _, b, k = op
-                assert done[b] < k + 2, f"phase aliasing: {r} waits on {b} phase {k} after {done[b]} completions"
-                if done[b] == k + 1:
-                    ready.append(r)
-        if not ready:
-            break
-        r = rnd.choice(ready)
-        op = roles[r][pc[r]]
-        pc[r] += 1
-        if op[0] == "arrive":
-            _, b, m = op
-            arrived[b] += m
-            assert arrived[b] <= cnt[b], f"over-arrival on {b}"
-            if arrived[b] == cnt[b]:
-                arrived[b] = 0
-                done[b] += 1
-        elif op[0] in ("begin", "end"):
-            _, key, v, k = op
-            buf = bufs.setdefault(key, _Buffer(STAGES[key[0]]))
-            (buf.begin if op[0] == "begin" else buf.end)(v, k)
-    stuck = {r: roles[r][pc[r]] for r in roles if pc[r] < len(roles[r])}
-    assert not stuck, f"deadlock: {stuck}"
-    assert all(a == 0 for a in arrived.values())  # every phase that was started was completed
+    sync_model.run(roles, cnt, STAGES, seed)
 
 
 @pytest.mark.parametrize("QS", [2, 4])

@@ -1,0 +1,272 @@
+"""A model of the synchronisation of the persistent forward kernel
+(``sqa_fwd_kernel``), run on the CPU under random schedules.
+
+Roles, in the kernel's program order: the TMA producer (a pair of Q tiles per
+work item into one of QBUF buffers, K/V tiles into a ring of STAGES), one MMA
+issuer per Q tile (S = Q K^T into two TMEM buffers per tile, O += P V), and
+the four softmax warps of each tile (P written over S in place, an occasional
+rescale of O, the epilogue).  Barrier arrival counts are the kernel's.
+
+Buffers checked by stage (see ``sync_model``): the Q buffers (producer writes,
+both issuers read), the K/V stages (producer writes, both issuers read until
+their release), and each tile's two S/P buffers (issuer's S MMA writes, the
+4 warps rewrite P, the P V MMA reads).  The O accumulator of each tile is
+shared by interleaved users and gets its own checker: no P V MMA, rescale or
+epilogue read overlaps another user, a rescale at step G comes after P V of
+step G - 1 completed and before P V of step G starts, the epilogue comes after
+the item's last P V, and the next item's first P V after all 4 warps have read
+O.  Whether a warp rescales O at a step depends on the data, so each step
+draws it at random.
+
+Work lists mirror the kernel's items: per item, nkv0 key tiles for Q tile 0,
+nkv1 for Q tile 1 (0 when the item has one tile; one more than nkv0 under a
+causal mask when the tiles straddle a key-tile boundary) and nkv = max of the
+two loaded.  Both buffer configurations of the kernel are run: QBUF 2 with 8
+stages (dh <= 32), QBUF 2 with 4 stages (dh 64) and QBUF 1 with 3 (dh 128).
+"""
+import random
+
+import pytest
+import sync_model
+
+WARPS_PER_TILE = 4
+
+STAGES = {
+    "q": [("producer writes the Q pair", 1), ("both issuers read", 2)],
+    "kv": [("producer writes K, V", 1), ("both issuers read", 2)],
+    "S0": [("issuer 0 writes S", 1), ("tile 0 warps write P", WARPS_PER_TILE), ("issuer 0 reads P (P V)", 1)],
+    "S1": [("issuer 1 writes S", 1), ("tile 1 warps write P", WARPS_PER_TILE), ("issuer 1 reads P (P V)", 1)],
+}
+
+
+class Accumulator:
+    """Users of one tile's O accumulator in TMEM."""
+
+    def __init__(self):
+        self.pv_started = self.pv_done = 0  # P V steps (across items)
+        self.active = {}                    # kind -> active users
+        self.epi_ended = {}                 # item -> warps that finished the epilogue
+
+    def _alone(self, kind):
+        others = {k: n for k, n in self.active.items() if k != kind and n}
+        assert not others, f"hazard on O: {kind} overlaps {others}"
+
+    def begin(self, slot, info):
+        kind = info[0]
+        self._alone(kind)
+        if kind == "pv":
+            _, step, item, first = info
+            assert self.active.get("pv", 0) == 0 and self.pv_started == step == self.pv_done, \
+                f"hazard on O: P V step {step} out of order"
+            if first and item > 0:
+                assert self.epi_ended.get(item - 1, 0) == WARPS_PER_TILE, \
+                    f"hazard on O: item {item} overwrites O before its epilogue read item {item - 1}"
+            self.pv_started += 1
+        elif kind == "rescale":
+            _, step = info
+            assert self.pv_done == step and self.pv_started == step, \
+                f"hazard on O: rescale at step {step} with {self.pv_done} P V done, {self.pv_started} started"
+        else:  # epilogue
+            _, item, steps_end = info
+            assert self.pv_done == steps_end, f"hazard on O: epilogue of item {item} before its last P V"
+        self.active[kind] = self.active.get(kind, 0) + 1
+
+    def end(self, slot, info):
+        kind = info[0]
+        self.active[kind] -= 1
+        if kind == "pv":
+            self.pv_done += 1
+        elif kind == "epi":
+            self.epi_ended[info[1]] = self.epi_ended.get(info[1], 0) + 1
+
+
+def _roles(items, QB, ST, rnd):
+    """items: [(nkv0, nkv1)] per work item of one CTA."""
+    cnt = {}
+    for qb in range(QB):
+        cnt[f"q_full{qb}"] = 1
+        cnt[f"q_empty{qb}"] = 2
+    for s in range(ST):
+        cnt[f"kv_full{s}"] = 1
+        cnt[f"kv_empty{s}"] = 2
+    for t in range(2):
+        for buf in range(2):
+            cnt[f"s_full{t}{buf}"] = 1
+            cnt[f"p_full{t}{buf}"] = 32 * WARPS_PER_TILE
+        cnt[f"o_done{t}"] = 1
+        cnt[f"o_final{t}"] = 1
+        cnt[f"o_free{t}"] = 32 * WARPS_PER_TILE
+
+    def W(b, k):
+        return ("wait", b, k)
+
+    def A(b, m=1):
+        return ("arrive", b, m)
+
+    def B(res, slot, v, stage=None):
+        return ("begin", (res, slot), v, stage)
+
+    def E(res, slot, v, stage=None):
+        return ("end", (res, slot), v, stage)
+
+    prod, g = [], 0
+    for r, (n0, n1) in enumerate(items):
+        qb, nkv = r % QB, max(n0, n1)
+        if r >= QB:
+            prod.append(W(f"q_empty{qb}", r // QB - 1))
+        prod += [B("q", qb, r, 0), E("q", qb, r, 0), A(f"q_full{qb}")]
+        for j in range(nkv):
+            s = (g + j) % ST
+            if g + j >= ST:
+                prod.append(W(f"kv_empty{s}", (g + j) // ST - 1))
+            prod += [B("kv", s, g + j, 0), E("kv", s, g + j, 0), A(f"kv_full{s}")]
+        g += nkv
+
+    def issuer(t):
+        ops, g, G, nd, loaded = [], 0, 0, 0, [0]
+        S = f"S{t}"
+
+        def ensure(gj):
+            out = []
+            while loaded[0] <= gj:
+                out.append(W(f"kv_full{loaded[0] % ST}", loaded[0] // ST))
+                loaded[0] += 1
+            return out
+
+        def qk(qb, gj, step):  # S of key tile gj into buffer step & 1; the MMA reads Q and K
+            return [B(S, step & 1, step, 0), E(S, step & 1, step, 0), A(f"s_full{t}{step & 1}")]
+
+        for r, (n0, n1) in enumerate(items):
+            nkv_t, nkv, qb = (n1 if t else n0), max(n0, n1), r % QB
+            ops += [W(f"q_full{qb}", r // QB), B("q", qb, r, 1)]
+            for j in range(min(2, nkv_t)):
+                ops += ensure(g + j) + [B("kv", (g + j) % ST, g + j, 1)] + qk(qb, g + j, G + j)
+            for j in range(nkv_t):
+                step = G + j
+                ops.append(W(f"p_full{t}{step & 1}", step >> 1))
+                if j == 0 and nd > 0:
+                    ops.append(W(f"o_free{t}", nd - 1))
+                # P V: reads P from the S buffer and V, accumulates into O; MMAs of one
+                # issuer run in order, so its read of P ends before the next S MMA.
+                ops += [B(S, step & 1, step, 2), B("O", t, ("pv", step, nd, j == 0)),
+                        E(S, step & 1, step, 2), E("O", t, ("pv",)), A(f"o_done{t}")]
+                if j + 2 < nkv_t:
+                    ops += ensure(g + j + 2) + [B("kv", (g + j + 2) % ST, g + j + 2, 1)] + qk(qb, g + j + 2, step + 2)
+                if j + 1 == nkv_t:
+                    ops.append(A(f"o_final{t}"))
+                ops += [E("kv", (g + j) % ST, g + j, 1), A(f"kv_empty{(g + j) % ST}")]
+            for j in range(nkv_t, nkv):  # tiles the other Q tile needs: released once loaded
+                ops += ensure(g + j) + [B("kv", (g + j) % ST, g + j, 1), E("kv", (g + j) % ST, g + j, 1),
+                                        A(f"kv_empty{(g + j) % ST}")]
+            ops += [E("q", qb, r, 1), A(f"q_empty{qb}")]
+            G += nkv_t
+            nd += 1 if nkv_t else 0
+            g += nkv
+        return ops
+
+    def softmax_warp(t):
+        ops, G, nd = [], 0, 0
+        S = f"S{t}"
+        for (n0, n1) in items:
+            nkv_t = n1 if t else n0
+            if nkv_t == 0:
+                continue
+            for j in range(nkv_t):
+                step = G + j
+                ops += [W(f"s_full{t}{step & 1}", step >> 1), B(S, step & 1, step, 1)]
+                if j > 0 and rnd.random() < 0.5:  # the running maximum rose: rescale O
+                    ops += [W(f"o_done{t}", step - 1), B("O", t, ("rescale", step)), E("O", t, ("rescale",))]
+                ops += [E(S, step & 1, step, 1), A(f"p_full{t}{step & 1}", 32)]
+            ops += [W(f"o_final{t}", nd), B("O", t, ("epi", nd, G + nkv_t)), E("O", t, ("epi", nd)),
+                    A(f"o_free{t}", 32)]
+            G += nkv_t
+            nd += 1
+        return ops
+
+    roles = {"producer": prod, "issuer0": issuer(0), "issuer1": issuer(1)}
+    for w in range(2 * WARPS_PER_TILE):
+        roles[f"warp{w}"] = softmax_warp(w // WARPS_PER_TILE)
+    return roles, cnt
+
+
+def _items(rnd):
+    out = []
+    for _ in range(rnd.randint(1, 5)):
+        kind = rnd.random()
+        n0 = rnd.randint(1, 6)
+        if kind < 0.15:
+            out.append((n0, 0))        # last, single-tile item
+        elif kind < 0.6:
+            out.append((n0, n0 + 1))   # causal: tile 1 needs one more key tile
+        else:
+            out.append((n0, n0))       # bidirectional, or both tiles in one key tile
+    return out
+
+
+def run(items, QB, ST, seed, drop=None):
+    rnd = random.Random(seed)
+    roles, cnt = _roles(items, QB, ST, rnd)
+    if drop is not None:
+        roles = {r: [op for op in ops if not drop(r, op)] for r, ops in roles.items()}
+    sync_model.run(roles, cnt, STAGES, seed, custom={"O": _OCheck()})
+
+
+class _OCheck:
+    """One Accumulator per Q tile."""
+
+    def __init__(self):
+        self.acc = {0: Accumulator(), 1: Accumulator()}
+
+    def begin(self, slot, info):
+        self.acc[slot].begin(slot, info)
+
+    def end(self, slot, info):
+        self.acc[slot].end(slot, info)
+
+
+@pytest.mark.parametrize("QB,ST", [(2, 8), (2, 4), (1, 3)])
+def test_forward_protocol_has_no_deadlock_aliasing_or_hazard(QB, ST):
+    rnd = random.Random(QB * 10 + ST)
+    for trial in range(150):
+        items = _items(rnd)
+        for seed in range(3):
+            run(items, QB, ST, trial * 100 + seed)
+
+
+def _drop(role_prefix, barrier):
+    return lambda r, op: r.startswith(role_prefix) and op[0] == "wait" and op[1].startswith(barrier)
+
+
+# Waits whose removal the model must notice.  (The issuers' o_free wait is
+# implied by the rest of the protocol: the first P V of the next item also
+# waits for p_full of that step, which every warp signals only after its
+# epilogue has read O.  The kernel keeps it as a second guard.)
+DROPS = {
+    # the warps would rescale O while a P V MMA still accumulates into it
+    "warps: o_done": _drop("warp", "o_done"),
+    # P V would read P before the warps wrote it
+    "issuer: p_full": _drop("issuer", "p_full"),
+    # the warps would read S before the MMA wrote it
+    "warps: s_full": _drop("warp", "s_full"),
+    # the epilogue would read O before the last P V
+    "warps: o_final": _drop("warp", "o_final"),
+    # the producer would overwrite a K/V stage or a Q buffer still in use
+    "producer: kv_empty": _drop("producer", "kv_empty"),
+    "producer: q_empty": _drop("producer", "q_empty"),
+    # an issuer would read K/V or Q before they landed
+    "issuer: kv_full": _drop("issuer", "kv_full"),
+    "issuer: q_full": _drop("issuer", "q_full"),
+}
+
+
+@pytest.mark.parametrize("name", list(DROPS))
+def test_model_detects_a_dropped_wait(name):
+    rnd = random.Random(17)
+    failures = 0
+    for trial in range(150):
+        items = _items(rnd)
+        try:
+            run(items, 2, 4, trial, drop=DROPS[name])
+        except AssertionError:
+            failures += 1
+    assert failures > 0, name
