@@ -18,8 +18,8 @@ The model fails on
   users; a use that starts before every user of the previous stage (or of the
   previous version) has finished is a hazard.
 
-Random schedules over random work lists (items of 1-6 Q tiles, several items
-per CTA) and both Q/dO stage counts the kernel uses (4 at dh 16, 2 at dh 32)
+The checker is ``sync_model.run``.  Random schedules over random work lists
+(items of 1-6 Q tiles, several items per CTA) and both Q/dO stage counts the kernel uses (4 at dh 16, 2 at dh 32)
 cover the interleavings a GPU may produce.
 """
 import random
