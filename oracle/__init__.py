@@ -9,7 +9,8 @@ The attention arithmetic lives in ``sqa_oracle.c`` (plain loops in fp64,
 OpenMP over rows).  This module only builds that file with gcc and marshals
 numpy arrays.  Inputs are converted to fp64 before the call; bf16 values
 convert exactly.  ``layer.py`` adds the full layer around that core
-(projections and rotary embedding, in numpy fp64).
+(projections and rotary embedding, in numpy fp64), ``block.py`` one decoder
+block around the layer (RMSNorm, SwiGLU feed-forward, residuals).
 
 What is computed follows the SQAT-m model card ("Architecture details": 16
 heads for the dimension split, 8 query groups, 4 key/value groups; "Model size
