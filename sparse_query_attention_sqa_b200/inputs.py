@@ -76,6 +76,10 @@ _add(Workload("decode_sqatm", 32, 32768, 8, 4, 16, False, False, decode=True,
               note="decode step, B=32 sequences, cache N=32768, dh=16 Hq=8 Hkv=4"))
 _add(Workload("decode_dh128", 8, 65536, 8, 4, 128, False, False, k_scale=0.1, decode=True,
               note="decode step, B=8 sequences, cache N=65536, dh=128 Hq=8 Hkv=4, K x 0.1"))
+# MQA head layout (16 query heads on one K/V head): a group of 16 takes the
+# shared-memory split path.
+_add(Workload("decode_mqa", 32, 32768, 16, 1, 16, False, False, decode=True,
+              note="decode step, B=32 sequences, cache N=32768, dh=16 Hq=16 Hkv=1"))
 
 
 def make_inputs(B: int, N: int, Hq: int, Hkv: int, dh: int, seed: int = 0, std: float = 1.0,
