@@ -1,5 +1,6 @@
-"""A Python model of the register-resident decoding split path's index
-arithmetic, run on the CPU against the fp64 oracle.
+"""Python models of the decoding split paths' index arithmetic, run on the
+CPU against the fp64 oracle: the register-resident path (below) and the
+shared-memory path (at the end of the file, with the rule that picks a path).
 
 The model follows the CUDA kernel's work split step by step: the range of
 positions per CTA chosen from the SM count and the CTAs resident per SM, the
@@ -11,6 +12,7 @@ ceil(len / span) ranges.  Arithmetic is fp64, so any mistake in the mapping
 shows as a mismatch far above rounding.  The grid size is a free parameter here
 (any SM count and occupancy), which the GPU tests cannot vary.
 """
+import itertools
 import math
 
 import numpy as np
@@ -171,3 +173,102 @@ def test_grid_of_the_decoding_workloads(B, N, Hkv, dh):
     # two resident CTAs per SM on 148 SMs give four full waves
     span = span_for(B, N, Hkv, dh, 148, 2)
     assert B * -(-N // span) == 4 * 148 * 2
+
+
+# ----------------------------------------------------------------------------- general path
+
+
+def decode_chunk(dh):
+    return 256 if dh <= 32 else (128 if dh == 64 else 64)
+
+
+def model_general(q, k, v, lens, scale):
+    """The shared-memory split path: one CTA per (range of 4 chunks, K/V head,
+    sequence); per chunk, all g heads' scores, block-wide online softmax."""
+    B, Hq, dh = q.shape
+    N, Hkv = k.shape[1], k.shape[2]
+    g = Hq // Hkv
+    CH = decode_chunk(dh)
+    span = 4 * CH
+    n_split = -(-N // span)
+    part = np.full((B, Hkv, n_split, g, dh + 2), np.nan)
+    sl2 = scale * math.log2(math.e)
+    for b, kvh, split in itertools.product(range(B), range(Hkv), range(n_split)):
+        ln = N if lens is None else min(max(lens[b], 0), N)
+        c_first = split * 4
+        n_chunks = max(0, min(4, -(-ln // CH) - c_first))
+        if n_chunks == 0:
+            part[b, kvh, split, :, :dh] = 0.0
+            part[b, kvh, split, :, dh] = -np.inf
+            part[b, kvh, split, :, dh + 1] = 0.0
+            continue
+        qs = q[b, kvh * g : (kvh + 1) * g] * sl2
+        m, l, o = np.full(g, -np.inf), np.zeros(g), np.zeros((g, dh))
+        for c in range(n_chunks):
+            j0 = (c_first + c) * CH
+            cnt = min(CH, ln - j0)
+            assert cnt > 0 and j0 + cnt <= ln
+            s = np.full((g, CH), -np.inf)
+            s[:, :cnt] = qs @ k[b, j0 : j0 + cnt, kvh].T
+            mn = np.maximum(m, s.max(axis=1))
+            w = np.exp2(s - mn[:, None])
+            with np.errstate(invalid="ignore"):
+                a = np.where(m == -np.inf, 0.0, np.exp2(m - mn))
+            l = l * a + w.sum(axis=1)
+            o = o * a[:, None] + w[:, :cnt] @ v[b, j0 : j0 + cnt, kvh]
+            m = mn
+        part[b, kvh, split, :, :dh] = o
+        part[b, kvh, split, :, dh] = m
+        part[b, kvh, split, :, dh + 1] = l
+    out, lse = np.zeros((B, Hq, dh)), np.zeros((B, Hq))
+    for b in range(B):
+        ln = N if lens is None else min(max(lens[b], 0), N)
+        n_used = -(-ln // span)
+        for hq in range(Hq):
+            kvh, hg = divmod(hq, g)
+            ps = part[b, kvh, :n_used, hg]
+            if n_used == 0:
+                out[b, hq], lse[b, hq] = 0.0, -np.inf
+                continue
+            M = ps[:, dh].max()
+            w = np.exp2(ps[:, dh] - M)
+            Ls = (ps[:, dh + 1] * w).sum()
+            out[b, hq] = (ps[:, :dh] * w[:, None]).sum(0) / Ls
+            lse[b, hq] = (M + math.log2(Ls)) * math.log(2)
+    return out, lse
+
+
+GENERAL_CASES = [
+    ((2, 1000, 16, 1, 16), [999, 257]),
+    ((2, 3000, 128, 1, 16), [2999, 3]),
+    ((2, 520, 16, 2, 128), [520, 131]),
+    ((2, 500, 6, 3, 32), [500, 250]),
+    ((2, 1100, 8, 1, 64), [0, 1100]),
+    ((1, 256, 32, 4, 16), None),  # exactly one chunk
+    ((1, 1025, 16, 2, 16), None),  # one position into the second range
+]
+
+
+@pytest.mark.parametrize("shape,lens", GENERAL_CASES, ids=lambda c: "x".join(map(str, c)) if isinstance(c, tuple) else str(c))
+def test_shared_memory_split_model_matches_oracle(shape, lens):
+    B, N, Hq, Hkv, dh = shape
+    rng = np.random.default_rng(N + Hq)
+    q = rng.standard_normal((B, Hq, dh))
+    k = rng.standard_normal((B, N, Hkv, dh))
+    v = rng.standard_normal((B, N, Hkv, dh))
+    out, lse = model_general(q, k, v, lens, 1 / math.sqrt(dh))
+    keep = [i for i in range(B) if lens is None or lens[i] > 0]
+    for i in set(range(B)) - set(keep):
+        assert np.all(out[i] == 0) and np.all(np.isneginf(lse[i]))
+    ref_out, ref_lse = oracle.sqa_decode(q[keep], k[keep], v[keep], None if lens is None else [lens[i] for i in keep])
+    np.testing.assert_allclose(out[keep], ref_out, rtol=0, atol=1e-10)
+    np.testing.assert_allclose(lse[keep], ref_lse, rtol=0, atol=1e-10)
+
+
+@pytest.mark.parametrize("g,hkv,dh,rows_path_expected", [(2, 4, 16, True), (4, 8, 128, True), (1, 16, 128, True),
+                                                         (5, 1, 16, False), (16, 1, 16, False), (2, 3, 32, False),
+                                                         (2, 32, 128, False), (4, 128, 16, True)])
+def test_path_selection(g, hkv, dh, rows_path_expected):
+    # the register-resident path takes groups of at most 4 heads whose K/V head
+    # count is a power of two no larger than the rows a CTA takes per step
+    assert rows_path(g, hkv, dh) == rows_path_expected
