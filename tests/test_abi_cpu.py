@@ -154,3 +154,31 @@ def _decode_ws_expected(B, N, Hq, Hkv, dh):
                                    (2, 500, 6, 3, 32), (2, 300, 16, 16, 128), (2, 300, 32, 32, 128), (1, 1, 4, 1, 64)])
 def test_decode_workspace_covers_both_split_paths(lib, shape):
     assert lib.sqa_decode_workspace_bytes(sqa.Shape(*shape)) == _decode_ws_expected(*shape)
+
+
+def test_plain_c_client_builds_links_and_runs(lib, tmp_path):
+    """include/sqa.h compiles as C11 (warnings as errors), a C program links
+    against libsqa.so, and its calls give the documented results without a GPU."""
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    pkg = os.path.join(ROOT, "sparse_query_attention_sqa_b200")
+    exe = str(tmp_path / "c_client")
+    subprocess.run([gcc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "abi", "c_client.c"), "-L", pkg, "-lsqa", f"-Wl,-rpath,{pkg}",
+                    "-o", exe], check=True, capture_output=True, text=True)
+    out = subprocess.run([exe], check=True, capture_output=True, text=True).stdout
+    got = dict(line.split(" ", 1) for line in out.strip().splitlines())
+    assert int(got["version"]) == lib.sqa_version()
+    assert int(got["bwd_workspace"]) == lib.sqa_bwd_workspace_bytes(sqa.Shape(32, 1024, 8, 4, 16))
+    assert int(got["decode_workspace"]) == lib.sqa_decode_workspace_bytes(sqa.Shape(32, 32768, 8, 4, 16))
+    assert int(got["decode_workspace_invalid"]) == 0
+    invalid, unsupported = "1", "2"
+    assert got["fwd_null"] == invalid and got["fwd_group"] == invalid
+    assert got["fwd_dh"] == unsupported and got["fwd_misaligned"] == unsupported
+    assert got["bwd_small_workspace"] == invalid and got["decode_null"] == invalid
+    assert got["timing_bad_kernel"] == invalid
+    assert got["status_string_ok"] == "1" and got["last_error_nonempty"] == "1"
