@@ -44,3 +44,47 @@ def test_traffic_table_names_a_capture_command_per_entry():
     for e in table["entries"]:
         assert e["command"].startswith("ncu ") and "--clock-control none" in e["command"]
         assert e["dram_bytes_per_launch"] > 0 and len(e["source_sha256"]) == 64
+
+
+def test_reference_arm_prints_one_complete_json_line():
+    import json
+    import subprocess
+
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                        "sqatm_layer_fwd", "--steps", "2", "--warmup", "1"], capture_output=True, text=True,
+                       timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["config"]["workload"] == "sqatm_layer_fwd"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_roofline_reports_the_stated_algorithmic_work():
+    from sparse_query_attention_sqa_b200.inputs import WORKLOADS
+
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1400.0}
+    ms = 0.5
+    # decode: HBM-bound on the caches plus q, out and lse
+    w = WORKLOADS["decode_sqatm"]
+    rl = bench.roofline_for(w, "sqa_decode_split_kernel", ms, peaks, "measured")
+    want = (2 * w.B * w.N * w.Hkv * w.dh * 2 + 2 * w.B * w.Hq * w.dh * 2 + 4 * w.B * w.Hq) / (ms * 1e-3) / 1e9
+    assert rl["bound"] == "hbm" and rl["unit"] == "GB/s" and rl["peak"] == 6000.0
+    assert abs(rl["achieved"] - want) < 1e-6 * want and abs(rl["frac"] - want / 6000.0) < 1e-12
+    # dh 16: one exp2 per unmasked score element against the derived special-function peak
+    w = WORKLOADS["sqatm_train_sqa"]
+    rl = bench.roofline_for(w, "sqa_bwd_kernel", ms, peaks, "measured")
+    causal_pairs = w.B * w.Hq * w.N * (w.N + 1) / 2
+    assert rl["bound"] == "alu" and rl["unit"] == "Gexp2/s"
+    assert abs(rl["achieved"] - causal_pairs / (ms * 1e-3) / 1e9) < 1e-6 * rl["achieved"]
+    assert abs(rl["peak"] - 148 * 16 * 1965e6 / 1e9) < 1e-9
+    for rl in (bench.roofline_for(WORKLOADS[n], k, ms, peaks, "measured")
+               for n, k in (("decode_sqatm", "sqa_decode_split_kernel"), ("sqatm_train_sqa", "sqa_fwd_kernel"))):
+        assert set(rl) >= {"bound", "achieved", "peak", "unit", "frac", "traffic"}
