@@ -182,3 +182,26 @@ def test_plain_c_client_builds_links_and_runs(lib, tmp_path):
     assert got["bwd_small_workspace"] == invalid and got["decode_null"] == invalid
     assert got["timing_bad_kernel"] == invalid
     assert got["status_string_ok"] == "1" and got["last_error_nonempty"] == "1"
+
+
+def _bwd_ws_expected(B, N, Hq, Hkv, dh):
+    """Workspace rule of sqa_bwd: -lse*log2(e) and -D per stacked-tile slot
+    (B * H_kv * n_qtiles * 128 fp32 each), the fp32 dQ accumulator
+    [B][N][H_q][dh], and for dh <= 32 fp32 images of every stacked Q and dO
+    tile (dh floats per slot each); every part rounded up to 256 bytes."""
+    def a256(x):
+        return -(-x // 256) * 256
+
+    g = Hq // Hkv
+    T = 128 // g
+    slots = B * Hkv * -(-N // T) * 128
+    total = 2 * a256(slots * 4) + a256(B * N * Hq * dh * 4)
+    if dh <= 32:
+        total += 2 * a256(slots * dh * 4)
+    return total
+
+
+@pytest.mark.parametrize("shape", [(32, 1024, 8, 4, 16), (2, 65536, 8, 4, 128), (1, 1000, 6, 2, 32),
+                                   (3, 77, 128, 1, 64), (1, 1, 16, 16, 16), (1, 200000, 8, 4, 16)])
+def test_bwd_workspace_follows_its_layout(lib, shape):
+    assert lib.sqa_bwd_workspace_bytes(sqa.Shape(*shape)) == _bwd_ws_expected(*shape)
