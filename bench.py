@@ -3,16 +3,21 @@
 
 One step is one pass of the whole path over one batch: sqa_fwd followed by
 sqa_bwd (for forward-only workloads, sqa_fwd alone).  The default workload is
-the SQAT-m training-step attention: B=32, N=1024, dh=16 (d=256 split over 16
-heads), H_q=8 query heads over H_kv=4 key/value heads, causal, forward and
-backward (SQAT-m model card, "Architecture details"; message length 1024).
+the largest single-GPU configuration: larger-model SQA attention, B=2,
+N=65536, dh=128 (d=2048 split over 16 heads), H_q=8 query heads over H_kv=4
+key/value heads, causal, forward and backward, K scaled by 0.1 (arXiv
+2510.01817 abstract: the gains are claimed for 32k-200k token sequences).
+After it the same kernels run the MHA (16/16), GQA (16/4) and MQA (16/1) head
+layouts of the same model for comparison (``--no-compare`` skips them); the
+SQAT-m training step (B=32, N=1024, dh=16, 8/4) and the other shapes are
+available with ``--workload``.
 
 Throughput counts 4*B*H_q*N^2*dh FLOPs for the forward (halved when causal)
 and 3.5 times that for forward plus backward.  Inputs are seeded synthetic bf16
 Gaussians; several buffer sets whose total exceeds the 126 MB L2 are used in
 rotation, so every step reads its inputs from HBM.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--no-compare]
   python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
 
 Under torchrun every rank runs its own copy of the workload (independent
@@ -46,7 +51,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="sqatm_train_sqa")
+    ap.add_argument("--workload", default="large_dh128")
+    ap.add_argument("--no-compare", action="store_true",
+                    help="skip the same-kernel MHA/GQA/MQA comparison after the workload")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="time budget of the CPU-baseline sample")
     ap.add_argument("--no-clocks", action="store_true")
@@ -265,6 +272,18 @@ def decode_bytes(w) -> float:
     return 2.0 * w.B * w.N * w.Hkv * w.dh * 2 + 2.0 * w.B * w.Hq * w.dh * 2 + 4.0 * w.B * w.Hq
 
 
+def launched_kernel(w, hook: int) -> str:
+    """Name (with template arguments) of the main kernel behind a timing hook:
+    0 the forward, 1 the backward, 2 the decoding split kernel."""
+    if hook == 0:
+        return f"sqa_fwd_kernel<{w.dh}>"
+    if hook == 1:
+        return f"sqa_bwd_tf32_kernel<{w.dh}>" if w.dh <= 32 else f"sqa_bwd_kernel<{w.dh}>"
+    g = w.Hq // w.Hkv
+    rows = g <= 4 and (w.Hkv & (w.Hkv - 1)) == 0  # register-resident path
+    return f"sqa_decode_split_kernel<{w.dh},{g if rows else 0}>"
+
+
 def roofline_for(w, kernel_name, ms, peaks, peak_kind):
     if w.decode:
         # HBM-bound: stream the caches once
@@ -285,8 +304,13 @@ def roofline_for(w, kernel_name, ms, peaks, peak_kind):
         flops *= 2.5
     achieved = flops / (ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops"]
-    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-            "traffic": traffic_for(kernel_name, w), "kernel": kernel_name, "peak_source": f"{peak_kind} bf16_tflops"}
+    sustained = peaks.get("bf16_tflops_sustained")
+    rl = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+          "traffic": traffic_for(kernel_name, w), "kernel": kernel_name, "peak_source": f"{peak_kind} bf16_tflops"}
+    if sustained:
+        rl["peak_sustained"] = sustained
+        rl["frac_sustained"] = achieved / sustained
+    return rl
 
 
 def strip_c_comments(text: str) -> str:
@@ -343,6 +367,78 @@ def traffic_for(kernel_name, w):
     return None
 
 
+def warm_up(lib, w, sets, warmup, torch):
+    """Warm-up steps; each times its main kernels with the library's hook.
+    Returns ({kernel: [ms]}, the dominant kernel's name, its hook index)."""
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    kern = {}
+    hooks = (2,) if w.decode else ((0, 1) if w.backward else (0,))  # timing-hook indices: fwd, bwd, decode
+    for i in range(max(warmup, 3)):
+        s = sets[i % len(sets)]
+        evs = {h: (ev(), ev()) for h in hooks}
+        for h, (e0, e1) in evs.items():
+            lib.set_timing_events(h, e0, e1)
+        step(lib, w, s)
+        for h in hooks:
+            lib.set_timing_events(h)
+        torch.cuda.synchronize()
+        for h, (e0, e1) in evs.items():
+            kern.setdefault(launched_kernel(w, h), []).append(e0.elapsed_time(e1))
+    assert lib.device_status() == 0, "a kernel wait gave up during warm-up"
+    dominant = max(kern, key=lambda n: statistics.median(kern[n]))
+    dom_idx = next(h for h in hooks if launched_kernel(w, h) == dominant)
+    return kern, dominant, dom_idx
+
+
+def compare_variants(args, w):
+    """Workloads run after the headline one for the same-kernel head-layout
+    comparison (the same model with every head kept, GQA and MQA)."""
+    from sparse_query_attention_sqa_b200.inputs import WORKLOADS
+
+    if args.no_compare:
+        return []
+    groups = {"large_dh128": ("large_dh128_mha", "large_dh128_gqa", "large_dh128_mqa"),
+              "sqatm_train_sqa": ("sqatm_train_mha", "sqatm_train_gqa", "sqatm_train_mqa"),
+              "enc32k_8_4": ("enc32k_16_16", "enc32k_16_4", "enc32k_16_1", "enc32k_8_8", "enc32k_4_4")}
+    return [WORKLOADS[n] for n in groups.get(w.name, ())]
+
+
+def time_variant(args, lib, w, torch, world, rank, peaks, peak_kind):
+    """Device time of the same kernels on another head layout: warm-up, then
+    args.steps steps with the dominant kernel timed by the library hook."""
+    from sparse_query_attention_sqa_b200.inputs import workload_inputs
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    q, k, v, dout = workload_inputs(w, seed=rank)
+    first = alloc_set(w, q, k, v, dout, lib, torch)
+    n_sets = max(2, math.ceil(2 * L2_BYTES / set_bytes(first)))
+    sets = [first] + [alloc_set(w, q, k, v, dout, lib, torch) for _ in range(n_sets - 1)]
+    del q, k, v, dout
+    kern, dominant, dom_idx = warm_up(lib, w, sets, args.warmup, torch)
+    starts = [ev() for _ in range(args.steps)]
+    stops = [ev() for _ in range(args.steps)]
+    t0, t1 = ev(), ev()
+    torch.cuda.synchronize()
+    t0.record()
+    for i in range(args.steps):
+        lib.set_timing_events(dom_idx, starts[i], stops[i])
+        step(lib, w, sets[i % n_sets])
+    t1.record()
+    lib.set_timing_events(dom_idx)
+    torch.cuda.synchronize()
+    assert lib.device_status() == 0, "a kernel wait gave up while timing a comparison layout"
+    ms_step = max_over_ranks(t0.elapsed_time(t1), world, "cuda") / args.steps
+    dom_ms = statistics.fmean(a.elapsed_time(b) for a, b in zip(starts, stops))
+    rl = roofline_for(w, dominant, dom_ms, peaks, peak_kind)
+    rl.pop("traffic", None)
+    out = {"workload": w.name, "H_q": w.Hq, "H_kv": w.Hkv, "ms_per_step": ms_step,
+           "value": job_tflops(w, world, ms_step), "unit": "TFLOP/s",
+           "kernel_ms": {n: statistics.median(v) for n, v in kern.items()}, "roofline": rl}
+    del sets
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -365,26 +461,8 @@ def run_ours(args, w):
     n_sets = max(2, math.ceil(2 * L2_BYTES / set_bytes(first)))
     sets = [first] + [alloc_set(w, q, k, v, dout, lib, torch) for _ in range(n_sets - 1)]
 
-    # Which kernel dominates: time both main kernels once per set during warm-up.
     ev = lambda: torch.cuda.Event(enable_timing=True)
-    kern = {}
-    hooks = (2,) if w.decode else (0, 1)  # library timing-hook indices: fwd, bwd, decode
-    names = {0: "sqa_fwd_kernel", 1: "sqa_bwd_kernel", 2: "sqa_decode_split_kernel"}
-    for i in range(max(args.warmup, 3)):
-        s = sets[i % n_sets]
-        evs = {h: (ev(), ev()) for h in hooks}
-        for h, (e0, e1) in evs.items():
-            lib.set_timing_events(h, e0, e1)
-        step(lib, w, s)
-        for h in hooks:
-            lib.set_timing_events(h)
-        torch.cuda.synchronize()
-        for h, (e0, e1) in evs.items():
-            if h != 1 or w.backward:
-                kern.setdefault(names[h], []).append(e0.elapsed_time(e1))
-    assert lib.device_status() == 0, "a kernel wait gave up during warm-up"
-    dominant = max(kern, key=lambda n: statistics.median(kern[n]))
-    dom_idx = next(h for h, n in names.items() if n == dominant)
+    kern, dominant, dom_idx = warm_up(lib, w, sets, args.warmup, torch)
 
     # Timed region: K steps, per-step events around the dominant kernel.
     starts = [ev() for _ in range(args.steps)]
@@ -485,6 +563,16 @@ def run_ours(args, w):
             "clocks": clk,
             "wall_s_timed_region": wall,
         }
+    # The same kernels on the MHA / GQA / MQA head layouts of the same model.
+    variants = compare_variants(args, w)
+    if variants:
+        sets.clear()
+        first = host_in = host_out = None
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        comp = [time_variant(args, lib, v, torch, world, rank, peaks, peak_kind) for v in variants]
+        if rank == 0:
+            line["compare"] = comp
     # CPU baseline: rank 0 at N=1 only, after all GPU work.
     if world == 1:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)

@@ -21,10 +21,15 @@
  *
  * Ownership and execution: the caller owns every buffer (device memory, e.g.
  * from PyTorch) and the stream.  Calls are asynchronous on `stream`; the library
- * never synchronises, never allocates device memory and keeps no per-call
- * state on the device.  Arguments are validated on the host before anything is
- * launched; a call that returns an error has launched nothing.  The calls are
- * thread-safe; error text is kept per host thread.
+ * allocates no device memory at run time and keeps no per-call state on the
+ * device, with two exceptions: sqa_bwd_static_scratch works in one file-scope
+ * device array that every GPU loading the library holds until exit and that
+ * keeps the last call's contents, and the kernels' wait-timeout status words
+ * persist until read.  No call synchronises except sqa_device_status and
+ * sqa_device_timeout_info, which synchronise the current device to read those
+ * words.  Arguments are validated on the host before anything is launched; a
+ * call that returns an error has launched nothing.  The calls are thread-safe;
+ * error text is kept per host thread.
  */
 #ifndef SQA_H_
 #define SQA_H_
@@ -104,8 +109,12 @@ sqa_status sqa_bwd(const void *dout, const void *q, const void *k, const void *v
  * are rejected with SQA_ERR_UNSUPPORTED before anything is launched.  Nothing
  * is allocated or freed by this call.
  *
- * The first call on a device looks up the array's device address (with that
- * device current), so make that first call before any stream capture.  All
+ * Every call made outside a stream capture looks up the array's device
+ * address on the current device (so a context torn down and rebuilt between
+ * calls, e.g. by cudaDeviceReset, leaves no stale pointer); a call made while
+ * `stream` is capturing uses the address found by the last call outside a
+ * capture on that device, and fails with SQA_ERR_INVALID_ARG if there was
+ * none.  So make a first call on each device before any stream capture.  All
  * calls share the one array and it keeps the last call's contents; the
  * kernels clear what must start at zero.  Calls whose GPU work overlaps (on
  * different streams, or from different threads) race on the array: order them.

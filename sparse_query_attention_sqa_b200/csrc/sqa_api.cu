@@ -3,6 +3,7 @@
 // stream.  This is the only translation unit of libsqa.so.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -177,20 +178,41 @@ int decode_rows_span(const sqa_shape& s, int ctas_per_sm) {
   return static_cast<int>(span < ms ? ms : span);
 }
 
+constexpr int kMaxDevices = 128;
+
+// Resident CTAs per SM of the register-resident split kernel on the current
+// device, queried once per device.  The kernel's shared-memory limit must be
+// raised first: asked before that, the query sees no resident CTA at all.
+template <int DH, int G>
+sqa_status decode_rows_occupancy(int smem, int* occ) {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(SQA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  int o = cache[dev].load(std::memory_order_relaxed);
+  if (o == 0) {
+    sqa_status st = set_smem(sqa::sqa_decode_split_kernel<DH, G>, smem);
+    if (st != SQA_OK) return st;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, sqa::sqa_decode_split_kernel<DH, G>, sqa::kDecodeThreads,
+                                                      smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (o < 1) o = 1;
+    cache[dev].store(o, std::memory_order_relaxed);
+  }
+  *occ = o;
+  return SQA_OK;
+}
+
 template <int DH, int G>
 sqa_status launch_decode_rows(sqa::DecodeParams& p, const sqa_shape& s, cudaStream_t stream) {
   const int smem = static_cast<int>(sqa::rows_smem_bytes(G, DH));
-  static const int occ = [smem] {
-    int o = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, sqa::sqa_decode_split_kernel<DH, G>, sqa::kDecodeThreads,
-                                                      smem) != cudaSuccess)
-      o = 0;
-    return o > 0 ? o : 1;
-  }();
-  p.span = decode_rows_span(s, occ);
-  p.n_split = (s.N + p.span - 1) / p.span;
   sqa_status st;
   if ((st = set_smem(sqa::sqa_decode_split_kernel<DH, G>, smem)) != SQA_OK) return st;
+  int occ = 1;
+  if ((st = decode_rows_occupancy<DH, G>(smem, &occ)) != SQA_OK) return st;
+  p.span = decode_rows_span(s, occ);
+  p.n_split = (s.N + p.span - 1) / p.span;
   if ((st = record_timing(2, 0, stream)) != SQA_OK) return st;
   sqa::sqa_decode_split_kernel<DH, G>
       <<<dim3(static_cast<unsigned>(p.n_split), static_cast<unsigned>(s.B)), sqa::kDecodeThreads, smem, stream>>>(p);
@@ -354,24 +376,32 @@ sqa_status launch_bwd(const void* dout, const void* q, const void* k, const void
 
 // Scratch for sqa_bwd_static_scratch: one device array per GPU that loads the
 // library.  In host code the name is only a handle; its device address comes
-// from cudaGetSymbolAddress, looked up once per device and cached.
+// from cudaGetSymbolAddress with the device current.  Outside a stream capture
+// the address is looked up on every call (cheap), so a context torn down and
+// rebuilt between calls (cudaDeviceReset) never leaves a stale pointer; inside
+// a capture the address from the last call outside one is used.
 static __device__ __align__(256) unsigned char g_static_scratch[SQA_STATIC_SCRATCH_BYTES];
 
 std::mutex g_static_scratch_mu;
-constexpr int kMaxDevices = 128;
 void* g_static_scratch_addr[kMaxDevices] = {};
 
-sqa_status static_scratch_address(void** addr) {
+sqa_status static_scratch_address(cudaStream_t stream, void** addr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(SQA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  e = cudaStreamIsCapturing(stream, &cap);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
   std::lock_guard<std::mutex> lock(g_static_scratch_mu);
-  if (!g_static_scratch_addr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress (static scratch)");
     g_static_scratch_addr[dev] = p;
+  } else if (!g_static_scratch_addr[dev]) {
+    return fail(SQA_ERR_INVALID_ARG,
+                "sqa_bwd_static_scratch: the first call on a device must come before any stream capture");
   }
   *addr = g_static_scratch_addr[dev];
   return SQA_OK;
@@ -477,7 +507,7 @@ sqa_status sqa_bwd_static_scratch(const void* dout, const void* q, const void* k
     return fail(SQA_ERR_UNSUPPORTED, "this shape needs %zu bytes of scratch; the static scratch holds %u (use sqa_bwd)",
                 need, SQA_STATIC_SCRATCH_BYTES);
   void* scratch = nullptr;
-  if ((st = static_scratch_address(&scratch)) != SQA_OK) return st;
+  if ((st = static_scratch_address(reinterpret_cast<cudaStream_t>(stream), &scratch)) != SQA_OK) return st;
   return sqa_bwd(dout, q, k, v, out, lse, dq, dk, dv, scratch, SQA_STATIC_SCRATCH_BYTES, s, causal, scale, stream);
 }
 

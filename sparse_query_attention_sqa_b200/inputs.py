@@ -67,9 +67,16 @@ for n in (131072, 200000):
     for hq, hkv in ((4, 4), (8, 4)):
         _add(Workload(f"enc{n // 1000}k_{hq}_{hkv}", 1, n, hq, hkv, 16, False, False, std=0.5,
                       note=f"encoder, B=1 N={n} dh=16 Hq={hq} Hkv={hkv} bidirectional, std 0.5"))
-# Larger-model SQA: d=2048 over 16 heads, dh=128.
+# Larger-model SQA: d=2048 over 16 heads, dh=128; the same kernel with every
+# head kept (MHA 16/16), GQA 16/4 and MQA 16/1 for comparison.
 _add(Workload("large_dh128", 2, 65536, 8, 4, 128, True, True, k_scale=0.1,
               note="larger model, B=2 N=65536 dh=128 Hq=8 Hkv=4 causal, K x 0.1"))
+for hq, hkv, tag in ((16, 16, "mha"), (16, 4, "gqa"), (16, 1, "mqa")):
+    _add(Workload(f"large_dh128_{tag}", 2, 65536, hq, hkv, 128, True, True, k_scale=0.1,
+                  note=f"larger model, B=2 N=65536 dh=128 Hq={hq} Hkv={hkv} causal, K x 0.1"))
+# The same head layout at 16384 tokens, small enough for full profiler captures.
+_add(Workload("large_dh128_16k", 1, 16384, 8, 4, 128, True, True, k_scale=0.1,
+              note="larger model, B=1 N=16384 dh=128 Hq=8 Hkv=4 causal, K x 0.1"))
 # Decoding step: a batch of sequences, each adding one token against a full
 # key/value cache (SQAT-m head layout, and the larger-model dh=128 layout).
 _add(Workload("decode_sqatm", 32, 32768, 8, 4, 16, False, False, decode=True,
