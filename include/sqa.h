@@ -123,6 +123,72 @@ sqa_status sqa_bwd_static_scratch(const void *dout, const void *q, const void *k
                                   const void *out, const float *lse, void *dq, void *dk, void *dv,
                                   sqa_shape s, int causal, float scale, sqa_stream_t stream);
 
+/*
+ * The full SQA layer around the attention core (SQAT-m model card, "Model size
+ * difference": the query and output projections shrink with the query-head
+ * count; "Architecture details": rotary position embedding):
+ *
+ *   [Q | K | V] = X W_qkv,   Q, K turned by the rotary embedding,
+ *   O = the attention core above (sqa_fwd),   Y = O W_o
+ *
+ * with no biases.  Layouts (row-major, contiguous, bf16 unless noted;
+ * M = B * N tokens, W = (H_q + 2 H_kv) * dh):
+ *   x, y, dy, dx : [B][N][d]
+ *   w_qkv        : [d][W]; columns [0, H_q dh) are W_q (query head h in
+ *                  columns h dh .. h dh + dh - 1), then H_kv dh columns of W_k,
+ *                  then H_kv dh columns of W_v
+ *   w_o          : [H_q dh][d]
+ *   q, out       : [B][N][H_q][dh];  k, v : [B][N][H_kv][dh];  lse fp32 [B][H_q][N]
+ *                  (the rotated projections and the core's outputs, as sqa_fwd
+ *                  takes and gives them; the backward needs them)
+ *   dw_qkv, dw_o : fp32, the shapes of w_qkv and w_o
+ * Rotary embedding: channels (2j, 2j+1) of every query and key head of the
+ * token at position i = token index within its sequence turn by the angle
+ * i * rope_base^(-2j/dh) (cos/sin formed in double precision, rounded to
+ * fp32); rope_base = 0 leaves Q and K unrotated.  d must be a multiple of 8;
+ * the other limits are sqa_fwd's.
+ */
+typedef struct {
+    int B, N;           /* batch, tokens per sequence */
+    int d;              /* model width */
+    int H_q, H_kv, dh;  /* as in sqa_shape */
+} sqa_layer_shape;
+
+/*
+ * Bytes of device scratch that sqa_layer_fwd (backward = 0) or sqa_layer_bwd
+ * (backward != 0) needs; 0 if the shape is invalid.  The caller allocates it,
+ * 256-byte aligned; its contents on entry do not matter.
+ */
+size_t sqa_layer_workspace_bytes(sqa_layer_shape s, int backward);
+
+/*
+ * Layer forward: writes y and the saved tensors q, k, v (rotated), out and lse.
+ * Three kernels on `stream` (a tcgen05 GEMM with the rotation in its epilogue,
+ * the attention core, the output GEMM), plus a small table kernel when
+ * rope_base > 0.  causal and scale as for sqa_fwd.  Errors as for sqa_fwd,
+ * returned before any launch; SQA_ERR_INVALID_ARG for a workspace smaller
+ * than sqa_layer_workspace_bytes(s, 0) or a negative or non-finite rope_base.
+ */
+sqa_status sqa_layer_fwd(const void *x, const void *w_qkv, const void *w_o, void *y, void *q, void *k,
+                         void *v, void *out, float *lse, void *workspace, size_t workspace_bytes,
+                         sqa_layer_shape s, int causal, float scale, float rope_base,
+                         sqa_stream_t stream);
+
+/*
+ * Layer backward of L = sum(dy * y): dx (bf16) and the weight gradients dw_qkv
+ * and dw_o (fp32, fully overwritten).  Takes the forward's x, weights and saved
+ * tensors.  Steps: dO = dY W_o^T; dW_o = O^T dY; the core backward (sqa_bwd)
+ * gives dQ, dK, dV of the rotated projections; the rotation is undone on dQ
+ * and dK; dW_qkv = X^T [dQ | dK | dV]; dX = [dQ | dK | dV] W_qkv^T.  The
+ * weight-gradient products reduce over all M tokens with fp32 reductions in a
+ * run-dependent order.  workspace: sqa_layer_workspace_bytes(s, 1) bytes.
+ */
+sqa_status sqa_layer_bwd(const void *dy, const void *x, const void *w_qkv, const void *w_o, const void *q,
+                         const void *k, const void *v, const void *out, const float *lse, void *dx,
+                         float *dw_qkv, float *dw_o, void *workspace, size_t workspace_bytes,
+                         sqa_layer_shape s, int causal, float scale, float rope_base,
+                         sqa_stream_t stream);
+
 /* Static text for a status code. */
 const char *sqa_status_string(sqa_status status);
 

@@ -14,7 +14,8 @@ import os
 __all__ = [
     "SqaError", "load_library", "library_path", "sqa_fwd", "sqa_bwd", "bwd_workspace_bytes", "sqa_decode",
     "decode_workspace_bytes",
-    "device_status", "timeout_info", "set_timing_events", "Shape",
+    "device_status", "timeout_info", "set_timing_events", "Shape", "LayerShape", "layer_workspace_bytes",
+    "sqa_layer_fwd", "sqa_layer_bwd",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -33,6 +34,11 @@ class SqaError(RuntimeError):
 class Shape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("N", ctypes.c_int), ("H_q", ctypes.c_int), ("H_kv", ctypes.c_int),
                 ("dh", ctypes.c_int)]
+
+
+class LayerShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("N", ctypes.c_int), ("d", ctypes.c_int), ("H_q", ctypes.c_int),
+                ("H_kv", ctypes.c_int), ("dh", ctypes.c_int)]
 
 
 def library_path() -> str:
@@ -68,6 +74,13 @@ def load_library():
     lib.sqa_device_timeout_info.restype = c_int
     lib.sqa_set_timing_events.argtypes = [c_int, vp, vp]
     lib.sqa_set_timing_events.restype = c_int
+    lib.sqa_layer_workspace_bytes.argtypes = [LayerShape, c_int]
+    lib.sqa_layer_workspace_bytes.restype = sz
+    lib.sqa_layer_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, fp, vp, sz, LayerShape, c_int, c_float, c_float, vp]
+    lib.sqa_layer_fwd.restype = c_int
+    lib.sqa_layer_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, fp, vp, fp, fp, vp, sz, LayerShape, c_int, c_float,
+                                  c_float, vp]
+    lib.sqa_layer_bwd.restype = c_int
     lib.sqa_version.argtypes = []
     lib.sqa_version.restype = c_int
     _lib = lib
@@ -236,3 +249,70 @@ def device_status(clear: bool = True) -> int:
     w = ctypes.c_uint(0)
     _check(lib.sqa_device_status(ctypes.byref(w), int(bool(clear))))
     return int(w.value)
+
+
+def layer_workspace_bytes(B: int, N: int, d: int, H_q: int, H_kv: int, dh: int, backward: bool) -> int:
+    return int(load_library().sqa_layer_workspace_bytes(LayerShape(B, N, d, H_q, H_kv, dh), int(bool(backward))))
+
+
+def _layer_shape(x, w_qkv, w_o, H_q, H_kv):
+    import torch
+
+    if x.dim() != 3:
+        raise ValueError("x must be [B, N, d]")
+    B, N, d = x.shape
+    dh = w_o.shape[0] // H_q
+    s = LayerShape(B, N, d, H_q, H_kv, dh)
+    _need(x, "x", (B, N, d), torch.bfloat16)
+    _need(w_qkv, "w_qkv", (d, (H_q + 2 * H_kv) * dh), torch.bfloat16)
+    _need(w_o, "w_o", (H_q * dh, d), torch.bfloat16)
+    return s
+
+
+def sqa_layer_fwd(x, w_qkv, w_o, H_q: int, H_kv: int, causal: bool = True, scale: float = 0.0,
+                  rope_base: float = 10000.0, workspace=None, stream=None):
+    """Layer forward.  x [B,N,d], w_qkv [d,(H_q+2H_kv)dh], w_o [H_q dh,d] (bf16 CUDA).
+    Returns (y, saved) with saved = dict(q, k, v, out, lse) for sqa_layer_bwd."""
+    import torch
+
+    lib = load_library()
+    s = _layer_shape(x, w_qkv, w_o, H_q, H_kv)
+    dev = x.device
+    y = torch.empty_like(x)
+    q = torch.empty((s.B, s.N, H_q, s.dh), dtype=torch.bfloat16, device=dev)
+    k = torch.empty((s.B, s.N, H_kv, s.dh), dtype=torch.bfloat16, device=dev)
+    v = torch.empty_like(k)
+    out = torch.empty_like(q)
+    lse = torch.empty((s.B, H_q, s.N), dtype=torch.float32, device=dev)
+    need = int(lib.sqa_layer_workspace_bytes(s, 0))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check(lib.sqa_layer_fwd(x.data_ptr(), w_qkv.data_ptr(), w_o.data_ptr(), y.data_ptr(), q.data_ptr(),
+                             k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
+                             workspace.numel() * workspace.element_size(), s, int(bool(causal)), float(scale),
+                             float(rope_base), _stream(stream)))
+    return y, {"q": q, "k": k, "v": v, "out": out, "lse": lse}
+
+
+def sqa_layer_bwd(dy, x, w_qkv, w_o, saved, H_q: int, H_kv: int, causal: bool = True, scale: float = 0.0,
+                  rope_base: float = 10000.0, workspace=None, stream=None):
+    """Layer backward of sum(dy * y).  Returns (dx bf16, dw_qkv fp32, dw_o fp32)."""
+    import torch
+
+    lib = load_library()
+    s = _layer_shape(x, w_qkv, w_o, H_q, H_kv)
+    _need(dy, "dy", tuple(x.shape), torch.bfloat16)
+    dev = x.device
+    dx = torch.empty_like(x)
+    dw_qkv = torch.empty(tuple(w_qkv.shape), dtype=torch.float32, device=dev)
+    dw_o = torch.empty(tuple(w_o.shape), dtype=torch.float32, device=dev)
+    need = int(lib.sqa_layer_workspace_bytes(s, 1))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    sv = saved
+    _check(lib.sqa_layer_bwd(dy.data_ptr(), x.data_ptr(), w_qkv.data_ptr(), w_o.data_ptr(), sv["q"].data_ptr(),
+                             sv["k"].data_ptr(), sv["v"].data_ptr(), sv["out"].data_ptr(), sv["lse"].data_ptr(),
+                             dx.data_ptr(), dw_qkv.data_ptr(), dw_o.data_ptr(), workspace.data_ptr(),
+                             workspace.numel() * workspace.element_size(), s, int(bool(causal)), float(scale),
+                             float(rope_base), _stream(stream)))
+    return dx, dw_qkv, dw_o

@@ -12,9 +12,11 @@
 
 #include "sqa.h"
 #include "sqa_bwd.cuh"
+#include "sqa_bwd_bf16.cuh"
 #include "sqa_bwd_tf32.cuh"
 #include "sqa_decode.cuh"
 #include "sqa_fwd.cuh"
+#include "sqa_gemm.cuh"
 
 namespace {
 
@@ -287,7 +289,6 @@ template <int DH>
 sqa_status launch_bwd(const void* dout, const void* q, const void* k, const void* v, const void* out,
                       const float* lse, void* dq, void* dk, void* dv, void* workspace, const sqa_shape& s,
                       int causal, float scale, cudaStream_t stream) {
-  using Tr = sqa::BwdTraits<DH>;
   const sqa::BwdLayout L = sqa::bwd_layout(s.B, s.N, s.H_q, s.H_kv, DH);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* lse2 = reinterpret_cast<float*>(ws);
@@ -322,10 +323,13 @@ sqa_status launch_bwd(const void* dout, const void* q, const void* k, const void
 
   CUtensorMap mq, mdo, mk, mv;
   sqa_status st;
-  if ((st = make_map(&mq, q, s.B, s.N, s.H_q, DH, Tr::PANEL, L.g, L.T)) != SQA_OK) return st;
-  if ((st = make_map(&mdo, dout, s.B, s.N, s.H_q, DH, Tr::PANEL, L.g, L.T)) != SQA_OK) return st;
-  if ((st = make_map(&mk, k, s.B, s.N, s.H_kv, DH, Tr::PANEL, 1, Tr::NK)) != SQA_OK) return st;
-  if ((st = make_map(&mv, v, s.B, s.N, s.H_kv, DH, Tr::PANEL, 1, Tr::NK)) != SQA_OK) return st;
+  // Tensor maps: boxes of one 32-, 64- or 128-byte swizzled row segment of dh
+  // (all of dh up to 64 elements, a 64-element panel at dh 128).
+  constexpr int PANEL = DH < 64 ? DH : 64;
+  if ((st = make_map(&mq, q, s.B, s.N, s.H_q, DH, PANEL, L.g, L.T)) != SQA_OK) return st;
+  if ((st = make_map(&mdo, dout, s.B, s.N, s.H_q, DH, PANEL, L.g, L.T)) != SQA_OK) return st;
+  if ((st = make_map(&mk, k, s.B, s.N, s.H_kv, DH, PANEL, 1, sqa::kBwdTile)) != SQA_OK) return st;
+  if ((st = make_map(&mv, v, s.B, s.N, s.H_kv, DH, PANEL, 1, sqa::kBwdTile)) != SQA_OK) return st;
   sqa::BwdParams p{};
   p.lse2 = lse2;
   p.D = Dst;
@@ -357,10 +361,12 @@ sqa_status launch_bwd(const void* dout, const void* q, const void* k, const void
     if ((st = record_timing(1, 0, stream)) != SQA_OK) return st;
     sqa::sqa_bwd_tf32_kernel<DH><<<grid, T32::THREADS, T32::SMEM_BYTES, stream>>>(mq, mdo, mk, mv, p);
   } else {
-    if ((st = set_smem(sqa::sqa_bwd_kernel<DH>, Tr::SMEM_BYTES)) != SQA_OK) return st;
+    // dh 64 and 128: one CTA per item, heaviest items first.
+    using Tr = sqa::BwdBf16Traits<DH < 64 ? 64 : DH>;
+    if ((st = set_smem(sqa::sqa_bwd_kernel<DH < 64 ? 64 : DH>, Tr::SMEM_BYTES)) != SQA_OK) return st;
     if ((st = record_timing(1, 0, stream)) != SQA_OK) return st;
-    sqa::sqa_bwd_kernel<DH><<<static_cast<unsigned>(grid_main), Tr::THREADS, Tr::SMEM_BYTES, stream>>>(mq, mdo, mk,
-                                                                                                       mv, p);
+    sqa::sqa_bwd_kernel<DH < 64 ? 64 : DH>
+        <<<static_cast<unsigned>(grid_main), Tr::THREADS, Tr::SMEM_BYTES, stream>>>(mq, mdo, mk, mv, p);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "sqa_bwd main launch");
@@ -404,6 +410,141 @@ sqa_status static_scratch_address(cudaStream_t stream, void** addr) {
                 "sqa_bwd_static_scratch: the first call on a device must come before any stream capture");
   }
   *addr = g_static_scratch_addr[dev];
+  return SQA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// The full layer: projections around the attention core.
+
+// 2-D tensor map over a row-major bf16 matrix [rows][cols] whose rows are ld
+// elements apart, box {64 columns, box_rows rows}, 128-byte swizzle (64 bf16
+// columns per swizzled row).
+sqa_status make_map_2d(CUtensorMap* map, const void* ptr, long long rows, long long cols, long long ld,
+                       int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(SQA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SQA_ERR_CUDA, "cuTensorMapEncodeTiled (2-D) failed (CUresult %d)", (int)r);
+  return SQA_OK;
+}
+
+int sm_count() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+// One K segment of a GEMM: A (K-major [M][k] or MN-major [k][M]) and B
+// (K-major [N][k] or MN-major [k][N]), row-major bf16 with row strides lda, ldb.
+struct GemmSeg {
+  const void* a;
+  const void* b;
+  int k;
+  long long lda, ldb;
+};
+
+// D[M x N] = sum_s A_s B_s with the epilogue in `p` (mode and outputs set by
+// the caller).  split_k > 1 only with the fp32 reduction epilogue.
+template <int BN, bool A_MN, bool B_MN>
+sqa_status launch_gemm(int M, int N, const GemmSeg* segs, int n_seg, int split_k, sqa::GemmParams p,
+                       cudaStream_t stream) {
+  using Tr = sqa::GemmTraits<BN>;
+  CUtensorMap ma[3], mb[3];
+  sqa_status st;
+  int blocks = 0;
+  for (int i = 0; i < 3; ++i) {
+    const GemmSeg& sg = segs[i < n_seg ? i : 0];
+    if ((st = A_MN ? make_map_2d(&ma[i], sg.a, sg.k, M, sg.lda, 64) : make_map_2d(&ma[i], sg.a, M, sg.k, sg.lda, 128)) !=
+        SQA_OK)
+      return st;
+    if ((st = B_MN ? make_map_2d(&mb[i], sg.b, sg.k, N, sg.ldb, 64) : make_map_2d(&mb[i], sg.b, N, sg.k, sg.ldb, BN)) !=
+        SQA_OK)
+      return st;
+    if (i < n_seg) {
+      p.kseg[i] = sg.k;
+      p.kblk0[i] = blocks;
+      blocks += (sg.k + Tr::BK - 1) / Tr::BK;
+    }
+  }
+  p.kblk0[n_seg] = blocks;
+  p.M = M;
+  p.N = N;
+  p.n_seg = n_seg;
+  p.tiles_m = (M + Tr::BM - 1) / Tr::BM;
+  p.tiles_n = (N + BN - 1) / BN;
+  p.split_k = split_k < 1 ? 1 : (split_k > blocks ? blocks : split_k);
+  const long long items = static_cast<long long>(p.tiles_m) * p.tiles_n * p.split_k;
+  if (items > 0x7fffffffLL) return fail(SQA_ERR_UNSUPPORTED, "GEMM too large for one launch");
+  p.n_items = static_cast<int>(items);
+  const int sms = sm_count();
+  const unsigned grid = static_cast<unsigned>(items < sms ? items : sms);
+  if ((st = set_smem(sqa::sqa_gemm_kernel<BN, A_MN, B_MN>, Tr::SMEM_BYTES)) != SQA_OK) return st;
+  sqa::sqa_gemm_kernel<BN, A_MN, B_MN>
+      <<<grid, Tr::THREADS, Tr::SMEM_BYTES, stream>>>(ma[0], ma[1], ma[2], mb[0], mb[1], mb[2], p);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "sqa_gemm launch");
+  return SQA_OK;
+}
+
+// Column tile width for an output of N columns.
+template <bool A_MN, bool B_MN>
+sqa_status gemm(int M, int N, const GemmSeg* segs, int n_seg, int split_k, const sqa::GemmParams& p,
+                cudaStream_t stream) {
+  if (N > 128) return launch_gemm<256, A_MN, B_MN>(M, N, segs, n_seg, split_k, p, stream);
+  if (N > 64) return launch_gemm<128, A_MN, B_MN>(M, N, segs, n_seg, split_k, p, stream);
+  return launch_gemm<64, A_MN, B_MN>(M, N, segs, n_seg, split_k, p, stream);
+}
+
+// K splits for a reduction GEMM with few output tiles: about one item per SM,
+// at least four K blocks per item.
+int split_for(int M, int N, int K) {
+  const long long tiles = static_cast<long long>((M + 127) / 128) * ((N + 255) / 256);
+  const int kblocks = (K + 63) / 64;
+  long long s = (sm_count() + tiles - 1) / tiles;
+  if (s > kblocks / 4) s = kblocks / 4;
+  return s < 1 ? 1 : static_cast<int>(s);
+}
+
+struct LayerLayout {
+  size_t off_dout, off_dq, off_dk, off_dv, off_core, fwd_bytes, bwd_bytes;
+};
+
+LayerLayout layer_layout(const sqa_layer_shape& s) {
+  LayerLayout L{};
+  const size_t M = static_cast<size_t>(s.B) * s.N;
+  const size_t table = sqa::align256(static_cast<size_t>(s.N) * (s.dh / 2) * sizeof(float2));
+  L.fwd_bytes = table;
+  L.off_dout = table;
+  L.off_dq = L.off_dout + sqa::align256(M * s.H_q * s.dh * 2);
+  L.off_dk = L.off_dq + sqa::align256(M * s.H_q * s.dh * 2);
+  L.off_dv = L.off_dk + sqa::align256(M * s.H_kv * s.dh * 2);
+  L.off_core = L.off_dv + sqa::align256(M * s.H_kv * s.dh * 2);
+  L.bwd_bytes = L.off_core + sqa::bwd_workspace_bytes(s.B, s.N, s.H_q, s.H_kv, s.dh);
+  return L;
+}
+
+sqa_status check_layer_shape(const sqa_layer_shape& s) {
+  const sqa_shape core{s.B, s.N, s.H_q, s.H_kv, s.dh};
+  sqa_status st = check_shape(core);
+  if (st != SQA_OK) return st;
+  if (s.d < 1) return fail(SQA_ERR_INVALID_ARG, "model width d=%d must be positive", s.d);
+  if (s.d % 8 != 0) return fail(SQA_ERR_UNSUPPORTED, "model width d=%d must be a multiple of 8", s.d);
+  if (static_cast<long long>(s.B) * s.N > 0x7fffffffLL)
+    return fail(SQA_ERR_UNSUPPORTED, "B * N must fit in a 32-bit int");
+  return SQA_OK;
+}
+
+sqa_status rope_table(float2* cs, const sqa_layer_shape& s, float base, cudaStream_t stream) {
+  const long long n = static_cast<long long>(s.N) * (s.dh / 2);
+  sqa::sqa_rope_table_kernel<<<grid_for(n, 256), 256, 0, stream>>>(cs, s.N, s.dh, static_cast<double>(base));
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "rotary table launch");
   return SQA_OK;
 }
 
@@ -509,6 +650,152 @@ sqa_status sqa_bwd_static_scratch(const void* dout, const void* q, const void* k
   void* scratch = nullptr;
   if ((st = static_scratch_address(reinterpret_cast<cudaStream_t>(stream), &scratch)) != SQA_OK) return st;
   return sqa_bwd(dout, q, k, v, out, lse, dq, dk, dv, scratch, SQA_STATIC_SCRATCH_BYTES, s, causal, scale, stream);
+}
+
+size_t sqa_layer_workspace_bytes(sqa_layer_shape s, int backward) {
+  if (check_layer_shape(s) != SQA_OK) return 0;
+  const LayerLayout L = layer_layout(s);
+  return backward ? L.bwd_bytes : L.fwd_bytes;
+}
+
+sqa_status sqa_layer_fwd(const void* x, const void* w_qkv, const void* w_o, void* y, void* q, void* k, void* v,
+                         void* out, float* lse, void* workspace, size_t workspace_bytes, sqa_layer_shape s,
+                         int causal, float scale, float rope_base, sqa_stream_t stream) {
+  g_last_error.clear();
+  if (!x || !w_qkv || !w_o || !y || !q || !k || !v || !out || !lse || !workspace)
+    return fail(SQA_ERR_INVALID_ARG, "null pointer argument");
+  sqa_status st = check_layer_shape(s);
+  if (st != SQA_OK) return st;
+  const void* bf[] = {x, w_qkv, w_o, y, q, k, v, out};
+  for (const void* ptr : bf)
+    if (!aligned(ptr, 16)) return fail(SQA_ERR_UNSUPPORTED, "bf16 tensors must be 16-byte aligned");
+  if (!aligned(lse, 4)) return fail(SQA_ERR_UNSUPPORTED, "lse must be 4-byte aligned");
+  if (!aligned(workspace, 256)) return fail(SQA_ERR_UNSUPPORTED, "workspace must be 256-byte aligned");
+  const LayerLayout L = layer_layout(s);
+  if (workspace_bytes < L.fwd_bytes)
+    return fail(SQA_ERR_INVALID_ARG, "workspace holds %zu bytes, %zu needed", workspace_bytes, L.fwd_bytes);
+  if (std::isnan(rope_base) || std::isinf(rope_base) || rope_base < 0.f)
+    return fail(SQA_ERR_INVALID_ARG, "rope_base must be finite and non-negative");
+  float sc;
+  if ((st = resolve_scale(scale, s.dh, &sc)) != SQA_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const int M = s.B * s.N, nq = s.H_q * s.dh, nk = s.H_kv * s.dh, wqkv = nq + 2 * nk;
+  float2* table = static_cast<float2*>(workspace);
+  if (rope_base > 0.f && (st = rope_table(table, s, rope_base, cs)) != SQA_OK) return st;
+  // Q | K | V = X W_qkv, rotary embedding on Q and K in the epilogue.
+  sqa::GemmParams gp{};
+  gp.mode = sqa::kQkvRope;
+  gp.q = static_cast<__nv_bfloat16*>(q);
+  gp.k = static_cast<__nv_bfloat16*>(k);
+  gp.v = static_cast<__nv_bfloat16*>(v);
+  gp.nq = nq;
+  gp.nk = nk;
+  gp.nv = nk;
+  gp.dh = s.dh;
+  gp.n_tokens = s.N;
+  gp.rope_cs = rope_base > 0.f ? table : nullptr;
+  const GemmSeg g_qkv{x, w_qkv, s.d, s.d, wqkv};
+  if ((st = gemm<false, true>(M, wqkv, &g_qkv, 1, 1, gp, cs)) != SQA_OK) return st;
+  // the attention core
+  const sqa_shape core{s.B, s.N, s.H_q, s.H_kv, s.dh};
+  switch (s.dh) {
+    case 16: st = launch_fwd<16>(q, k, v, out, lse, core, causal, sc, cs); break;
+    case 32: st = launch_fwd<32>(q, k, v, out, lse, core, causal, sc, cs); break;
+    case 64: st = launch_fwd<64>(q, k, v, out, lse, core, causal, sc, cs); break;
+    default: st = launch_fwd<128>(q, k, v, out, lse, core, causal, sc, cs); break;
+  }
+  if (st != SQA_OK) return st;
+  // Y = O W_o
+  sqa::GemmParams go{};
+  go.mode = sqa::kStoreBf16;
+  go.out = static_cast<__nv_bfloat16*>(y);
+  go.ld_out = s.d;
+  const GemmSeg g_o{out, w_o, nq, nq, s.d};
+  return gemm<false, true>(M, s.d, &g_o, 1, 1, go, cs);
+}
+
+sqa_status sqa_layer_bwd(const void* dy, const void* x, const void* w_qkv, const void* w_o, const void* q,
+                         const void* k, const void* v, const void* out, const float* lse, void* dx, float* dw_qkv,
+                         float* dw_o, void* workspace, size_t workspace_bytes, sqa_layer_shape s, int causal,
+                         float scale, float rope_base, sqa_stream_t stream) {
+  g_last_error.clear();
+  if (!dy || !x || !w_qkv || !w_o || !q || !k || !v || !out || !lse || !dx || !dw_qkv || !dw_o || !workspace)
+    return fail(SQA_ERR_INVALID_ARG, "null pointer argument");
+  sqa_status st = check_layer_shape(s);
+  if (st != SQA_OK) return st;
+  const void* bf[] = {dy, x, w_qkv, w_o, q, k, v, out, dx, dw_qkv, dw_o};
+  for (const void* ptr : bf)
+    if (!aligned(ptr, 16)) return fail(SQA_ERR_UNSUPPORTED, "tensors must be 16-byte aligned");
+  if (!aligned(lse, 4)) return fail(SQA_ERR_UNSUPPORTED, "lse must be 4-byte aligned");
+  if (!aligned(workspace, 256)) return fail(SQA_ERR_UNSUPPORTED, "workspace must be 256-byte aligned");
+  const LayerLayout L = layer_layout(s);
+  if (workspace_bytes < L.bwd_bytes)
+    return fail(SQA_ERR_INVALID_ARG, "workspace holds %zu bytes, %zu needed", workspace_bytes, L.bwd_bytes);
+  if (std::isnan(rope_base) || std::isinf(rope_base) || rope_base < 0.f)
+    return fail(SQA_ERR_INVALID_ARG, "rope_base must be finite and non-negative");
+  float sc;
+  if ((st = resolve_scale(scale, s.dh, &sc)) != SQA_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const int M = s.B * s.N, nq = s.H_q * s.dh, nk = s.H_kv * s.dh, wqkv = nq + 2 * nk;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float2* table = reinterpret_cast<float2*>(ws);
+  void* dout = ws + L.off_dout;
+  void* dq = ws + L.off_dq;
+  void* dk = ws + L.off_dk;
+  void* dv = ws + L.off_dv;
+  void* core_ws = ws + L.off_core;
+  if (rope_base > 0.f && (st = rope_table(table, s, rope_base, cs)) != SQA_OK) return st;
+  // dO = dY W_o^T (W_o is [H_q dh][d]: K-major for this product)
+  sqa::GemmParams p1{};
+  p1.mode = sqa::kStoreBf16;
+  p1.out = static_cast<__nv_bfloat16*>(dout);
+  p1.ld_out = nq;
+  const GemmSeg g1{dy, w_o, s.d, s.d, s.d};
+  if ((st = gemm<false, false>(M, nq, &g1, 1, 1, p1, cs)) != SQA_OK) return st;
+  // dW_o = O^T dY, reduced over all tokens (split over K, fp32 reductions)
+  cudaError_t e = cudaMemsetAsync(dw_o, 0, static_cast<size_t>(nq) * s.d * sizeof(float), cs);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dw_qkv, 0, static_cast<size_t>(s.d) * wqkv * sizeof(float), cs);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (weight gradients)");
+  sqa::GemmParams p2{};
+  p2.mode = sqa::kAtomicF32;
+  p2.out32 = dw_o;
+  p2.ld_out32 = s.d;
+  const GemmSeg g2{out, dy, M, nq, s.d};
+  if ((st = gemm<true, true>(nq, s.d, &g2, 1, split_for(nq, s.d, M), p2, cs)) != SQA_OK) return st;
+  // the attention core's backward, then the rotation undone on dQ and dK
+  const sqa_shape core{s.B, s.N, s.H_q, s.H_kv, s.dh};
+  const size_t core_bytes = sqa::bwd_workspace_bytes(s.B, s.N, s.H_q, s.H_kv, s.dh);
+  if ((st = sqa_bwd(dout, q, k, v, out, lse, dq, dk, dv, core_ws, core_bytes, core, causal, scale, stream)) !=
+      SQA_OK)
+    return st;
+  if (rope_base > 0.f) {
+    sqa::sqa_rope_inverse_kernel<<<grid_for(static_cast<long long>(M) * nq / 8, 256), 256, 0, cs>>>(
+        static_cast<__nv_bfloat16*>(dq), M, nq, s.dh, s.N, table);
+    sqa::sqa_rope_inverse_kernel<<<grid_for(static_cast<long long>(M) * nk / 8, 256), 256, 0, cs>>>(
+        static_cast<__nv_bfloat16*>(dk), M, nk, s.dh, s.N, table);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "inverse rotary launch");
+  }
+  // dW_qkv = X^T [dQ | dK | dV], one product per part into its columns
+  const void* parts[3] = {dq, dk, dv};
+  const int widths[3] = {nq, nk, nk}, col0[3] = {0, nq, nq + nk};
+  for (int i = 0; i < 3; ++i) {
+    sqa::GemmParams p3{};
+    p3.mode = sqa::kAtomicF32;
+    p3.out32 = dw_qkv + col0[i];
+    p3.ld_out32 = wqkv;
+    const GemmSeg g3{x, parts[i], M, s.d, widths[i]};
+    if ((st = gemm<true, true>(s.d, widths[i], &g3, 1, split_for(s.d, widths[i], M), p3, cs)) != SQA_OK) return st;
+  }
+  // dX = dQ W_q^T + dK W_k^T + dV W_v^T: three K segments, W_qkv's column
+  // blocks as K-major B operands
+  sqa::GemmParams p4{};
+  p4.mode = sqa::kStoreBf16;
+  p4.out = static_cast<__nv_bfloat16*>(dx);
+  p4.ld_out = s.d;
+  const __nv_bfloat16* w = static_cast<const __nv_bfloat16*>(w_qkv);
+  const GemmSeg g4[3] = {{dq, w, nq, nq, wqkv}, {dk, w + nq, nk, nk, wqkv}, {dv, w + nq + nk, nk, nk, wqkv}};
+  return gemm<false, false>(M, s.d, g4, 3, 1, p4, cs);
 }
 
 sqa_status sqa_selftest_exp2_poly(const float* x, float* y, int n, sqa_stream_t stream) {

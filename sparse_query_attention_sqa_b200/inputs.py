@@ -116,3 +116,16 @@ def workload_inputs(w: Workload, seed: int = 0):
         return (*make_decode_inputs(w.B, w.N, w.Hq, w.Hkv, w.dh, seed=seed, std=w.std, k_scale=w.k_scale), None)
     return make_inputs(w.B, w.N, w.Hq, w.Hkv, w.dh, seed=seed, std=w.std, k_scale=w.k_scale,
                        with_dout=w.backward)
+
+
+def make_layer_inputs(B: int, N: int, d: int, Hq: int, Hkv: int, dh: int, seed: int = 0):
+    """Draw x [B,N,d], the fused projection w_qkv [d, (Hq + 2 Hkv) dh], w_o
+    [Hq dh, d] and the upstream gradient dy [B,N,d] (CPU bf16), in that order.
+    x and dy are standard normal; each weight has standard deviation
+    1/sqrt(fan-in), so the projections keep unit variance."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    x = torch.randn(B, N, d, generator=g).to(torch.bfloat16)
+    w_qkv = (torch.randn(d, (Hq + 2 * Hkv) * dh, generator=g) * d ** -0.5).to(torch.bfloat16)
+    w_o = (torch.randn(Hq * dh, d, generator=g) * (Hq * dh) ** -0.5).to(torch.bfloat16)
+    dy = torch.randn(B, N, d, generator=g).to(torch.bfloat16)
+    return x, w_qkv, w_o, dy

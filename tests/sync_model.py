@@ -51,15 +51,18 @@ class Buffer:
         self.ended += 1
 
 
-def run(roles, counts, stages, seed, custom=None):
+def run(roles, counts, stages, seed, custom=None, skewed=False):
     """One random interleaving of ``roles``; ``counts``: barrier -> arrivals per
     phase; ``stages``: buffer kind -> [(description, users)]; ``custom``:
-    buffer name -> object with begin(slot, info) and end(slot, info)."""
+    buffer name -> object with begin(slot, info) and end(slot, info).
+    ``skewed``: give each role a random speed for the whole run (a role may then
+    lag far behind the others), instead of picking ready roles uniformly."""
     done = {b: 0 for b in counts}
     arrived = {b: 0 for b in counts}
     bufs = {}
     pc = {r: 0 for r in roles}
     rnd = random.Random(seed)
+    speed = {r: (10.0 ** rnd.uniform(-3, 0) if skewed else 1.0) for r in roles}
     while True:
         ready = []
         for r, ops in roles.items():
@@ -75,7 +78,7 @@ def run(roles, counts, stages, seed, custom=None):
                     ready.append(r)
         if not ready:
             break
-        r = rnd.choice(ready)
+        r = rnd.choices(ready, weights=[speed[x] for x in ready])[0] if skewed else rnd.choice(ready)
         op = roles[r][pc[r]]
         pc[r] += 1
         if op[0] == "arrive":

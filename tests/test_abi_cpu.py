@@ -205,3 +205,32 @@ def _bwd_ws_expected(B, N, Hq, Hkv, dh):
                                    (3, 77, 128, 1, 64), (1, 1, 16, 16, 16), (1, 200000, 8, 4, 16)])
 def test_bwd_workspace_follows_its_layout(lib, shape):
     assert lib.sqa_bwd_workspace_bytes(sqa.Shape(*shape)) == _bwd_ws_expected(*shape)
+
+
+def test_layer_rejects_bad_arguments_before_launch(lib):
+    s = sqa.LayerShape(2, 256, 256, 8, 4, 16)
+    need_f = lib.sqa_layer_workspace_bytes(s, 0)
+    need_b = lib.sqa_layer_workspace_bytes(s, 1)
+    # forward: the rotary table [N][dh/2] of (cos, sin); backward adds dO, dQ,
+    # dK, dV and the core's workspace
+    assert need_f == 256 * 8 * 8
+    core = lib.sqa_bwd_workspace_bytes(sqa.Shape(2, 256, 8, 4, 16))
+    assert need_b == need_f + 2 * (2 * 256 * 128 * 2) + 2 * (2 * 256 * 64 * 2) + core
+    assert lib.sqa_layer_workspace_bytes(sqa.LayerShape(2, 256, 250, 8, 4, 16), 0) == 0  # d % 8 != 0
+    p = 0x10000
+    args = [p] * 9 + [p, need_f]
+    st = lib.sqa_layer_fwd(*([0] + args[1:]), s, 1, 0.0, 10000.0, None)
+    assert st == sqa.SQA_ERR_INVALID_ARG
+    st = lib.sqa_layer_fwd(*args[:10], need_f - 1, s, 1, 0.0, 10000.0, None)
+    assert st == sqa.SQA_ERR_INVALID_ARG and b"workspace" in lib.sqa_last_error()
+    st = lib.sqa_layer_fwd(*args, s, 1, 0.0, -1.0, None)
+    assert st == sqa.SQA_ERR_INVALID_ARG and b"rope_base" in lib.sqa_last_error()
+    st = lib.sqa_layer_fwd(*args, sqa.LayerShape(2, 256, 250, 8, 4, 16), 1, 0.0, 10000.0, None)
+    assert st == sqa.SQA_ERR_UNSUPPORTED
+    st = lib.sqa_layer_fwd(*args, sqa.LayerShape(2, 256, 256, 6, 4, 16), 1, 0.0, 10000.0, None)
+    assert st == sqa.SQA_ERR_INVALID_ARG
+    bargs = [p] * 13 + [need_b]
+    st = lib.sqa_layer_bwd(*bargs[:12], 0, need_b, s, 1, 0.0, 10000.0, None)
+    assert st == sqa.SQA_ERR_INVALID_ARG
+    st = lib.sqa_layer_bwd(*bargs[:13], need_b - 256, s, 1, 0.0, 10000.0, None)
+    assert st == sqa.SQA_ERR_INVALID_ARG and b"workspace" in lib.sqa_last_error()
