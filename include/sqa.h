@@ -273,6 +273,20 @@ sqa_status sqa_decode(const void *q, const void *k_cache, const void *v_cache, c
  */
 sqa_status sqa_selftest_exp2_poly(const float *x, float *y, int n, sqa_stream_t stream);
 
+/*
+ * Self-test hook for the kernels' bounded waits, so that tests can exercise
+ * the failure path without faulting or hanging a GPU; the pages have no
+ * counterpart.  Launches one small kernel on `stream` whose thread waits on an
+ * mbarrier that nothing ever completes, through the same bounded wait the
+ * attention kernels use, but giving up after limit_us microseconds (1 to
+ * 100000) instead of about two seconds.  It then sets bit `site` (0 to 4, the
+ * roles of sqa_device_timeout_info) in the device status word, records itself
+ * in the timeout record if that is empty (block 0, thread 0, parity 0) and
+ * returns; the context stays usable.  SQA_ERR_INVALID_ARG for limits or sites
+ * out of range, before any launch.
+ */
+sqa_status sqa_selftest_wait_timeout(unsigned int limit_us, unsigned int site, sqa_stream_t stream);
+
 /* Library version as an integer (major * 10000 + minor * 100 + patch). */
 int sqa_version(void);
 

@@ -277,6 +277,24 @@ __global__ void exp2_poly_kernel(const float* x, float* y, int n) {
   }
 }
 
+// Self-test of the bounded waits: one thread waits on an mbarrier that nothing
+// ever arrives on, with the given limit, through the same slow path the
+// kernels use; it gives up, records `site` in the device status word and the
+// timeout record, and the kernel returns.
+__global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns, unsigned site) {
+  __shared__ __align__(8) unsigned long long bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    sqa::dev::mbar_init(sqa::dev::smem_u32(&bar), 1);
+    abort_flag = 0;
+    sqa::dev::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)
+    sqa::dev::mbar_wait_slow(sqa::dev::smem_u32(&bar), 0, &abort_flag, site, limit_ns);
+  __syncthreads();
+}
+
 int grid_for(long long work, int threads) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -807,6 +825,16 @@ sqa_status sqa_selftest_exp2_poly(const float* x, float* y, int n, sqa_stream_t 
   exp2_poly_kernel<<<grid_for(pairs, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "sqa_selftest_exp2_poly launch");
+  return SQA_OK;
+}
+
+sqa_status sqa_selftest_wait_timeout(unsigned int limit_us, unsigned int site, sqa_stream_t stream) {
+  g_last_error.clear();
+  if (limit_us < 1 || limit_us > 100000) return fail(SQA_ERR_INVALID_ARG, "limit_us must be in [1, 100000]");
+  if (site > 4) return fail(SQA_ERR_INVALID_ARG, "site must be in [0, 4]");
+  wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(1000ull * limit_us, site);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "sqa_selftest_wait_timeout launch");
   return SQA_OK;
 }
 

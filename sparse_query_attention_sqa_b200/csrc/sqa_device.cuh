@@ -84,18 +84,18 @@ __device__ __forceinline__ bool mbar_test_sleep(uint32_t bar, uint32_t parity, u
 
 // Wait for the phase of `bar` with the given parity (mbar_wait below is the
 // entry point).  Gives up when another
-// role of the CTA has raised `abort_flag`, or after kWaitLimitNs (then it
+// role of the CTA has raised `abort_flag`, or after limit_ns (then it
 // raises the flag and records `site` in the device status word).  Returns
 // true when the phase completed.
 __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                            unsigned site) {
+                                            unsigned site, unsigned long long limit_ns = kWaitLimitNs) {
   const unsigned long long t0 = global_timer_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 8; ++i)
       if (mbar_test_sleep(bar, parity, 20000u)) return true;
     if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       atomicOr(&g_wait_status, 1u << site);
       if (atomicCAS(&g_timeout_info[0], 0u, 1u) == 0u) {

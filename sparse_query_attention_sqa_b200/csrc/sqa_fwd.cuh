@@ -54,7 +54,12 @@ struct FwdParams {
 template <int DH>
 struct FwdTraits {
   static constexpr int BM = 128;  // stacked rows per Q tile
-  static constexpr int NK = 64;   // keys per K/V tile
+  // Keys per K/V tile.  At dh = 128 a tile of 128 keys makes S = Q K^T an
+  // N = 128 MMA, which reads its operands from shared memory no faster than it
+  // computes (at N = 64 the reads take longer than the math); the 128 columns
+  // of a tile's S region then hold one S buffer instead of two.
+  static constexpr int NK = DH == 128 ? 128 : 64;
+  static constexpr int NSBUF = NK == 128 ? 1 : 2;  // S buffers per Q tile
   static constexpr int PANEL = DH < 64 ? DH : 64;  // elements per swizzled row segment
   static constexpr int NPANEL = DH / PANEL;
   static constexpr int ROWB = PANEL * 2;  // bytes per row segment
@@ -62,7 +67,7 @@ struct FwdTraits {
   static constexpr int Q_BYTES = BM * DH * 2;
   static constexpr int KV_BYTES = NK * DH * 2;
   static constexpr int QBUF = DH <= 64 ? 2 : 1;  // Q-tile pairs in flight
-  static constexpr int STAGES = DH <= 32 ? 8 : (DH == 64 ? 4 : 3);
+  static constexpr int STAGES = DH <= 32 ? 8 : (DH == 64 ? 4 : (NK == 128 ? 2 : 3));
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + QBUF * 2 * Q_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
@@ -114,6 +119,7 @@ __global__ void __launch_bounds__(384, 1)
   using Tr = FwdTraits<DH>;
   using namespace dev;
   constexpr int BM = Tr::BM, NK = Tr::NK, ROWB = Tr::ROWB, PANEL = Tr::PANEL, ST = Tr::STAGES, QB = Tr::QBUF;
+  constexpr int NSB = Tr::NSBUF;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -248,8 +254,9 @@ __global__ void __launch_bounds__(384, 1)
     auto issue_pv = [&](int s, int buf, bool acc) {
       const uint64_t b0 = dv0 + static_cast<uint64_t>((s * Tr::KV_BYTES) >> 4);
 #pragma unroll
-      for (int ks = 0; ks < NK / 16; ++ks)
-        mma_ts_w(tO, tS0 + 64u * buf + ks * 8, b0 + ((ks * 16 * ROWB) >> 4), idesc_pv, (acc || ks > 0) ? 1u : 0u);
+      for (int ks = 0; ks < NK / 16; ++ks)  // P of keys 16 ks .. + 15: column 64 (ks / 4) + 8 (ks % 4)
+        mma_ts_w(tO, tS0 + 64u * buf + 64u * (ks >> 2) + 8u * (ks & 3), b0 + ((ks * 16 * ROWB) >> 4), idesc_pv,
+                 (acc || ks > 0) ? 1u : 0u);
       mma_commit_w(o_done(t));
     };
     int loaded = 0;  // K/V tiles whose kv_full phase this warp has observed
@@ -275,13 +282,13 @@ __global__ void __launch_bounds__(384, 1)
         ok = false;
         break;
       }
-      for (int j = 0; ok && j < 2 && j < nkv_t; ++j) {  // prologue: S for key tiles 0 and 1
+      for (int j = 0; ok && j < NSB && j < nkv_t; ++j) {  // prologue: S for the first key tiles
         ok = ensure_loaded(g + j);
-        if (ok) issue_qk(qb, (g + j) % ST, (G + j) & 1);
+        if (ok) issue_qk(qb, (g + j) % ST, (G + j) % NSB);
       }
       for (int j = 0; ok && j < nkv_t; ++j) {
         const int Gt = G + j;
-        if (!mbar_wait_warp(p_full(t, Gt & 1), (Gt >> 1) & 1, abort_flag, kSiteMma)) {
+        if (!mbar_wait_warp(p_full(t, Gt % NSB), (Gt / NSB) & 1, abort_flag, kSiteMma)) {
           ok = false;
           break;
         }
@@ -291,15 +298,15 @@ __global__ void __launch_bounds__(384, 1)
           break;
         }
         tc_fence_after();
-        issue_pv((g + j) % ST, Gt & 1, j > 0);
-        if (j + 2 < nkv_t) {
+        issue_pv((g + j) % ST, Gt % NSB, j > 0);
+        if (j + NSB < nkv_t) {
           // The next S in this buffer: the PV just issued reads P from it first
           // (MMAs from one issuer execute in order).
-          if (!ensure_loaded(g + j + 2)) {
+          if (!ensure_loaded(g + j + NSB)) {
             ok = false;
             break;
           }
-          issue_qk(qb, (g + j + 2) % ST, Gt & 1);
+          issue_qk(qb, (g + j + NSB) % ST, Gt % NSB);
         }
         if (j + 1 == nkv_t) mma_commit_w(o_final(t));
         mma_commit_w(kv_empty((g + j) % ST));
@@ -342,34 +349,44 @@ __global__ void __launch_bounds__(384, 1)
         const int Gt = G + j;
         // Every lane waits; the verdict is made warp-uniform so that the
         // warp-wide TMEM instructions below are never reached divergently.
-        ok = __all_sync(0xffffffffu, mbar_wait(s_full(t, Gt & 1), (Gt >> 1) & 1, abort_flag, kSiteSoftmax));
+        ok = __all_sync(0xffffffffu, mbar_wait(s_full(t, Gt % NSB), (Gt / NSB) & 1, abort_flag, kSiteSoftmax));
         if (!ok) break;
         tc_fence_after();
-        const uint32_t tS = lane_addr + Tr::tm_s(t, Gt & 1);
+        const uint32_t tS = lane_addr + Tr::tm_s(t, Gt % NSB);
         const int k0 = j * NK;
         const bool masked = (k0 + NK > p.N) || (p.causal && k0 + NK - 1 > qt * p.T);
-        uint32_t sr[NK];
-        tmem_ld32x2(tS, tS + 32, sr);
-        if (masked) {
-          // last visible key of this tile, relative to k0 (may be negative)
-          const int last = min(p.N - 1, p.causal ? tok : p.N - 1) - k0;
+        // The tile's scores are handled 64 columns (a half at NK = 128) at a time.
+        // last visible key of this tile, relative to k0 (may be negative)
+        const int last = min(p.N - 1, p.causal ? tok : p.N - 1) - k0;
+        uint32_t sr[64];
+        auto load64 = [&](int h) {
+          tmem_ld32x2(tS + 64 * h, tS + 64 * h + 32, sr);
+          if (masked) {
 #pragma unroll
-          for (int i = 0; i < NK; ++i)
-            if (i > last) sr[i] = __float_as_uint(-INFINITY);
+            for (int i = 0; i < 64; ++i)
+              if (i + 64 * h > last) sr[i] = __float_as_uint(-INFINITY);
+          }
+        };
+        // Row maximum: eight independent chains of three-input maxima per half.
+        auto max64 = [&]() {
+          float acc[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            acc[c] = fmax3(__uint_as_float(sr[c]), __uint_as_float(sr[8 + c]), __uint_as_float(sr[16 + c]));
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            acc[c] = fmax3(acc[c], __uint_as_float(sr[24 + c]), __uint_as_float(sr[32 + c]));
+            acc[c] = fmax3(acc[c], __uint_as_float(sr[40 + c]), __uint_as_float(sr[48 + c]));
+            acc[c] = fmaxf(acc[c], __uint_as_float(sr[56 + c]));
+          }
+          return fmax3(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], acc[5]), fmaxf(acc[6], acc[7]));
+        };
+        float mx = -INFINITY;
+#pragma unroll
+        for (int h = 0; h < NK / 64; ++h) {
+          load64(h);
+          mx = fmaxf(mx, max64());
         }
-        // Row maximum: eight independent chains of three-input maxima.
-        float acc[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          acc[c] = fmax3(__uint_as_float(sr[c]), __uint_as_float(sr[8 + c]), __uint_as_float(sr[16 + c]));
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          acc[c] = fmax3(acc[c], __uint_as_float(sr[24 + c]), __uint_as_float(sr[32 + c]));
-          acc[c] = fmax3(acc[c], __uint_as_float(sr[40 + c]), __uint_as_float(sr[48 + c]));
-          acc[c] = fmaxf(acc[c], __uint_as_float(sr[56 + c]));
-        }
-        const float mx =
-            fmax3(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], acc[5]), fmaxf(acc[6], acc[7]));
         const float mnew = fmaxf(m, mx * sl2);
         const bool raise = mnew > m + 8.f;
         const float alpha = (raise && m != -INFINITY) ? ex2(m - mnew) : 1.f;
@@ -396,43 +413,52 @@ __global__ void __launch_bounds__(384, 1)
         float sum0[8], sum1[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) sum0[c] = sum1[c] = 0.f;
-        uint32_t pk[NK / 2];
-        if (!masked) {
-          // POLY of every 8 pairs take the FMA-pipe exponential, the rest the
-          // special-function unit, so that neither pipe alone sets the pace.
+        // P (bf16 pairs) of the 64 keys of half h goes to columns 64 h .. 64 h + 31,
+        // over scores already consumed.  At NK = 128 the second half is still in
+        // registers from the maximum pass and goes first, then the first half is
+        // loaded again.
 #pragma unroll
-          for (int i = 0; i < NK / 2; ++i) {
-            float x0, x1, p0, p1;
-            ffma2(x0, x1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), sl2, sl2, nref, nref);
-            if ((i & 7) * POLY % 8 + POLY >= 8) {  // POLY evenly spread indices of 0..7
-              const float2 pp = exp2_poly2(x0, x1);
-              p0 = pp.x;
-              p1 = pp.y;
-            } else {
-              p0 = ex2(x0);
-              p1 = ex2(x1);
+        for (int hh = 0; hh < NK / 64; ++hh) {
+          const int h = NK / 64 - 1 - hh;
+          if (hh > 0) load64(h);
+          uint32_t pk[32];
+          if (!masked) {
+            // POLY of every 8 pairs take the FMA-pipe exponential, the rest the
+            // special-function unit, so that neither pipe alone sets the pace.
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              float x0, x1, p0, p1;
+              ffma2(x0, x1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), sl2, sl2, nref, nref);
+              if ((i & 7) * POLY % 8 + POLY >= 8) {  // POLY evenly spread indices of 0..7
+                const float2 pp = exp2_poly2(x0, x1);
+                p0 = pp.x;
+                p1 = pp.y;
+              } else {
+                p0 = ex2(x0);
+                p1 = ex2(x1);
+              }
+              fadd2(sum0[i & 7], sum1[i & 7], sum0[i & 7], sum1[i & 7], p0, p1);
+              pk[i] = pack_bf16x2(p0, p1);
             }
-            fadd2(sum0[i & 7], sum1[i & 7], sum0[i & 7], sum1[i & 7], p0, p1);
-            pk[i] = pack_bf16x2(p0, p1);
-          }
-        } else {
-          // Masked scores are -inf: the special-function unit gives exactly 0 there.
+          } else {
+            // Masked scores are -inf: the special-function unit gives exactly 0 there.
 #pragma unroll
-          for (int i = 0; i < NK / 2; ++i) {
-            float x0, x1;
-            ffma2(x0, x1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), sl2, sl2, nref, nref);
-            const float p0 = ex2(x0), p1 = ex2(x1);
-            fadd2(sum0[i & 7], sum1[i & 7], sum0[i & 7], sum1[i & 7], p0, p1);
-            pk[i] = pack_bf16x2(p0, p1);
+            for (int i = 0; i < 32; ++i) {
+              float x0, x1;
+              ffma2(x0, x1, __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]), sl2, sl2, nref, nref);
+              const float p0 = ex2(x0), p1 = ex2(x1);
+              fadd2(sum0[i & 7], sum1[i & 7], sum0[i & 7], sum1[i & 7], p0, p1);
+              pk[i] = pack_bf16x2(p0, p1);
+            }
           }
+          tmem_st32(tS + 64 * h, pk);
         }
-        tmem_st32(tS, pk);
 #pragma unroll
         for (int c = 0; c < 4; ++c) fadd2(sum0[c], sum1[c], sum0[c], sum1[c], sum0[c + 4], sum1[c + 4]);
         l += ((sum0[0] + sum1[0]) + (sum0[1] + sum1[1])) + ((sum0[2] + sum1[2]) + (sum0[3] + sum1[3]));
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(p_full(t, Gt & 1));
+        mbar_arrive(p_full(t, Gt % NSB));
       }
       if (!ok) break;
       ok = __all_sync(0xffffffffu, mbar_wait(o_final(t), nd & 1, abort_flag, kSiteEpilogue));
