@@ -189,6 +189,64 @@ sqa_status sqa_layer_bwd(const void *dy, const void *x, const void *w_qkv, const
                          sqa_layer_shape s, int causal, float scale, float rope_base,
                          sqa_stream_t stream);
 
+/*
+ * One SQAT-m decoder block (SQAT-m model card, "Architecture details": SQA,
+ * RoPE, RMS Norm and a SwiGLU feed-forward of hidden width 768), read as the
+ * plain pre-norm residual block with no biases:
+ *
+ *   n1 = RMSNorm(x; g1),  h = x + SQA layer(n1),
+ *   n2 = RMSNorm(h; g2),  y = h + (silu(n2 W1) * (n2 W3)) W2,
+ *   RMSNorm(x; g) = g * x / sqrt(mean over the d features of x^2 + 1e-6),
+ *   silu(a) = a / (1 + e^-a).
+ *
+ * Weights (bf16): g1, g2 [d]; w_qkv, w_o as for sqa_layer_fwd; w1, w3
+ * [d][hidden]; w2 [hidden][d].  x, y, dy, dx: bf16 [B][N][d].  Gradients
+ * (fp32, fully overwritten; the weight gradients reduce over all tokens in a
+ * run-dependent order) have the weights' shapes.  Every activation the
+ * backward needs (the normalised rows and their 1/RMS, the layer's q, k, v,
+ * core output and lse, h, the feed-forward's a = n2 W1, b = n2 W3 and
+ * silu(a) * b, all bf16 but the statistics) is kept in `state`, which the
+ * forward writes and the backward reads, plus the backward's scratch: the
+ * caller allocates sqa_block_state_bytes(s) bytes, 256-byte aligned, and keeps
+ * it between the two calls.  Additional limits: hidden a multiple of 8,
+ * d <= 8192.
+ */
+typedef struct {
+    int B, N, d, H_q, H_kv, dh;
+    int hidden; /* feed-forward width */
+} sqa_block_shape;
+
+typedef struct {
+    const void *g1, *w_qkv, *w_o, *g2, *w1, *w3, *w2;
+} sqa_block_weights;
+
+typedef struct {
+    float *g1, *w_qkv, *w_o, *g2, *w1, *w3, *w2;
+} sqa_block_grads;
+
+/* Bytes of the forward-to-backward state of one block; 0 if s is invalid. */
+size_t sqa_block_state_bytes(sqa_block_shape s);
+
+/*
+ * Block forward: y, and the saved activations in `state`.  causal, scale and
+ * rope_base as for sqa_layer_fwd.  Errors as for sqa_layer_fwd, returned
+ * before any launch.
+ */
+sqa_status sqa_block_fwd(const void *x, const sqa_block_weights *w, void *y, void *state, size_t state_bytes,
+                         sqa_block_shape s, int causal, float scale, float rope_base, sqa_stream_t stream);
+
+/*
+ * Block backward of L = sum(dy * y), after sqa_block_fwd on the same x,
+ * weights and state: dx and every gradient in *grads.  Steps: dM = dY W2^T
+ * with da = dM b silu'(a), db = dM silu(a) in the same product's epilogue;
+ * dW2 = m^T dY, dW1 = n2^T da, dW3 = n2^T db; dn2 = da W1^T + db W3^T;
+ * dh = dY + RMSNorm'(h) dn2 (and dg2); the layer's backward (sqa_layer_bwd)
+ * with X = n1 and dY = dh; dx = dh + RMSNorm'(x) dn1 (and dg1).
+ */
+sqa_status sqa_block_bwd(const void *dy, const void *x, const sqa_block_weights *w, void *state,
+                         size_t state_bytes, void *dx, const sqa_block_grads *grads, sqa_block_shape s,
+                         int causal, float scale, float rope_base, sqa_stream_t stream);
+
 /* Static text for a status code. */
 const char *sqa_status_string(sqa_status status);
 

@@ -15,7 +15,7 @@ __all__ = [
     "SqaError", "load_library", "library_path", "sqa_fwd", "sqa_bwd", "bwd_workspace_bytes", "sqa_decode",
     "decode_workspace_bytes",
     "device_status", "timeout_info", "set_timing_events", "Shape", "LayerShape", "layer_workspace_bytes",
-    "sqa_layer_fwd", "sqa_layer_bwd",
+    "sqa_layer_fwd", "sqa_layer_bwd", "BlockShape", "block_state_bytes", "sqa_block_fwd", "sqa_block_bwd",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -316,3 +316,91 @@ def sqa_layer_bwd(dy, x, w_qkv, w_o, saved, H_q: int, H_kv: int, causal: bool = 
                              workspace.numel() * workspace.element_size(), s, int(bool(causal)), float(scale),
                              float(rope_base), _stream(stream)))
     return dx, dw_qkv, dw_o
+
+
+class BlockShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("N", ctypes.c_int), ("d", ctypes.c_int), ("H_q", ctypes.c_int),
+                ("H_kv", ctypes.c_int), ("dh", ctypes.c_int), ("hidden", ctypes.c_int)]
+
+
+_BLOCK_PARAMS = ("g1", "w_qkv", "w_o", "g2", "w1", "w3", "w2")
+
+
+class BlockWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in _BLOCK_PARAMS]
+
+
+class BlockGrads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in _BLOCK_PARAMS]
+
+
+def _block_lib():
+    lib = load_library()
+    if not getattr(lib, "_block_bound", False):
+        vp, sz, c_int, c_float = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
+        lib.sqa_block_state_bytes.argtypes = [BlockShape]
+        lib.sqa_block_state_bytes.restype = sz
+        lib.sqa_block_fwd.argtypes = [vp, ctypes.POINTER(BlockWeights), vp, vp, sz, BlockShape, c_int, c_float,
+                                      c_float, vp]
+        lib.sqa_block_fwd.restype = c_int
+        lib.sqa_block_bwd.argtypes = [vp, vp, ctypes.POINTER(BlockWeights), vp, sz, vp, ctypes.POINTER(BlockGrads),
+                                      BlockShape, c_int, c_float, c_float, vp]
+        lib.sqa_block_bwd.restype = c_int
+        lib._block_bound = True
+    return lib
+
+
+def _block_shape(x, w, H_q, H_kv):
+    import torch
+
+    if x.dim() != 3:
+        raise ValueError("x must be [B, N, d]")
+    B, N, d = x.shape
+    dh = w["w_o"].shape[0] // H_q
+    hidden = w["w1"].shape[1]
+    shapes = {"g1": (d,), "w_qkv": (d, (H_q + 2 * H_kv) * dh), "w_o": (H_q * dh, d), "g2": (d,),
+              "w1": (d, hidden), "w3": (d, hidden), "w2": (hidden, d)}
+    _need(x, "x", (B, N, d), torch.bfloat16)
+    for n in _BLOCK_PARAMS:
+        _need(w[n], n, shapes[n], torch.bfloat16)
+    return BlockShape(B, N, d, H_q, H_kv, dh, hidden), shapes
+
+
+def block_state_bytes(B, N, d, H_q, H_kv, dh, hidden) -> int:
+    return int(_block_lib().sqa_block_state_bytes(BlockShape(B, N, d, H_q, H_kv, dh, hidden)))
+
+
+def sqa_block_fwd(x, weights: dict, H_q: int, H_kv: int, state=None, causal: bool = True, scale: float = 0.0,
+                  rope_base: float = 10000.0, stream=None):
+    """One SQAT-m block forward.  weights: dict of bf16 CUDA tensors g1, w_qkv,
+    w_o, g2, w1, w3, w2.  Returns (y, state); pass state to sqa_block_bwd."""
+    import torch
+
+    lib = _block_lib()
+    s, _ = _block_shape(x, weights, H_q, H_kv)
+    if state is None:
+        state = torch.empty(max(int(lib.sqa_block_state_bytes(s)), 256), dtype=torch.uint8, device=x.device)
+    y = torch.empty_like(x)
+    w = BlockWeights(*(weights[n].data_ptr() for n in _BLOCK_PARAMS))
+    _check(lib.sqa_block_fwd(x.data_ptr(), ctypes.byref(w), y.data_ptr(), state.data_ptr(),
+                             state.numel() * state.element_size(), s, int(bool(causal)), float(scale),
+                             float(rope_base), _stream(stream)))
+    return y, state
+
+
+def sqa_block_bwd(dy, x, weights: dict, state, H_q: int, H_kv: int, causal: bool = True, scale: float = 0.0,
+                  rope_base: float = 10000.0, stream=None):
+    """Block backward of sum(dy * y).  Returns (dx bf16, dict of fp32 gradients)."""
+    import torch
+
+    lib = _block_lib()
+    s, shapes = _block_shape(x, weights, H_q, H_kv)
+    _need(dy, "dy", tuple(x.shape), torch.bfloat16)
+    dx = torch.empty_like(x)
+    grads = {n: torch.empty(shapes[n], dtype=torch.float32, device=x.device) for n in _BLOCK_PARAMS}
+    w = BlockWeights(*(weights[n].data_ptr() for n in _BLOCK_PARAMS))
+    gr = BlockGrads(*(grads[n].data_ptr() for n in _BLOCK_PARAMS))
+    _check(lib.sqa_block_bwd(dy.data_ptr(), x.data_ptr(), ctypes.byref(w), state.data_ptr(),
+                             state.numel() * state.element_size(), dx.data_ptr(), ctypes.byref(gr), s,
+                             int(bool(causal)), float(scale), float(rope_base), _stream(stream)))
+    return dx, grads

@@ -11,6 +11,7 @@
 #include <string>
 
 #include "sqa.h"
+#include "sqa_block.cuh"
 #include "sqa_bwd.cuh"
 #include "sqa_bwd_bf16.cuh"
 #include "sqa_bwd_tf32.cuh"
@@ -477,7 +478,9 @@ sqa_status launch_gemm(int M, int N, const GemmSeg* segs, int n_seg, int split_k
   sqa_status st;
   int blocks = 0;
   for (int i = 0; i < 3; ++i) {
-    const GemmSeg& sg = segs[i < n_seg ? i : 0];
+    // kSwiGLU reads a second B operand (W3) from segs[1] over the same K.
+    const int n_maps = p.mode == sqa::kSwiGLU ? 2 : n_seg;
+    const GemmSeg& sg = segs[i < n_maps ? i : 0];
     if ((st = A_MN ? make_map_2d(&ma[i], sg.a, sg.k, M, sg.lda, 64) : make_map_2d(&ma[i], sg.a, M, sg.k, sg.lda, 128)) !=
         SQA_OK)
       return st;
@@ -495,7 +498,8 @@ sqa_status launch_gemm(int M, int N, const GemmSeg* segs, int n_seg, int split_k
   p.N = N;
   p.n_seg = n_seg;
   p.tiles_m = (M + Tr::BM - 1) / Tr::BM;
-  p.tiles_n = (N + BN - 1) / BN;
+  const int tile_cols = p.mode == sqa::kSwiGLU ? BN / 2 : BN;  // output columns per tile
+  p.tiles_n = (N + tile_cols - 1) / tile_cols;
   p.split_k = split_k < 1 ? 1 : (split_k > blocks ? blocks : split_k);
   const long long items = static_cast<long long>(p.tiles_m) * p.tiles_n * p.split_k;
   if (items > 0x7fffffffLL) return fail(SQA_ERR_UNSUPPORTED, "GEMM too large for one launch");
@@ -563,6 +567,160 @@ sqa_status rope_table(float2* cs, const sqa_layer_shape& s, float base, cudaStre
   sqa::sqa_rope_table_kernel<<<grid_for(n, 256), 256, 0, stream>>>(cs, s.N, s.dh, static_cast<double>(base));
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "rotary table launch");
+  return SQA_OK;
+}
+
+// The layer forward after validation: Q | K | V = X W_qkv with the rotation in
+// the epilogue, the attention core, Y = O W_o (+ resid when given).
+sqa_status layer_forward(const void* x, const void* w_qkv, const void* w_o, void* y, const void* resid, void* q,
+                         void* k, void* v, void* out, float* lse, float2* table, const sqa_layer_shape& s,
+                         int causal, float sc, float rope_base, cudaStream_t cs) {
+  sqa_status st;
+  const int M = s.B * s.N, nq = s.H_q * s.dh, nk = s.H_kv * s.dh, wqkv = nq + 2 * nk;
+  if (rope_base > 0.f && (st = rope_table(table, s, rope_base, cs)) != SQA_OK) return st;
+  sqa::GemmParams gp{};
+  gp.mode = sqa::kQkvRope;
+  gp.q = static_cast<__nv_bfloat16*>(q);
+  gp.k = static_cast<__nv_bfloat16*>(k);
+  gp.v = static_cast<__nv_bfloat16*>(v);
+  gp.nq = nq;
+  gp.nk = nk;
+  gp.nv = nk;
+  gp.dh = s.dh;
+  gp.n_tokens = s.N;
+  gp.rope_cs = rope_base > 0.f ? table : nullptr;
+  const GemmSeg g_qkv{x, w_qkv, s.d, s.d, wqkv};
+  if ((st = gemm<false, true>(M, wqkv, &g_qkv, 1, 1, gp, cs)) != SQA_OK) return st;
+  const sqa_shape core{s.B, s.N, s.H_q, s.H_kv, s.dh};
+  switch (s.dh) {
+    case 16: st = launch_fwd<16>(q, k, v, out, lse, core, causal, sc, cs); break;
+    case 32: st = launch_fwd<32>(q, k, v, out, lse, core, causal, sc, cs); break;
+    case 64: st = launch_fwd<64>(q, k, v, out, lse, core, causal, sc, cs); break;
+    default: st = launch_fwd<128>(q, k, v, out, lse, core, causal, sc, cs); break;
+  }
+  if (st != SQA_OK) return st;
+  sqa::GemmParams go{};
+  go.mode = sqa::kStoreBf16;
+  go.out = static_cast<__nv_bfloat16*>(y);
+  go.ld_out = s.d;
+  go.resid = static_cast<const __nv_bfloat16*>(resid);
+  const GemmSeg g_o{out, w_o, nq, nq, s.d};
+  return gemm<false, true>(M, s.d, &g_o, 1, 1, go, cs);
+}
+
+// ---------------------------------------------------------------------------
+// One decoder block: RMSNorm, the layer, residuals, SwiGLU feed-forward.
+
+sqa_status check_block_shape(const sqa_block_shape& s) {
+  const sqa_layer_shape ls{s.B, s.N, s.d, s.H_q, s.H_kv, s.dh};
+  sqa_status st = check_layer_shape(ls);
+  if (st != SQA_OK) return st;
+  if (s.hidden < 1) return fail(SQA_ERR_INVALID_ARG, "hidden width %d must be positive", s.hidden);
+  if (s.hidden % 8 != 0) return fail(SQA_ERR_UNSUPPORTED, "hidden width %d must be a multiple of 8", s.hidden);
+  if (s.d > 8192) return fail(SQA_ERR_UNSUPPORTED, "model width d=%d exceeds 8192", s.d);
+  return SQA_OK;
+}
+
+sqa_status check_block_weights(const sqa_block_weights* w) {
+  const void* all[] = {w->g1, w->w_qkv, w->w_o, w->g2, w->w1, w->w3, w->w2};
+  for (const void* ptr : all) {
+    if (!ptr) return fail(SQA_ERR_INVALID_ARG, "null weight pointer");
+    if (!aligned(ptr, 16)) return fail(SQA_ERR_UNSUPPORTED, "weights must be 16-byte aligned");
+  }
+  return SQA_OK;
+}
+
+struct BlockLayout {
+  size_t n1, rstd1, q, k, v, out, lse, h, n2, rstd2, a, b, act, da, db, dn, dh, layer_ws, layer_ws_bytes, bytes;
+};
+
+BlockLayout block_layout(const sqa_block_shape& s) {
+  BlockLayout L{};
+  const size_t M = static_cast<size_t>(s.B) * s.N, bf = 2;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o += sqa::align256(bytes);
+    return at;
+  };
+  L.n1 = take(M * s.d * bf);
+  L.rstd1 = take(M * sizeof(float));
+  L.q = take(M * s.H_q * s.dh * bf);
+  L.k = take(M * s.H_kv * s.dh * bf);
+  L.v = take(M * s.H_kv * s.dh * bf);
+  L.out = take(M * s.H_q * s.dh * bf);
+  L.lse = take(M * s.H_q * sizeof(float));
+  L.h = take(M * s.d * bf);
+  L.n2 = take(M * s.d * bf);
+  L.rstd2 = take(M * sizeof(float));
+  L.a = take(M * s.hidden * bf);
+  L.b = take(M * s.hidden * bf);
+  L.act = take(M * s.hidden * bf);
+  L.da = take(M * s.hidden * bf);
+  L.db = take(M * s.hidden * bf);
+  L.dn = take(M * s.d * bf);
+  L.dh = take(M * s.d * bf);
+  const sqa_layer_shape ls{s.B, s.N, s.d, s.H_q, s.H_kv, s.dh};
+  L.layer_ws_bytes = layer_layout(ls).bwd_bytes;
+  L.layer_ws = take(L.layer_ws_bytes);
+  L.bytes = o;
+  return L;
+}
+
+struct BlockPtrs {
+  void *n1, *q, *k, *v, *out, *h, *n2, *a, *b, *act, *da, *db, *dn, *dh, *layer_ws;
+  float *rstd1, *rstd2, *lse;
+  float2* table;
+};
+
+BlockPtrs block_ptrs(void* state, const sqa_block_shape& s, const BlockLayout& L) {
+  uint8_t* base = static_cast<uint8_t*>(state);
+  BlockPtrs b;
+  b.n1 = base + L.n1;
+  b.q = base + L.q;
+  b.k = base + L.k;
+  b.v = base + L.v;
+  b.out = base + L.out;
+  b.h = base + L.h;
+  b.n2 = base + L.n2;
+  b.a = base + L.a;
+  b.b = base + L.b;
+  b.act = base + L.act;
+  b.da = base + L.da;
+  b.db = base + L.db;
+  b.dn = base + L.dn;
+  b.dh = base + L.dh;
+  b.layer_ws = base + L.layer_ws;
+  b.rstd1 = reinterpret_cast<float*>(base + L.rstd1);
+  b.rstd2 = reinterpret_cast<float*>(base + L.rstd2);
+  b.lse = reinterpret_cast<float*>(base + L.lse);
+  b.table = reinterpret_cast<float2*>(base + L.layer_ws);  // the layer workspace starts with the rotary table
+  (void)s;
+  return b;
+}
+
+sqa_status rmsnorm(const void* x, const void* g, void* n, float* rstd, int M, int d, cudaStream_t cs) {
+  const int blocks = grid_for(static_cast<long long>(M) * 32, 256);
+  sqa::sqa_rmsnorm_kernel<<<blocks, 256, 0, cs>>>(static_cast<const __nv_bfloat16*>(x),
+                                                  static_cast<const __nv_bfloat16*>(g),
+                                                  static_cast<__nv_bfloat16*>(n), rstd, M, d);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "rmsnorm launch");
+  return SQA_OK;
+}
+
+sqa_status rmsnorm_bwd(const void* x, const void* g, const float* rstd, const void* dn, const void* resid, void* dx,
+                       float* dg, int M, int d, cudaStream_t cs) {
+  const int blocks = grid_for(static_cast<long long>(M) * 32, 256);
+  const int smem = d * static_cast<int>(sizeof(float));
+  sqa_status st;
+  if (smem > 48 * 1024 && (st = set_smem(sqa::sqa_rmsnorm_bwd_kernel, smem)) != SQA_OK) return st;
+  sqa::sqa_rmsnorm_bwd_kernel<<<blocks, 256, smem, cs>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(g), rstd,
+      static_cast<const __nv_bfloat16*>(dn), static_cast<const __nv_bfloat16*>(resid),
+      static_cast<__nv_bfloat16*>(dx), dg, M, d);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "rmsnorm backward launch");
   return SQA_OK;
 }
 
@@ -696,40 +854,8 @@ sqa_status sqa_layer_fwd(const void* x, const void* w_qkv, const void* w_o, void
     return fail(SQA_ERR_INVALID_ARG, "rope_base must be finite and non-negative");
   float sc;
   if ((st = resolve_scale(scale, s.dh, &sc)) != SQA_OK) return st;
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-  const int M = s.B * s.N, nq = s.H_q * s.dh, nk = s.H_kv * s.dh, wqkv = nq + 2 * nk;
-  float2* table = static_cast<float2*>(workspace);
-  if (rope_base > 0.f && (st = rope_table(table, s, rope_base, cs)) != SQA_OK) return st;
-  // Q | K | V = X W_qkv, rotary embedding on Q and K in the epilogue.
-  sqa::GemmParams gp{};
-  gp.mode = sqa::kQkvRope;
-  gp.q = static_cast<__nv_bfloat16*>(q);
-  gp.k = static_cast<__nv_bfloat16*>(k);
-  gp.v = static_cast<__nv_bfloat16*>(v);
-  gp.nq = nq;
-  gp.nk = nk;
-  gp.nv = nk;
-  gp.dh = s.dh;
-  gp.n_tokens = s.N;
-  gp.rope_cs = rope_base > 0.f ? table : nullptr;
-  const GemmSeg g_qkv{x, w_qkv, s.d, s.d, wqkv};
-  if ((st = gemm<false, true>(M, wqkv, &g_qkv, 1, 1, gp, cs)) != SQA_OK) return st;
-  // the attention core
-  const sqa_shape core{s.B, s.N, s.H_q, s.H_kv, s.dh};
-  switch (s.dh) {
-    case 16: st = launch_fwd<16>(q, k, v, out, lse, core, causal, sc, cs); break;
-    case 32: st = launch_fwd<32>(q, k, v, out, lse, core, causal, sc, cs); break;
-    case 64: st = launch_fwd<64>(q, k, v, out, lse, core, causal, sc, cs); break;
-    default: st = launch_fwd<128>(q, k, v, out, lse, core, causal, sc, cs); break;
-  }
-  if (st != SQA_OK) return st;
-  // Y = O W_o
-  sqa::GemmParams go{};
-  go.mode = sqa::kStoreBf16;
-  go.out = static_cast<__nv_bfloat16*>(y);
-  go.ld_out = s.d;
-  const GemmSeg g_o{out, w_o, nq, nq, s.d};
-  return gemm<false, true>(M, s.d, &g_o, 1, 1, go, cs);
+  return layer_forward(x, w_qkv, w_o, y, nullptr, q, k, v, out, lse, static_cast<float2*>(workspace), s, causal, sc,
+                       rope_base, reinterpret_cast<cudaStream_t>(stream));
 }
 
 sqa_status sqa_layer_bwd(const void* dy, const void* x, const void* w_qkv, const void* w_o, const void* q,
@@ -814,6 +940,127 @@ sqa_status sqa_layer_bwd(const void* dy, const void* x, const void* w_qkv, const
   const __nv_bfloat16* w = static_cast<const __nv_bfloat16*>(w_qkv);
   const GemmSeg g4[3] = {{dq, w, nq, nq, wqkv}, {dk, w + nq, nk, nk, wqkv}, {dv, w + nq + nk, nk, nk, wqkv}};
   return gemm<false, false>(M, s.d, g4, 3, 1, p4, cs);
+}
+
+size_t sqa_block_state_bytes(sqa_block_shape s) {
+  if (check_block_shape(s) != SQA_OK) return 0;
+  return block_layout(s).bytes;
+}
+
+sqa_status sqa_block_fwd(const void* x, const sqa_block_weights* w, void* y, void* state, size_t state_bytes,
+                         sqa_block_shape s, int causal, float scale, float rope_base, sqa_stream_t stream) {
+  g_last_error.clear();
+  if (!x || !w || !y || !state) return fail(SQA_ERR_INVALID_ARG, "null pointer argument");
+  sqa_status st = check_block_shape(s);
+  if (st != SQA_OK) return st;
+  if ((st = check_block_weights(w)) != SQA_OK) return st;
+  if (!aligned(x, 16) || !aligned(y, 16)) return fail(SQA_ERR_UNSUPPORTED, "x and y must be 16-byte aligned");
+  if (!aligned(state, 256)) return fail(SQA_ERR_UNSUPPORTED, "state must be 256-byte aligned");
+  const BlockLayout L = block_layout(s);
+  if (state_bytes < L.bytes) return fail(SQA_ERR_INVALID_ARG, "state holds %zu bytes, %zu needed", state_bytes, L.bytes);
+  if (std::isnan(rope_base) || std::isinf(rope_base) || rope_base < 0.f)
+    return fail(SQA_ERR_INVALID_ARG, "rope_base must be finite and non-negative");
+  float sc;
+  if ((st = resolve_scale(scale, s.dh, &sc)) != SQA_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const BlockPtrs b = block_ptrs(state, s, L);
+  const sqa_layer_shape ls{s.B, s.N, s.d, s.H_q, s.H_kv, s.dh};
+  const int M = s.B * s.N;
+  // n1 = RMSNorm(x; g1); h = x + SQA(n1)
+  if ((st = rmsnorm(x, w->g1, b.n1, b.rstd1, M, s.d, cs)) != SQA_OK) return st;
+  if ((st = layer_forward(b.n1, w->w_qkv, w->w_o, b.h, x, b.q, b.k, b.v, b.out, b.lse, b.table, ls, causal, sc,
+                          rope_base, cs)) != SQA_OK)
+    return st;
+  // n2 = RMSNorm(h; g2); a = n2 W1, b = n2 W3, m = silu(a) * b; y = h + m W2
+  if ((st = rmsnorm(b.h, w->g2, b.n2, b.rstd2, M, s.d, cs)) != SQA_OK) return st;
+  sqa::GemmParams p1{};
+  p1.mode = sqa::kSwiGLU;
+  p1.out = static_cast<__nv_bfloat16*>(b.act);
+  p1.sw_a = static_cast<__nv_bfloat16*>(b.a);
+  p1.sw_b = static_cast<__nv_bfloat16*>(b.b);
+  p1.ld_out = s.hidden;
+  const GemmSeg g1[2] = {{b.n2, w->w1, s.d, s.d, s.hidden}, {b.n2, w->w3, s.d, s.d, s.hidden}};
+  if ((st = launch_gemm<256, false, true>(M, s.hidden, g1, 1, 1, p1, cs)) != SQA_OK) return st;
+  sqa::GemmParams p2{};
+  p2.mode = sqa::kStoreBf16;
+  p2.out = static_cast<__nv_bfloat16*>(y);
+  p2.ld_out = s.d;
+  p2.resid = static_cast<const __nv_bfloat16*>(b.h);
+  const GemmSeg g2{b.act, w->w2, s.hidden, s.hidden, s.d};
+  return gemm<false, true>(M, s.d, &g2, 1, 1, p2, cs);
+}
+
+sqa_status sqa_block_bwd(const void* dy, const void* x, const sqa_block_weights* w, void* state, size_t state_bytes,
+                         void* dx, const sqa_block_grads* gr, sqa_block_shape s, int causal, float scale,
+                         float rope_base, sqa_stream_t stream) {
+  g_last_error.clear();
+  if (!dy || !x || !w || !state || !dx || !gr) return fail(SQA_ERR_INVALID_ARG, "null pointer argument");
+  if (!gr->g1 || !gr->w_qkv || !gr->w_o || !gr->g2 || !gr->w1 || !gr->w3 || !gr->w2)
+    return fail(SQA_ERR_INVALID_ARG, "null gradient pointer");
+  sqa_status st = check_block_shape(s);
+  if (st != SQA_OK) return st;
+  if ((st = check_block_weights(w)) != SQA_OK) return st;
+  const void* al[] = {dy, x, dx, gr->g1, gr->w_qkv, gr->w_o, gr->g2, gr->w1, gr->w3, gr->w2};
+  for (const void* ptr : al)
+    if (!aligned(ptr, 16)) return fail(SQA_ERR_UNSUPPORTED, "tensors must be 16-byte aligned");
+  if (!aligned(state, 256)) return fail(SQA_ERR_UNSUPPORTED, "state must be 256-byte aligned");
+  const BlockLayout L = block_layout(s);
+  if (state_bytes < L.bytes) return fail(SQA_ERR_INVALID_ARG, "state holds %zu bytes, %zu needed", state_bytes, L.bytes);
+  if (std::isnan(rope_base) || std::isinf(rope_base) || rope_base < 0.f)
+    return fail(SQA_ERR_INVALID_ARG, "rope_base must be finite and non-negative");
+  float sc;
+  if ((st = resolve_scale(scale, s.dh, &sc)) != SQA_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const BlockPtrs b = block_ptrs(state, s, L);
+  const int M = s.B * s.N;
+  const size_t dsz = static_cast<size_t>(s.d) * sizeof(float);
+  const size_t whid = static_cast<size_t>(s.d) * s.hidden * sizeof(float);
+  cudaError_t e = cudaMemsetAsync(gr->g1, 0, dsz, cs);
+  if (e == cudaSuccess) e = cudaMemsetAsync(gr->g2, 0, dsz, cs);
+  if (e == cudaSuccess) e = cudaMemsetAsync(gr->w1, 0, whid, cs);
+  if (e == cudaSuccess) e = cudaMemsetAsync(gr->w3, 0, whid, cs);
+  if (e == cudaSuccess) e = cudaMemsetAsync(gr->w2, 0, whid, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync (block gradients)");
+  // dM = dY W2^T, and with the saved a, b: da = dM b silu'(a), db = dM silu(a)
+  sqa::GemmParams p1{};
+  p1.mode = sqa::kSwiGLUBwd;
+  p1.out = static_cast<__nv_bfloat16*>(b.da);
+  p1.out2 = static_cast<__nv_bfloat16*>(b.db);
+  p1.sw_a = static_cast<__nv_bfloat16*>(b.a);
+  p1.sw_b = static_cast<__nv_bfloat16*>(b.b);
+  p1.ld_out = s.hidden;
+  const GemmSeg g1{dy, w->w2, s.d, s.d, s.d};
+  if ((st = gemm<false, false>(M, s.hidden, &g1, 1, 1, p1, cs)) != SQA_OK) return st;
+  // dW2 = m^T dY; dW1 = n2^T da; dW3 = n2^T db (fp32 reductions over the tokens)
+  sqa::GemmParams pw{};
+  pw.mode = sqa::kAtomicF32;
+  pw.out32 = gr->w2;
+  pw.ld_out32 = s.d;
+  const GemmSeg gw2{b.act, dy, M, s.hidden, s.d};
+  if ((st = gemm<true, true>(s.hidden, s.d, &gw2, 1, split_for(s.hidden, s.d, M), pw, cs)) != SQA_OK) return st;
+  pw.ld_out32 = s.hidden;
+  pw.out32 = gr->w1;
+  const GemmSeg gw1{b.n2, b.da, M, s.d, s.hidden};
+  if ((st = gemm<true, true>(s.d, s.hidden, &gw1, 1, split_for(s.d, s.hidden, M), pw, cs)) != SQA_OK) return st;
+  pw.out32 = gr->w3;
+  const GemmSeg gw3{b.n2, b.db, M, s.d, s.hidden};
+  if ((st = gemm<true, true>(s.d, s.hidden, &gw3, 1, split_for(s.d, s.hidden, M), pw, cs)) != SQA_OK) return st;
+  // dn2 = da W1^T + db W3^T
+  sqa::GemmParams p2{};
+  p2.mode = sqa::kStoreBf16;
+  p2.out = static_cast<__nv_bfloat16*>(b.dn);
+  p2.ld_out = s.d;
+  const GemmSeg g2[2] = {{b.da, w->w1, s.hidden, s.hidden, s.hidden}, {b.db, w->w3, s.hidden, s.hidden, s.hidden}};
+  if ((st = gemm<false, false>(M, s.d, g2, 2, 1, p2, cs)) != SQA_OK) return st;
+  // dh = dY + RMSNorm'(h; g2) dn2
+  if ((st = rmsnorm_bwd(b.h, w->g2, b.rstd2, b.dn, dy, b.dh, gr->g2, M, s.d, cs)) != SQA_OK) return st;
+  // the layer's backward with X = n1, dY = dh: dn1, dW_qkv, dW_o
+  const sqa_layer_shape ls{s.B, s.N, s.d, s.H_q, s.H_kv, s.dh};
+  if ((st = sqa_layer_bwd(b.dh, b.n1, w->w_qkv, w->w_o, b.q, b.k, b.v, b.out, b.lse, b.dn, gr->w_qkv, gr->w_o,
+                          b.layer_ws, L.layer_ws_bytes, ls, causal, scale, rope_base, stream)) != SQA_OK)
+    return st;
+  // dx = dh + RMSNorm'(x; g1) dn1
+  return rmsnorm_bwd(x, w->g1, b.rstd1, b.dn, b.dh, dx, gr->g1, M, s.d, cs);
 }
 
 sqa_status sqa_selftest_exp2_poly(const float* x, float* y, int n, sqa_stream_t stream) {

@@ -10,6 +10,14 @@
 //               is written bf16 to its own [M][width] tensor
 //   kAtomicF32  D added to an fp32 row-major output with vector reductions
 //               (split-K: each work item covers a range of K blocks)
+//   kSwiGLU     the SwiGLU feed-forward's first product: each 256-column tile
+//               is 128 columns of U W1 (the gate, from the first B map) beside
+//               the same 128 columns of U W3 (from the second); the epilogue
+//               writes a = U W1, b = U W3 and silu(a) * b, bf16
+//   kSwiGLUBwd  its backward: D = dM (the gradient of silu(a) * b); with the
+//               saved a and b the epilogue writes da = dM * b * silu'(a) and
+//               db = dM * silu(a), bf16
+// kStoreBf16 can add a bf16 residual (same layout as the output) before rounding.
 // SQAT-m model card, "Model size difference": the query and output
 // projections shrink with the query-head count (W_q is d x H_q dh, W_o is
 // H_q dh x d); "Architecture details": rotary position embedding.
@@ -31,7 +39,7 @@
 
 namespace sqa {
 
-enum GemmEpilogue : int { kStoreBf16 = 0, kQkvRope = 1, kAtomicF32 = 2 };
+enum GemmEpilogue : int { kStoreBf16 = 0, kQkvRope = 1, kAtomicF32 = 2, kSwiGLU = 3, kSwiGLUBwd = 4 };
 
 struct GemmParams {
   int M, N;
@@ -40,9 +48,14 @@ struct GemmParams {
   int kblk0[4];   // first K block (of 64) of each segment; kblk0[n_seg] = total blocks
   int tiles_m, tiles_n, split_k, n_items;
   int mode;
-  // kStoreBf16
+  // kStoreBf16 (and the outputs of the SwiGLU epilogues)
   __nv_bfloat16* out;
   long long ld_out;
+  const __nv_bfloat16* resid;  // kStoreBf16: added before rounding, or null
+  // kSwiGLU: a, b written beside out; kSwiGLUBwd: a, b read, da -> out, db -> out2
+  __nv_bfloat16* sw_a;
+  __nv_bfloat16* sw_b;
+  __nv_bfloat16* out2;
   // kAtomicF32
   float* out32;
   long long ld_out32;
@@ -148,7 +161,7 @@ __global__ void __launch_bounds__(256, 1)
       int g = 0;  // K blocks issued so far (across items)
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-        const GemmItem it = gemm_item(p, item, BN);
+        const GemmItem it = gemm_item(p, item, p.mode == kSwiGLU ? BN / 2 : BN);
         const int n0 = it.n0;
         int sgi = 0;
         for (int kb = it.kb0; kb < it.kb1; ++kb, ++g) {
@@ -167,7 +180,12 @@ __global__ void __launch_bounds__(256, 1)
           } else {  // [M][K]: 128 rows x 128 bytes
             tma_load_2d(a_dst, mA[sgi], full(s), k0, it.m0);
           }
-          if (B_MN) {  // [K][N]: BN / 64 panels of N, each 64 K rows x 128 bytes
+          if (BN >= 128 && B_MN && p.mode == kSwiGLU) {  // BN / 2 columns of W1, then the same of W3
+            constexpr int HALF = BN >= 128 ? BN / 128 : 1;  // 64-column panels per half
+#pragma unroll
+            for (int pn = 0; pn < BN / 64; ++pn)
+              tma_load_2d(b_dst + pn * 8192, pn < HALF ? mB[0] : mB[1], full(s), n0 + 64 * (pn % HALF), k0);
+          } else if (B_MN) {  // [K][N]: BN / 64 panels of N, each 64 K rows x 128 bytes
 #pragma unroll
             for (int pn = 0; pn < BN / 64; ++pn) tma_load_2d(b_dst + pn * 8192, mB[sgi], full(s), n0 + 64 * pn, k0);
           } else {  // [N][K]: BN rows x 128 bytes
@@ -185,7 +203,7 @@ __global__ void __launch_bounds__(256, 1)
     int g = 0, r = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++r) {
-      const GemmItem it = gemm_item(p, item, BN);
+      const GemmItem it = gemm_item(p, item, p.mode == kSwiGLU ? BN / 2 : BN);
       const int ab = r & 1;
       if (r >= 2 && !(ok = mbar_wait_warp(acc_empty(ab), ((r >> 1) - 1) & 1, abort_flag, kSiteMma))) break;
       const uint32_t d_tmem = tmem + static_cast<uint32_t>(ab * BN);
@@ -221,7 +239,7 @@ __global__ void __launch_bounds__(256, 1)
     int r = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++r) {
-      const GemmItem it = gemm_item(p, item, BN);
+      const GemmItem it = gemm_item(p, item, p.mode == kSwiGLU ? BN / 2 : BN);
       const int ab = r & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(acc_full(ab), (r >> 1) & 1, abort_flag, kSiteEpilogue));
       if (!ok) break;
@@ -229,6 +247,44 @@ __global__ void __launch_bounds__(256, 1)
       const int m = it.m0 + row;
       const bool row_ok = m < p.M;
       const int n_base = it.n0;
+      if (p.mode == kSwiGLU) {
+        // columns [0, BN/2): a = U W1, [BN/2, BN): b = U W3, for hidden columns n_base ..
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN / 2; c0 += 32) {
+          uint32_t ra[32], rb[32];
+          tmem_ld32(lane_addr + static_cast<uint32_t>(ab * BN + c0), ra);
+          tmem_ld32(lane_addr + static_cast<uint32_t>(ab * BN + BN / 2 + c0), rb);
+          if (c0 + 32 == BN / 2) {
+            tc_fence_before();
+            mbar_arrive(acc_empty(ab));
+          }
+          if (!row_ok) continue;
+          const long long o = static_cast<long long>(m) * p.ld_out + n_base + c0;
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            if (n_base + c0 + e >= p.N) continue;
+            uint4 oa, ob, om;
+            uint32_t* pa = &oa.x;
+            uint32_t* pb = &ob.x;
+            uint32_t* pm = &om.x;
+#pragma unroll
+            for (int u = 0; u < 8; u += 2) {
+              const float a0 = __uint_as_float(ra[e + u]), a1 = __uint_as_float(ra[e + u + 1]);
+              const float b0 = __uint_as_float(rb[e + u]), b1 = __uint_as_float(rb[e + u + 1]);
+              // silu(a) = a / (1 + 2^(-a log2 e))
+              const float s0 = a0 / (1.f + ex2(-1.4426950408889634f * a0));
+              const float s1 = a1 / (1.f + ex2(-1.4426950408889634f * a1));
+              pa[u >> 1] = pack_bf16x2(a0, a1);
+              pb[u >> 1] = pack_bf16x2(b0, b1);
+              pm[u >> 1] = pack_bf16x2(s0 * b0, s1 * b1);
+            }
+            *reinterpret_cast<uint4*>(p.sw_a + o + e) = oa;
+            *reinterpret_cast<uint4*>(p.sw_b + o + e) = ob;
+            *reinterpret_cast<uint4*>(p.out + o + e) = om;
+          }
+        }
+        continue;
+      }
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t rr[32];
@@ -247,17 +303,57 @@ __global__ void __launch_bounds__(256, 1)
                         make_float4(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1]), __uint_as_float(rr[e + 2]),
                                     __uint_as_float(rr[e + 3])));
         } else if (p.mode == kStoreBf16) {
-          __nv_bfloat16* dst = p.out + static_cast<long long>(m) * p.ld_out + n_base + c0;
+          const long long o0 = static_cast<long long>(m) * p.ld_out + n_base + c0;
+          __nv_bfloat16* dst = p.out + o0;
 #pragma unroll
           for (int e = 0; e < 32; e += 8)
             if (n_base + c0 + e < p.N) {
+              float y[8];
+#pragma unroll
+              for (int u = 0; u < 8; ++u) y[u] = __uint_as_float(rr[e + u]);
+              if (p.resid) {
+                const uint4 rv = *reinterpret_cast<const uint4*>(p.resid + o0 + e);
+                const __nv_bfloat162* r2 = reinterpret_cast<const __nv_bfloat162*>(&rv);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  const float2 f = __bfloat1622float2(r2[u]);
+                  y[2 * u] += f.x;
+                  y[2 * u + 1] += f.y;
+                }
+              }
               uint4 o;
-              o.x = pack_bf16x2(__uint_as_float(rr[e]), __uint_as_float(rr[e + 1]));
-              o.y = pack_bf16x2(__uint_as_float(rr[e + 2]), __uint_as_float(rr[e + 3]));
-              o.z = pack_bf16x2(__uint_as_float(rr[e + 4]), __uint_as_float(rr[e + 5]));
-              o.w = pack_bf16x2(__uint_as_float(rr[e + 6]), __uint_as_float(rr[e + 7]));
+              o.x = pack_bf16x2(y[0], y[1]);
+              o.y = pack_bf16x2(y[2], y[3]);
+              o.z = pack_bf16x2(y[4], y[5]);
+              o.w = pack_bf16x2(y[6], y[7]);
               *reinterpret_cast<uint4*>(dst + e) = o;
             }
+        } else if (p.mode == kSwiGLUBwd) {
+          // D = dM; with the saved a, b: da = dM b silu'(a), db = dM silu(a),
+          // silu'(a) = s + a s (1 - s), s = 1 / (1 + e^-a)
+          const long long o0 = static_cast<long long>(m) * p.ld_out + n_base + c0;
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            if (n_base + c0 + e >= p.N) continue;
+            const uint4 av = *reinterpret_cast<const uint4*>(p.sw_a + o0 + e);
+            const uint4 bv = *reinterpret_cast<const uint4*>(p.sw_b + o0 + e);
+            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&av);
+            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&bv);
+            uint4 oa, ob;
+            uint32_t* pa = &oa.x;
+            uint32_t* pb = &ob.x;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float2 a = __bfloat1622float2(a2[u]), b = __bfloat1622float2(b2[u]);
+              const float dm0 = __uint_as_float(rr[e + 2 * u]), dm1 = __uint_as_float(rr[e + 2 * u + 1]);
+              const float s0 = 1.f / (1.f + ex2(-1.4426950408889634f * a.x));
+              const float s1 = 1.f / (1.f + ex2(-1.4426950408889634f * a.y));
+              pa[u] = pack_bf16x2(dm0 * b.x * (s0 + a.x * s0 * (1.f - s0)), dm1 * b.y * (s1 + a.y * s1 * (1.f - s1)));
+              pb[u] = pack_bf16x2(dm0 * a.x * s0, dm1 * a.y * s1);
+            }
+            *reinterpret_cast<uint4*>(p.out + o0 + e) = oa;
+            *reinterpret_cast<uint4*>(p.out2 + o0 + e) = ob;
+          }
         } else {  // kQkvRope
           const int pos = m % p.n_tokens;
 #pragma unroll

@@ -129,3 +129,21 @@ def make_layer_inputs(B: int, N: int, d: int, Hq: int, Hkv: int, dh: int, seed: 
     w_o = (torch.randn(Hq * dh, d, generator=g) * (Hq * dh) ** -0.5).to(torch.bfloat16)
     dy = torch.randn(B, N, d, generator=g).to(torch.bfloat16)
     return x, w_qkv, w_o, dy
+
+
+def make_block_inputs(B: int, N: int, d: int, Hq: int, Hkv: int, dh: int, hidden: int, seed: int = 0):
+    """Draw x [B,N,d], the block's weights and dy [B,N,d] (CPU bf16), in the
+    order x, g1, w_qkv, w_o, g2, w1, w3, w2, dy.  The norm gains are 1 + 0.1
+    N(0,1); each matrix has standard deviation 1/sqrt(fan-in)."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+
+    def mat(rows, cols):
+        return (torch.randn(rows, cols, generator=g) * rows ** -0.5).to(torch.bfloat16)
+
+    x = torch.randn(B, N, d, generator=g).to(torch.bfloat16)
+    w = {"g1": (1.0 + 0.1 * torch.randn(d, generator=g)).to(torch.bfloat16),
+         "w_qkv": mat(d, (Hq + 2 * Hkv) * dh), "w_o": mat(Hq * dh, d),
+         "g2": (1.0 + 0.1 * torch.randn(d, generator=g)).to(torch.bfloat16),
+         "w1": mat(d, hidden), "w3": mat(d, hidden), "w2": mat(hidden, d)}
+    dy = torch.randn(B, N, d, generator=g).to(torch.bfloat16)
+    return x, w, dy

@@ -234,3 +234,24 @@ def test_layer_rejects_bad_arguments_before_launch(lib):
     assert st == sqa.SQA_ERR_INVALID_ARG
     st = lib.sqa_layer_bwd(*bargs[:13], need_b - 256, s, 1, 0.0, 10000.0, None)
     assert st == sqa.SQA_ERR_INVALID_ARG and b"workspace" in lib.sqa_last_error()
+
+
+def test_block_rejects_bad_arguments_before_launch(lib):
+    b = sqa._block_lib()
+    s = sqa.BlockShape(2, 256, 256, 8, 4, 16, 768)
+    need = b.sqa_block_state_bytes(s)
+    assert need > 0
+    assert b.sqa_block_state_bytes(sqa.BlockShape(2, 256, 256, 8, 4, 16, 700)) == 0  # hidden % 8 != 0
+    assert b.sqa_block_state_bytes(sqa.BlockShape(2, 256, 16384, 8, 4, 16, 768)) == 0  # d > 8192
+    p = 0x10000
+    w = sqa.BlockWeights(*([p] * 7))
+    st = b.sqa_block_fwd(p, ctypes.byref(w), p, p, need - 1, s, 1, 0.0, 10000.0, None)
+    assert st == sqa.SQA_ERR_INVALID_ARG and b"state" in b.sqa_last_error()
+    w0 = sqa.BlockWeights(*([p] * 6 + [0]))
+    st = b.sqa_block_fwd(p, ctypes.byref(w0), p, p, need, s, 1, 0.0, 10000.0, None)
+    assert st == sqa.SQA_ERR_INVALID_ARG and b"weight" in b.sqa_last_error()
+    g = sqa.BlockGrads(*([p] * 7))
+    st = b.sqa_block_bwd(p, p, ctypes.byref(w), p, need, p, ctypes.byref(g), s, 1, 0.0, -2.0, None)
+    assert st == sqa.SQA_ERR_INVALID_ARG and b"rope_base" in b.sqa_last_error()
+    st = b.sqa_block_bwd(p, p, ctypes.byref(w), p, need, p, None, s, 1, 0.0, 10000.0, None)
+    assert st == sqa.SQA_ERR_INVALID_ARG

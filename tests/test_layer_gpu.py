@@ -17,26 +17,10 @@ import pytest
 import torch
 
 from oracle.layer import sqa_layer_bwd, sqa_layer_fwd
-from parity import record, to_np
+from parity import assert_scaled_close as assert_layer_close, to_np
 from sparse_query_attention_sqa_b200.inputs import make_layer_inputs
 
 pytestmark = pytest.mark.gpu
-
-REL_FRO = 1e-2
-
-
-def assert_layer_close(name, got, ref):
-    got = np.asarray(got, dtype=np.float64)
-    ref = np.asarray(ref, dtype=np.float64)
-    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
-    err = np.abs(got - ref)
-    rms = float(np.sqrt(np.mean(ref ** 2)))
-    bound = 2e-2 + 0.1 * rms
-    rf = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
-    record({"name": name, "max_abs": float(err.max()), "rms_ref": rms, "rel_fro": rf, "n": int(ref.size)})
-    assert err.max() <= bound and rf <= REL_FRO, (
-        f"{name}: max-abs {err.max():.3e} (<= {bound:.3e}), rel-Frobenius {rf:.3e} (<= {REL_FRO})")
-
 
 # (B, N, d, H_q, H_kv, dh, causal): the SQAT-m layer (d = 256 over 16 heads,
 # 8 query heads, 4 key/value heads), a ragged token count (M not a multiple of
