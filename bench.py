@@ -277,8 +277,8 @@ def launched_kernel(w, hook: int) -> str:
     0 the forward, 1 the backward, 2 the decoding split kernel."""
     if hook == 0:
         return f"sqa_fwd_kernel<{w.dh}>"
-    if hook == 1:
-        return f"sqa_bwd_tf32_kernel<{w.dh}>" if w.dh <= 32 else f"sqa_bwd_kernel<{w.dh}>"
+    if hook == 1:  # at dh 64 / 128 the hook brackets the dK/dV and the dQ kernels
+        return f"sqa_bwd_tf32_kernel<{w.dh}>" if w.dh <= 32 else f"sqa_bwd_kernel<{w.dh}>+sqa_bwd_q_kernel<{w.dh}>"
     g = w.Hq // w.Hkv
     rows = g <= 4 and (w.Hkv & (w.Hkv - 1)) == 0  # register-resident path
     return f"sqa_decode_split_kernel<{w.dh},{g if rows else 0}>"
@@ -559,6 +559,8 @@ def run_ours(args, w):
             "e2e": {"value": job_tflops(w, world, e2e_ms), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "streams": n_pipe,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            # fwd + bwd: the forward, the backward's preprocess, its main kernel and
+            # either the dQ conversion (dh <= 32) or the dQ kernel (dh 64 / 128)
             "gpu_launches": args.steps * (4 if w.backward else (2 if w.decode else 1)),
             "clocks": clk,
             "wall_s_timed_region": wall,

@@ -114,6 +114,12 @@ sqa_status set_smem(Kernel k, int bytes) {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+int sm_count() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
 template <int DH>
 sqa_status launch_fwd(const void* q, const void* k, const void* v, void* out, float* lse, const sqa_shape& s,
                       int causal, float scale, cudaStream_t stream) {
@@ -312,9 +318,11 @@ sqa_status launch_bwd(const void* dout, const void* q, const void* k, const void
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* lse2 = reinterpret_cast<float*>(ws);
   float* Dst = reinterpret_cast<float*>(ws + L.off_D);
-  float* dq_acc = reinterpret_cast<float*>(ws + L.off_dq);
+  float* dq_acc = DH <= 32 ? reinterpret_cast<float*>(ws + L.off_dq) : nullptr;
   const long long grid_main = static_cast<long long>(L.n_kt) * s.B * s.H_kv;
-  if (grid_main > 0x7fffffffLL) return fail(SQA_ERR_UNSUPPORTED, "problem too large for one launch");
+  const long long grid_q = static_cast<long long>(L.n_qt) * s.B * s.H_kv;
+  if (grid_main > 0x7fffffffLL || grid_q > 0x7fffffffLL)
+    return fail(SQA_ERR_UNSUPPORTED, "problem too large for one launch");
 
   sqa::BwdPrepParams pp{};
   pp.dout = static_cast<const __nv_bfloat16*>(dout);
@@ -334,7 +342,7 @@ sqa_status launch_bwd(const void* dout, const void* q, const void* k, const void
   pp.rows = L.rows;
   pp.n_qt = L.n_qt;
   pp.n_slots = static_cast<long long>(L.n_slots);
-  pp.dq_vec4 = static_cast<long long>(s.B) * s.N * s.H_q * DH / 4;
+  pp.dq_vec4 = DH <= 32 ? static_cast<long long>(s.B) * s.N * s.H_q * DH / 4 : 0;
   const long long prep_work = pp.n_slots > pp.dq_vec4 ? pp.n_slots : pp.dq_vec4;
   sqa::sqa_bwd_prep_kernel<DH><<<grid_for(prep_work, 256), 256, 0, stream>>>(pp);
   cudaError_t e = cudaGetLastError();
@@ -369,34 +377,64 @@ sqa_status launch_bwd(const void* dout, const void* q, const void* k, const void
   p.scale_log2 = scale * kLog2e;
   p.scale = scale;
   if constexpr (DH <= 32) {
-    // dh 16 and 32: tf32 gradient contractions, half-tile pipelining
+    // dh 16 and 32: tf32 gradient contractions, half-tile pipelining, dQ added
+    // to an fp32 accumulator and converted by a third kernel.
     // Persistent: one CTA per SM walks the items.
     using T32 = sqa::BwdTf32Traits<DH>;
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = sm_count();
     p.n_items = static_cast<int>(grid_main);
     const unsigned grid = static_cast<unsigned>(grid_main < sms ? grid_main : sms);
     if ((st = set_smem(sqa::sqa_bwd_tf32_kernel<DH>, T32::SMEM_BYTES)) != SQA_OK) return st;
     if ((st = record_timing(1, 0, stream)) != SQA_OK) return st;
     sqa::sqa_bwd_tf32_kernel<DH><<<grid, T32::THREADS, T32::SMEM_BYTES, stream>>>(mq, mdo, mk, mv, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "sqa_bwd main launch");
+    if ((st = record_timing(1, 1, stream)) != SQA_OK) return st;
+    const long long n_vec8 = static_cast<long long>(s.B) * s.N * s.H_q * DH / 8;
+    sqa::sqa_bwd_dq_kernel<<<grid_for(n_vec8, 256), 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq),
+                                                                      n_vec8, scale);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "sqa_bwd dq launch");
+    return SQA_OK;
   } else {
-    // dh 64 and 128: one CTA per item, heaviest items first.
-    using Tr = sqa::BwdBf16Traits<DH < 64 ? 64 : DH>;
-    if ((st = set_smem(sqa::sqa_bwd_kernel<DH < 64 ? 64 : DH>, Tr::SMEM_BYTES)) != SQA_OK) return st;
+    // dh 64 and 128: dK / dV key-major, then dQ query-major (one CTA per item,
+    // heaviest items first); the timing hook brackets both.
+    constexpr int D2 = DH < 64 ? 64 : DH;
+    using Tr = sqa::BwdBf16Traits<D2>;
+    using TQ = sqa::BwdQTraits<D2>;
+    CUtensorMap mk64, mv64;
+    if ((st = make_map(&mk64, k, s.B, s.N, s.H_kv, DH, PANEL, 1, TQ::NK)) != SQA_OK) return st;
+    if ((st = make_map(&mv64, v, s.B, s.N, s.H_kv, DH, PANEL, 1, TQ::NK)) != SQA_OK) return st;
+    sqa::BwdQParams pq{};
+    pq.q = static_cast<const __nv_bfloat16*>(q);
+    pq.dout = static_cast<const __nv_bfloat16*>(dout);
+    pq.lse2 = lse2;
+    pq.D = Dst;
+    pq.dq = static_cast<__nv_bfloat16*>(dq);
+    pq.N = s.N;
+    pq.Hq = s.H_q;
+    pq.Hkv = s.H_kv;
+    pq.g = L.g;
+    pq.T = L.T;
+    pq.rows = L.rows;
+    pq.n_qt = L.n_qt;
+    pq.n_bh = s.B * s.H_kv;
+    pq.causal = causal;
+    pq.scale_log2 = scale * kLog2e;
+    pq.scale = scale;
+    if ((st = set_smem(sqa::sqa_bwd_kernel<D2>, Tr::SMEM_BYTES)) != SQA_OK) return st;
+    if ((st = set_smem(sqa::sqa_bwd_q_kernel<D2>, TQ::SMEM_BYTES)) != SQA_OK) return st;
     if ((st = record_timing(1, 0, stream)) != SQA_OK) return st;
-    sqa::sqa_bwd_kernel<DH < 64 ? 64 : DH>
-        <<<static_cast<unsigned>(grid_main), Tr::THREADS, Tr::SMEM_BYTES, stream>>>(mq, mdo, mk, mv, p);
+    sqa::sqa_bwd_kernel<D2><<<static_cast<unsigned>(grid_main), Tr::THREADS, Tr::SMEM_BYTES, stream>>>(mq, mdo, mk,
+                                                                                                     mv, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "sqa_bwd dK/dV launch");
+    sqa::sqa_bwd_q_kernel<D2><<<static_cast<unsigned>(grid_q), TQ::THREADS, TQ::SMEM_BYTES, stream>>>(mk64, mv64,
+                                                                                                     pq);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "sqa_bwd dQ launch");
+    return record_timing(1, 1, stream);
   }
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "sqa_bwd main launch");
-  if ((st = record_timing(1, 1, stream)) != SQA_OK) return st;
-
-  const long long n_vec8 = static_cast<long long>(s.B) * s.N * s.H_q * DH / 8;
-  sqa::sqa_bwd_dq_kernel<<<grid_for(n_vec8, 256), 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq),
-                                                                    n_vec8, scale);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "sqa_bwd dq launch");
-  return SQA_OK;
 }
 
 // Scratch for sqa_bwd_static_scratch: one device array per GPU that loads the
@@ -451,12 +489,6 @@ sqa_status make_map_2d(CUtensorMap* map, const void* ptr, long long rows, long l
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SQA_ERR_CUDA, "cuTensorMapEncodeTiled (2-D) failed (CUresult %d)", (int)r);
   return SQA_OK;
-}
-
-int sm_count() {
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return sms;
 }
 
 // One K segment of a GEMM: A (K-major [M][k] or MN-major [k][M]) and B

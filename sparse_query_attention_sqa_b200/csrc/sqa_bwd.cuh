@@ -39,7 +39,7 @@ struct BwdLayout {
   int g, T, rows, n_qt, n_kt;
   size_t n_slots;     // B * H_kv * n_qt * 128
   size_t off_D;       // byte offsets inside the workspace
-  size_t off_dq;
+  size_t off_dq;       // dh <= 32 only: the fp32 dQ accumulator
   size_t off_q32;     // dh <= 32 only: fp32 transposed images of the stacked Q and dO tiles
   size_t off_do32;
   size_t bytes;
@@ -55,8 +55,9 @@ inline BwdLayout bwd_layout(int B, int N, int Hq, int Hkv, int dh) {
   L.n_slots = static_cast<size_t>(B) * Hkv * L.n_qt * kBwdTile;
   L.off_D = align256(L.n_slots * sizeof(float));
   L.off_dq = L.off_D + align256(L.n_slots * sizeof(float));
-  L.bytes = L.off_dq + align256(static_cast<size_t>(B) * N * Hq * dh * sizeof(float));
-  if (dh <= 32) {
+  L.bytes = L.off_dq;
+  if (dh <= 32) {  // dh 64 / 128: dQ comes from its own kernel, with no accumulator
+    L.bytes += align256(static_cast<size_t>(B) * N * Hq * dh * sizeof(float));
     const size_t img = align256(L.n_slots * dh * sizeof(float));
     L.off_q32 = L.bytes;
     L.off_do32 = L.bytes + img;

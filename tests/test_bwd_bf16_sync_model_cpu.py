@@ -1,24 +1,23 @@
-"""A model of the synchronisation of the dh 64/128 backward kernel
-(``sqa_bwd_kernel`` in sqa_bwd_bf16.cuh: one CTA per 128-key tile), run on
-the CPU under random schedules with the checker in ``sync_model``.
+"""Models of the synchronisation of the dh 64/128 backward kernels, run on the
+CPU under random schedules with the checker in ``sync_model``.
 
-Roles, in the kernel's program order:
+``sqa_bwd_kernel`` (dK and dV, one CTA per 128-key tile), in program order:
 * the TMA producer: K and V once; the first two Q/dO stages; then, per tile,
   the next tile's -lse2 once the warps have finished P^T (p_ready of the second
-  half), its -D once they have finished dS (ds_ready), and the Q/dO tile two
+  half), its -D once they have finished dS^T (ds_ready), and the Q/dO tile two
   ahead once the stage is free (qd_empty);
-* the MMA-issuing warp: S^T, dP^T (after the dQ of the previous tile was read
-  out), dV per half of 64 query rows (after that half's p_ready), dK and dQ
-  (after ds_ready); MMAs of one issuer run in order, so they are modelled at
-  their place in its program, and everything the other roles learn about them
-  comes through commits that follow them;
+* the MMA-issuing warp: S^T and dP^T of the first tile, then per tile dV per
+  half of 64 query rows (after that half's p_ready), S^T of the next tile,
+  dK (after ds_ready) and dP^T of the next tile; MMAs of one issuer run in
+  order, so they are modelled at their place in its program, and everything the
+  other roles learn about them comes through commits that follow them;
 * the eight softmax warps: P^T of both halves (rewriting S^T's columns), dS^T
-  (rewriting dP^T's columns) and dS into shared memory, the dQ read-out, the
-  dV/dK epilogue.
+  (rewriting dP^T's columns), the dV/dK epilogue.
 
-TMEM columns [128, 256) go through dP^T written, dS^T rewritten, dS^T read by
-the dK MMA, dQ written and dQ read out before the next tile's dP^T.  Barrier
-arrival counts are the kernel's.
+``sqa_bwd_q_kernel`` (dQ, one CTA per stacked Q tile): the producer streams
+K/V through a ring; the warps put Q and dO into TMEM; the issuer runs S_j and
+dP_j into buffer j % 2 and then dQ of j - 1; the warps turn S_j and dP_j into
+dS_j in place; the epilogue reads dQ.  Barrier arrival counts are the kernels'.
 """
 import random
 
@@ -36,9 +35,7 @@ def _stages():
         "lse": [("producer writes -lse2", 1), ("warps read -lse2", WARPS)],
         "dbuf": [("producer writes -D", 1), ("warps read -D", WARPS)],
         "ST": [("S^T write", 1), ("warps rewrite P^T", WARPS), ("dV MMA reads P^T", 1)],
-        "DPT": [("dP^T write", 1), ("warps rewrite dS^T", WARPS), ("dK MMA reads dS^T", 1),
-                ("dQ write (same columns)", 1), ("warps read dQ", WARPS)],
-        "dsbuf": [("warps write dS", WARPS), ("dQ MMA reads dS", 1)],
+        "DPT": [("dP^T write", 1), ("warps rewrite dS^T", WARPS), ("dK MMA reads dS^T", 1)],
         "acc_dv": [("issuer accumulates dV", 1), ("warps read dV", WARPS)],
         "acc_dk": [("issuer accumulates dK", 1), ("warps read dK", WARPS)],
     }
@@ -46,7 +43,7 @@ def _stages():
 
 def _roles(nq):
     cnt = {"kv_full": 1, "lse_full": 1, "d_full": 1, "s_full": 1, "dp_full": 1, "p_ready0": 32 * WARPS,
-           "p_ready1": 32 * WARPS, "ds_ready": 32 * WARPS, "dq_full": 1, "dq_empty": 32 * WARPS, "dkv_final": 1}
+           "p_ready1": 32 * WARPS, "ds_ready": 32 * WARPS, "dkv_final": 1}
     for s in range(QS):
         cnt[f"qd_full{s}"] = 1
         cnt[f"qd_empty{s}"] = 1
@@ -78,17 +75,20 @@ def _roles(nq):
             prod += [W(f"qd_empty{s}", i // QS)] + write("stage", i + QS, 0, s) + [A(f"qd_full{s}")]
 
     iss = [W("kv_full", 0), B("kv", 0, 1), B("acc_dv", 0, 0), B("acc_dk", 0, 0)]
+    iss += [W("qd_full0", 0), B("stage", 0, 1, 0)]
+    iss += [B("ST", 0, 0, 0), B("ST", 0, 0, 1), E("ST", 0, 0, 0), E("ST", 0, 0, 1), A("s_full")]
+    iss += write("DPT", 0, 0) + [A("dp_full")]
     for i in range(nq):
-        s = i % QS
-        iss += [W(f"qd_full{s}", i // QS), B("stage", i, 1, s)]
-        iss += [B("ST", i, 0, 0), B("ST", i, 0, 1), E("ST", i, 0, 0), E("ST", i, 0, 1), A("s_full")]
-        if i > 0:
-            iss.append(W("dq_empty", i - 1))
-        iss += write("DPT", i, 0) + [A("dp_full")]
+        s, s1 = i % QS, (i + 1) % QS
         for hh in range(2):
             iss += [W(f"p_ready{hh}", i)] + write("ST", i, 2, hh)
+        if i + 1 < nq:
+            iss += [W(f"qd_full{s1}", (i + 1) // QS), B("stage", i + 1, 1, s1)]
+            iss += [B("ST", i + 1, 0, 0), B("ST", i + 1, 0, 1), E("ST", i + 1, 0, 0), E("ST", i + 1, 0, 1),
+                    A("s_full")]
         iss += [W("ds_ready", i)] + write("DPT", i, 2) + [E("stage", i, 1, s), A(f"qd_empty{s}")]
-        iss += [B("dsbuf", i, 1), B("DPT", i, 3), E("dsbuf", i, 1), E("DPT", i, 3), A("dq_full")]
+        if i + 1 < nq:
+            iss += write("DPT", i + 1, 0) + [A("dp_full")]
     iss += [E("acc_dv", 0, 0), E("acc_dk", 0, 0), A("dkv_final"), E("kv", 0, 1)]
 
     def warp():
@@ -100,9 +100,8 @@ def _roles(nq):
                 if hh == 1:
                     ops.append(E("lse", i, 1))
                 ops.append(A(f"p_ready{hh}", 32))
-            ops += [W("dp_full", i), W("d_full", i), B("dbuf", i, 1), B("DPT", i, 1), B("dsbuf", i, 0),
-                    E("DPT", i, 1), E("dsbuf", i, 0), E("dbuf", i, 1), A("ds_ready", 32)]
-            ops += [W("dq_full", i)] + write("DPT", i, 4) + [A("dq_empty", 32)]
+            ops += [W("dp_full", i), W("d_full", i), B("dbuf", i, 1), B("DPT", i, 1), E("DPT", i, 1),
+                    E("dbuf", i, 1), A("ds_ready", 32)]
         ops += [W("dkv_final", 0), B("acc_dv", 0, 1), B("acc_dk", 0, 1), E("acc_dv", 0, 1), E("acc_dk", 0, 1)]
         return ops
 
@@ -130,18 +129,16 @@ def _drop(role_prefix, barrier):
 
 
 DROPS = {
-    # dP^T of the next tile would overwrite dQ the warps still read
-    "issuer: dq_empty": _drop("issuer", "dq_empty"),
     # dV would read P^T before the warps wrote it
     "issuer: p_ready": _drop("issuer", "p_ready"),
-    # dK / dQ would read dS^T / dS before the warps wrote them
+    # dK would read dS^T before the warps wrote it; S^T / dP^T of the next tile
+    # would overwrite P^T / dS^T still in use
     "issuer: ds_ready": _drop("issuer", "ds_ready"),
     # the MMAs would read a Q/dO stage before it landed
     "issuer: qd_full": _drop("issuer", "qd_full"),
-    # the warps would read S^T, dP^T or dQ before the MMA wrote it
+    # the warps would read S^T or dP^T before the MMA wrote it
     "warps: s_full": _drop("warp", "s_full"),
     "warps: dp_full": _drop("warp", "dp_full"),
-    "warps: dq_full": _drop("warp", "dq_full"),
     # the warps would read statistics before they landed
     "warps: lse_full": _drop("warp", "lse_full"),
     "warps: d_full": _drop("warp", "d_full"),
@@ -161,6 +158,115 @@ def test_model_detects_a_dropped_wait(name):
     for trial in range(300):
         try:
             run(rnd.randint(2, 10), trial, drop=DROPS[name])
+        except AssertionError:
+            failures += 1
+    assert failures > 0, name
+
+
+# --------------------------------------------------------------------------- sqa_bwd_q_kernel
+
+
+def _q_stages():
+    return {
+        "kv": [("producer writes K, V", 1), ("S, dP, dQ MMAs read", 1)],
+        "QD": [("warps write Q, dO into TMEM", WARPS), ("S, dP MMAs read", 1)],
+        "SB": [("S, dP write", 1), ("warps rewrite dS", WARPS), ("dQ MMA reads dS", 1)],
+        "acc_dq": [("issuer accumulates dQ", 1), ("warps read dQ", WARPS)],
+    }
+
+
+def _q_roles(nkv, ST):
+    cnt = {"qd_ready": 32 * WARPS, "dq_final": 1}
+    for s in range(ST):
+        cnt[f"kv_full{s}"] = 1
+        cnt[f"kv_empty{s}"] = 1
+    for x in range(2):
+        cnt[f"sd_full{x}"] = 1
+        cnt[f"ds_ready{x}"] = 32 * WARPS
+
+    def W(b, k):
+        return ("wait", b, k)
+
+    def A(b, m=1):
+        return ("arrive", b, m)
+
+    def B(res, v, stage, slot=0):
+        return ("begin", (res, slot), v, stage)
+
+    def E(res, v, stage, slot=0):
+        return ("end", (res, slot), v, stage)
+
+    prod = []
+    for j in range(nkv):
+        s = j % ST
+        if j >= ST:
+            prod.append(W(f"kv_empty{s}", j // ST - 1))
+        prod += [B("kv", j, 0, s), E("kv", j, 0, s), A(f"kv_full{s}")]
+
+    def dq(j):
+        x = j & 1
+        return [W(f"ds_ready{x}", j >> 1), B("SB", j, 2, x), E("SB", j, 2, x), E("kv", j, 1, j % ST),
+                A(f"kv_empty{j % ST}")]
+
+    iss = [W("qd_ready", 0), B("QD", 0, 1), B("acc_dq", 0, 0)]
+    for j in range(nkv):
+        x = j & 1
+        iss += [W(f"kv_full{j % ST}", j // ST), B("kv", j, 1, j % ST), B("SB", j, 0, x), E("SB", j, 0, x),
+                A(f"sd_full{x}")]
+        if j > 0:
+            iss += dq(j - 1)
+    iss += dq(nkv - 1) + [E("QD", 0, 1), E("acc_dq", 0, 0), A("dq_final")]
+
+    def warp():
+        ops = [B("QD", 0, 0), E("QD", 0, 0), A("qd_ready", 32)]
+        for j in range(nkv):
+            x = j & 1
+            ops += [W(f"sd_full{x}", j >> 1), B("SB", j, 1, x), E("SB", j, 1, x), A(f"ds_ready{x}", 32)]
+        ops += [W("dq_final", 0), B("acc_dq", 0, 1), E("acc_dq", 0, 1)]
+        return ops
+
+    roles = {"producer": prod, "issuer": iss}
+    for w in range(WARPS):
+        roles[f"warp{w}"] = warp()
+    return roles, cnt
+
+
+def run_q(nkv, ST, seed, drop=None):
+    roles, cnt = _q_roles(nkv, ST)
+    if drop is not None:
+        roles = {r: [op for op in ops if not drop(r, op)] for r, ops in roles.items()}
+    sync_model.run(roles, cnt, _q_stages(), seed, skewed=seed % 2 == 1)
+
+
+@pytest.mark.parametrize("ST", [6, 8, 2])
+def test_q_kernel_protocol_has_no_deadlock_aliasing_or_hazard(ST):
+    rnd = random.Random(ST)
+    for trial in range(300):
+        run_q(rnd.randint(1, 14), ST, trial)
+
+
+Q_DROPS = {
+    # S / dP would read Q, dO before the warps put them into TMEM
+    "issuer: qd_ready": _drop("issuer", "qd_ready"),
+    # dQ would read dS before the warps wrote it (and S of j + 2 would overwrite it)
+    "issuer: ds_ready": _drop("issuer", "ds_ready"),
+    # the MMAs would read a K/V stage before it landed
+    "issuer: kv_full": _drop("issuer", "kv_full"),
+    # the warps would read S / dP before the MMA wrote them, or dQ before the last MMA
+    "warps: sd_full": _drop("warp", "sd_full"),
+    "warps: dq_final": _drop("warp", "dq_final"),
+    # the producer would overwrite a K/V stage still in use
+    "producer: kv_empty": _drop("producer", "kv_empty"),
+}
+
+
+@pytest.mark.parametrize("name", list(Q_DROPS))
+def test_q_model_detects_a_dropped_wait(name):
+    rnd = random.Random(29)
+    failures = 0
+    for trial in range(300):
+        try:
+            run_q(rnd.randint(3, 12), 2, trial, drop=Q_DROPS[name])
         except AssertionError:
             failures += 1
     assert failures > 0, name
