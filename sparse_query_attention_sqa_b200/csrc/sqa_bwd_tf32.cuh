@@ -72,11 +72,6 @@ __device__ __forceinline__ void mma_ts_tf32_w(uint32_t d_tmem, uint32_t a_tmem, 
 }
 }  // namespace dev
 
-// Whether tiles whose keys are all visible to every row skip the mask test,
-// and whether dS is rounded to the nearest tf32 value before the dK MMA.
-constexpr bool kBwdMaskBranch = false;
-constexpr bool kBwdRoundDs = true;
-
 template <int DH>
 struct BwdTf32Traits {
   static_assert(DH == 16 || DH == 32, "tf32 backward handles dh 16 and 32");
@@ -126,10 +121,6 @@ struct BwdTf32Traits {
 // lim > rtok[column].  dS is rounded to the nearest tf32 value by
 // Veltkamp splitting (with C = 2^13 + 1, C x - (C x - x) keeps the 11 leading
 // significant bits, rounded to nearest), in packed fp32 pairs.
-// MASK = false skips the mask test (tiles where every key is visible to every
-// row of the Q tile); ROUND = false passes dS to the tf32 MMA unrounded (the
-// tensor core then ignores its low 13 mantissa bits).
-template <bool MASK, bool ROUND>
 __device__ __forceinline__ void bwd_p_ds16(const uint32_t (&sr)[32], const float* nl2, const float* nd,
                                            const int* rtok, int lim, float2 sl2, uint32_t (&pt)[16],
                                            uint32_t (&dst)[16], uint32_t (&dsb)[8]) {
@@ -139,22 +130,19 @@ __device__ __forceinline__ void bwd_p_ds16(const uint32_t (&sr)[32], const float
   for (int e = 0; e < 16; e += 4) {
     const float4 l4 = *reinterpret_cast<const float4*>(nl2 + e);
     const float4 d4 = *reinterpret_cast<const float4*>(nd + e);
-    const int4 r4 = MASK ? *reinterpret_cast<const int4*>(rtok + e) : make_int4(0, 0, 0, 0);
+    const int4 r4 = *reinterpret_cast<const int4*>(rtok + e);
 #pragma unroll
     for (int u = 0; u < 4; u += 2) {
       const float2 l = u == 0 ? make_float2(l4.x, l4.y) : make_float2(l4.z, l4.w);
       const float2 d = u == 0 ? make_float2(d4.x, d4.y) : make_float2(d4.z, d4.w);
       const float2 xx = __ffma2_rn(make_float2(__uint_as_float(sr[e + u]), __uint_as_float(sr[e + u + 1])), sl2, l);
       float p0 = ex2(xx.x), p1 = ex2(xx.y);
-      if (MASK && lim > (u == 0 ? r4.x : r4.z)) p0 = 0.f;
-      if (MASK && lim > (u == 0 ? r4.y : r4.w)) p1 = 0.f;
+      if (lim > (u == 0 ? r4.x : r4.z)) p0 = 0.f;
+      if (lim > (u == 0 ? r4.y : r4.w)) p1 = 0.f;
       const float2 t = __fadd2_rn(make_float2(__uint_as_float(sr[16 + e + u]), __uint_as_float(sr[16 + e + u + 1])), d);
       const float2 ds = __fmul2_rn(make_float2(p0, p1), t);
-      float2 hi = ds;
-      if (ROUND) {
-        const float2 cx = __fmul2_rn(ds, split);
-        hi = __ffma2_rn(__ffma2_rn(ds, minus1, cx), minus1, cx);
-      }
+      const float2 cx = __fmul2_rn(ds, split);
+      const float2 hi = __ffma2_rn(__ffma2_rn(ds, minus1, cx), minus1, cx);
       pt[e + u] = __float_as_uint(p0);
       pt[e + u + 1] = __float_as_uint(p1);
       dst[e + u] = __float_as_uint(hi.x);
@@ -447,8 +435,6 @@ __global__ void __launch_bounds__(384, 1)
         // P is zeroed where lim > rtok[row]: keys past N always, keys after the
         // row's token on the causal diagonal.
         const int lim = !key_ok ? 0x7fffffff : (masked ? key - qt * p.T : -0x7fffffff);
-        // Whether any key of this warp can be hidden from any row of the tile.
-        const bool edge = __any_sync(0xffffffffu, lim != -0x7fffffff);
         uint8_t* ds_smem = smem + Tr::OFF_DS + (G & 1) * Tr::DS_BYTES;
         // dS (bf16) for the dQ MMA goes to this buffer, which the dQ of tile G - 2 read.
         if (G >= 2) {
@@ -477,12 +463,8 @@ __global__ void __launch_bounds__(384, 1)
             // The mask test runs on every tile (lim makes it a no-op off the
             // diagonal): cheaper than branching between two versions.
             uint32_t pt[16], dst[16], dsb[8];
-            if (kBwdMaskBranch && !edge)
-              bwd_p_ds16<false, kBwdRoundDs>(c16 ? cb : ca, nl2 + 16 * c16, nl2 + 128 + 16 * c16,
-                                             rtok + col0 + 16 * c16, lim, sl2, pt, dst, dsb);
-            else
-              bwd_p_ds16<true, kBwdRoundDs>(c16 ? cb : ca, nl2 + 16 * c16, nl2 + 128 + 16 * c16,
-                                            rtok + col0 + 16 * c16, lim, sl2, pt, dst, dsb);
+            bwd_p_ds16(c16 ? cb : ca, nl2 + 16 * c16, nl2 + 128 + 16 * c16, rtok + col0 + 16 * c16, lim, sl2, pt,
+                             dst, dsb);
             tmem_st16x2(tS + 16 * c16, tP + 16 * c16, pt, dst);
             // dS[q][key] for q = col0 + 16 c16 .. + 15 into the MN-major 128B-swizzled
             // tile: panel q / 64, key row kk (128 bytes), 16-byte chunk (q % 64) / 8.
