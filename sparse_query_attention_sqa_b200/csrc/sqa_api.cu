@@ -138,14 +138,18 @@ sqa_status launch_fwd(const void* q, const void* k, const void* v, void* out, fl
   p.n_bh = s.B * s.H_kv;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * kLog2e;
-  const long long items = static_cast<long long>(p.n_pairs) * p.n_bh;
-  if (items > 0x7fffffffLL) return fail(SQA_ERR_UNSUPPORTED, "problem too large for one launch");
-  p.n_items = static_cast<int>(items);
-  // Persistent kernel: at most one CTA per SM, each walking several work items.
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return cuda_fail(e, "querying the SM count");
+  // Small problems, whose pairs of Q tiles would fill less than half the SMs:
+  // one Q tile per CTA, its key tiles shared between the two tile slots
+  // (needs a K/V ring of at least four stages: dh <= 64).
+  p.split = (DH <= 64 && static_cast<long long>(p.n_pairs) * p.n_bh < sms / 2) ? 1 : 0;
+  const long long items = static_cast<long long>(p.split ? p.n_qtiles : p.n_pairs) * p.n_bh;
+  if (items > 0x7fffffffLL) return fail(SQA_ERR_UNSUPPORTED, "problem too large for one launch");
+  p.n_items = static_cast<int>(items);
+  // Persistent kernel: at most one CTA per SM, each walking several work items.
   const long long grid = items < sms ? items : sms;
 
   CUtensorMap mq, mk, mv;

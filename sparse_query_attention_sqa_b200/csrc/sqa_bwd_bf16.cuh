@@ -308,13 +308,15 @@ __global__ void __launch_bounds__(384, 1)
                                        mbar_wait(lse_full, i & 1, abort_flag, kSiteSoftmax));
       if (!ok) break;
       tc_fence_after();
-      // P^T of both halves; kept in registers (fp32) for dS.
+      // P^T of both halves (their S^T columns loaded with one wait); kept in
+      // registers (fp32) for dS.
       float pr[2][32];
+      uint32_t sr2[64];  // [0, 32): half 0, [32, 64): half 1
+      tmem_ld32x2(lane_addr + Tr::TM_ST + 32 * w, lane_addr + Tr::TM_ST + 64 + 32 * w, sr2);
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         const int col0 = 64 * hh + 32 * w;
-        uint32_t sr[32];
-        tmem_ld32(lane_addr + Tr::TM_ST + col0, sr);
+        const uint32_t* sr = sr2 + 32 * hh;
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           const float4 l4 = *reinterpret_cast<const float4*>(nl2 + col0 + e);
@@ -341,11 +343,12 @@ __global__ void __launch_bounds__(384, 1)
                                        mbar_wait(d_full, i & 1, abort_flag, kSiteSoftmax));
       if (!ok) break;
       tc_fence_after();
+      uint32_t dr2[64];  // dP^T of both halves, one wait
+      tmem_ld32x2(lane_addr + Tr::TM_DPT + 32 * w, lane_addr + Tr::TM_DPT + 64 + 32 * w, dr2);
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         const int col0 = 64 * hh + 32 * w;
-        uint32_t dr[32];
-        tmem_ld32(lane_addr + Tr::TM_DPT + col0, dr);
+        const uint32_t* dr = dr2 + 32 * hh;
         uint32_t dk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
@@ -632,21 +635,20 @@ __global__ void __launch_bounds__(384, 1)
       if (!ok) break;
       tc_fence_after();
       const int k0 = j * NK + 32 * w;  // this warpgroup's first key
-      uint32_t sr[32], dr[32];
-      tmem_ld32(lane_addr + Tr::tm_s(x) + 32 * w, sr);
-      tmem_ld32(lane_addr + Tr::tm_dp(x) + 32 * w, dr);
+      uint32_t sd[64];                 // [0, 32): S, [32, 64): dP (one wait for both loads)
+      tmem_ld32x2(lane_addr + Tr::tm_s(x) + 32 * w, lane_addr + Tr::tm_dp(x) + 32 * w, sd);
       const bool edge = __any_sync(0xffffffffu, k0 + 31 > last);
       uint32_t pk[16];
 #pragma unroll
       for (int e = 0; e < 32; e += 2) {
-        float p0 = ex2(fmaf(__uint_as_float(sr[e]), sl2, nl2));
-        float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), sl2, nl2));
+        float p0 = ex2(fmaf(__uint_as_float(sd[e]), sl2, nl2));
+        float p1 = ex2(fmaf(__uint_as_float(sd[e + 1]), sl2, nl2));
         if (edge) {
           if (k0 + e > last) p0 = 0.f;
           if (k0 + e + 1 > last) p1 = 0.f;
         }
         const float2 ds = __fmul2_rn(make_float2(p0, p1),
-                                     __fadd2_rn(make_float2(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])),
+                                     __fadd2_rn(make_float2(__uint_as_float(sd[32 + e]), __uint_as_float(sd[33 + e])),
                                                 make_float2(nd, nd)));
         pk[e >> 1] = pack_bf16x2(ds.x, ds.y);
       }

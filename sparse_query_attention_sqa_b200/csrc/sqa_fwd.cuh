@@ -48,6 +48,7 @@ struct FwdParams {
   int n_bh;      // B * Hkv
   int n_items;   // n_pairs * n_bh
   int causal;
+  int split;         // 1: both tile slots of a CTA work on one Q tile, even / odd key tiles
   float scale_log2;  // scale * log2(e)
 };
 
@@ -73,9 +74,11 @@ struct FwdTraits {
   static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
   // q_full[QB] | q_empty[QB] | kv_full[S] | kv_empty[S] | s_full[2][2] | p_full[2][2] |
-  // o_done[2] | o_final[2] | o_free[2] | drain[2]
-  static constexpr int N_BARS = 2 * QBUF + 2 * STAGES + 4 + 4 + 2 + 2 + 2 + 2;
-  static constexpr int SMEM_USED = OFF_BAR + N_BARS * 8 + 16;
+  // o_done[2] | o_final[2] | o_free[2] | drain[2] | split_ready | split_done
+  static constexpr int N_BARS = 2 * QBUF + 2 * STAGES + 4 + 4 + 2 + 2 + 2 + 2 + 2;
+  // split mode: slot 1's running maximum and sum per row, for slot 0's combine
+  static constexpr int OFF_ML = OFF_BAR + N_BARS * 8 + 16;
+  static constexpr int SMEM_USED = OFF_ML + 2 * BM * 4;
   // Ask for enough shared memory that only one CTA fits per SM (each CTA holds
   // all 512 TMEM columns), plus slack to align the base to 1024 bytes.
   static constexpr int SMEM_BYTES = (SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024) + 1024;
@@ -96,10 +99,20 @@ struct FwdItem {
 
 __device__ __forceinline__ FwdItem fwd_decode(const FwdParams& p, int item, int NK) {
   FwdItem it;
-  const int pair = p.n_pairs - 1 - item / p.n_bh;  // latest tokens (heaviest under a causal mask) first
   const int bh = item % p.n_bh;
   it.b = bh / p.Hkv;
   it.kvh = bh % p.Hkv;
+  if (p.split) {
+    // One Q tile; slot 0 takes its even key tiles, slot 1 the odd ones.
+    it.qt0 = p.n_qtiles - 1 - item / p.n_bh;  // latest tokens (heaviest under a causal mask) first
+    const int end = p.causal ? min(p.N, (it.qt0 + 1) * p.T) : p.N;
+    it.nkv = (end + NK - 1) / NK;
+    it.nkv0 = (it.nkv + 1) / 2;
+    it.nkv1 = it.nkv / 2;
+    it.has1 = false;  // one Q tile to load
+    return it;
+  }
+  const int pair = p.n_pairs - 1 - item / p.n_bh;  // latest tokens (heaviest under a causal mask) first
   it.qt0 = 2 * pair;
   it.has1 = it.qt0 + 1 < p.n_qtiles;
   const int end0 = p.causal ? min(p.N, (it.qt0 + 1) * p.T) : p.N;
@@ -142,6 +155,10 @@ __global__ void __launch_bounds__(384, 1)
   auto o_final = [&](int t) { return bar0 + 8u * (2 * QB + 2 * ST + 10 + t); };
   auto o_free = [&](int t) { return bar0 + 8u * (2 * QB + 2 * ST + 12 + t); };
   auto drain = [&](int t) { return bar0 + 8u * (2 * QB + 2 * ST + 14 + t); };
+  const uint32_t split_ready = bar0 + 8u * (2 * QB + 2 * ST + 16);  // slot 1's O, m, l are final
+  const uint32_t split_done = bar0 + 8u * (2 * QB + 2 * ST + 17);   // slot 0 has read them
+  float* sm_m = reinterpret_cast<float*>(smem + Tr::OFF_ML);
+  float* sm_l = sm_m + BM;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Tr::OFF_BAR + Tr::N_BARS * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -165,6 +182,8 @@ __global__ void __launch_bounds__(384, 1)
     }
     mbar_init(drain(0), 1);
     mbar_init(drain(1), 1);
+    mbar_init(split_ready, 128);
+    mbar_init(split_done, 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -236,7 +255,8 @@ __global__ void __launch_bounds__(384, 1)
     constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, DH, false, true);
     // Descriptors of Q buffer 0 / stage 0; other buffers, stages and K-steps add
     // their byte offset (in 16-byte units) to the start-address field.
-    const uint64_t dq0 = smem_desc(sbase + Tr::OFF_Q + t * Tr::Q_BYTES, 16, 8 * ROWB, Tr::LAYOUT);
+    // (In split mode both slots read the one Q tile, in slot 0's buffer.)
+    const uint64_t dq0 = smem_desc(sbase + Tr::OFF_Q + (p.split ? 0 : t) * Tr::Q_BYTES, 16, 8 * ROWB, Tr::LAYOUT);
     const uint64_t dk0 = smem_desc(sbase + Tr::OFF_K, 16, 8 * ROWB, Tr::LAYOUT);
     const uint64_t dv0 = smem_desc(sbase + Tr::OFF_V, NK * ROWB, 8 * ROWB, Tr::LAYOUT);
     const uint32_t tS0 = tmem + Tr::tm_s(t, 0), tO = tmem + Tr::tm_o(t);
@@ -260,15 +280,20 @@ __global__ void __launch_bounds__(384, 1)
       mma_commit_w(o_done(t));
     };
     int loaded = 0;  // K/V tiles whose kv_full phase this warp has observed
+    int g = 0;       // first K/V tile (global index) of the current item
+    // In split mode a slot releases the other slot's key tiles as soon as it
+    // has observed them loaded.
     auto ensure_loaded = [&](int gj) {
       while (loaded <= gj) {
         if (!mbar_wait_warp(kv_full(loaded % ST), (loaded / ST) & 1, abort_flag, kSiteMma)) return false;
+        if (p.split && ((loaded - g) & 1) != t) mma_commit_w(kv_empty(loaded % ST));
         ++loaded;
       }
       tc_fence_after();
       return true;
     };
-    int g = 0;   // first K/V tile (global index) of the current item
+    // item-relative index of this slot's j-th key tile
+    auto own = [&](int j) { return p.split ? 2 * j + t : j; };
     int G = 0;   // S steps of this Q tile so far (across items)
     int nd = 0;  // items finished by this Q tile
     bool ok = true;
@@ -283,8 +308,8 @@ __global__ void __launch_bounds__(384, 1)
         break;
       }
       for (int j = 0; ok && j < NSB && j < nkv_t; ++j) {  // prologue: S for the first key tiles
-        ok = ensure_loaded(g + j);
-        if (ok) issue_qk(qb, (g + j) % ST, (G + j) % NSB);
+        ok = ensure_loaded(g + own(j));
+        if (ok) issue_qk(qb, (g + own(j)) % ST, (G + j) % NSB);
       }
       for (int j = 0; ok && j < nkv_t; ++j) {
         const int Gt = G + j;
@@ -298,24 +323,31 @@ __global__ void __launch_bounds__(384, 1)
           break;
         }
         tc_fence_after();
-        issue_pv((g + j) % ST, Gt % NSB, j > 0);
+        issue_pv((g + own(j)) % ST, Gt % NSB, j > 0);
+        if (j + 1 == nkv_t) mma_commit_w(o_final(t));
+        // The stage is released when the PV just issued has read V (a commit
+        // covers every MMA issued before it), before waiting for a later one.
+        mma_commit_w(kv_empty((g + own(j)) % ST));
         if (j + NSB < nkv_t) {
           // The next S in this buffer: the PV just issued reads P from it first
           // (MMAs from one issuer execute in order).
-          if (!ensure_loaded(g + j + NSB)) {
+          if (!ensure_loaded(g + own(j + NSB))) {
             ok = false;
             break;
           }
-          issue_qk(qb, (g + j + NSB) % ST, Gt % NSB);
+          issue_qk(qb, (g + own(j + NSB)) % ST, Gt % NSB);
         }
-        if (j + 1 == nkv_t) mma_commit_w(o_final(t));
-        mma_commit_w(kv_empty((g + j) % ST));
       }
-      // K/V tiles of this item that this Q tile does not need (causal: the other
-      // tile reaches one tile further) are released too, once they are loaded.
-      for (int j = nkv_t; ok && j < it.nkv; ++j) {
-        ok = ensure_loaded(g + j);
-        if (ok) mma_commit_w(kv_empty((g + j) % ST));
+      if (p.split) {
+        // the other slot's tiles after this slot's last one
+        if (ok && it.nkv > 0) ok = ensure_loaded(g + it.nkv - 1);
+      } else {
+        // K/V tiles of this item that this Q tile does not need (causal: the other
+        // tile reaches one tile further) are released too, once they are loaded.
+        for (int j = nkv_t; ok && j < it.nkv; ++j) {
+          ok = ensure_loaded(g + j);
+          if (ok) mma_commit_w(kv_empty((g + j) % ST));
+        }
       }
       if (!ok) break;
       mma_commit_w(q_empty(qb));
@@ -335,12 +367,14 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tO = lane_addr + Tr::tm_o(t);
     const float sl2 = p.scale_log2;
     int G = 0, nd = 0;
+    int nc = 0;  // split mode: combines done (phases of split_ready / split_done)
     bool ok = true;
     for (int r = 0, item; ok && (item = fwd_item(r, p.n_items)) >= 0; ++r) {
       const FwdItem it = fwd_decode(p, item, NK);
       const int nkv_t = t ? it.nkv1 : it.nkv0;
       if (nkv_t == 0) continue;
-      const int qt = it.qt0 + t;
+      const int qt = p.split ? it.qt0 : it.qt0 + t;
+      const bool combine = p.split && it.nkv1 > 0;  // slot 1 holds part of this row's sums
       const int tok = qt * p.T + row / p.g;
       const int head = it.kvh * p.g + row % p.g;
       const bool row_valid = row < p.rows && tok < p.N;
@@ -353,7 +387,7 @@ __global__ void __launch_bounds__(384, 1)
         if (!ok) break;
         tc_fence_after();
         const uint32_t tS = lane_addr + Tr::tm_s(t, Gt % NSB);
-        const int k0 = j * NK;
+        const int k0 = (p.split ? 2 * j + t : j) * NK;
         const bool masked = (k0 + NK > p.N) || (p.causal && k0 + NK - 1 > qt * p.T);
         // The tile's scores are handled 64 columns (a half at NK = 128) at a time.
         // last visible key of this tile, relative to k0 (may be negative)
@@ -464,30 +498,75 @@ __global__ void __launch_bounds__(384, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(o_final(t), nd & 1, abort_flag, kSiteEpilogue));
       if (!ok) break;
       tc_fence_after();
+      if (combine && t == 1) {
+        // Slot 1 hands its row statistics to slot 0, which reads O_1 from TMEM
+        // too; O_1 stays until slot 0 is done with it.
+        sm_m[row] = m;
+        sm_l[row] = l;
+        tc_fence_before();
+        mbar_arrive(split_ready);
+        ok = __all_sync(0xffffffffu, mbar_wait(split_done, nc & 1, abort_flag, kSiteEpilogue));
+        if (!ok) break;
+        tc_fence_before();
+        mbar_arrive(o_free(t));
+        G += nkv_t;
+        ++nd;
+        ++nc;
+        continue;
+      }
+      // Split mode: O = O_0 2^(m_0 - M) + O_1 2^(m_1 - M) over L = l_0 2^(m_0 - M) +
+      // l_1 2^(m_1 - M), M = max(m_0, m_1).
+      float a0 = 1.f, a1 = 0.f;
+      const uint32_t tO1 = lane_addr + Tr::tm_o(1);
+      if (combine) {
+        ok = __all_sync(0xffffffffu, mbar_wait(split_ready, nc & 1, abort_flag, kSiteEpilogue));
+        if (!ok) break;
+        tc_fence_after();
+        const float m1 = sm_m[row], l1 = sm_l[row];
+        const float M = fmaxf(m, m1);
+        a0 = M == -INFINITY ? 0.f : ex2(m - M);
+        a1 = M == -INFINITY ? 0.f : ex2(m1 - M);
+        l = l * a0 + l1 * a1;
+        m = M;
+      }
       const float inv_l = row_valid ? 1.f / l : 0.f;
+      const float c0 = a0 * inv_l, c1 = a1 * inv_l;
       __nv_bfloat16* dst =
           p.out + ((static_cast<size_t>(it.b) * p.N + (row_valid ? tok : 0)) * p.Hq + head) * DH;
 #pragma unroll 1
       for (int c = 0; c < DH; c += 16) {
         uint32_t rr[16];
+        float y[16];
         tmem_ld16(tO + c, rr);  // warp-wide: every lane loads, only valid rows store
+#pragma unroll
+        for (int i = 0; i < 16; ++i) y[i] = __uint_as_float(rr[i]) * c0;
+        if (combine) {
+          tmem_ld16(tO1 + c, rr);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) y[i] = fmaf(__uint_as_float(rr[i]), c1, y[i]);
+        }
         uint4 lo, hi;
-        lo.x = pack_bf16x2(__uint_as_float(rr[0]) * inv_l, __uint_as_float(rr[1]) * inv_l);
-        lo.y = pack_bf16x2(__uint_as_float(rr[2]) * inv_l, __uint_as_float(rr[3]) * inv_l);
-        lo.z = pack_bf16x2(__uint_as_float(rr[4]) * inv_l, __uint_as_float(rr[5]) * inv_l);
-        lo.w = pack_bf16x2(__uint_as_float(rr[6]) * inv_l, __uint_as_float(rr[7]) * inv_l);
-        hi.x = pack_bf16x2(__uint_as_float(rr[8]) * inv_l, __uint_as_float(rr[9]) * inv_l);
-        hi.y = pack_bf16x2(__uint_as_float(rr[10]) * inv_l, __uint_as_float(rr[11]) * inv_l);
-        hi.z = pack_bf16x2(__uint_as_float(rr[12]) * inv_l, __uint_as_float(rr[13]) * inv_l);
-        hi.w = pack_bf16x2(__uint_as_float(rr[14]) * inv_l, __uint_as_float(rr[15]) * inv_l);
+        lo.x = pack_bf16x2(y[0], y[1]);
+        lo.y = pack_bf16x2(y[2], y[3]);
+        lo.z = pack_bf16x2(y[4], y[5]);
+        lo.w = pack_bf16x2(y[6], y[7]);
+        hi.x = pack_bf16x2(y[8], y[9]);
+        hi.y = pack_bf16x2(y[10], y[11]);
+        hi.z = pack_bf16x2(y[12], y[13]);
+        hi.w = pack_bf16x2(y[14], y[15]);
         if (row_valid) {
           *reinterpret_cast<uint4*>(dst + c) = lo;
           *reinterpret_cast<uint4*>(dst + c + 8) = hi;
         }
       }
-      // O has been read: the next item's first PV may overwrite it.
+      // O has been read: the next item's first PV may overwrite it (and, in
+      // split mode, slot 1's).
       tc_fence_before();
       mbar_arrive(o_free(t));
+      if (combine) {
+        mbar_arrive(split_done);
+        ++nc;
+      }
       if (row_valid)
         p.lse[(static_cast<size_t>(it.b) * p.Hq + head) * p.N + tok] = (m + __log2f(l)) * 0.69314718055994531f;
       G += nkv_t;

@@ -82,9 +82,11 @@ class Accumulator:
             self.epi_ended[info[1]] = self.epi_ended.get(info[1], 0) + 1
 
 
-def _roles(items, QB, ST, rnd, NSB=2):
-    """items: [(nkv0, nkv1)] per work item of one CTA."""
-    cnt = {}
+def _roles(items, QB, ST, rnd, NSB=2, split=False):
+    """items: [(nkv0, nkv1)] per work item of one CTA.  split: both slots on one
+    Q tile, slot t taking the item's key tiles t, t + 2, ... (nkv0 = ceil(n / 2),
+    nkv1 = floor(n / 2)), slot 1's O read by slot 0's warps in the combine."""
+    cnt = {"split_ready": 32 * WARPS_PER_TILE, "split_done": 32 * WARPS_PER_TILE}
     for qb in range(QB):
         cnt[f"q_full{qb}"] = 1
         cnt[f"q_empty{qb}"] = 2
@@ -111,9 +113,12 @@ def _roles(items, QB, ST, rnd, NSB=2):
     def E(res, slot, v, stage=None):
         return ("end", (res, slot), v, stage)
 
+    def nkv_of(n0, n1):
+        return n0 + n1 if split else max(n0, n1)
+
     prod, g = [], 0
     for r, (n0, n1) in enumerate(items):
-        qb, nkv = r % QB, max(n0, n1)
+        qb, nkv = r % QB, nkv_of(n0, n1)
         if r >= QB:
             prod.append(W(f"q_empty{qb}", r // QB - 1))
         prod += [B("q", qb, r, 0), E("q", qb, r, 0), A(f"q_full{qb}")]
@@ -125,13 +130,19 @@ def _roles(items, QB, ST, rnd, NSB=2):
         g += nkv
 
     def issuer(t):
-        ops, g, G, nd, loaded = [], 0, 0, 0, [0]
+        ops, g, G, nd, loaded = [], [0], 0, 0, [0]
         S = f"S{t}"
+
+        def own(j):
+            return 2 * j + t if split else j
 
         def ensure(gj):
             out = []
             while loaded[0] <= gj:
-                out.append(W(f"kv_full{loaded[0] % ST}", loaded[0] // ST))
+                i = loaded[0]
+                out.append(W(f"kv_full{i % ST}", i // ST))
+                if split and (i - g[0]) % 2 != t:  # the other slot's tile: released at once
+                    out += [B("kv", i % ST, i, 1), E("kv", i % ST, i, 1), A(f"kv_empty{i % ST}")]
                 loaded[0] += 1
             return out
 
@@ -139,12 +150,14 @@ def _roles(items, QB, ST, rnd, NSB=2):
             return [B(S, step % NSB, step, 0), E(S, step % NSB, step, 0), A(f"s_full{t}{step % NSB}")]
 
         for r, (n0, n1) in enumerate(items):
-            nkv_t, nkv, qb = (n1 if t else n0), max(n0, n1), r % QB
+            nkv_t, nkv, qb = (n1 if t else n0), nkv_of(n0, n1), r % QB
+            base = g[0]
             ops += [W(f"q_full{qb}", r // QB), B("q", qb, r, 1)]
             for j in range(min(NSB, nkv_t)):
-                ops += ensure(g + j) + [B("kv", (g + j) % ST, g + j, 1)] + qk(qb, g + j, G + j)
+                gi = base + own(j)
+                ops += ensure(gi) + [B("kv", gi % ST, gi, 1)] + qk(qb, gi, G + j)
             for j in range(nkv_t):
-                step = G + j
+                step, gi = G + j, base + own(j)
                 ops.append(W(f"p_full{t}{step % NSB}", step // NSB))
                 if j == 0 and nd > 0:
                     ops.append(W(f"o_free{t}", nd - 1))
@@ -152,26 +165,33 @@ def _roles(items, QB, ST, rnd, NSB=2):
                 # issuer run in order, so its read of P ends before the next S MMA.
                 ops += [B(S, step % NSB, step, 2), B("O", t, ("pv", step, nd, j == 0)),
                         E(S, step % NSB, step, 2), E("O", t, ("pv",)), A(f"o_done{t}")]
-                if j + NSB < nkv_t:
-                    ops += ensure(g + j + NSB) + [B("kv", (g + j + NSB) % ST, g + j + NSB, 1)] + \
-                        qk(qb, g + j + NSB, step + NSB)
                 if j + 1 == nkv_t:
                     ops.append(A(f"o_final{t}"))
-                ops += [E("kv", (g + j) % ST, g + j, 1), A(f"kv_empty{(g + j) % ST}")]
-            for j in range(nkv_t, nkv):  # tiles the other Q tile needs: released once loaded
-                ops += ensure(g + j) + [B("kv", (g + j) % ST, g + j, 1), E("kv", (g + j) % ST, g + j, 1),
-                                        A(f"kv_empty{(g + j) % ST}")]
+                # the stage is released (after the P V just issued) before a later one is awaited
+                ops += [E("kv", gi % ST, gi, 1), A(f"kv_empty{gi % ST}")]
+                if j + NSB < nkv_t:
+                    gn = base + own(j + NSB)
+                    ops += ensure(gn) + [B("kv", gn % ST, gn, 1)] + qk(qb, gn, step + NSB)
+            if split:
+                if nkv > 0:
+                    ops += ensure(base + nkv - 1)
+            else:
+                for j in range(nkv_t, nkv):  # tiles the other Q tile needs: released once loaded
+                    ops += ensure(base + j) + [B("kv", (base + j) % ST, base + j, 1),
+                                               E("kv", (base + j) % ST, base + j, 1),
+                                               A(f"kv_empty{(base + j) % ST}")]
             ops += [E("q", qb, r, 1), A(f"q_empty{qb}")]
             G += nkv_t
             nd += 1 if nkv_t else 0
-            g += nkv
+            g[0] = base + nkv
         return ops
 
     def softmax_warp(t):
-        ops, G, nd = [], 0, 0
+        ops, G, nd, G1, nd1, nc = [], 0, 0, 0, 0, 0
         S = f"S{t}"
         for (n0, n1) in items:
             nkv_t = n1 if t else n0
+            combine = split and n1 > 0
             if nkv_t == 0:
                 continue
             for j in range(nkv_t):
@@ -180,10 +200,23 @@ def _roles(items, QB, ST, rnd, NSB=2):
                 if j > 0 and rnd.random() < 0.5:  # the running maximum rose: rescale O
                     ops += [W(f"o_done{t}", step - 1), B("O", t, ("rescale", step)), E("O", t, ("rescale",))]
                 ops += [E(S, step % NSB, step, 1), A(f"p_full{t}{step % NSB}", 32)]
-            ops += [W(f"o_final{t}", nd), B("O", t, ("epi", nd, G + nkv_t)), E("O", t, ("epi", nd)),
-                    A(f"o_free{t}", 32)]
+            ops.append(W(f"o_final{t}", nd))
+            if combine and t == 1:
+                # hand m, l to slot 0; O_1 stays until slot 0 has read it
+                ops += [A("split_ready", 32), W("split_done", nc), A(f"o_free{t}", 32)]
+            else:
+                if combine:  # slot 0 reads O_1 as well
+                    ops += [W("split_ready", nc), B("O", 1, ("epi", nd1, G1 + n1)), E("O", 1, ("epi", nd1))]
+                ops += [B("O", t, ("epi", nd, G + nkv_t)), E("O", t, ("epi", nd)), A(f"o_free{t}", 32)]
+                if combine:
+                    ops.append(A("split_done", 32))
             G += nkv_t
             nd += 1
+            if combine:
+                nc += 1
+            if split and n1 > 0:
+                G1 += n1
+                nd1 += 1
         return ops
 
     roles = {"producer": prod, "issuer0": issuer(0), "issuer1": issuer(1)}
@@ -206,12 +239,12 @@ def _items(rnd):
     return out
 
 
-def run(items, QB, ST, seed, drop=None, NSB=2):
+def run(items, QB, ST, seed, drop=None, NSB=2, split=False):
     rnd = random.Random(seed)
-    roles, cnt = _roles(items, QB, ST, rnd, NSB)
+    roles, cnt = _roles(items, QB, ST, rnd, NSB, split)
     if drop is not None:
         roles = {r: [op for op in ops if not drop(r, op)] for r, ops in roles.items()}
-    sync_model.run(roles, cnt, STAGES, seed, custom={"O": _OCheck()})
+    sync_model.run(roles, cnt, STAGES, seed, custom={"O": _OCheck()}, skewed=seed % 2 == 1)
 
 
 class _OCheck:
@@ -276,6 +309,46 @@ def test_model_detects_a_dropped_wait(name, NSB):
         items = _items(rnd)
         try:
             run(items, 2 if NSB == 2 else 1, 4 if NSB == 2 else 2, trial, drop=DROPS[name], NSB=NSB)
+        except AssertionError:
+            failures += 1
+    assert failures > 0, name
+
+
+def _split_items(rnd):
+    out = []
+    for _ in range(rnd.randint(1, 5)):
+        n = rnd.randint(1, 9)
+        out.append(((n + 1) // 2, n // 2))
+    return out
+
+
+@pytest.mark.parametrize("QB,ST", [(2, 8), (2, 4)])
+def test_split_mode_has_no_deadlock_aliasing_or_hazard(QB, ST):
+    """One Q tile per item, the two slots on alternate key tiles, slot 1's
+    results combined into slot 0's (dh <= 64)."""
+    rnd = random.Random(QB * 100 + ST)
+    for trial in range(200):
+        items = _split_items(rnd)
+        for seed in range(3):
+            run(items, QB, ST, trial * 100 + seed, split=True)
+
+
+SPLIT_DROPS = dict(DROPS, **{
+    # slot 0 would read slot 1's O, m, l before they are final
+    "warps: split_ready": _drop("warp", "split_ready"),
+    # slot 1 would free O_1 for the next item while slot 0 still reads it
+    "warps: split_done": _drop("warp", "split_done"),
+})
+
+
+@pytest.mark.parametrize("name", list(SPLIT_DROPS))
+def test_split_model_detects_a_dropped_wait(name):
+    rnd = random.Random(31)
+    failures = 0
+    for trial in range(200):
+        items = _split_items(rnd)
+        try:
+            run(items, 2, 4, trial, drop=SPLIT_DROPS[name], split=True)
         except AssertionError:
             failures += 1
     assert failures > 0, name

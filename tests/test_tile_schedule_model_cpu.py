@@ -175,3 +175,39 @@ def test_snake_order_evens_out_causal_work(B, N, Hkv, g, kind):
     rr_totals = [sum(costs[i::grid]) for i in range(grid)]
     assert max(snake_totals) - min(snake_totals) <= max(costs) / 2
     assert max(snake_totals) < max(rr_totals)
+
+
+def fwd_split_items(B, N, Hkv, g, causal):
+    """The forward's split-mode items (small problems): one Q tile each, slot
+    t taking the key tiles t, t + 2, ...: (b, kvh, qt, [key tiles of slot 0],
+    [key tiles of slot 1])."""
+    T = BM // g
+    n_qt = -(-N // T)
+    n_bh = B * Hkv
+    out = []
+    for item in range(n_qt * n_bh):
+        qt = n_qt - 1 - item // n_bh
+        bh = item % n_bh
+        end = min(N, (qt + 1) * T) if causal else N
+        nkv = -(-end // NK_FWD)
+        n0, n1 = (nkv + 1) // 2, nkv // 2
+        out.append((bh // Hkv, bh % Hkv, qt, [2 * j for j in range(n0)], [2 * j + 1 for j in range(n1)]))
+    return out
+
+
+@pytest.mark.parametrize("B,N,Hkv,g", SHAPES)
+@pytest.mark.parametrize("causal", [True, False])
+def test_forward_split_mode_visits_exactly_the_needed_key_tiles(B, N, Hkv, g, causal):
+    T = BM // g
+    need = _tile_pairs_needed(N, T, NK_FWD, causal)
+    seen = {}
+    for b, kvh, qt, tiles0, tiles1 in fwd_split_items(B, N, Hkv, g, causal):
+        assert len(tiles0) >= len(tiles1) and not set(tiles0) & set(tiles1)
+        for kt in tiles0 + tiles1:
+            seen[(b, kvh, qt, kt)] = seen.get((b, kvh, qt, kt), 0) + 1
+            assert (qt, kt) in need, f"fully masked tile pair visited: q tile {qt}, k tile {kt}"
+            if _hidden(qt, kt, T, NK_FWD, N, causal):
+                assert fwd_masked(kt * NK_FWD, qt, T, N, causal), f"unflagged tile pair {qt}, {kt}"
+    for b, kvh in itertools.product(range(B), range(Hkv)):
+        for qt, kt in need:
+            assert seen.get((b, kvh, qt, kt)) == 1
