@@ -280,8 +280,11 @@ def launched_kernel(w, hook: int) -> str:
     if hook == 1:  # at dh 64 / 128 the hook brackets the dK/dV and the dQ kernels
         return f"sqa_bwd_tf32_kernel<{w.dh}>" if w.dh <= 32 else f"sqa_bwd_kernel<{w.dh}>+sqa_bwd_q_kernel<{w.dh}>"
     g = w.Hq // w.Hkv
-    rows = g <= 4 and (w.Hkv & (w.Hkv - 1)) == 0  # register-resident path
-    return f"sqa_decode_split_kernel<{w.dh},{g if rows else 0}>"
+    if g <= 4 and (w.Hkv & (w.Hkv - 1)) == 0 and w.Hkv <= 2048 // w.dh:  # register-resident path
+        return f"sqa_decode_split_kernel<{w.dh},{g}>"
+    if 5 <= g <= 16:  # tensor-core path
+        return f"sqa_decode_mma_kernel<{w.dh}>"
+    return f"sqa_decode_split_kernel<{w.dh},0>"
 
 
 def roofline_for(w, kernel_name, ms, peaks, peak_kind):
@@ -564,6 +567,8 @@ def run_ours(args, w):
             "gpu_launches": args.steps * (4 if w.backward else (2 if w.decode else 1)),
             "clocks": clk,
             "wall_s_timed_region": wall,
+            # the CUDA sources this run was built from (profiles/traffic.json entries are keyed to it)
+            "source_sha256": kernel_source_sha256(),
         }
     # The same kernels on the MHA / GQA / MQA head layouts of the same model.
     variants = compare_variants(args, w)

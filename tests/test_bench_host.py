@@ -88,3 +88,15 @@ def test_roofline_reports_the_stated_algorithmic_work():
     for rl in (bench.roofline_for(WORKLOADS[n], k, ms, peaks, "measured")
                for n, k in (("decode_sqatm", "sqa_decode_split_kernel"), ("sqatm_train_sqa", "sqa_fwd_kernel"))):
         assert set(rl) >= {"bound", "achieved", "peak", "unit", "frac", "traffic"}
+
+
+def test_launched_kernel_names_the_decoding_path_that_runs():
+    # the same selection rule as the library: register-resident (g <= 4, H_kv a
+    # power of two within one CTA step), tensor cores (5 <= g <= 16), else shared memory
+    from sparse_query_attention_sqa_b200.inputs import WORKLOADS
+
+    assert bench.launched_kernel(WORKLOADS["decode_sqatm"], 2) == "sqa_decode_split_kernel<16,2>"
+    assert bench.launched_kernel(WORKLOADS["decode_dh128"], 2) == "sqa_decode_split_kernel<128,2>"
+    assert bench.launched_kernel(WORKLOADS["decode_mqa"], 2) == "sqa_decode_mma_kernel<16>"
+    assert bench.launched_kernel(WORKLOADS["large_dh128"], 1) == "sqa_bwd_kernel<128>+sqa_bwd_q_kernel<128>"
+    assert bench.launched_kernel(WORKLOADS["sqatm_train_sqa"], 1) == "sqa_bwd_tf32_kernel<16>"
