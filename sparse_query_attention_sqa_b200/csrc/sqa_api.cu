@@ -259,6 +259,16 @@ sqa_status launch_decode(const void* q, const void* k, const void* v, const int*
       default: st = launch_decode_rows<DH, 4>(p, s, stream); break;
     }
     if (st != SQA_OK) return st;
+  } else if (sqa::mma_path(p.g) && aligned(q, 4)) {
+    p.span = sqa::decode_span(DH);
+    p.n_split = (s.N + p.span - 1) / p.span;
+    const int smem = static_cast<int>(sqa::mma_smem_bytes(DH));
+    if ((st = set_smem(sqa::sqa_decode_mma_kernel<DH>, smem)) != SQA_OK) return st;
+    const dim3 grid(static_cast<unsigned>(p.n_split * s.H_kv), static_cast<unsigned>(s.B));
+    if ((st = record_timing(2, 0, stream)) != SQA_OK) return st;
+    sqa::sqa_decode_mma_kernel<DH><<<grid, sqa::kMmaThreads, smem, stream>>>(p);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "sqa_decode mma split launch");
   } else {
     p.span = sqa::decode_span(DH);
     p.n_split = (s.N + p.span - 1) / p.span;

@@ -6,15 +6,16 @@
 // position), not the scores: reducing the query heads saves nothing here
 // (arXiv 2510.01817 abstract: the gains are in compute-bound settings; the
 // GQA summary, "The idea": the K/V head count sets the cache size).  So the
-// kernels are built to stream the cache from HBM once at full width, on the
-// CUDA cores: with g query heads per K/V head there are only 2 g dh
-// multiply-adds per cached position, far below what tensor cores are for.
+// kernels are built to stream the cache from HBM once at full width.  With g
+// query heads per K/V head there are 4 g dh flops per cached position (scores
+// and P V): for small groups the CUDA cores keep up with HBM; from about five
+// heads up they do not, and warp-level tensor-core MMAs take the products.
 //
 // Two launches, split-K over the cache:
 //   1. split:   one CTA per (range of positions, batch entry[, K/V head]),
 //               writing per query head the range's unnormalised output o with
 //               its running maximum m and sum l (log2 units) to the workspace.
-//               Two paths:
+//               Three paths:
 //               - register-resident (groups of at most 4 query heads, a
 //                 power-of-two K/V head count): the range's cache rows of all
 //                 K/V heads are one contiguous run; dh / 8 lanes share a row,
@@ -22,6 +23,9 @@
 //                 registers with several rows' loads in flight, and the slots
 //                 of each K/V head merge once at the end.  The number of
 //                 ranges makes about four waves of resident CTAs.
+//               - tensor cores (groups of 5 to 16 heads): one CTA of four
+//                 warps per (range, K/V head, batch entry), mma.sync on a
+//                 16-head by 16-key tile per warp step (see the kernel).
 //               - general (any group up to 128 heads): one CTA per (4 chunks
 //                 of positions, K/V head, batch entry); chunks (256 positions
 //                 at dh <= 32, 128 at dh = 64, 64 at dh = 128) are copied into
@@ -498,6 +502,246 @@ __device__ __forceinline__ void decode_split_rows(const DecodeParams& p) {
       }
     }
     p.part[((static_cast<size_t>(b) * Hkv + hk) * p.n_split + split) * REC + rem] = val;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Warp-level tensor-core split path for groups of 5 to 16 query heads (MQA-like
+// layouts).  There the g queries that share a cached row make the scores and
+// P V a dense contraction (16 x dh by dh x keys, then 16 x keys by keys x dh)
+// that the CUDA cores cannot finish while HBM delivers the row; one
+// mma.sync.m16n8k16 (bf16 in, fp32 out) computes a 16-head by 8-key block.
+// The g heads are the 16 rows of the A operand (rows past g are zero).
+//
+// One CTA of 4 warps per (range of positions, K/V head, batch entry); the
+// range streams through a ring of chunks in shared memory (16-byte cp.async
+// copies; 128 keys, or 64 at dh 128 so that two CTAs fit on an SM), each warp
+// taking a quarter of a chunk in 16-key steps:
+//   S = Q K^T (B fragments by ldmatrix from the K rows), online softmax on
+//   the accumulator fragments (row r = lane / 4 and r + 8; the four lanes of a
+//   row reduce with shuffles), P re-packed as the A fragment of P V (the
+//   accumulator layout of two 8-key blocks is the A layout of one 16-key
+//   step), O += P V (B fragments by ldmatrix.trans from the V rows).
+// At the end the four warps' (m, l, O) are merged in shared memory into the
+// range's partial record, in the general path's format.
+constexpr int kMmaThreads = 128, kMmaStages = 3;
+__host__ __device__ constexpr bool mma_path(int g) { return g >= 5 && g <= 16; }
+__host__ __device__ constexpr int mma_chunk(int dh) { return dh == 128 ? 64 : 128; }
+__host__ __device__ constexpr size_t mma_smem_bytes(int dh) {
+  return static_cast<size_t>(kMmaStages) * 2 * mma_chunk(dh) * dh * 2;  // the ring; the merge reuses it
+}
+// 16-byte piece j of cached row `row` in a chunk buffer: XOR-swizzled so that
+// the eight rows one ldmatrix phase reads (same piece, consecutive rows) fall
+// in eight different 16-byte bank groups.
+template <int DH>
+__device__ __forceinline__ int mma_piece(int row, int j) {
+  constexpr int P = DH / 8;  // pieces per row
+  if constexpr (P >= 8) {
+    return row * P + (j ^ (row & 7));
+  } else {
+    constexpr int SH = P == 4 ? 1 : 2;  // rows per 128 bytes: 2 or 4
+    return row * P + (j ^ ((row >> SH) & (P - 1)));
+  }
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* smem_row) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(dev::smem_u32(smem_row)));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const void* smem_row) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(dev::smem_u32(smem_row)));
+}
+// d (+)= a b, m16n8k16, bf16 operands, fp32 accumulators
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int DH>
+__global__ void __launch_bounds__(kMmaThreads) sqa_decode_mma_kernel(const DecodeParams p) {
+  constexpr int KS = DH / 16;   // 16-wide steps over dh (scores)
+  constexpr int NB = DH / 8;    // 8-wide output column blocks
+  constexpr int ROWB = DH * 2;  // bytes per cached row
+  constexpr int CH = mma_chunk(DH), SPW = CH / 64;  // keys per chunk; 16-key steps per warp
+  constexpr int CHUNK_BYTES = CH * ROWB;
+  const int split = blockIdx.x / p.Hkv, kvh = blockIdx.x % p.Hkv, b = blockIdx.y;
+  const int bk = b * p.Hkv + kvh, g = p.g;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int r = lane >> 2, c = lane & 3;  // fragment row (and row + 8) and column pair
+  const int len = decode_len(p, b);
+  const int r0 = split * p.span, r1 = min(len, r0 + p.span);
+  float* part = p.part + (static_cast<size_t>(bk) * p.n_split + split) * g * (DH + 2);
+  if (r1 <= r0) {  // range past this sequence's length: an empty partial
+    for (int i = tid; i < g * (DH + 2); i += kMmaThreads) part[i] = i % (DH + 2) == DH ? -INFINITY : 0.f;
+    return;
+  }
+  extern __shared__ __align__(128) uint8_t msm[];
+  const int n_chunks = (r1 - r0 + CH - 1) / CH;
+  const __nv_bfloat16* kg = p.k + (static_cast<size_t>(b) * p.N * p.Hkv + kvh) * DH;
+  const __nv_bfloat16* vg = p.v + (static_cast<size_t>(b) * p.N * p.Hkv + kvh) * DH;
+  const size_t pos_stride = static_cast<size_t>(p.Hkv) * DH;  // elements between cached positions
+  // chunk ci -> ring stage ci % kMmaStages: K rows at stage * 2 CHUNK_BYTES, V rows after them
+  auto load_chunk = [&](int ci) {
+    uint8_t* st = msm + (ci % kMmaStages) * 2 * CHUNK_BYTES;
+    const int base = r0 + ci * CH;
+    for (int i = tid; i < CH * (ROWB / 16); i += kMmaThreads) {
+      const int row = i / (ROWB / 16), j = i % (ROWB / 16);
+      const size_t pos = min(base + row, len - 1);  // rows past the length repeat the last (masked below)
+      const int at = mma_piece<DH>(row, j) * 16;
+      cp_async16(st + at, kg + pos * pos_stride + j * 8);
+      cp_async16(st + CHUNK_BYTES + at, vg + pos * pos_stride + j * 8);
+    }
+  };
+  for (int ci = 0; ci < kMmaStages - 1; ++ci) {
+    if (ci < n_chunks) load_chunk(ci);
+    cp_async_commit();
+  }
+  // A fragments of the queries, one per 16-wide dh step: rows r and r + 8 are
+  // heads of the group (zero past g).
+  uint32_t qa[KS][4];
+  {
+    const __nv_bfloat16* qh = p.q + (static_cast<size_t>(b) * p.Hq + kvh * g) * DH;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const int k0 = ks * 16 + 2 * c;
+      auto ld = [&](int row, int col) -> uint32_t {
+        return row < g ? *reinterpret_cast<const uint32_t*>(qh + row * DH + col) : 0u;
+      };
+      qa[ks][0] = ld(r, k0);
+      qa[ks][1] = ld(r + 8, k0);
+      qa[ks][2] = ld(r, k0 + 8);
+      qa[ks][3] = ld(r + 8, k0 + 8);
+    }
+  }
+  const float sl2 = p.scale_log2;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // rows r and r + 8
+  float o[NB][4];
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) o[nb][0] = o[nb][1] = o[nb][2] = o[nb][3] = 0.f;
+
+  for (int ci = 0; ci < n_chunks; ++ci) {
+    if (ci + kMmaStages - 1 < n_chunks) load_chunk(ci + kMmaStages - 1);
+    cp_async_commit();
+    cp_async_wait<kMmaStages - 1>();
+    __syncthreads();
+    const uint8_t* ks_base = msm + (ci % kMmaStages) * 2 * CHUNK_BYTES;
+    const uint8_t* vs_base = ks_base + CHUNK_BYTES;
+    const int chunk_pos = r0 + ci * CH;
+#pragma unroll
+    for (int step = 0; step < SPW; ++step) {
+      const int key0 = (warp * SPW + step) * 16;  // this step's first key in the chunk
+      // S for keys key0 .. key0 + 15: two 8-key blocks
+      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        uint32_t kb[4];
+        // lanes 0-7: keys key0 + 0..7 at dh 16 ks; 8-15: same keys at 16 ks + 8;
+        // 16-23 / 24-31: keys key0 + 8..15
+        const int krow = key0 + (lane & 7) + ((lane >> 4) << 3);
+        ldmatrix_x4(kb, ks_base + mma_piece<DH>(krow, 2 * ks + ((lane >> 3) & 1)) * 16);
+        mma16816(s0, qa[ks], kb[0], kb[1]);
+        mma16816(s1, qa[ks], kb[2], kb[3]);
+      }
+      // mask keys past the length; scale to log2 units
+      const int kp = chunk_pos + key0 + 2 * c;  // position of s0[0]
+      float x[8] = {s0[0], s0[1], s1[0], s1[1], s0[2], s0[3], s1[2], s1[3]};  // row r: 0-3, row r + 8: 4-7
+      const int kpos[4] = {kp, kp + 1, kp + 8, kp + 9};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = kpos[i & 3] < r1 ? x[i] * sl2 : -INFINITY;
+      float mx0 = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+      float mx1 = fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7]));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+      const float a0 = n0 == -INFINITY ? 1.f : dev::ex2(m0 - n0), a1 = n1 == -INFINITY ? 1.f : dev::ex2(m1 - n1);
+      m0 = n0;
+      m1 = n1;
+      const float b0 = n0 == -INFINITY ? 0.f : n0, b1 = n1 == -INFINITY ? 0.f : n1;
+      float pr[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) pr[i] = dev::ex2(x[i] - b0);
+#pragma unroll
+      for (int i = 4; i < 8; ++i) pr[i] = dev::ex2(x[i] - b1);
+      l0 = l0 * a0 + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
+      l1 = l1 * a1 + ((pr[4] + pr[5]) + (pr[6] + pr[7]));
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) {
+        o[nb][0] *= a0;
+        o[nb][1] *= a0;
+        o[nb][2] *= a1;
+        o[nb][3] *= a1;
+      }
+      // P as the A fragment of the 16-key step: k 0-7 from block 0, 8-15 from block 1
+      const uint32_t pa[4] = {dev::pack_bf16x2(pr[0], pr[1]), dev::pack_bf16x2(pr[4], pr[5]),
+                              dev::pack_bf16x2(pr[2], pr[3]), dev::pack_bf16x2(pr[6], pr[7])};
+#pragma unroll
+      for (int nb = 0; nb < NB; nb += 2) {
+        uint32_t vb[4];
+        // lanes 0-7: keys key0 + 0..7 at dh 8 nb; 8-15: keys key0 + 8..15 at 8 nb;
+        // 16-23 / 24-31: the same at dh 8 (nb + 1)
+        const int vrow = key0 + (lane & 7) + (((lane >> 3) & 1) << 3);
+        ldmatrix_x4_trans(vb, vs_base + mma_piece<DH>(vrow, nb + (lane >> 4)) * 16);
+        mma16816(o[nb], pa, vb[0], vb[1]);
+        mma16816(o[nb + 1], pa, vb[2], vb[3]);
+      }
+    }
+    __syncthreads();  // the stage is reloaded next
+  }
+  cp_async_wait<0>();
+  // Row sums over the row's four lanes.
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  // Merge the four warps: M = max of their m, each O and l scaled by 2^(m - M).
+  __syncthreads();
+  float* ms = reinterpret_cast<float*>(msm);  // [4 warps][16 rows]
+  float* ls = ms + 4 * 16;
+  float* os = ls + 4 * 16;                    // [4 warps][16 rows][DH]
+  if (c == 0) {
+    ms[warp * 16 + r] = m0;
+    ms[warp * 16 + r + 8] = m1;
+  }
+  __syncthreads();
+  float M0 = -INFINITY, M1 = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    M0 = fmaxf(M0, ms[w * 16 + r]);
+    M1 = fmaxf(M1, ms[w * 16 + r + 8]);
+  }
+  const float f0 = m0 == -INFINITY ? 0.f : dev::ex2(m0 - M0), f1 = m1 == -INFINITY ? 0.f : dev::ex2(m1 - M1);
+  if (c == 0) {
+    ls[warp * 16 + r] = l0 * f0;
+    ls[warp * 16 + r + 8] = l1 * f1;
+  }
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb) {
+    const int col = nb * 8 + 2 * c;
+    os[(warp * 16 + r) * DH + col] = o[nb][0] * f0;
+    os[(warp * 16 + r) * DH + col + 1] = o[nb][1] * f0;
+    os[(warp * 16 + r + 8) * DH + col] = o[nb][2] * f1;
+    os[(warp * 16 + r + 8) * DH + col + 1] = o[nb][3] * f1;
+  }
+  __syncthreads();
+  for (int i = tid; i < g * (DH + 2); i += kMmaThreads) {
+    const int h = i / (DH + 2), col = i % (DH + 2);
+    float v;
+    if (col < DH) {
+      v = os[h * DH + col] + os[(16 + h) * DH + col] + os[(32 + h) * DH + col] + os[(48 + h) * DH + col];
+    } else if (col == DH) {
+      v = fmaxf(fmaxf(ms[h], ms[16 + h]), fmaxf(ms[32 + h], ms[48 + h]));
+    } else {
+      v = ls[h] + ls[16 + h] + ls[32 + h] + ls[48 + h];
+    }
+    part[i] = v;
   }
 }
 

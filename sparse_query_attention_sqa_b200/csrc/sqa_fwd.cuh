@@ -26,6 +26,14 @@
 // on the current one; O_t sits at 256 + 128 t.  P_t (bf16 pairs) overwrites the
 // first 32 columns of its S buffer.
 //
+// With one S buffer per tile (dh 128) a tile's next S = Q K^T can only start
+// after its P V, so each tile alternates between softmax and MMAs.  The two
+// tiles' softmax warpgroups take turns for the exponentials (a token passed
+// through two mbarriers): while one warpgroup works on the special-function
+// unit, the other tile's P V and next S run on the tensor core.  Left to
+// themselves the two tiles fall into step, share the special-function unit and
+// then queue their MMAs together, and each unit idles while the other works.
+//
 // Online softmax (exact): each row keeps a reference maximum m (log2 units) and
 // l = sum 2^(s*scale*log2e - m).  m is raised only when a tile's maximum exceeds
 // it by more than 8, so P <= 256 and O is rescaled rarely; the final O / l and
@@ -74,8 +82,10 @@ struct FwdTraits {
   static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
   // q_full[QB] | q_empty[QB] | kv_full[S] | kv_empty[S] | s_full[2][2] | p_full[2][2] |
-  // o_done[2] | o_final[2] | o_free[2] | drain[2] | split_ready | split_done
-  static constexpr int N_BARS = 2 * QBUF + 2 * STAGES + 4 + 4 + 2 + 2 + 2 + 2 + 2;
+  // o_done[2] | o_final[2] | o_free[2] | drain[2] | split_ready | split_done | turn[2]
+  static constexpr int N_BARS = 2 * QBUF + 2 * STAGES + 4 + 4 + 2 + 2 + 2 + 2 + 2 + 2;
+  // The softmax warpgroups take turns for the exponentials (one S buffer per tile).
+  static constexpr bool TOKEN = NSBUF == 1;
   // split mode: slot 1's running maximum and sum per row, for slot 0's combine
   static constexpr int OFF_ML = OFF_BAR + N_BARS * 8 + 16;
   static constexpr int SMEM_USED = OFF_ML + 2 * BM * 4;
@@ -157,6 +167,8 @@ __global__ void __launch_bounds__(384, 1)
   auto drain = [&](int t) { return bar0 + 8u * (2 * QB + 2 * ST + 14 + t); };
   const uint32_t split_ready = bar0 + 8u * (2 * QB + 2 * ST + 16);  // slot 1's O, m, l are final
   const uint32_t split_done = bar0 + 8u * (2 * QB + 2 * ST + 17);   // slot 0 has read them
+  // turn(t): the softmax warpgroup of slot t finished the exponentials of a step
+  auto turn = [&](int t) { return bar0 + 8u * (2 * QB + 2 * ST + 18 + t); };
   float* sm_m = reinterpret_cast<float*>(smem + Tr::OFF_ML);
   float* sm_l = sm_m + BM;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Tr::OFF_BAR + Tr::N_BARS * 8);
@@ -184,6 +196,8 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(drain(1), 1);
     mbar_init(split_ready, 128);
     mbar_init(split_done, 128);
+    mbar_init(turn(0), 128);
+    mbar_init(turn(1), 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -368,10 +382,20 @@ __global__ void __launch_bounds__(384, 1)
     const float sl2 = p.scale_log2;
     int G = 0, nd = 0;
     int nc = 0;  // split mode: combines done (phases of split_ready / split_done)
+    // Token order within an item: slot 0's step j follows slot 1's step j - 1,
+    // slot 1's step j follows slot 0's step j, where the other slot has such a
+    // step.  (Across items there is no order: the next item's Q tile may wait
+    // for this item's last steps to release the Q buffer.)  Phases of turn(t)
+    // count slot t's steps over all items; G_other is the other slot's count
+    // before this item.
+    int G_other = 0;
     bool ok = true;
     for (int r = 0, item; ok && (item = fwd_item(r, p.n_items)) >= 0; ++r) {
       const FwdItem it = fwd_decode(p, item, NK);
       const int nkv_t = t ? it.nkv1 : it.nkv0;
+      const int nkv_o = t ? it.nkv0 : it.nkv1;
+      const int G_o = G_other;
+      G_other += nkv_o;
       if (nkv_t == 0) continue;
       const int qt = p.split ? it.qt0 : it.qt0 + t;
       const bool combine = p.split && it.nkv1 > 0;  // slot 1 holds part of this row's sums
@@ -442,6 +466,13 @@ __global__ void __launch_bounds__(384, 1)
         }
         l *= alpha;
         if (raise) m = mnew;
+        if constexpr (Tr::TOKEN) {
+          const int k_other = t ? j : j - 1;  // the other slot's step of this item that goes first
+          if (k_other >= 0 && k_other < nkv_o) {
+            ok = __all_sync(0xffffffffu, mbar_wait(turn(1 - t), (G_o + k_other) & 1, abort_flag, kSiteSoftmax));
+            if (!ok) break;
+          }
+        }
         // Masked scores are -inf, so their P is exactly 0 (the scale is positive).
         const float nref = m == -INFINITY ? 0.f : -m;
         float sum0[8], sum1[8];
@@ -493,6 +524,7 @@ __global__ void __launch_bounds__(384, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full(t, Gt % NSB));
+        if constexpr (Tr::TOKEN) mbar_arrive(turn(t));
       }
       if (!ok) break;
       ok = __all_sync(0xffffffffu, mbar_wait(o_final(t), nd & 1, abort_flag, kSiteEpilogue));

@@ -2,7 +2,8 @@
 cache) with the fp64 oracle, on seeded inputs; ragged cache lengths, group
 sizes 1-128, every head dim, K/V head counts that are and are not powers of
 two (the register-resident split path takes groups of at most four heads with a
-power-of-two K/V head count, the shared-memory path the rest), a one-entry
+power-of-two K/V head count, the tensor-core path groups of 5 to 16 heads, the
+shared-memory path the rest), a one-entry
 cache, the whole cache, an empty sequence, and the full-size decoding
 workloads."""
 import numpy as np
@@ -41,6 +42,12 @@ CASES = [
     ((2, 300, 16, 16, 128), [300, 17]),
     ((2, 500, 6, 3, 32), [500, 250]),
     ((1, 5000, 8, 2, 128), [4999]),
+    # groups of 5 to 16 heads: the tensor-core split path
+    ((2, 777, 10, 2, 64), [777, 300]),
+    ((3, 1500, 36, 3, 32), [1500, 1, 1025]),
+    ((2, 2049, 16, 1, 128), [2049, 64]),
+    ((1, 200, 7, 1, 16), None),
+    ((2, 130, 40, 4, 128), [1, 130]),
 ]
 
 
@@ -93,7 +100,7 @@ def test_workspace_contents_do_not_matter(cuda_lib):
     assert_lse_close("lse", lse.cpu().numpy(), ref_lse)
 
 
-@pytest.mark.parametrize("name", ["decode_sqatm", "decode_dh128"])
+@pytest.mark.parametrize("name", ["decode_sqatm", "decode_dh128", "decode_mqa"])
 def test_decode_workloads_full_size(cuda_lib, name):
     w = WORKLOADS[name]
     q, k, v = _inputs(w.B, w.N, w.Hq, w.Hkv, w.dh, seed=0, k_scale=w.k_scale, std=w.std)

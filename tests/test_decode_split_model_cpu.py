@@ -1,6 +1,7 @@
 """Python models of the decoding split paths' index arithmetic, run on the
-CPU against the fp64 oracle: the register-resident path (below) and the
-shared-memory path (at the end of the file, with the rule that picks a path).
+CPU against the fp64 oracle: the register-resident path (below), the
+shared-memory path (with the rule that picks a path) and the tensor-core path
+(at the end of the file, at the level of mma.sync and ldmatrix fragments).
 
 The model follows the CUDA kernel's work split step by step: the range of
 positions per CTA chosen from the SM count and the CTAs resident per SM, the
@@ -272,3 +273,248 @@ def test_path_selection(g, hkv, dh, rows_path_expected):
     # the register-resident path takes groups of at most 4 heads whose K/V head
     # count is a power of two no larger than the rows a CTA takes per step
     assert rows_path(g, hkv, dh) == rows_path_expected
+
+
+# ----------------------------------------------------------------------------- tensor-core path
+#
+# Fragment layouts of mma.sync.m16n8k16 (bf16 operands, fp32 accumulators) and
+# ldmatrix, as the PTX ISA defines them, for lane t with r = t // 4, c = t % 4:
+#   A (16 x 16, row-major):  a0 = A[r][2c:2c+2], a1 = A[r+8][2c:2c+2],
+#                            a2 = A[r][2c+8:2c+10], a3 = A[r+8][2c+8:2c+10]
+#   B (16 x 8, "col"):       b0 = B[2c:2c+2][r], b1 = B[2c+8:2c+10][r]
+#   C/D (16 x 8):            d0, d1 = D[r][2c], D[r][2c+1]; d2, d3 = D[r+8][2c], D[r+8][2c+1]
+#   ldmatrix .x4: lanes 8i..8i+7 give the row addresses of matrix i; lane t
+#   receives M_i[r][2c:2c+2] (.trans: M_i[2c][r], M_i[2c+1][r]).
+# The model holds registers as per-lane arrays and shared memory as 16-byte
+# pieces, and runs the kernel's index arithmetic through these definitions.
+
+MMA_STAGES = 3
+LANES = np.arange(32)
+FR, FC = LANES // 4, LANES % 4
+
+
+def mma_path(g):
+    return 5 <= g <= 16
+
+
+def mma_chunk(dh):
+    return 64 if dh == 128 else 128
+
+
+def mma_piece(dh, row, j):
+    p = dh // 8
+    if p >= 8:
+        return row * p + (j ^ (row & 7))
+    sh = 1 if p == 4 else 2
+    return row * p + (j ^ ((row >> sh) & (p - 1)))
+
+
+def ldmatrix_x4(pieces, addr, trans=False):
+    """pieces: [n][8] shared-memory pieces; addr[lane] = piece index.  Returns
+    regs[4][32][2]."""
+    regs = np.zeros((4, 32, 2))
+    for i in range(4):
+        m = pieces[addr[8 * i : 8 * i + 8]]  # 8 x 8, rows as addressed
+        if trans:
+            regs[i, :, 0] = m[2 * FC, FR]
+            regs[i, :, 1] = m[2 * FC + 1, FR]
+        else:
+            regs[i, :, 0] = m[FR, 2 * FC]
+            regs[i, :, 1] = m[FR, 2 * FC + 1]
+    return regs
+
+
+def mma16816(d, a, b0, b1):
+    """d[32][4] += A B, A from a[4][32][2], B from b0, b1 [32][2]."""
+    A = np.zeros((16, 16))
+    B = np.zeros((16, 8))
+    for h in range(2):
+        A[FR, 2 * FC + h] = a[0][:, h]
+        A[FR + 8, 2 * FC + h] = a[1][:, h]
+        A[FR, 2 * FC + 8 + h] = a[2][:, h]
+        A[FR + 8, 2 * FC + 8 + h] = a[3][:, h]
+        B[2 * FC + h, FR] = b0[:, h]
+        B[2 * FC + 8 + h, FR] = b1[:, h]
+    D = A @ B
+    d[:, 0] += D[FR, 2 * FC]
+    d[:, 1] += D[FR, 2 * FC + 1]
+    d[:, 2] += D[FR + 8, 2 * FC]
+    d[:, 3] += D[FR + 8, 2 * FC + 1]
+
+
+def shfl_xor(x, m):
+    return x[LANES ^ m]
+
+
+def model_mma(q, k, v, lens, scale):
+    B, Hq, dh = q.shape
+    N, Hkv = k.shape[1], k.shape[2]
+    g = Hq // Hkv
+    assert mma_path(g)
+    CH, P = mma_chunk(dh), dh // 8
+    SPW, KS, NB = CH // 64, dh // 16, dh // 8
+    span = 4 * decode_chunk(dh)  # the shared-memory path's span: the same workspace
+    n_split = -(-N // span)
+    part = np.full((B, Hkv, n_split, g, dh + 2), np.nan)
+    sl2 = scale * math.log2(math.e)
+    for b, kvh, split in itertools.product(range(B), range(Hkv), range(n_split)):
+        ln = N if lens is None else min(max(lens[b], 0), N)
+        r0, r1 = split * span, min(ln, split * span + span)
+        rec = part[b, kvh, split]
+        if r1 <= r0:
+            rec[:, :dh], rec[:, dh], rec[:, dh + 1] = 0.0, -np.inf, 0.0
+            continue
+        n_chunks = -(-(r1 - r0) // CH)
+        ring_k = np.full((MMA_STAGES, CH * P, 8), np.nan)
+        ring_v = np.full((MMA_STAGES, CH * P, 8), np.nan)
+
+        def load_chunk(ci):
+            st = ci % MMA_STAGES
+            for i in range(CH * P):
+                row, j = divmod(i, P)
+                pos = min(r0 + ci * CH + row, ln - 1)
+                at = mma_piece(dh, row, j)
+                ring_k[st, at] = k[b, pos, kvh, 8 * j : 8 * j + 8]
+                ring_v[st, at] = v[b, pos, kvh, 8 * j : 8 * j + 8]
+
+        qh = q[b, kvh * g : (kvh + 1) * g]
+        qa = np.zeros((KS, 4, 32, 2))
+        for ks in range(KS):
+            k0 = ks * 16 + 2 * FC
+            for slot, (rows, cols) in enumerate([(FR, k0), (FR + 8, k0), (FR, k0 + 8), (FR + 8, k0 + 8)]):
+                for h in range(2):
+                    qa[ks, slot, :, h] = np.where(rows < g, qh[np.minimum(rows, g - 1), cols + h], 0.0)
+        for ci in range(min(n_chunks, MMA_STAGES - 1)):
+            load_chunk(ci)
+        warps = []
+        for w in range(4):
+            warps.append(dict(m0=np.full(32, -np.inf), m1=np.full(32, -np.inf), l0=np.zeros(32), l1=np.zeros(32),
+                              o=np.zeros((NB, 32, 4))))
+        for ci in range(n_chunks):
+            if ci + MMA_STAGES - 1 < n_chunks:
+                load_chunk(ci + MMA_STAGES - 1)
+            kbuf, vbuf = ring_k[ci % MMA_STAGES], ring_v[ci % MMA_STAGES]
+            chunk_pos = r0 + ci * CH
+            for w, st in enumerate(warps):
+                for step in range(SPW):
+                    key0 = (w * SPW + step) * 16
+                    s0, s1 = np.zeros((32, 4)), np.zeros((32, 4))
+                    for ks in range(KS):
+                        krow = key0 + (LANES & 7) + ((LANES >> 4) << 3)
+                        kb = ldmatrix_x4(kbuf, mma_piece(dh, krow, 2 * ks + ((LANES >> 3) & 1)))
+                        mma16816(s0, qa[ks], kb[0], kb[1])
+                        mma16816(s1, qa[ks], kb[2], kb[3])
+                    kp = chunk_pos + key0 + 2 * FC
+                    x = np.stack([s0[:, 0], s0[:, 1], s1[:, 0], s1[:, 1], s0[:, 2], s0[:, 3], s1[:, 2], s1[:, 3]], 1)
+                    kpos = np.stack([kp, kp + 1, kp + 8, kp + 9], 1)
+                    valid = np.concatenate([kpos, kpos], 1) < r1
+                    x = np.where(valid, x * sl2, -np.inf)
+                    mx0, mx1 = x[:, :4].max(1), x[:, 4:].max(1)
+                    for sh in (1, 2):
+                        mx0 = np.maximum(mx0, shfl_xor(mx0, sh))
+                        mx1 = np.maximum(mx1, shfl_xor(mx1, sh))
+                    n0, n1 = np.maximum(st["m0"], mx0), np.maximum(st["m1"], mx1)
+                    with np.errstate(invalid="ignore"):
+                        a0 = np.where(n0 == -np.inf, 1.0, np.exp2(st["m0"] - n0))
+                        a1 = np.where(n1 == -np.inf, 1.0, np.exp2(st["m1"] - n1))
+                    st["m0"], st["m1"] = n0, n1
+                    b0, b1 = np.where(n0 == -np.inf, 0.0, n0), np.where(n1 == -np.inf, 0.0, n1)
+                    pr = np.concatenate([np.exp2(x[:, :4] - b0[:, None]), np.exp2(x[:, 4:] - b1[:, None])], 1)
+                    st["l0"] = st["l0"] * a0 + pr[:, :4].sum(1)
+                    st["l1"] = st["l1"] * a1 + pr[:, 4:].sum(1)
+                    st["o"][:, :, 0:2] *= a0[None, :, None]
+                    st["o"][:, :, 2:4] *= a1[None, :, None]
+                    pa = np.stack([pr[:, 0:2], pr[:, 4:6], pr[:, 2:4], pr[:, 6:8]])
+                    for nb in range(0, NB, 2):
+                        vrow = key0 + (LANES & 7) + (((LANES >> 3) & 1) << 3)
+                        vb = ldmatrix_x4(vbuf, mma_piece(dh, vrow, nb + (LANES >> 4)), trans=True)
+                        mma16816(st["o"][nb], pa, vb[0], vb[1])
+                        mma16816(st["o"][nb + 1], pa, vb[2], vb[3])
+        # merge the four warps into the record
+        ms = np.zeros((4, 16))
+        ls = np.zeros((4, 16))
+        os_ = np.full((4, 16, dh), np.nan)
+        for w, st in enumerate(warps):
+            for nm in ("l0", "l1"):
+                for sh in (1, 2):
+                    st[nm] = st[nm] + shfl_xor(st[nm], sh)
+            ms[w, FR], ms[w, FR + 8] = st["m0"], st["m1"]
+        M = ms.max(0)
+        for w, st in enumerate(warps):
+            with np.errstate(invalid="ignore"):
+                f0 = np.where(st["m0"] == -np.inf, 0.0, np.exp2(st["m0"] - M[FR]))
+                f1 = np.where(st["m1"] == -np.inf, 0.0, np.exp2(st["m1"] - M[FR + 8]))
+            ls[w, FR], ls[w, FR + 8] = st["l0"] * f0, st["l1"] * f1
+            for nb in range(NB):
+                col = nb * 8 + 2 * FC
+                os_[w, FR, col] = st["o"][nb][:, 0] * f0
+                os_[w, FR, col + 1] = st["o"][nb][:, 1] * f0
+                os_[w, FR + 8, col] = st["o"][nb][:, 2] * f1
+                os_[w, FR + 8, col + 1] = st["o"][nb][:, 3] * f1
+        rec[:, :dh] = os_.sum(0)[:g]
+        rec[:, dh] = M[:g]
+        rec[:, dh + 1] = ls.sum(0)[:g]
+    out, lse = np.zeros((B, Hq, dh)), np.zeros((B, Hq))
+    for b in range(B):
+        ln = N if lens is None else min(max(lens[b], 0), N)
+        n_used = -(-ln // span)
+        for hq in range(Hq):
+            kvh, hg = divmod(hq, g)
+            ps = part[b, kvh, :n_used, hg]
+            assert not np.isnan(ps).any()
+            if n_used == 0:
+                out[b, hq], lse[b, hq] = 0.0, -np.inf
+                continue
+            M = ps[:, dh].max()
+            w = np.exp2(ps[:, dh] - M)
+            Ls = (ps[:, dh + 1] * w).sum()
+            out[b, hq] = (ps[:, :dh] * w[:, None]).sum(0) / Ls
+            lse[b, hq] = (M + math.log2(Ls)) * math.log(2)
+    return out, lse
+
+
+MMA_CASES = [
+    ((2, 1100, 16, 1, 16), [1100, 257]),
+    ((2, 300, 5, 1, 32), [300, 1]),
+    ((1, 600, 24, 2, 64), [600]),
+    ((2, 280, 8, 1, 128), [280, 65]),
+    ((2, 200, 21, 3, 16), [0, 129]),
+]
+
+
+@pytest.mark.parametrize("shape,lens", MMA_CASES, ids=lambda c: "x".join(map(str, c)) if isinstance(c, tuple) else str(c))
+def test_tensor_core_split_model_matches_oracle(shape, lens):
+    B, N, Hq, Hkv, dh = shape
+    rng = np.random.default_rng(N * 7 + Hq)
+    q = rng.standard_normal((B, Hq, dh))
+    k = rng.standard_normal((B, N, Hkv, dh))
+    v = rng.standard_normal((B, N, Hkv, dh))
+    out, lse = model_mma(q, k, v, lens, 1 / math.sqrt(dh))
+    keep = [i for i in range(B) if lens is None or lens[i] > 0]
+    for i in set(range(B)) - set(keep):
+        assert np.all(out[i] == 0) and np.all(np.isneginf(lse[i]))
+    ref_out, ref_lse = oracle.sqa_decode(q[keep], k[keep], v[keep], None if lens is None else [lens[i] for i in keep])
+    np.testing.assert_allclose(out[keep], ref_out, rtol=0, atol=1e-10)
+    np.testing.assert_allclose(lse[keep], ref_lse, rtol=0, atol=1e-10)
+
+
+@pytest.mark.parametrize("dh", [16, 32, 64, 128])
+def test_tensor_core_path_swizzle_is_conflict_free(dh):
+    # every ldmatrix phase (8 consecutive rows, one 16-byte piece each) hits 8
+    # different 16-byte bank groups, and the swizzle permutes each row's pieces
+    p = dh // 8
+    for row in range(mma_chunk(dh)):
+        assert sorted(mma_piece(dh, row, j) for j in range(p)) == list(range(row * p, row * p + p))
+    for row0 in range(0, mma_chunk(dh), 8):
+        for j in range(p):
+            groups = {mma_piece(dh, row0 + i, j) % 8 for i in range(8)}
+            assert len(groups) == 8
+
+
+@pytest.mark.parametrize("g,hkv,dh,path", [(4, 4, 16, "rows"), (5, 1, 16, "mma"), (16, 1, 16, "mma"),
+                                           (8, 2, 128, "mma"), (17, 1, 64, "general"), (2, 3, 32, "general"),
+                                           (3, 32, 128, "general"), (128, 1, 16, "general")])
+def test_three_way_path_selection(g, hkv, dh, path):
+    # register-resident first, then tensor cores for 5-16 heads, else shared memory
+    got = "rows" if rows_path(g, hkv, dh) else ("mma" if mma_path(g) else "general")
+    assert got == path

@@ -25,6 +25,14 @@ two loaded.  The kernel's buffer configurations are run: QBUF 2 with 8 stages
 (dh <= 32), QBUF 2 with 4 stages (dh 64), each with two S buffers per tile,
 and QBUF 1 with 2 stages and one S buffer per tile (dh 128, 128-key tiles);
 QBUF 1 with 3 stages and two S buffers is kept as a further case.
+
+With one S buffer per tile the two tiles' softmax warpgroups also pass a token
+(mbarriers tok0 / tok1) around their exponentials, within each item: slot 0's
+step j after slot 1's step j - 1, slot 1's step j after slot 0's step j, where
+the other slot has such a step (an order across items deadlocks: the next
+item's Q load waits for the Q buffer this item's last steps hold).  A custom
+checker asserts that the two tiles' exponential phases never overlap within
+an item.
 """
 import random
 
@@ -93,6 +101,7 @@ def _roles(items, QB, ST, rnd, NSB=2, split=False):
     for s in range(ST):
         cnt[f"kv_full{s}"] = 1
         cnt[f"kv_empty{s}"] = 2
+    cnt["tok0"] = cnt["tok1"] = 32 * WARPS_PER_TILE
     for t in range(2):
         for buf in range(2):
             cnt[f"s_full{t}{buf}"] = 1
@@ -186,11 +195,15 @@ def _roles(items, QB, ST, rnd, NSB=2, split=False):
             g[0] = base + nkv
         return ops
 
+    token = NSB == 1
+
     def softmax_warp(t):
         ops, G, nd, G1, nd1, nc = [], 0, 0, 0, 0, 0
         S = f"S{t}"
-        for (n0, n1) in items:
-            nkv_t = n1 if t else n0
+        G_other = 0
+        for r, (n0, n1) in enumerate(items):
+            nkv_t, nkv_o = (n1, n0) if t else (n0, n1)
+            G_o, G_other = G_other, G_other + nkv_o
             combine = split and n1 > 0
             if nkv_t == 0:
                 continue
@@ -199,7 +212,14 @@ def _roles(items, QB, ST, rnd, NSB=2, split=False):
                 ops += [W(f"s_full{t}{step % NSB}", step // NSB), B(S, step % NSB, step, 1)]
                 if j > 0 and rnd.random() < 0.5:  # the running maximum rose: rescale O
                     ops += [W(f"o_done{t}", step - 1), B("O", t, ("rescale", step)), E("O", t, ("rescale",))]
+                if token:
+                    k_other = j if t else j - 1
+                    if 0 <= k_other < nkv_o:
+                        ops.append(W(f"tok{1 - t}", G_o + k_other))
+                ops += [B("X", t, ("exp", r)), E("X", t, ("exp", r))]
                 ops += [E(S, step % NSB, step, 1), A(f"p_full{t}{step % NSB}", 32)]
+                if token:
+                    ops.append(A(f"tok{t}", 32))
             ops.append(W(f"o_final{t}", nd))
             if combine and t == 1:
                 # hand m, l to slot 0; O_1 stays until slot 0 has read it
@@ -244,7 +264,26 @@ def run(items, QB, ST, seed, drop=None, NSB=2, split=False):
     roles, cnt = _roles(items, QB, ST, rnd, NSB, split)
     if drop is not None:
         roles = {r: [op for op in ops if not drop(r, op)] for r, ops in roles.items()}
-    sync_model.run(roles, cnt, STAGES, seed, custom={"O": _OCheck()}, skewed=seed % 2 == 1)
+    sync_model.run(roles, cnt, STAGES, seed, custom={"O": _OCheck(), "X": _ExpCheck(NSB == 1)},
+                   skewed=seed % 2 == 1)
+
+
+class _ExpCheck:
+    """With the token (one S buffer per tile), the two tiles' exponential
+    phases of one item never overlap."""
+
+    def __init__(self, exclusive):
+        self.exclusive = exclusive
+        self.active = {0: {}, 1: {}}  # slot -> item -> warps in their exponentials
+
+    def begin(self, slot, info):
+        item = info[1]
+        if self.exclusive:
+            assert self.active[1 - slot].get(item, 0) == 0, "both tiles in their exponentials at once"
+        self.active[slot][item] = self.active[slot].get(item, 0) + 1
+
+    def end(self, slot, info):
+        self.active[slot][info[1]] -= 1
 
 
 class _OCheck:
@@ -292,13 +331,15 @@ DROPS = {
     # an issuer would read K/V or Q before they landed
     "issuer: kv_full": _drop("issuer", "kv_full"),
     "issuer: q_full": _drop("issuer", "q_full"),
+    # with one S buffer per tile: both tiles would run their exponentials at once
+    "warps: tok": _drop("warp", "tok"),
 }
 
 
 # With one S buffer per tile (dh 128) the next S MMA of a tile comes after its
 # P V MMA in the issuer's order, so the warps' s_full wait also implies the
 # P V of the previous step completed: there the o_done wait is implied.
-IMPLIED = {("warps: o_done", 1)}
+IMPLIED = {("warps: o_done", 1), ("warps: tok", 2)}  # no token with two S buffers
 
 
 @pytest.mark.parametrize("name,NSB", [(n, b) for n in DROPS for b in (2, 1) if (n, b) not in IMPLIED])
@@ -333,7 +374,7 @@ def test_split_mode_has_no_deadlock_aliasing_or_hazard(QB, ST):
             run(items, QB, ST, trial * 100 + seed, split=True)
 
 
-SPLIT_DROPS = dict(DROPS, **{
+SPLIT_DROPS = dict({n: d for n, d in DROPS.items() if n != "warps: tok"}, **{  # split mode: dh <= 64, no token
     # slot 0 would read slot 1's O, m, l before they are final
     "warps: split_ready": _drop("warp", "split_ready"),
     # slot 1 would free O_1 for the next item while slot 0 still reads it
