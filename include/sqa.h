@@ -332,6 +332,20 @@ sqa_status sqa_decode(const void *q, const void *k_cache, const void *v_cache, c
 sqa_status sqa_selftest_exp2_poly(const float *x, float *y, int n, sqa_stream_t stream);
 
 /*
+ * Throughput probe of the special-function unit's exponential (ex2.approx,
+ * the instruction the softmax uses for 2^x), behind the exp2 roofline that the
+ * dh <= 32 kernels are measured against; the pages have no counterpart.
+ * Launches n_blocks blocks of 256 threads on `stream`; every thread runs 8
+ * independent chains of `iters` dependent exponentials (8 * iters per thread)
+ * and writes one float (the chains' sum, so nothing is optimised away) to
+ * out[block * 256 + thread].  out: device fp32 array of n_blocks * 256
+ * elements, owned by the caller.  The caller times the launch (events on the
+ * stream).  SQA_ERR_INVALID_ARG for a null `out`, n_blocks outside 1..65535 or
+ * iters outside 1..1048576, before any launch.
+ */
+sqa_status sqa_selftest_exp2_rate(float *out, int n_blocks, int iters, sqa_stream_t stream);
+
+/*
  * Self-test hook for the kernels' bounded waits, so that tests can exercise
  * the failure path without faulting or hanging a GPU; the pages have no
  * counterpart.  Launches one small kernel on `stream` whose thread waits on an

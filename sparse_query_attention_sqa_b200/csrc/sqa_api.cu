@@ -298,6 +298,19 @@ __global__ void exp2_poly_kernel(const float* x, float* y, int n) {
   }
 }
 
+// Exponential throughput: 8 independent chains of dependent ex2.approx per
+// thread, so the special-function unit, not latency, sets the pace.
+__global__ void __launch_bounds__(256) exp2_rate_kernel(float* out, int iters) {
+  float v[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) v[c] = -0.5f + 0.01f * c + 1e-6f * threadIdx.x;
+  for (int it = 0; it < iters; ++it) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) v[c] = sqa::dev::ex2(v[c]) - 1.5f;  // stays in [-1, 0.5]
+  }
+  out[blockIdx.x * 256 + threadIdx.x] = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+}
+
 // Self-test of the bounded waits: one thread waits on an mbarrier that nothing
 // ever arrives on, with the given limit, through the same slow path the
 // kernels use; it gives up, records `site` in the device status word and the
@@ -1118,6 +1131,17 @@ sqa_status sqa_selftest_exp2_poly(const float* x, float* y, int n, sqa_stream_t 
   exp2_poly_kernel<<<grid_for(pairs, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "sqa_selftest_exp2_poly launch");
+  return SQA_OK;
+}
+
+sqa_status sqa_selftest_exp2_rate(float* out, int n_blocks, int iters, sqa_stream_t stream) {
+  g_last_error.clear();
+  if (!out) return fail(SQA_ERR_INVALID_ARG, "null pointer");
+  if (n_blocks < 1 || n_blocks > 65535) return fail(SQA_ERR_INVALID_ARG, "n_blocks must be in [1, 65535]");
+  if (iters < 1 || iters > (1 << 20)) return fail(SQA_ERR_INVALID_ARG, "iters must be in [1, 1048576]");
+  exp2_rate_kernel<<<n_blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(out, iters);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "sqa_selftest_exp2_rate launch");
   return SQA_OK;
 }
 

@@ -329,6 +329,11 @@ __global__ void __launch_bounds__(384, 1)
       for (int hl = 0; ok && hl < NBUF && hl < nh; ++hl) ok = issue_half(hl);
       for (int i = 0; ok && i < it.nq; ++i) {
         const int G = gt + i;
+        // S^T / dP^T of the next tile's second half go ahead of this tile's dQ,
+        // so that the softmax warps find them computed when they get there.
+        // (The next-but-one tile's first half stays behind dQ: with two Q / dO
+        // stages its load waits for the stage this dQ releases.)
+        if (2 * i + 3 < nh && !(ok = issue_half(2 * i + 3))) break;
         // dQ of tile G once both warpgroups wrote their columns of dS, into the
         // dQ buffer the epilogue of tile G - 2 has emptied.
         if (!mbar_wait_warp(dsq_ready(0), G & 1, abort_flag, kSiteMma) ||
@@ -342,7 +347,6 @@ __global__ void __launch_bounds__(384, 1)
           mma_ss_w(tmem + Tr::tm_dq(G), dsb + 128 * ks, dkmn0 + koff + ((ks * 16 * ROWB) >> 4), idesc_q, ks > 0);
         mma_commit_w(dq_full(G & 1));
         mma_commit_w(qd_empty(G % QS));
-        if (2 * i + 3 < nh && !(ok = issue_half(2 * i + 3))) break;
         if (2 * i + 4 < nh && !(ok = issue_half(2 * i + 4))) break;
       }
       if (!ok) break;

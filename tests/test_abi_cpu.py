@@ -256,3 +256,14 @@ def test_block_rejects_bad_arguments_before_launch(lib):
     assert st == sqa.SQA_ERR_INVALID_ARG and b"rope_base" in b.sqa_last_error()
     st = b.sqa_block_bwd(p, p, ctypes.byref(w), p, need, p, None, s, 1, 0.0, 10000.0, None)
     assert st == sqa.SQA_ERR_INVALID_ARG
+
+
+def test_exp2_rate_probe_rejects_bad_arguments_before_launch(lib):
+    f = lib.sqa_selftest_exp2_rate
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    assert f(None, 1, 1, None) == 1
+    assert f(0x100, 0, 1, None) == 1
+    assert f(0x100, 65536, 1, None) == 1
+    assert f(0x100, 1, 0, None) == 1
+    assert f(0x100, 1, (1 << 20) + 1, None) == 1

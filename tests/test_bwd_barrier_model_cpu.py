@@ -115,14 +115,14 @@ def _roles(nqs, QS):
             issuer_a += half(hl)
         for i in range(nq):
             G = gt + i
+            if 2 * i + 3 < nh:  # the next tile's second half goes ahead of this tile's dQ
+                issuer_a += half(2 * i + 3)
             issuer_a += [W(f"dsq_ready{w}", G) for w in range(NWG)]
             issuer_a.append(B("dsbuf", G & 1, G, 1))
             if G >= 2:
                 issuer_a.append(W(f"dq_empty{G & 1}", (G >> 1) - 1))
             issuer_a += [B("dqtm", G & 1, G, 0), E("dsbuf", G & 1, G, 1), E("dqtm", G & 1, G, 0)]
             issuer_a += [A(f"dq_full{G & 1}"), A(f"qd_empty{G % QS}")]
-            if 2 * i + 3 < nh:
-                issuer_a += half(2 * i + 3)
             if 2 * i + 4 < nh:
                 issuer_a += half(2 * i + 4)
         issuer_a += [E("kv", kb, r, 1), A(f"kv_empty{kb}")]

@@ -1,7 +1,9 @@
 """The polynomial exponential the forward uses for part of its softmax
 exponentials (sqa_selftest_exp2_poly runs it elementwise), against 2^x in fp64
 and against CUDA's own exp2f.  The forward's parity tests cover it inside the
-kernel too; this pins its error bound directly."""
+kernel too; this pins its error bound directly.  Also the throughput probe of
+the special-function unit's exponential (sqa_selftest_exp2_rate), which stands
+behind the derived exp2 roofline of the dh <= 32 kernels."""
 import ctypes
 
 import numpy as np
@@ -56,3 +58,31 @@ def test_odd_length_and_tail(cuda_lib):
     y = _run(cuda_lib, x)
     assert not torch.isnan(y).any()
     assert abs(float(y[-1]) / 8.0 - 1.0) <= 7.6e-5
+
+
+def test_exponential_rate_is_near_the_derived_unit_count(cuda_lib):
+    # 16 exponentials per clock per SM; the probe's rate divided by SMs x the
+    # SM clock it ran at must come out near 16 (the clock is read from the
+    # device's max clock, so a throttled GPU reads low: the bound is loose)
+    lib = cuda_lib.load_library()
+    f = lib.sqa_selftest_exp2_rate
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    props = torch.cuda.get_device_properties(0)
+    sms = props.multi_processor_count
+    blocks, iters = sms * 8, 2048
+    out = torch.empty(blocks * 256, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for _ in range(2):
+        assert f(out.data_ptr(), blocks, iters, stream) == 0, lib.sqa_last_error()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(5):
+        f(out.data_ptr(), blocks, iters, stream)
+    b.record()
+    torch.cuda.synchronize()
+    rate = 5 * blocks * 256 * 8 * iters / (a.elapsed_time(b) * 1e-3)
+    clock_hz = props.clock_rate * 1e3 if hasattr(props, "clock_rate") else 1.965e9
+    per_clk = rate / sms / clock_hz
+    assert torch.isfinite(out).all()
+    assert 8.0 <= per_clk <= 16.5, per_clk
