@@ -20,18 +20,21 @@
 //    over keys and runs in bf16 (dS as bf16 in shared memory, K as loaded).
 //    S^T = K Q^T and dP^T = V dO^T run in bf16 (exact products).
 //
-//  * The 128-row Q tile is split into two 64-column halves, processed one after
-//    the other by both warpgroups (32 columns each).  Halves rotate through
-//    three TMEM buffers: while the warpgroups work on one, the dV / dK MMAs of
-//    the previous one run and S^T / dP^T of the next one are ready.
+//  * The 128-row Q tile is split into two 64-column halves; warpgroup w takes
+//    half w of every tile, all 64 columns, in four 16-column chunks whose
+//    TMEM loads run one chunk ahead of the arithmetic.  (Splitting each half's
+//    columns between the warpgroups instead pays every hand-off twice per half
+//    and keeps both warpgroups in the same phase.)  Halves rotate through
+//    three TMEM buffers: while the warpgroups work on two of them, the dV / dK
+//    MMAs of the previous half run and S^T / dP^T of the next are ready.
 //
 //  * Three MMA-issuing threads, each in its own warp: A issues S^T / dP^T and
 //    dQ, DV issues the dV MMAs, DK the dK MMAs.  dS has two shared-memory
 //    buffers, so the softmax warps never wait for the dQ of the previous tile.
 //
 // Roles (384 threads):
-//   warps 0-7   P^T / dS^T (warpgroup w: columns 32 w .. 32 w + 31 of each half),
-//               the dQ epilogue (fp32 atomics) and the dK / dV epilogue
+//   warps 0-7   P^T / dS^T (warpgroup w: half w of each Q tile), the dQ
+//               epilogue (fp32 atomics) and the dK / dV epilogue
 //   warp 8      TMA producer (K, V once; Q, dO, their fp32 images, lse2, D per Q tile)
 //   warp 9      TMEM allocator and MMA issuer A; warp 10 issuer DV; warp 11 issuer DK
 // TMEM: buffer x (0..2): S^T at 128 x, dP^T at 128 x + 64 (64 columns each);
@@ -214,7 +217,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int x = 0; x < NBUF; ++x) {
       mbar_init(s_full(x), 1);
-      mbar_init(ds_ready(x), 256);  // both warpgroups
+      mbar_init(ds_ready(x), 128);  // the warpgroup that owns the half
       mbar_init(kvmma_done(x), 2);  // DV and DK
       mbar_init(drain(x), 1);
     }
@@ -445,30 +448,28 @@ __global__ void __launch_bounds__(384, 1)
           ok = __all_sync(0xffffffffu, mbar_wait(dq_full(G & 1), ((G >> 1) - 1) & 1, abort_flag, kSiteSoftmax));
           if (!ok) break;
         }
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          // Both warpgroups work on half hh of the tile: this one on its 32
-          // query columns col0 .. col0 + 31.
-          const int H = 2 * G + hh, x = H % NBUF;
-          const int col0 = 64 * hh + 32 * w;
+        {
+          // This warpgroup's half of the tile: query columns col0 .. col0 + 63.
+          const int H = 2 * G + w, x = H % NBUF;
+          const int col0 = 64 * w;
           ok = __all_sync(0xffffffffu, mbar_wait(s_full(x), (H / NBUF) & 1, abort_flag, kSiteSoftmax));
           if (!ok) break;
           tc_fence_after();
           const float* nl2 = reinterpret_cast<const float*>(smem + Tr::OFF_STAT + s * 1024) + col0;
-          const uint32_t tS = lane_addr + Tr::tm_st(x) + 32 * w, tP = lane_addr + Tr::tm_dpt(x) + 32 * w;
-          // Two chunks of 16 columns: the second one's TMEM load is in flight
-          // while the first one is computed.
+          const uint32_t tS = lane_addr + Tr::tm_st(x), tP = lane_addr + Tr::tm_dpt(x);
+          // Four chunks of 16 columns; the next chunk's TMEM load is in flight
+          // while one chunk is computed.
           uint32_t ca[32], cb[32];  // [0,16): S^T, [16,32): dP^T
           tmem_ld16x2(tS, tP, ca);
-          tmem_ld16x2_nowait(tS + 16, tP + 16, cb);
 #pragma unroll
-          for (int c16 = 0; c16 < 2; ++c16) {
-            if (c16 == 1) tmem_wait_ld32(cb);
+          for (int c16 = 0; c16 < 4; ++c16) {
+            uint32_t(&cur)[32] = (c16 & 1) ? cb : ca;
+            uint32_t(&nxt)[32] = (c16 & 1) ? ca : cb;
+            if (c16 + 1 < 4) tmem_ld16x2_nowait(tS + 16 * (c16 + 1), tP + 16 * (c16 + 1), nxt);
             // The mask test runs on every tile (lim makes it a no-op off the
             // diagonal): cheaper than branching between two versions.
             uint32_t pt[16], dst[16], dsb[8];
-            bwd_p_ds16(c16 ? cb : ca, nl2 + 16 * c16, nl2 + 128 + 16 * c16, rtok + col0 + 16 * c16, lim, sl2, pt,
-                             dst, dsb);
+            bwd_p_ds16(cur, nl2 + 16 * c16, nl2 + 128 + 16 * c16, rtok + col0 + 16 * c16, lim, sl2, pt, dst, dsb);
             tmem_st16x2(tS + 16 * c16, tP + 16 * c16, pt, dst);
             // dS[q][key] for q = col0 + 16 c16 .. + 15 into the MN-major 128B-swizzled
             // tile: panel q / 64, key row kk (128 bytes), 16-byte chunk (q % 64) / 8.
@@ -479,8 +480,8 @@ __global__ void __launch_bounds__(384, 1)
               *reinterpret_cast<uint4*>(ds_smem + panel * 16384 + kk * 128 + ((chunk ^ (kk & 7)) << 4)) =
                   make_uint4(dsb[4 * ch], dsb[4 * ch + 1], dsb[4 * ch + 2], dsb[4 * ch + 3]);
             }
+            if (c16 + 1 < 4) tmem_wait_ld32(nxt);
           }
-          if (!ok) break;
           tmem_wait_st();
           fence_async_smem();
           tc_fence_before();

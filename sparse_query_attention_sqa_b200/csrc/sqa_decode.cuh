@@ -516,12 +516,15 @@ __device__ __forceinline__ void decode_split_rows(const DecodeParams& p) {
 // One CTA of 4 warps per (range of positions, K/V head, batch entry); the
 // range streams through a ring of chunks in shared memory (16-byte cp.async
 // copies; 128 keys, or 64 at dh 128 so that two CTAs fit on an SM), each warp
-// taking a quarter of a chunk in 16-key steps:
+// taking a quarter of a chunk (32 keys, 16 at dh 128) per step:
 //   S = Q K^T (B fragments by ldmatrix from the K rows), online softmax on
 //   the accumulator fragments (row r = lane / 4 and r + 8; the four lanes of a
-//   row reduce with shuffles), P re-packed as the A fragment of P V (the
-//   accumulator layout of two 8-key blocks is the A layout of one 16-key
-//   step), O += P V (B fragments by ldmatrix.trans from the V rows).
+//   row reduce with shuffles; the reference maximum is raised only when a
+//   step's maximum exceeds it by more than 8, so O is rarely rescaled; keys
+//   are masked only in the chunk where the range ends), P re-packed as the A
+//   fragments of P V (the accumulator layout of two 8-key blocks is the A
+//   layout of one 16-key step), O += P V (B fragments by ldmatrix.trans from
+//   the V rows).
 // At the end the four warps' (m, l, O) are merged in shared memory into the
 // range's partial record, in the general path's format.
 constexpr int kMmaThreads = 128, kMmaStages = 3;
@@ -567,9 +570,13 @@ template <int DH>
 __global__ void __launch_bounds__(kMmaThreads) sqa_decode_mma_kernel(const DecodeParams p) {
   constexpr int KS = DH / 16;   // 16-wide steps over dh (scores)
   constexpr int NB = DH / 8;    // 8-wide output column blocks
-  constexpr int ROWB = DH * 2;  // bytes per cached row
-  constexpr int CH = mma_chunk(DH), SPW = CH / 64;  // keys per chunk; 16-key steps per warp
-  constexpr int CHUNK_BYTES = CH * ROWB;
+  constexpr int P = DH / 8;     // 16-byte pieces per cached row
+  constexpr int CH = mma_chunk(DH);
+  constexpr int KW = CH / 4;    // keys per warp per chunk: 32, or 16 at dh 128
+  constexpr int NKB = KW / 8;   // 8-key blocks of a warp's scores
+  constexpr int CHUNK_BYTES = CH * DH * 2;
+  constexpr int PIECES = CH * P / kMmaThreads;  // pieces of K (and of V) each thread copies per chunk
+  static_assert(CH * P % kMmaThreads == 0 && NKB % 2 == 0, "chunk shape");
   const int split = blockIdx.x / p.Hkv, kvh = blockIdx.x % p.Hkv, b = blockIdx.y;
   const int bk = b * p.Hkv + kvh, g = p.g;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -583,19 +590,39 @@ __global__ void __launch_bounds__(kMmaThreads) sqa_decode_mma_kernel(const Decod
   }
   extern __shared__ __align__(128) uint8_t msm[];
   const int n_chunks = (r1 - r0 + CH - 1) / CH;
+  const size_t pos_stride = static_cast<size_t>(p.Hkv) * DH;  // elements between cached positions
   const __nv_bfloat16* kg = p.k + (static_cast<size_t>(b) * p.N * p.Hkv + kvh) * DH;
   const __nv_bfloat16* vg = p.v + (static_cast<size_t>(b) * p.N * p.Hkv + kvh) * DH;
-  const size_t pos_stride = static_cast<size_t>(p.Hkv) * DH;  // elements between cached positions
+  // This thread's pieces (the same in every chunk): piece i = tid + k * threads
+  // is row i / P, 16-byte piece i % P; its place in a chunk buffer and its
+  // offset from the chunk's first cached row.
+  uint32_t poff[PIECES];
+  size_t goff[PIECES];
+#pragma unroll
+  for (int k = 0; k < PIECES; ++k) {
+    const int i = tid + k * kMmaThreads, row = i / P, j = i % P;
+    poff[k] = mma_piece<DH>(row, j) * 16;
+    goff[k] = row * pos_stride + j * 8;
+  }
   // chunk ci -> ring stage ci % kMmaStages: K rows at stage * 2 CHUNK_BYTES, V rows after them
   auto load_chunk = [&](int ci) {
     uint8_t* st = msm + (ci % kMmaStages) * 2 * CHUNK_BYTES;
     const int base = r0 + ci * CH;
-    for (int i = tid; i < CH * (ROWB / 16); i += kMmaThreads) {
-      const int row = i / (ROWB / 16), j = i % (ROWB / 16);
-      const size_t pos = min(base + row, len - 1);  // rows past the length repeat the last (masked below)
-      const int at = mma_piece<DH>(row, j) * 16;
-      cp_async16(st + at, kg + pos * pos_stride + j * 8);
-      cp_async16(st + CHUNK_BYTES + at, vg + pos * pos_stride + j * 8);
+    if (base + CH <= len) {
+#pragma unroll
+      for (int k = 0; k < PIECES; ++k) {
+        const size_t go = base * pos_stride + goff[k];
+        cp_async16(st + poff[k], kg + go);
+        cp_async16(st + CHUNK_BYTES + poff[k], vg + go);
+      }
+    } else {  // the sequence ends in this chunk: rows past it repeat the last one (masked below)
+#pragma unroll
+      for (int k = 0; k < PIECES; ++k) {
+        const int i = tid + k * kMmaThreads, row = i / P, j = i % P;
+        const size_t go = static_cast<size_t>(min(base + row, len - 1)) * pos_stride + j * 8;
+        cp_async16(st + poff[k], kg + go);
+        cp_async16(st + CHUNK_BYTES + poff[k], vg + go);
+      }
     }
   };
   for (int ci = 0; ci < kMmaStages - 1; ++ci) {
@@ -620,7 +647,10 @@ __global__ void __launch_bounds__(kMmaThreads) sqa_decode_mma_kernel(const Decod
     }
   }
   const float sl2 = p.scale_log2;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // rows r and r + 8
+  // Running reference maxima m (log2 units, rows r and r + 8), raised only when
+  // a step's maximum exceeds them by more than 8 (P <= 256), and per-lane
+  // partial sums l of 2^(s - m) over this lane's columns.
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   float o[NB][4];
 #pragma unroll
   for (int nb = 0; nb < NB; ++nb) o[nb][0] = o[nb][1] = o[nb][2] = o[nb][3] = 0.f;
@@ -633,45 +663,52 @@ __global__ void __launch_bounds__(kMmaThreads) sqa_decode_mma_kernel(const Decod
     const uint8_t* ks_base = msm + (ci % kMmaStages) * 2 * CHUNK_BYTES;
     const uint8_t* vs_base = ks_base + CHUNK_BYTES;
     const int chunk_pos = r0 + ci * CH;
+    const int key0 = warp * KW;  // this warp's first key in the chunk
+    // S for the warp's KW keys: NKB blocks of 8
+    float s[NKB][4];
 #pragma unroll
-    for (int step = 0; step < SPW; ++step) {
-      const int key0 = (warp * SPW + step) * 16;  // this step's first key in the chunk
-      // S for keys key0 .. key0 + 15: two 8-key blocks
-      float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int nb = 0; nb < NKB; ++nb) s[nb][0] = s[nb][1] = s[nb][2] = s[nb][3] = 0.f;
 #pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
+    for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+      for (int h = 0; h < NKB / 2; ++h) {
         uint32_t kb[4];
-        // lanes 0-7: keys key0 + 0..7 at dh 16 ks; 8-15: same keys at 16 ks + 8;
-        // 16-23 / 24-31: keys key0 + 8..15
-        const int krow = key0 + (lane & 7) + ((lane >> 4) << 3);
+        // lanes 0-7: keys 16 h + 0..7 at dh 16 ks; 8-15: same keys at 16 ks + 8;
+        // 16-23 / 24-31: keys 16 h + 8..15
+        const int krow = key0 + 16 * h + (lane & 7) + ((lane >> 4) << 3);
         ldmatrix_x4(kb, ks_base + mma_piece<DH>(krow, 2 * ks + ((lane >> 3) & 1)) * 16);
-        mma16816(s0, qa[ks], kb[0], kb[1]);
-        mma16816(s1, qa[ks], kb[2], kb[3]);
+        mma16816(s[2 * h], qa[ks], kb[0], kb[1]);
+        mma16816(s[2 * h + 1], qa[ks], kb[2], kb[3]);
       }
-      // mask keys past the length; scale to log2 units
-      const int kp = chunk_pos + key0 + 2 * c;  // position of s0[0]
-      float x[8] = {s0[0], s0[1], s1[0], s1[1], s0[2], s0[3], s1[2], s1[3]};  // row r: 0-3, row r + 8: 4-7
-      const int kpos[4] = {kp, kp + 1, kp + 8, kp + 9};
+    }
+    if (chunk_pos + CH > r1) {  // the range ends in this chunk: keys past it get -inf
 #pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] = kpos[i & 3] < r1 ? x[i] * sl2 : -INFINITY;
-      float mx0 = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-      float mx1 = fmaxf(fmaxf(x[4], x[5]), fmaxf(x[6], x[7]));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-      const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-      const float a0 = n0 == -INFINITY ? 1.f : dev::ex2(m0 - n0), a1 = n1 == -INFINITY ? 1.f : dev::ex2(m1 - n1);
-      m0 = n0;
-      m1 = n1;
-      const float b0 = n0 == -INFINITY ? 0.f : n0, b1 = n1 == -INFINITY ? 0.f : n1;
-      float pr[8];
+      for (int nb = 0; nb < NKB; ++nb) {
+        const int kp = chunk_pos + key0 + 8 * nb + 2 * c;  // key of s[nb][0] and s[nb][2]
+        if (kp >= r1) s[nb][0] = s[nb][2] = -INFINITY;
+        if (kp + 1 >= r1) s[nb][1] = s[nb][3] = -INFINITY;
+      }
+    }
+    // Row maxima of the raw scores (the scale is positive), over the row's four lanes.
+    float mx0 = fmaxf(s[0][0], s[0][1]), mx1 = fmaxf(s[0][2], s[0][3]);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) pr[i] = dev::ex2(x[i] - b0);
-#pragma unroll
-      for (int i = 4; i < 8; ++i) pr[i] = dev::ex2(x[i] - b1);
-      l0 = l0 * a0 + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
-      l1 = l1 * a1 + ((pr[4] + pr[5]) + (pr[6] + pr[7]));
+    for (int nb = 1; nb < NKB; ++nb) {
+      mx0 = dev::fmax3(mx0, s[nb][0], s[nb][1]);
+      mx1 = dev::fmax3(mx1, s[nb][2], s[nb][3]);
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    const float t0 = mx0 * sl2, t1 = mx1 * sl2;
+    const bool up0 = t0 > m0 + 8.f, up1 = t1 > m1 + 8.f;
+    if (__any_sync(0xffffffffu, up0 || up1)) {
+      const float a0 = (up0 && m0 != -INFINITY) ? dev::ex2(m0 - t0) : 1.f;
+      const float a1 = (up1 && m1 != -INFINITY) ? dev::ex2(m1 - t1) : 1.f;
+      if (up0) m0 = t0;
+      if (up1) m1 = t1;
+      l0 *= a0;
+      l1 *= a1;
 #pragma unroll
       for (int nb = 0; nb < NB; ++nb) {
         o[nb][0] *= a0;
@@ -679,18 +716,32 @@ __global__ void __launch_bounds__(kMmaThreads) sqa_decode_mma_kernel(const Decod
         o[nb][2] *= a1;
         o[nb][3] *= a1;
       }
-      // P as the A fragment of the 16-key step: k 0-7 from block 0, 8-15 from block 1
-      const uint32_t pa[4] = {dev::pack_bf16x2(pr[0], pr[1]), dev::pack_bf16x2(pr[4], pr[5]),
-                              dev::pack_bf16x2(pr[2], pr[3]), dev::pack_bf16x2(pr[6], pr[7])};
+    }
+    // P = 2^(s sl2 - m); rows with no key seen yet (m = -inf) have only -inf scores.
+    const float nm0 = m0 == -INFINITY ? 0.f : -m0, nm1 = m1 == -INFINITY ? 0.f : -m1;
+    uint32_t pa[NKB / 2][4];
+#pragma unroll
+    for (int nb = 0; nb < NKB; ++nb) {
+      const float p0 = dev::ex2(fmaf(s[nb][0], sl2, nm0)), p1 = dev::ex2(fmaf(s[nb][1], sl2, nm0));
+      const float p2 = dev::ex2(fmaf(s[nb][2], sl2, nm1)), p3 = dev::ex2(fmaf(s[nb][3], sl2, nm1));
+      l0 += p0 + p1;
+      l1 += p2 + p3;
+      // the accumulator layout of 8-key blocks 2 h and 2 h + 1 is the A layout
+      // of 16-key step h: keys 0-7 in registers 0 / 1, keys 8-15 in 2 / 3
+      pa[nb >> 1][(nb & 1) * 2 + 0] = dev::pack_bf16x2(p0, p1);
+      pa[nb >> 1][(nb & 1) * 2 + 1] = dev::pack_bf16x2(p2, p3);
+    }
+#pragma unroll
+    for (int h = 0; h < NKB / 2; ++h) {
 #pragma unroll
       for (int nb = 0; nb < NB; nb += 2) {
         uint32_t vb[4];
-        // lanes 0-7: keys key0 + 0..7 at dh 8 nb; 8-15: keys key0 + 8..15 at 8 nb;
+        // lanes 0-7: keys 16 h + 0..7 at dh 8 nb; 8-15: keys 16 h + 8..15 at 8 nb;
         // 16-23 / 24-31: the same at dh 8 (nb + 1)
-        const int vrow = key0 + (lane & 7) + (((lane >> 3) & 1) << 3);
+        const int vrow = key0 + 16 * h + (lane & 7) + (((lane >> 3) & 1) << 3);
         ldmatrix_x4_trans(vb, vs_base + mma_piece<DH>(vrow, nb + (lane >> 4)) * 16);
-        mma16816(o[nb], pa, vb[0], vb[1]);
-        mma16816(o[nb + 1], pa, vb[2], vb[3]);
+        mma16816(o[nb], pa[h], vb[0], vb[1]);
+        mma16816(o[nb + 1], pa[h], vb[2], vb[3]);
       }
     }
     __syncthreads();  // the stage is reloaded next
@@ -701,7 +752,7 @@ __global__ void __launch_bounds__(kMmaThreads) sqa_decode_mma_kernel(const Decod
   l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
   l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  // Merge the four warps: M = max of their m, each O and l scaled by 2^(m - M).
+  // Merge the four warps: M = max of their references m, each O and l scaled by 2^(m - M).
   __syncthreads();
   float* ms = reinterpret_cast<float*>(msm);  // [4 warps][16 rows]
   float* ls = ms + 4 * 16;

@@ -5,7 +5,7 @@ Each role of the kernel is a list of what it does, in the kernel's order: the
 mbarrier waits and arrives, and the windows in which it uses a buffer.  The
 roles are the TMA producer, issuer A (S^T / dP^T halves into three TMEM
 buffers, then dQ), the DV and DK issuers, and the eight softmax warps (two
-warpgroups).  Every barrier has the kernel's arrival count; a use window of an
+warpgroups; warpgroup w takes half w of every Q tile).  Every barrier has the kernel's arrival count; a use window of an
 asynchronous copy or MMA ends where its completion arrives on a barrier.
 
 The model fails on
@@ -14,7 +14,7 @@ The model fails on
 * over-arrival, or deadlock (no role can move while some have not finished);
 * a data hazard: every buffer version goes through its stages in order (for
   example an S^T buffer: written by issuer A's MMAs, rewritten in place by the
-  8 softmax warps, read by the DV and DK MMAs), each stage with its number of
+  4 warps of its half's warpgroup, read by the DV and DK MMAs), each stage with its number of
   users; a use that starts before every user of the previous stage (or of the
   previous version) has finished is a hazard.
 
@@ -35,7 +35,7 @@ WARPS = 4 * NWG
 STAGES = {
     "kv": [("producer writes K, V", 1), ("issuer A reads", 1)],
     "stage": [("producer writes Q, dO, images, stats", 1), ("issuer A, DV, DK and the warps read", 3 + WARPS)],
-    "S": [("issuer A writes S^T, dP^T", 1), ("warps rewrite P^T, dS^T", WARPS), ("DV and DK read", 2)],
+    "S": [("issuer A writes S^T, dP^T", 1), ("the half's warpgroup rewrites P^T, dS^T", 4), ("DV and DK read", 2)],
     "dsbuf": [("warps write dS", WARPS), ("issuer A reads (dQ)", 1)],
     "dqtm": [("issuer A writes dQ", 1), ("warps read dQ", WARPS)],
     "acc_dv": [("DV accumulates dV", 1), ("warps read dV", WARPS)],
@@ -57,7 +57,7 @@ def _roles(nqs, QS):
         bar(f"qd_empty{s}", 3)  # issuer A (after dQ), DV and DK
     for x in range(NBUF):
         bar(f"s_full{x}", 1)
-        bar(f"ds_ready{x}", 32 * WARPS)
+        bar(f"ds_ready{x}", 128)  # the warpgroup that owns the half
         bar(f"kvmma_done{x}", 2)
     for w in range(NWG):
         bar(f"dsq_ready{w}", 128)
@@ -158,10 +158,9 @@ def _roles(nqs, QS):
                 if G >= 2:  # the dQ MMA of tile G - 2 has read this dS buffer
                     ops.append(W(f"dq_full{G & 1}", (G >> 1) - 1))
                 ops.append(B("dsbuf", G & 1, G, 0))
-                for hh in range(2):
-                    H = 2 * G + hh
-                    x = H % NBUF
-                    ops += [W(f"s_full{x}", H // NBUF), B("S", x, H, 1), E("S", x, H, 1), A(f"ds_ready{x}", 32)]
+                H = 2 * G + w  # warpgroup w owns half w of every tile
+                x = H % NBUF
+                ops += [W(f"s_full{x}", H // NBUF), B("S", x, H, 1), E("S", x, H, 1), A(f"ds_ready{x}", 32)]
                 ops.append(E("dsbuf", G & 1, G, 0))
                 if G > 0:
                     ops.append(W(f"dq_full{(G - 1) & 1}", (G - 1) >> 1))

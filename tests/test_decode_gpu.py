@@ -89,6 +89,31 @@ def test_cache_past_the_length_is_not_read(cuda_lib):
     np.testing.assert_array_equal(a[1], b[1])
 
 
+@pytest.mark.parametrize("Hq,Hkv,dh", [(10, 1, 16), (16, 2, 128)])
+def test_tensor_core_path_ignores_the_cache_past_the_length(cuda_lib, Hq, Hkv, dh):
+    q, k, v = _inputs(1, 1500, Hq, Hkv, dh, seed=8)
+    a = _run(cuda_lib, q, k, v, [1100])
+    k2, v2 = k.clone(), v.clone()
+    k2[:, 1100:] = float("nan")
+    v2[:, 1100:] = float("inf")
+    b = _run(cuda_lib, q, k2, v2, [1100])
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("Hq,Hkv,dh", [(10, 1, 16), (12, 2, 64), (16, 2, 128), (5, 1, 32)])
+def test_growing_scores_raise_the_running_maximum(cuda_lib, Hq, Hkv, dh):
+    # keys scaled up along the cache: later positions raise the running maximum
+    # by more than the kernels' lazy-rescale threshold, inside and across ranges
+    q, k, v = _inputs(2, 3000, Hq, Hkv, dh, seed=9)
+    ramp = (1.0 + torch.arange(3000, dtype=torch.float32) / 300.0).to(torch.bfloat16)
+    k = (k.float() * ramp[None, :, None, None].float()).to(torch.bfloat16)
+    out, lse = _run(cuda_lib, q, k, v, [3000, 1777])
+    ref_out, ref_lse = oracle.sqa_decode(q, k, v, [3000, 1777])
+    assert_lse_close("lse", lse, ref_lse)
+    assert_close("out", out, ref_out)
+
+
 def test_workspace_contents_do_not_matter(cuda_lib):
     B, N, Hq, Hkv, dh = 2, 900, 8, 4, 32
     q, k, v = _inputs(B, N, Hq, Hkv, dh, seed=6)

@@ -352,7 +352,7 @@ def model_mma(q, k, v, lens, scale):
     g = Hq // Hkv
     assert mma_path(g)
     CH, P = mma_chunk(dh), dh // 8
-    SPW, KS, NB = CH // 64, dh // 16, dh // 8
+    KS, NB = dh // 16, dh // 8
     span = 4 * decode_chunk(dh)  # the shared-memory path's span: the same workspace
     n_split = -(-N // span)
     part = np.full((B, Hkv, n_split, g, dh + 2), np.nan)
@@ -390,46 +390,61 @@ def model_mma(q, k, v, lens, scale):
         for w in range(4):
             warps.append(dict(m0=np.full(32, -np.inf), m1=np.full(32, -np.inf), l0=np.zeros(32), l1=np.zeros(32),
                               o=np.zeros((NB, 32, 4))))
+        KW = CH // 4
+        NKB = KW // 8
         for ci in range(n_chunks):
             if ci + MMA_STAGES - 1 < n_chunks:
                 load_chunk(ci + MMA_STAGES - 1)
             kbuf, vbuf = ring_k[ci % MMA_STAGES], ring_v[ci % MMA_STAGES]
             chunk_pos = r0 + ci * CH
             for w, st in enumerate(warps):
-                for step in range(SPW):
-                    key0 = (w * SPW + step) * 16
-                    s0, s1 = np.zeros((32, 4)), np.zeros((32, 4))
-                    for ks in range(KS):
-                        krow = key0 + (LANES & 7) + ((LANES >> 4) << 3)
+                key0 = w * KW
+                s_ = [np.zeros((32, 4)) for _ in range(NKB)]
+                for ks in range(KS):
+                    for h in range(NKB // 2):
+                        krow = key0 + 16 * h + (LANES & 7) + ((LANES >> 4) << 3)
                         kb = ldmatrix_x4(kbuf, mma_piece(dh, krow, 2 * ks + ((LANES >> 3) & 1)))
-                        mma16816(s0, qa[ks], kb[0], kb[1])
-                        mma16816(s1, qa[ks], kb[2], kb[3])
-                    kp = chunk_pos + key0 + 2 * FC
-                    x = np.stack([s0[:, 0], s0[:, 1], s1[:, 0], s1[:, 1], s0[:, 2], s0[:, 3], s1[:, 2], s1[:, 3]], 1)
-                    kpos = np.stack([kp, kp + 1, kp + 8, kp + 9], 1)
-                    valid = np.concatenate([kpos, kpos], 1) < r1
-                    x = np.where(valid, x * sl2, -np.inf)
-                    mx0, mx1 = x[:, :4].max(1), x[:, 4:].max(1)
-                    for sh in (1, 2):
-                        mx0 = np.maximum(mx0, shfl_xor(mx0, sh))
-                        mx1 = np.maximum(mx1, shfl_xor(mx1, sh))
-                    n0, n1 = np.maximum(st["m0"], mx0), np.maximum(st["m1"], mx1)
+                        mma16816(s_[2 * h], qa[ks], kb[0], kb[1])
+                        mma16816(s_[2 * h + 1], qa[ks], kb[2], kb[3])
+                if chunk_pos + CH > r1:  # the range ends in this chunk
+                    for nb in range(NKB):
+                        kp = chunk_pos + key0 + 8 * nb + 2 * FC
+                        s_[nb][kp >= r1, 0] = -np.inf
+                        s_[nb][kp >= r1, 2] = -np.inf
+                        s_[nb][kp + 1 >= r1, 1] = -np.inf
+                        s_[nb][kp + 1 >= r1, 3] = -np.inf
+                mx0 = np.max([np.maximum(x[:, 0], x[:, 1]) for x in s_], axis=0)
+                mx1 = np.max([np.maximum(x[:, 2], x[:, 3]) for x in s_], axis=0)
+                for sh in (1, 2):
+                    mx0 = np.maximum(mx0, shfl_xor(mx0, sh))
+                    mx1 = np.maximum(mx1, shfl_xor(mx1, sh))
+                t0, t1 = mx0 * sl2, mx1 * sl2
+                up0, up1 = t0 > st["m0"] + 8.0, t1 > st["m1"] + 8.0
+                if (up0 | up1).any():  # warp vote
                     with np.errstate(invalid="ignore"):
-                        a0 = np.where(n0 == -np.inf, 1.0, np.exp2(st["m0"] - n0))
-                        a1 = np.where(n1 == -np.inf, 1.0, np.exp2(st["m1"] - n1))
-                    st["m0"], st["m1"] = n0, n1
-                    b0, b1 = np.where(n0 == -np.inf, 0.0, n0), np.where(n1 == -np.inf, 0.0, n1)
-                    pr = np.concatenate([np.exp2(x[:, :4] - b0[:, None]), np.exp2(x[:, 4:] - b1[:, None])], 1)
-                    st["l0"] = st["l0"] * a0 + pr[:, :4].sum(1)
-                    st["l1"] = st["l1"] * a1 + pr[:, 4:].sum(1)
+                        a0 = np.where(up0 & (st["m0"] != -np.inf), np.exp2(st["m0"] - t0), 1.0)
+                        a1 = np.where(up1 & (st["m1"] != -np.inf), np.exp2(st["m1"] - t1), 1.0)
+                    st["m0"] = np.where(up0, t0, st["m0"])
+                    st["m1"] = np.where(up1, t1, st["m1"])
+                    st["l0"], st["l1"] = st["l0"] * a0, st["l1"] * a1
                     st["o"][:, :, 0:2] *= a0[None, :, None]
                     st["o"][:, :, 2:4] *= a1[None, :, None]
-                    pa = np.stack([pr[:, 0:2], pr[:, 4:6], pr[:, 2:4], pr[:, 6:8]])
+                nm0 = np.where(st["m0"] == -np.inf, 0.0, -st["m0"])
+                nm1 = np.where(st["m1"] == -np.inf, 0.0, -st["m1"])
+                pa = np.zeros((NKB // 2, 4, 32, 2))
+                for nb in range(NKB):
+                    p01 = np.exp2(s_[nb][:, 0:2] * sl2 + nm0[:, None])
+                    p23 = np.exp2(s_[nb][:, 2:4] * sl2 + nm1[:, None])
+                    st["l0"] = st["l0"] + p01.sum(1)
+                    st["l1"] = st["l1"] + p23.sum(1)
+                    pa[nb >> 1, (nb & 1) * 2 + 0] = p01
+                    pa[nb >> 1, (nb & 1) * 2 + 1] = p23
+                for h in range(NKB // 2):
                     for nb in range(0, NB, 2):
-                        vrow = key0 + (LANES & 7) + (((LANES >> 3) & 1) << 3)
+                        vrow = key0 + 16 * h + (LANES & 7) + (((LANES >> 3) & 1) << 3)
                         vb = ldmatrix_x4(vbuf, mma_piece(dh, vrow, nb + (LANES >> 4)), trans=True)
-                        mma16816(st["o"][nb], pa, vb[0], vb[1])
-                        mma16816(st["o"][nb + 1], pa, vb[2], vb[3])
+                        mma16816(st["o"][nb], pa[h], vb[0], vb[1])
+                        mma16816(st["o"][nb + 1], pa[h], vb[2], vb[3])
         # merge the four warps into the record
         ms = np.zeros((4, 16))
         ls = np.zeros((4, 16))
@@ -518,3 +533,19 @@ def test_three_way_path_selection(g, hkv, dh, path):
     # register-resident first, then tensor cores for 5-16 heads, else shared memory
     got = "rows" if rows_path(g, hkv, dh) else ("mma" if mma_path(g) else "general")
     assert got == path
+
+
+@pytest.mark.parametrize("dh", [16, 128])
+def test_tensor_core_model_raises_the_reference_maximum(dh):
+    # scores that grow along the cache (keys scaled up with their position) make
+    # later steps exceed the reference maximum by more than 8 (log2 units), so
+    # the rescale of O and l runs, mid-range and across warps
+    B, N, Hq, Hkv = 1, 700, 10, 1
+    rng = np.random.default_rng(dh)
+    q = rng.standard_normal((B, Hq, dh))
+    k = rng.standard_normal((B, N, Hkv, dh)) * (1.0 + np.arange(N) / 40.0)[None, :, None, None]
+    v = rng.standard_normal((B, N, Hkv, dh))
+    out, lse = model_mma(q, k, v, [N], 1 / math.sqrt(dh))
+    ref_out, ref_lse = oracle.sqa_decode(q, k, v, [N])
+    np.testing.assert_allclose(out, ref_out, rtol=0, atol=1e-10)
+    np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-9)
