@@ -86,6 +86,11 @@ struct FwdTraits {
   static constexpr int N_BARS = 2 * QBUF + 2 * STAGES + 4 + 4 + 2 + 2 + 2 + 2 + 2 + 2;
   // The softmax warpgroups take turns for the exponentials (one S buffer per tile).
   static constexpr bool TOKEN = NSBUF == 1;
+  // With one Q buffer a slot cannot start the next item before the other slot
+  // has finished this one, so a slot that skips the other's turns (an item with
+  // one Q tile) stays within one phase of the turn barriers; with two Q buffers
+  // it could run a whole item ahead and alias their phases.
+  static_assert(!TOKEN || QBUF == 1, "turns need one Q buffer");
   // split mode: slot 1's running maximum and sum per row, for slot 0's combine
   static constexpr int OFF_ML = OFF_BAR + N_BARS * 8 + 16;
   static constexpr int SMEM_USED = OFF_ML + 2 * BM * 4;

@@ -342,6 +342,23 @@ DROPS = {
 IMPLIED = {("warps: o_done", 1), ("warps: tok", 2)}  # no token with two S buffers
 
 
+def test_turns_with_two_q_buffers_would_alias_their_phases():
+    # why the kernel keeps turns to one Q buffer: with two, a slot runs a whole
+    # item ahead through an item the other slot has no tile in
+    rnd = random.Random(5)
+    failures = 0
+    for trial in range(100):
+        items = _items(rnd)
+        rnd2 = random.Random(trial)
+        roles, cnt = _roles(items, 2, 4, rnd2, 1)
+        try:
+            sync_model.run(roles, cnt, STAGES, trial, custom={"O": _OCheck(), "X": _ExpCheck(True)},
+                           skewed=trial % 2 == 1)
+        except AssertionError as e:
+            failures += "aliasing" in str(e)
+    assert failures > 0
+
+
 @pytest.mark.parametrize("name,NSB", [(n, b) for n in DROPS for b in (2, 1) if (n, b) not in IMPLIED])
 def test_model_detects_a_dropped_wait(name, NSB):
     rnd = random.Random(17)
