@@ -416,17 +416,18 @@ __global__ void __launch_bounds__(384, 1)
 //     S_j  = Q K_j^T, dP_j = dO V_j^T        (TMEM, query rows on lanes)
 //     dS_j = 2^(S_j scale log2e - lse2) (dP_j - D), rewritten in place (bf16)
 //     dQ  += dS_j K_j                         (A = dS_j from TMEM)
-// Two issuers: one runs S_{j+1} and dP_{j+1} ahead while the warps turn S_j
-// and dP_j into dS_j, the other issues dQ of j as soon as dS_j is ready.  (With
-// one issuer for all three products, its instruction stream, which shares its
-// sub-partition with two busy softmax warps, took twice as long per key tile
-// as the warps and set the pace.)  S_{j+2} reuses buffer j % 2 once the dQ of j
-// has read dS_j (dq_done).  dQ is scaled and written once, in bf16.
+// Three issuers: one runs S_{j+1} ahead and one dP_{j+1} while the warps turn
+// S_j and dP_j into dS_j, the third issues dQ of j as soon as dS_j is ready.
+// (With one issuer for all three products its instruction stream, which shares
+// its sub-partition with two busy softmax warps, took twice as long per key
+// tile as the warps and set the pace: an N = 64 MMA takes longer to issue than
+// to run.)  S_{j+2} and dP_{j+2} reuse buffer j % 2 once the dQ of j has read
+// dS_j (dq_done).  dQ is scaled and written once, in bf16.
 //
 // TMEM (dh 128): Q [0, 64), dO [64, 128), S buffers 128 + 64 b, dP buffers
 // 256 + 64 b, dQ [384, 512); at dh 64 the same with Q, dO of 32 columns.
-// Roles (384 threads): warp 0 producer, warp 1 TMEM allocator and S / dP
-// issuer, warp 2 dQ issuer, warps 4-11 two warpgroups (warpgroup w: keys 32 w .. 32 w + 31 of each
+// Roles (384 threads): warp 0 producer, warp 1 TMEM allocator and S issuer,
+// warp 2 dQ issuer, warp 3 dP issuer, warps 4-11 two warpgroups (warpgroup w: keys 32 w .. 32 w + 31 of each
 // stage, query row = TMEM lane), which also load Q and dO into TMEM and write
 // dQ.
 
@@ -451,8 +452,8 @@ struct BwdQTraits {
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
-  // kv_full[S], kv_empty[S], qd_ready, sd_full[2], ds_ready[2], dq_final, drain[2], dq_done[2]
-  static constexpr int N_BARS = 2 * STAGES + 10;
+  // kv_full[S], kv_empty[S], qd_ready, sd_full[2], ds_ready[2], dq_final, drain[3], dq_done[2]
+  static constexpr int N_BARS = 2 * STAGES + 11;
   static constexpr int SMEM_USED = OFF_BAR + N_BARS * 8 + 16;
   static constexpr int SMEM_BYTES = (SMEM_USED > 120 * 1024 ? SMEM_USED : 120 * 1024) + 1024;
   static constexpr uint32_t TM_Q = 0, TM_DO = DH / 2;
@@ -460,7 +461,7 @@ struct BwdQTraits {
   __host__ __device__ static constexpr uint32_t tm_dp(int b) { return 256u + 64u * b; }
   static constexpr uint32_t TM_DQ = 384, TM_COLS = 512;
   static constexpr int THREADS = 384;
-  static constexpr int WARP_PRODUCER = 0, WARP_MMA = 1, WARP_MMA_Q = 2, WARP_SOFTMAX0 = 4;
+  static constexpr int WARP_PRODUCER = 0, WARP_MMA = 1, WARP_MMA_Q = 2, WARP_MMA_DP = 3, WARP_SOFTMAX0 = 4;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   static_assert(TM_DQ + DH <= TM_COLS, "TMEM budget");
 };
@@ -494,7 +495,7 @@ __global__ void __launch_bounds__(384, 1)
   auto ds_ready = [&](int x) { return bar0 + 8u * (2 * ST + 3 + x); };
   const uint32_t dq_final = bar0 + 8u * (2 * ST + 5);
   auto drain = [&](int i) { return bar0 + 8u * (2 * ST + 6 + i); };  // one per issuer
-  auto dq_done = [&](int x) { return bar0 + 8u * (2 * ST + 8 + x); };  // dQ of a tile in buffer x has read its dS
+  auto dq_done = [&](int x) { return bar0 + 8u * (2 * ST + 9 + x); };  // dQ of a tile in buffer x has read its dS
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Tr::OFF_BAR + Tr::N_BARS * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -505,14 +506,12 @@ __global__ void __launch_bounds__(384, 1)
     }
     mbar_init(qd_ready, 256);
     for (int x = 0; x < 2; ++x) {
-      mbar_init(sd_full(x), 1);
+      mbar_init(sd_full(x), 2);  // the S and the dP issuer
       mbar_init(ds_ready(x), 256);
+      mbar_init(dq_done(x), 1);
     }
     mbar_init(dq_final, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(drain(i), 1);
-      mbar_init(dq_done(i), 1);
-    }
+    for (int i = 0; i < 3; ++i) mbar_init(drain(i), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -546,35 +545,34 @@ __global__ void __launch_bounds__(384, 1)
         for (int i = max(0, j - ST); i < j; ++i) mbar_wait_drain(kv_full(i % ST), (i / ST) & 1);
       }
     }
-  } else if (warp == Tr::WARP_MMA) {
-    // ------------------------------------------------------------ S / dP issuer
-    constexpr uint32_t idesc_s = idesc_bf16_f32(128, NK, false, false);  // S, dP: A (Q, dO) in TMEM, B K-major
-    // Descriptors of stage 0, K-step 0; a stage and a K-step add their byte offsets / 16.
-    const uint64_t dk0 = smem_desc(sbase + Tr::OFF_K, 16, 8 * ROWB, Tr::LAYOUT);
-    const uint64_t dv0 = smem_desc(sbase + Tr::OFF_V, 16, 8 * ROWB, Tr::LAYOUT);
-    // S_j and dP_j: M = 128 rows, N = 64 keys, K = dh in steps of 16 (8 TMEM columns of Q / dO).
-    auto issue_sd = [&](int j) {
+  } else if (warp == Tr::WARP_MMA || warp == Tr::WARP_MMA_DP) {
+    // ------------------------------------------------------------ S issuer (warp 1), dP issuer (warp 3)
+    // S_j = Q K_j^T or dP_j = dO V_j^T: M = 128 rows, N = 64 keys, K = dh in
+    // steps of 16 (8 TMEM columns of Q / dO); A from TMEM, B K-major in smem.
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, NK, false, false);
+    const bool is_s = warp == Tr::WARP_MMA;
+    const uint64_t db0 = smem_desc(sbase + (is_s ? Tr::OFF_K : Tr::OFF_V), 16, 8 * ROWB, Tr::LAYOUT);
+    const uint32_t ta = tmem + (is_s ? Tr::TM_Q : Tr::TM_DO);
+    bool ok = mbar_wait_warp(qd_ready, 0, abort_flag, kSiteMma);
+    for (int j = 0; ok && j < nkv; ++j) {
       const int x = j & 1;
+      if (!(ok = mbar_wait_warp(kv_full(j % ST), (j / ST) & 1, abort_flag, kSiteMma))) break;
+      // buffer j % 2 held dS_{j-2} (and dP_{j-2}): the dQ MMA has read it
+      if (j >= 2 && !(ok = mbar_wait_warp(dq_done(x), ((j - 2) >> 1) & 1, abort_flag, kSiteMma))) break;
+      tc_fence_after();
+      const uint32_t td = tmem + (is_s ? Tr::tm_s(x) : Tr::tm_dp(x));
       const uint64_t so = static_cast<uint64_t>(((j % ST) * Tr::KV_BYTES) >> 4);
 #pragma unroll
       for (int ks = 0; ks < DH / 16; ++ks) {
         const uint64_t ko = so + ((((ks * 16) / PANEL) * NK * ROWB + ((ks * 16) % PANEL) * 2) >> 4);
-        mma_ts_w(tmem + Tr::tm_s(x), tmem + Tr::TM_Q + 8u * ks, dk0 + ko, idesc_s, ks > 0);
-        mma_ts_w(tmem + Tr::tm_dp(x), tmem + Tr::TM_DO + 8u * ks, dv0 + ko, idesc_s, ks > 0);
+        mma_ts_w(td, ta + 8u * ks, db0 + ko, idesc_s, ks > 0);
       }
       mma_commit_w(sd_full(x));
-    };
-    bool ok = mbar_wait_warp(qd_ready, 0, abort_flag, kSiteMma);
-    for (int j = 0; ok && j < nkv; ++j) {
-      if (!(ok = mbar_wait_warp(kv_full(j % ST), (j / ST) & 1, abort_flag, kSiteMma))) break;
-      // buffer j % 2 held dS_{j-2}: the dQ MMA has read it
-      if (j >= 2 && !(ok = mbar_wait_warp(dq_done(j & 1), ((j - 2) >> 1) & 1, abort_flag, kSiteMma))) break;
-      tc_fence_after();
-      issue_sd(j);
     }
     if (!ok) {
-      mma_commit_w(drain(0));
-      mbar_wait_drain(drain(0), 0);
+      const int d = is_s ? 0 : 2;
+      mma_commit_w(drain(d));
+      mbar_wait_drain(drain(d), 0);
     }
   } else if (warp == Tr::WARP_MMA_Q) {
     // ------------------------------------------------------------ dQ issuer

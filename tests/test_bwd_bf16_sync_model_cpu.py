@@ -15,8 +15,8 @@ CPU under random schedules with the checker in ``sync_model``.
   (rewriting dP^T's columns), the dV/dK epilogue.
 
 ``sqa_bwd_q_kernel`` (dQ, one CTA per stacked Q tile): the producer streams
-K/V through a ring; the warps put Q and dO into TMEM; one issuer runs S_j and
-dP_j into buffer j % 2 and then dQ of j - 1; the warps turn S_j and dP_j into
+K/V through a ring; the warps put Q and dO into TMEM; two issuers run S_j and
+dP_j into buffer j % 2, a third dQ of j once dS_j is ready; the warps turn S_j and dP_j into
 dS_j in place; the epilogue reads dQ.  Barrier arrival counts are the kernels'.
 """
 import random
@@ -168,22 +168,23 @@ def test_model_detects_a_dropped_wait(name):
 
 def _q_stages():
     return {
-        "kv": [("producer writes K, V", 1), ("S, dP MMAs and the dQ MMA read", 2)],
-        "QD": [("warps write Q, dO into TMEM", WARPS), ("S, dP MMAs read", 1)],
-        "SB": [("S, dP write", 1), ("warps rewrite dS", WARPS), ("dQ MMA reads dS", 1)],
+        "kv": [("producer writes K, V", 1), ("S, dP and dQ MMAs read", 3)],
+        "QD": [("warps write Q, dO into TMEM", WARPS), ("S, dP MMAs read", 2)],
+        "SB": [("S and dP MMAs write", 2), ("warps rewrite dS", WARPS), ("dQ MMA reads dS", 1)],
         "acc_dq": [("dQ issuer accumulates dQ", 1), ("warps read dQ", WARPS)],
     }
 
 
 def _q_roles(nkv, ST):
-    """Two issuers: S / dP of tile j into buffer j % 2 once the dQ of j - 2 has
-    read that buffer (dq_done), and dQ of j once the warps made dS_j."""
+    """Three issuers: S and dP (one each) of tile j into buffer j % 2 once the
+    dQ of j - 2 has read that buffer (dq_done), and dQ of j once the warps made
+    dS_j."""
     cnt = {"qd_ready": 32 * WARPS, "dq_final": 1}
     for s in range(ST):
         cnt[f"kv_full{s}"] = 1
         cnt[f"kv_empty{s}"] = 1
     for x in range(2):
-        cnt[f"sd_full{x}"] = 1
+        cnt[f"sd_full{x}"] = 2  # the S and the dP issuer
         cnt[f"ds_ready{x}"] = 32 * WARPS
         cnt[f"dq_done{x}"] = 1
 
@@ -206,16 +207,18 @@ def _q_roles(nkv, ST):
             prod.append(W(f"kv_empty{s}", j // ST - 1))
         prod += [B("kv", j, 0, s), E("kv", j, 0, s), A(f"kv_full{s}")]
 
-    iss_s = [W("qd_ready", 0), B("QD", 0, 1)]
-    for j in range(nkv):
-        x = j & 1
-        iss_s.append(W(f"kv_full{j % ST}", j // ST))
-        if j >= 2:
-            iss_s.append(W(f"dq_done{x}", (j - 2) >> 1))
-        # the S / dP MMAs read K_j, V_j and write buffer x; done when sd_full arrives
-        iss_s += [B("kv", j, 1, j % ST), B("SB", j, 0, x), E("SB", j, 0, x), E("kv", j, 1, j % ST),
-                  A(f"sd_full{x}")]
-    iss_s.append(E("QD", 0, 1))
+    def sd_issuer():
+        ops = [W("qd_ready", 0), B("QD", 0, 1)]
+        for j in range(nkv):
+            x = j & 1
+            ops.append(W(f"kv_full{j % ST}", j // ST))
+            if j >= 2:
+                ops.append(W(f"dq_done{x}", (j - 2) >> 1))
+            # the MMAs read K_j or V_j and write buffer x; done when sd_full arrives
+            ops += [B("kv", j, 1, j % ST), B("SB", j, 0, x), E("SB", j, 0, x), E("kv", j, 1, j % ST),
+                    A(f"sd_full{x}")]
+        ops.append(E("QD", 0, 1))
+        return ops
 
     iss_q = [B("acc_dq", 0, 0)]
     for j in range(nkv):
@@ -232,7 +235,7 @@ def _q_roles(nkv, ST):
         ops += [W("dq_final", 0), B("acc_dq", 0, 1), E("acc_dq", 0, 1)]
         return ops
 
-    roles = {"producer": prod, "issuer_s": iss_s, "issuer_q": iss_q}
+    roles = {"producer": prod, "issuer_s": sd_issuer(), "issuer_dp": sd_issuer(), "issuer_q": iss_q}
     for w in range(WARPS):
         roles[f"warp{w}"] = warp()
     return roles, cnt
@@ -255,10 +258,12 @@ def test_q_kernel_protocol_has_no_deadlock_aliasing_or_hazard(ST):
 Q_DROPS = {
     # S / dP would read Q, dO before the warps put them into TMEM
     "issuer: qd_ready": _drop("issuer_s", "qd_ready"),
+    "dP issuer: qd_ready": _drop("issuer_dp", "qd_ready"),
     # dQ would read dS before the warps wrote it
     "issuer: ds_ready": _drop("issuer_q", "ds_ready"),
     # S of j + 2 would overwrite dS_j before the dQ MMA read it
     "issuer: dq_done": _drop("issuer_s", "dq_done"),
+    "dP issuer: dq_done": _drop("issuer_dp", "dq_done"),
     # the MMAs would read a K/V stage before it landed
     "issuer: kv_full": _drop("issuer_s", "kv_full"),
     # the warps would read S / dP before the MMA wrote them, or dQ before the last MMA
