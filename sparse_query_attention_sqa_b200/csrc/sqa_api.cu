@@ -157,9 +157,11 @@ sqa_status launch_fwd(const void* q, const void* k, const void* v, void* out, fl
   if ((st = make_map(&mq, q, s.B, s.N, s.H_q, DH, Tr::PANEL, p.g, p.T)) != SQA_OK) return st;
   if ((st = make_map(&mk, k, s.B, s.N, s.H_kv, DH, Tr::PANEL, 1, Tr::NK)) != SQA_OK) return st;
   if ((st = make_map(&mv, v, s.B, s.N, s.H_kv, DH, Tr::PANEL, 1, Tr::NK)) != SQA_OK) return st;
-  if ((st = set_smem(sqa::sqa_fwd_kernel<DH>, Tr::SMEM_BYTES)) != SQA_OK) return st;
+  // split mode is compiled as its own kernel (dh <= 64 only)
+  auto kernel = p.split ? sqa::sqa_fwd_kernel<DH, DH <= 64> : sqa::sqa_fwd_kernel<DH, false>;
+  if ((st = set_smem(kernel, Tr::SMEM_BYTES)) != SQA_OK) return st;
   if ((st = record_timing(0, 0, stream)) != SQA_OK) return st;
-  sqa::sqa_fwd_kernel<DH><<<static_cast<unsigned>(grid), Tr::THREADS, Tr::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  kernel<<<static_cast<unsigned>(grid), Tr::THREADS, Tr::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "sqa_fwd launch");
   return record_timing(0, 1, stream);

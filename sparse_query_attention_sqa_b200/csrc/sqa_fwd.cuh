@@ -112,12 +112,13 @@ struct FwdItem {
   bool has1;
 };
 
+template <bool SPLIT>
 __device__ __forceinline__ FwdItem fwd_decode(const FwdParams& p, int item, int NK) {
   FwdItem it;
   const int bh = item % p.n_bh;
   it.b = bh / p.Hkv;
   it.kvh = bh % p.Hkv;
-  if (p.split) {
+  if (SPLIT) {
     // One Q tile; slot 0 takes its even key tiles, slot 1 the odd ones.
     it.qt0 = p.n_qtiles - 1 - item / p.n_bh;  // latest tokens (heaviest under a causal mask) first
     const int end = p.causal ? min(p.N, (it.qt0 + 1) * p.T) : p.N;
@@ -138,9 +139,11 @@ __device__ __forceinline__ FwdItem fwd_decode(const FwdParams& p, int item, int 
   return it;
 }
 
-// POLY: of every 8 pairs of scores in an unmasked tile, how many take the
-// polynomial exponential (exp2_poly2) instead of the special-function unit.
-template <int DH, int POLY = (DH <= 32 ? 2 : 0)>
+// SPLIT: split mode (FwdParams::split), compiled separately so that the
+// ordinary kernel carries none of its code.  POLY: of every 8 pairs of scores
+// in an unmasked tile, how many take the polynomial exponential (exp2_poly2)
+// instead of the special-function unit.
+template <int DH, bool SPLIT, int POLY = (DH <= 32 ? 2 : 0)>
 __global__ void __launch_bounds__(384, 1)
     sqa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -237,7 +240,7 @@ __global__ void __launch_bounds__(384, 1)
       int g = 0;  // K/V tiles issued so far (across items)
       bool ok = true;
       for (int r = 0, item; ok && (item = fwd_item(r, p.n_items)) >= 0; ++r) {
-        const FwdItem it = fwd_decode(p, item, NK);
+        const FwdItem it = fwd_decode<SPLIT>(p, item, NK);
         const int qb = r % QB;
         if (r >= QB && !mbar_wait(q_empty(qb), ((r / QB) - 1) & 1, abort_flag, kSiteProducer)) break;
         mbar_expect_tx(q_full(qb), q_bytes * (it.has1 ? 2u : 1u));
@@ -275,7 +278,7 @@ __global__ void __launch_bounds__(384, 1)
     // Descriptors of Q buffer 0 / stage 0; other buffers, stages and K-steps add
     // their byte offset (in 16-byte units) to the start-address field.
     // (In split mode both slots read the one Q tile, in slot 0's buffer.)
-    const uint64_t dq0 = smem_desc(sbase + Tr::OFF_Q + (p.split ? 0 : t) * Tr::Q_BYTES, 16, 8 * ROWB, Tr::LAYOUT);
+    const uint64_t dq0 = smem_desc(sbase + Tr::OFF_Q + (SPLIT ? 0 : t) * Tr::Q_BYTES, 16, 8 * ROWB, Tr::LAYOUT);
     const uint64_t dk0 = smem_desc(sbase + Tr::OFF_K, 16, 8 * ROWB, Tr::LAYOUT);
     const uint64_t dv0 = smem_desc(sbase + Tr::OFF_V, NK * ROWB, 8 * ROWB, Tr::LAYOUT);
     const uint32_t tS0 = tmem + Tr::tm_s(t, 0), tO = tmem + Tr::tm_o(t);
@@ -305,19 +308,19 @@ __global__ void __launch_bounds__(384, 1)
     auto ensure_loaded = [&](int gj) {
       while (loaded <= gj) {
         if (!mbar_wait_warp(kv_full(loaded % ST), (loaded / ST) & 1, abort_flag, kSiteMma)) return false;
-        if (p.split && ((loaded - g) & 1) != t) mma_commit_w(kv_empty(loaded % ST));
+        if (SPLIT && ((loaded - g) & 1) != t) mma_commit_w(kv_empty(loaded % ST));
         ++loaded;
       }
       tc_fence_after();
       return true;
     };
     // item-relative index of this slot's j-th key tile
-    auto own = [&](int j) { return p.split ? 2 * j + t : j; };
+    auto own = [&](int j) { return SPLIT ? 2 * j + t : j; };
     int G = 0;   // S steps of this Q tile so far (across items)
     int nd = 0;  // items finished by this Q tile
     bool ok = true;
     for (int r = 0, item; ok && (item = fwd_item(r, p.n_items)) >= 0; ++r) {
-      const FwdItem it = fwd_decode(p, item, NK);
+      const FwdItem it = fwd_decode<SPLIT>(p, item, NK);
       const int nkv_t = t ? it.nkv1 : it.nkv0;
       const int qb = r % QB;
       // Both issuers observe this item's Q load before releasing its buffer, so a
@@ -357,7 +360,7 @@ __global__ void __launch_bounds__(384, 1)
           issue_qk(qb, (g + own(j + NSB)) % ST, Gt % NSB);
         }
       }
-      if (p.split) {
+      if (SPLIT) {
         // the other slot's tiles after this slot's last one
         if (ok && it.nkv > 0) ok = ensure_loaded(g + it.nkv - 1);
       } else {
@@ -396,14 +399,14 @@ __global__ void __launch_bounds__(384, 1)
     int G_other = 0;
     bool ok = true;
     for (int r = 0, item; ok && (item = fwd_item(r, p.n_items)) >= 0; ++r) {
-      const FwdItem it = fwd_decode(p, item, NK);
+      const FwdItem it = fwd_decode<SPLIT>(p, item, NK);
       const int nkv_t = t ? it.nkv1 : it.nkv0;
-      const int nkv_o = t ? it.nkv0 : it.nkv1;
+      const int nkv_o = Tr::TOKEN ? (t ? it.nkv0 : it.nkv1) : 0;
       const int G_o = G_other;
-      G_other += nkv_o;
+      if constexpr (Tr::TOKEN) G_other += nkv_o;
       if (nkv_t == 0) continue;
-      const int qt = p.split ? it.qt0 : it.qt0 + t;
-      const bool combine = p.split && it.nkv1 > 0;  // slot 1 holds part of this row's sums
+      const int qt = SPLIT ? it.qt0 : it.qt0 + t;
+      const bool combine = SPLIT && it.nkv1 > 0;  // slot 1 holds part of this row's sums
       const int tok = qt * p.T + row / p.g;
       const int head = it.kvh * p.g + row % p.g;
       const bool row_valid = row < p.rows && tok < p.N;
@@ -416,7 +419,7 @@ __global__ void __launch_bounds__(384, 1)
         if (!ok) break;
         tc_fence_after();
         const uint32_t tS = lane_addr + Tr::tm_s(t, Gt % NSB);
-        const int k0 = (p.split ? 2 * j + t : j) * NK;
+        const int k0 = (SPLIT ? 2 * j + t : j) * NK;
         const bool masked = (k0 + NK > p.N) || (p.causal && k0 + NK - 1 > qt * p.T);
         // The tile's scores are handled 64 columns (a half at NK = 128) at a time.
         // last visible key of this tile, relative to k0 (may be negative)
