@@ -57,7 +57,14 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="time budget of the CPU-baseline sample")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch every step from the host even where the workload asks for CUDA-graph replay")
     return ap.parse_args()
+
+
+def block_gemm_params(w) -> int:
+    """Weights of one decoder block's matrix products: W_q|W_k|W_v, W_o, W1, W3, W2."""
+    return w.d * (w.Hq + 2 * w.Hkv) * w.dh + w.Hq * w.dh * w.d + 3 * w.d * w.hidden
 
 
 def counted_flops(w) -> float:
@@ -66,7 +73,10 @@ def counted_flops(w) -> float:
     fwd = 4.0 * w.B * w.Hq * w.N * w.N * w.dh
     if w.causal:
         fwd /= 2
-    return fwd * (3.5 if w.backward else 1.0)
+    attn = fwd * (3.5 if w.backward else 1.0)
+    if w.block:  # per block: the attention plus its matrix products (forward once, backward twice)
+        return w.layers * (attn + 2.0 * w.B * w.N * block_gemm_params(w) * (3.0 if w.backward else 1.0))
+    return attn
 
 
 def max_over_ranks(x: float, world: int, device) -> float:
@@ -105,9 +115,20 @@ def load_peaks():
 # --------------------------------------------------------------------------- CPU oracle
 def oracle_subproblem(w, seed=0):
     """One independent slice of the workload: batch entry 0, KV head 0 and its
-    g query heads (the oracle's work on it scales with the counted FLOPs)."""
-    from sparse_query_attention_sqa_b200.inputs import make_decode_inputs, make_inputs
+    g query heads (the oracle's work on it scales with the counted FLOPs); for
+    a block stack, one block of batch entry 0."""
+    from sparse_query_attention_sqa_b200.inputs import make_block_inputs, make_decode_inputs, make_inputs
 
+    if w.block:
+        x, wd, dy = make_block_inputs(1, w.N, w.d, w.Hq, w.Hkv, w.dh, w.hidden, seed=seed)
+        sub = type(w)(name=w.name + "_slice", B=1, N=w.N, Hq=w.Hq, Hkv=w.Hkv, dh=w.dh, causal=w.causal,
+                      backward=w.backward, d=w.d, hidden=w.hidden, layers=1)
+        # the oracle block takes fp64 arrays and the fused projection split into W_q, W_k, W_v
+        wf = {n: t.double().numpy() for n, t in wd.items()}
+        nq, nk = w.Hq * w.dh, w.Hkv * w.dh
+        p = {"g1": wf["g1"], "g2": wf["g2"], "wq": wf["w_qkv"][:, :nq], "wk": wf["w_qkv"][:, nq:nq + nk],
+             "wv": wf["w_qkv"][:, nq + nk:], "wo": wf["w_o"], "w1": wf["w1"], "w3": wf["w3"], "w2": wf["w2"]}
+        return sub, (x.double().numpy(), p, dy.double().numpy(), None)
     g = w.Hq // w.Hkv
     if w.decode:
         q, k, v = make_decode_inputs(1, w.N, g, 1, w.dh, seed=seed, std=w.std, k_scale=w.k_scale)
@@ -123,6 +144,14 @@ def oracle_subproblem(w, seed=0):
 def run_oracle_step(sub, data):
     import oracle
 
+    if sub.block:
+        from oracle import block as oblock
+
+        x, wd, dy, _ = data
+        oblock.block_fwd(x, wd, sub.Hq, sub.Hkv, sub.causal)
+        if sub.backward:
+            oblock.block_bwd(x, wd, dy, sub.Hq, sub.Hkv, sub.causal)
+        return
     q, k, v, dout = data
     if sub.decode:
         oracle.sqa_decode(q, k, v, None, sub.softmax_scale)
@@ -161,7 +190,7 @@ def cpu_baseline_rows(w, seconds):
 
 def cpu_baseline(w, seconds):
     g = w.Hq // w.Hkv
-    if not w.decode and g * w.N * w.N * w.dh > 2 ** 34:  # one slice would take minutes
+    if not w.decode and not w.block and g * w.N * w.N * w.dh > 2 ** 34:  # one slice would take minutes
         return cpu_baseline_rows(w, seconds)
     sub, data = oracle_subproblem(w)
     run_oracle_step(sub, data)  # builds the oracle and warms caches
@@ -174,9 +203,10 @@ def cpu_baseline(w, seconds):
         if el >= seconds:
             break
     rate = counted_flops(sub) * n / el / 1e12
+    what = (f"one decoder block of batch entry 0 (N={w.N}, d={w.d})" if w.block else
+            f"batch entry 0, KV head 0 and its {sub.Hq} query heads (N={w.N}, dh={w.dh})")
     return {"value": rate, "unit": "TFLOP/s", "cores": omp_threads(), "kind": "oracle",
-            "sample": f"fp64 oracle {pass_name(w)} on batch entry 0, KV head 0 and its "
-                      f"{sub.Hq} query heads (N={w.N}, dh={w.dh}), {n} runs in {el:.1f} s"}
+            "sample": f"fp64 oracle {pass_name(w)} on {what}, {n} runs in {el:.1f} s"}
 
 
 # --------------------------------------------------------------------------- clocks
@@ -229,8 +259,20 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- GPU arm
+BLOCK_PARAMS = ("g1", "w_qkv", "w_o", "g2", "w1", "w3", "w2")
+
+
 def alloc_set(w, q, k, v, dout, lib, torch):
     dev = "cuda"
+    if w.block:  # q, k, v are x, the weights, dy
+        s = {"x": q.to(dev), "dy": v.to(dev)}
+        s.update({"w_" + n: k[n].to(dev) for n in BLOCK_PARAMS})
+        nbytes = max(lib.block_state_bytes(w.B, w.N, w.d, w.Hq, w.Hkv, w.dh, w.hidden), 256)
+        for layer in range(w.layers):
+            s[f"state{layer}"] = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        s["y"] = torch.empty_like(s["x"])
+        s["dx"] = torch.empty_like(s["x"])
+        return s
     s = {"q": q.to(dev), "k": k.to(dev), "v": v.to(dev)}
     s["out"] = torch.empty_like(s["q"])
     if w.decode:
@@ -253,6 +295,19 @@ def set_bytes(s) -> int:
 
 
 def step(lib, w, s):
+    if w.block:
+        # every block runs with the same random weights (a timing stack); the
+        # weight gradients of each block are produced and dropped
+        wd = {n: s["w_" + n] for n in BLOCK_PARAMS}
+        xs = [s["x"]]
+        for layer in range(w.layers):
+            y, _ = lib.sqa_block_fwd(xs[-1], wd, w.Hq, w.Hkv, state=s[f"state{layer}"], causal=w.causal)
+            xs.append(y)
+        g = s["dy"]
+        for layer in reversed(range(w.layers)):
+            g, _ = lib.sqa_block_bwd(g, xs[layer], wd, s[f"state{layer}"], w.Hq, w.Hkv, causal=w.causal)
+        s["y"], s["dx"] = xs[-1], g
+        return
     if w.decode:
         lib.sqa_decode(s["q"], s["k"], s["v"], out=s["out"], lse=s["lse"], workspace=s["ws"], scale=w.scale)
         return
@@ -262,7 +317,26 @@ def step(lib, w, s):
                     workspace=s["ws"], causal=w.causal, scale=w.scale)
 
 
+def metric_name(w) -> str:
+    return "SQAT-m decoder-block stack" if w.block else "SQA attention"
+
+
+def launches_per_step(w) -> int:
+    """Kernels of this library launched per step (memsets not counted)."""
+    if w.block:
+        # forward: RMSNorm, rotary table, W_qkv, attention, W_o, RMSNorm, W1|W3, W2;
+        # backward: dM (SwiGLU), dW2, dW1, dW3, dN, RMSNorm; the layer (rotary
+        # table, dO, dW_o, attention preprocess / main / dQ, two inverse
+        # rotations, three dW_qkv parts, dX); RMSNorm
+        return w.layers * (8 + 6 + 12 + 1)
+    # the forward, the backward's preprocess, its main kernel and either the dQ
+    # conversion (dh <= 32) or the dQ kernel (dh 64 / 128)
+    return 4 if w.backward else (2 if w.decode else 1)
+
+
 def pass_name(w) -> str:
+    if w.block:
+        return f"{w.layers}-block fwd+bwd"
     return "decode" if w.decode else ("fwd+bwd" if w.backward else "fwd")
 
 
@@ -370,6 +444,23 @@ def traffic_for(kernel_name, w):
     return None
 
 
+def make_graphs(lib, w, sets, torch):
+    """One CUDA graph per buffer set holding a whole step (launch-bound
+    workloads: the step's launches cost the host more than the device's work).
+    The timing hooks are off while capturing."""
+    graphs = []
+    for s in sets:
+        gph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gph, capture_error_mode="thread_local"):
+            step(lib, w, s)
+        graphs.append(gph)
+    for gph in graphs:
+        gph.replay()
+    torch.cuda.synchronize()
+    assert lib.device_status() == 0, "a kernel wait gave up in a graph's first replay"
+    return graphs
+
+
 def warm_up(lib, w, sets, warmup, torch):
     """Warm-up steps; each times its main kernels with the library's hook.
     Returns ({kernel: [ms]}, the dominant kernel's name, its hook index)."""
@@ -401,6 +492,7 @@ def compare_variants(args, w):
     if args.no_compare:
         return []
     groups = {"large_dh128": ("large_dh128_mha", "large_dh128_gqa", "large_dh128_mqa"),
+              "sqatm_block_sqa": ("sqatm_block_mha", "sqatm_block_gqa", "sqatm_block_mqa"),
               "sqatm_train_sqa": ("sqatm_train_mha", "sqatm_train_gqa", "sqatm_train_mqa"),
               "enc32k_8_4": ("enc32k_16_16", "enc32k_16_4", "enc32k_16_1", "enc32k_8_8", "enc32k_4_4")}
     return [WORKLOADS[n] for n in groups.get(w.name, ())]
@@ -418,20 +510,26 @@ def time_variant(args, lib, w, torch, world, rank, peaks, peak_kind):
     sets = [first] + [alloc_set(w, q, k, v, dout, lib, torch) for _ in range(n_sets - 1)]
     del q, k, v, dout
     kern, dominant, dom_idx = warm_up(lib, w, sets, args.warmup, torch)
+    graphs = make_graphs(lib, w, sets, torch) if w.graph and not args.no_graph else None
     starts = [ev() for _ in range(args.steps)]
     stops = [ev() for _ in range(args.steps)]
     t0, t1 = ev(), ev()
     torch.cuda.synchronize()
     t0.record()
     for i in range(args.steps):
-        lib.set_timing_events(dom_idx, starts[i], stops[i])
-        step(lib, w, sets[i % n_sets])
+        if graphs:
+            graphs[i % n_sets].replay()
+        else:
+            lib.set_timing_events(dom_idx, starts[i], stops[i])
+            step(lib, w, sets[i % n_sets])
     t1.record()
     lib.set_timing_events(dom_idx)
     torch.cuda.synchronize()
     assert lib.device_status() == 0, "a kernel wait gave up while timing a comparison layout"
     ms_step = max_over_ranks(t0.elapsed_time(t1), world, "cuda") / args.steps
-    dom_ms = statistics.fmean(a.elapsed_time(b) for a, b in zip(starts, stops))
+    # with graphs the dominant kernel's time is the warm-up's (the hook records outside graphs)
+    dom_ms = (statistics.fmean(kern[dominant]) if graphs else
+              statistics.fmean(a.elapsed_time(b) for a, b in zip(starts, stops)))
     rl = roofline_for(w, dominant, dom_ms, peaks, peak_kind)
     rl.pop("traffic", None)
     out = {"workload": w.name, "H_q": w.Hq, "H_kv": w.Hkv, "ms_per_step": ms_step,
@@ -466,8 +564,11 @@ def run_ours(args, w):
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
     kern, dominant, dom_idx = warm_up(lib, w, sets, args.warmup, torch)
+    graphs = make_graphs(lib, w, sets, torch) if w.graph and not args.no_graph else None
 
-    # Timed region: K steps, per-step events around the dominant kernel.
+    # Timed region: K steps, per-step events around the dominant kernel (graph
+    # replays instead for launch-bound workloads; the dominant kernel's time is
+    # then the warm-up's).
     starts = [ev() for _ in range(args.steps)]
     stops = [ev() for _ in range(args.steps)]
     t0, t1 = ev(), ev()
@@ -479,8 +580,11 @@ def run_ours(args, w):
     wall0 = time.perf_counter()
     t0.record()
     for i in range(args.steps):
-        lib.set_timing_events(dom_idx, starts[i], stops[i])
-        step(lib, w, sets[i % n_sets])
+        if graphs:
+            graphs[i % n_sets].replay()
+        else:
+            lib.set_timing_events(dom_idx, starts[i], stops[i])
+            step(lib, w, sets[i % n_sets])
     t1.record()
     lib.set_timing_events(dom_idx)
     torch.cuda.synchronize()
@@ -489,7 +593,8 @@ def run_ours(args, w):
     wall = time.perf_counter() - wall0
     clk = clocks.stop()
     ms_total = max_over_ranks(t0.elapsed_time(t1), world, "cuda")
-    dom_ms = statistics.fmean(a.elapsed_time(b) for a, b in zip(starts, stops))
+    dom_ms = (statistics.fmean(kern[dominant]) if graphs else
+              statistics.fmean(a.elapsed_time(b) for a, b in zip(starts, stops)))
     assert lib.device_status() == 0, "a kernel wait gave up during the timed region"
     ms_step = ms_total / args.steps
     value = job_tflops(w, world, ms_step)
@@ -505,9 +610,9 @@ def run_ours(args, w):
     streams = [torch.cuda.Stream() for _ in range(n_pipe)]
     # (A decoding step's input is the new token's queries; its key/value cache
     # stays resident on the device, as in serving.)
-    in_names = ("q",) if w.decode else ("q", "k", "v", "dout")
+    in_names = ("x", "dy") if w.block else (("q",) if w.decode else ("q", "k", "v", "dout"))
     host_in = {n: sets[0][n].cpu().pin_memory() for n in in_names if n in sets[0]}
-    outs = ("out", "lse", "dq", "dk", "dv") if w.backward else ("out", "lse")
+    outs = ("y", "dx") if w.block else (("out", "lse", "dq", "dk", "dv") if w.backward else ("out", "lse"))
     host_out = [{n: torch.empty(sets[0][n].shape, dtype=sets[0][n].dtype, pin_memory=True) for n in outs}
                 for _ in range(n_pipe)]
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
@@ -546,7 +651,7 @@ def run_ours(args, w):
     line = None
     if rank == 0:
         line = {
-            "metric": f"SQA attention {pass_name(w)} TFLOP/s ({w.note})",
+            "metric": f"{metric_name(w)} {pass_name(w)} TFLOP/s ({w.note})",
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic (seeded Gaussian bf16 inputs)",
@@ -554,7 +659,10 @@ def run_ours(args, w):
                        "causal": w.causal, "pass": pass_name(w),
                        "parallelism": f"{world} independent replicas" if world > 1 else "single GPU",
                        "l2": f"{n_sets} rotating buffer sets of {set_bytes(first) / 2**20:.0f} MiB "
-                             f"(> L2 in total), no flush"},
+                             f"(> L2 in total), no flush",
+                       "launch": "CUDA-graph replay of each step" if graphs else "host launches",
+                       **({"d": w.d, "hidden": w.hidden, "layers": w.layers,
+                           "weights": "random, one set shared by every block"} if w.block else {})},
             "tokens_per_s": (w.B if w.decode else w.B * w.N) * world / (ms_step * 1e-3),
             "tensor_frac_of_bf16_peak": value / peaks["bf16_tflops"],
             "roofline": roofline_for(w, dominant, dom_ms, peaks, peak_kind),
@@ -562,9 +670,7 @@ def run_ours(args, w):
             "e2e": {"value": job_tflops(w, world, e2e_ms), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "streams": n_pipe,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            # fwd + bwd: the forward, the backward's preprocess, its main kernel and
-            # either the dQ conversion (dh <= 32) or the dQ kernel (dh 64 / 128)
-            "gpu_launches": args.steps * (4 if w.backward else (2 if w.decode else 1)),
+            "gpu_launches": args.steps * launches_per_step(w),
             "clocks": clk,
             "wall_s_timed_region": wall,
             # the CUDA sources this run was built from (profiles/traffic.json entries are keyed to it)
@@ -596,7 +702,7 @@ def run_reference(args, w):
         return None
     if not w.decode and (w.Hq // w.Hkv) * w.N * w.N * w.dh > 2 ** 34:  # one slice would take minutes: sample rows
         cb = cpu_baseline_rows(w, 60.0)
-        return {"impl": "reference", "metric": f"SQA attention {pass_name(w)} TFLOP/s ({w.note})",
+        return {"impl": "reference", "metric": f"{metric_name(w)} {pass_name(w)} TFLOP/s ({w.note})",
                 "value": cb["value"], "unit": "TFLOP/s", "n_gpus": world, "steps": 1, "warmup": 0,
                 "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f64", "data": "synthetic",
@@ -624,7 +730,7 @@ def run_reference(args, w):
     value = counted_flops(sub) / (ms * 1e-3) / 1e12
     sample = (f"fp64 oracle {pass_name(w)} on batch entry 0, KV head 0 and its {sub.Hq} "
               f"query heads (N={w.N}, dh={w.dh}); {steps} of the requested {args.steps} steps run")
-    return {"impl": "reference", "metric": f"SQA attention {pass_name(w)} TFLOP/s ({w.note})",
+    return {"impl": "reference", "metric": f"{metric_name(w)} {pass_name(w)} TFLOP/s ({w.note})",
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "N": w.N, "H_q": w.Hq, "H_kv": w.Hkv, "dh": w.dh,

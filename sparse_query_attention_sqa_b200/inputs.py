@@ -36,10 +36,18 @@ class Workload:
     scale: float = 0.0  # <= 0 selects 1/sqrt(dh)
     note: str = ""
     decode: bool = False  # one new query token per sequence against a cache of N positions
+    d: int = 0            # decoder-block stacks: model width, SwiGLU width, number of blocks
+    hidden: int = 0
+    layers: int = 0
+    graph: bool = False   # launch-bound: the benchmark replays each step as a CUDA graph
 
     @property
     def softmax_scale(self) -> float:
         return self.scale if self.scale > 0 else self.dh ** -0.5
+
+    @property
+    def block(self) -> bool:
+        return self.layers > 0
 
 
 # Workload shapes.  Each is one (B, N, H_q, H_kv, dh) point; sweeps list one
@@ -52,7 +60,7 @@ def _add(w: Workload):
 
 
 # SQAT-m single-layer attention, forward only.
-_add(Workload("sqatm_layer_fwd", 1, 1024, 8, 4, 16, True, False, scale=0.25,
+_add(Workload("sqatm_layer_fwd", 1, 1024, 8, 4, 16, True, False, scale=0.25, graph=True,
               note="SQAT-m single layer, B=1 N=1024 dh=16 Hq=8 Hkv=4 causal"))
 # SQAT-m training-step attention (forward + backward) and its same-kernel comparisons.
 for hq, hkv, tag in ((8, 4, "sqa"), (16, 4, "gqa"), (16, 16, "mha"), (16, 1, "mqa")):
@@ -77,6 +85,14 @@ for hq, hkv, tag in ((16, 16, "mha"), (16, 4, "gqa"), (16, 1, "mqa")):
 # The same head layout at 16384 tokens, small enough for full profiler captures.
 _add(Workload("large_dh128_16k", 1, 16384, 8, 4, 128, True, True, k_scale=0.1,
               note="larger model, B=1 N=16384 dh=128 Hq=8 Hkv=4 causal, K x 0.1"))
+# SQAT-m decoder-block stack (RMSNorm, the SQA layer with its projections and
+# the rotary embedding, SwiGLU 768; 8 blocks, d = 256, dh = 16, causal), one
+# forward and backward step with random weights (SQAT-m card, "Architecture
+# details"; its "Time per batch" table compares whole-model steps of the head
+# layouts), with the same comparisons as the training-step attention.
+for hq, hkv, tag in ((8, 4, "sqa"), (16, 4, "gqa"), (16, 16, "mha"), (16, 1, "mqa")):
+    _add(Workload(f"sqatm_block_{tag}", 32, 1024, hq, hkv, 16, True, True, d=256, hidden=768, layers=8, graph=True,
+                  note=f"SQAT-m 8-block stack, B=32 N=1024 d=256 dh=16 Hq={hq} Hkv={hkv} SwiGLU 768 causal"))
 # Decoding step: a batch of sequences, each adding one token against a full
 # key/value cache (SQAT-m head layout, and the larger-model dh=128 layout).
 _add(Workload("decode_sqatm", 32, 32768, 8, 4, 16, False, False, decode=True,
@@ -111,7 +127,10 @@ def make_decode_inputs(B: int, N: int, Hq: int, Hkv: int, dh: int, seed: int = 0
 
 
 def workload_inputs(w: Workload, seed: int = 0):
-    """(q, k, v, dout); for a decoding workload q is [B,Hq,dh] and dout is None."""
+    """(q, k, v, dout); for a decoding workload q is [B,Hq,dh] and dout is None;
+    for a block stack (x, weights, dy, None) from make_block_inputs."""
+    if w.block:
+        return (*make_block_inputs(w.B, w.N, w.d, w.Hq, w.Hkv, w.dh, w.hidden, seed=seed), None)
     if w.decode:
         return (*make_decode_inputs(w.B, w.N, w.Hq, w.Hkv, w.dh, seed=seed, std=w.std, k_scale=w.k_scale), None)
     return make_inputs(w.B, w.N, w.Hq, w.Hkv, w.dh, seed=seed, std=w.std, k_scale=w.k_scale,

@@ -100,3 +100,19 @@ def test_launched_kernel_names_the_decoding_path_that_runs():
     assert bench.launched_kernel(WORKLOADS["decode_mqa"], 2) == "sqa_decode_mma_kernel<16>"
     assert bench.launched_kernel(WORKLOADS["large_dh128"], 1) == "sqa_bwd_kernel<128>+sqa_bwd_q_kernel<128>"
     assert bench.launched_kernel(WORKLOADS["sqatm_train_sqa"], 1) == "sqa_bwd_tf32_kernel<16>"
+
+
+def test_block_stack_counts_attention_and_matrix_products():
+    from sparse_query_attention_sqa_b200.inputs import WORKLOADS
+
+    w = WORKLOADS["sqatm_block_sqa"]
+    attn = 4.0 * 32 * 8 * 1024 * 1024 * 16 / 2 * 3.5
+    params = 256 * (8 + 8) * 16 + 8 * 16 * 256 + 3 * 256 * 768
+    assert bench.block_gemm_params(w) == params
+    assert bench.counted_flops(w) == 8 * (attn + 2.0 * 32 * 1024 * params * 3)
+    assert bench.launches_per_step(w) == 8 * 27
+    assert bench.launches_per_step(WORKLOADS["large_dh128"]) == 4
+    assert bench.pass_name(w) == "8-block fwd+bwd"
+    # the MHA stack does the same matrix products as SQAT-m plus wider attention ones
+    m = WORKLOADS["sqatm_block_mha"]
+    assert bench.block_gemm_params(m) - params == 256 * (16 + 32 - 16) * 16 + 8 * 16 * 256
