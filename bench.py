@@ -351,9 +351,12 @@ def launched_kernel(w, hook: int) -> str:
     0 the forward, 1 the backward, 2 the decoding split kernel."""
     if hook == 0:
         return f"sqa_fwd_kernel<{w.dh}>"
-    if hook == 1:  # at dh 64 / 128 the hook brackets the dK/dV and the dQ kernels
-        return f"sqa_bwd_tf32_kernel<{w.dh}>" if w.dh <= 32 else f"sqa_bwd_kernel<{w.dh}>+sqa_bwd_q_kernel<{w.dh}>"
     g = w.Hq // w.Hkv
+    if hook == 1:  # at dh 64 / 128 the hook brackets the dK/dV and the dQ kernels
+        if w.dh <= 32:
+            return f"sqa_bwd_tf32_kernel<{w.dh}>"
+        lo = "true" if g >= 8 else "false"  # groups of 8+ carry P and dS as bf16 hi + lo
+        return f"sqa_bwd_kernel<{w.dh},{lo}>+sqa_bwd_q_kernel<{w.dh}>"
     if g <= 4 and (w.Hkv & (w.Hkv - 1)) == 0 and w.Hkv <= 2048 // w.dh:  # register-resident path
         return f"sqa_decode_split_kernel<{w.dh},{g}>"
     if 5 <= g <= 16:  # tensor-core path

@@ -451,11 +451,11 @@ sqa_status launch_bwd(const void* dout, const void* q, const void* k, const void
     pq.causal = causal;
     pq.scale_log2 = scale * kLog2e;
     pq.scale = scale;
-    if ((st = set_smem(sqa::sqa_bwd_kernel<D2>, Tr::SMEM_BYTES)) != SQA_OK) return st;
+    auto kern_kv = L.g >= sqa::kBwdSplitGroup ? sqa::sqa_bwd_kernel<D2, true> : sqa::sqa_bwd_kernel<D2, false>;
+    if ((st = set_smem(kern_kv, Tr::SMEM_BYTES)) != SQA_OK) return st;
     if ((st = set_smem(sqa::sqa_bwd_q_kernel<D2>, TQ::SMEM_BYTES)) != SQA_OK) return st;
     if ((st = record_timing(1, 0, stream)) != SQA_OK) return st;
-    sqa::sqa_bwd_kernel<D2><<<static_cast<unsigned>(grid_main), Tr::THREADS, Tr::SMEM_BYTES, stream>>>(mq, mdo, mk,
-                                                                                                     mv, p);
+    kern_kv<<<static_cast<unsigned>(grid_main), Tr::THREADS, Tr::SMEM_BYTES, stream>>>(mq, mdo, mk, mv, p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "sqa_bwd dK/dV launch");
     sqa::sqa_bwd_q_kernel<D2><<<static_cast<unsigned>(grid_q), TQ::THREADS, TQ::SMEM_BYTES, stream>>>(mk64, mv64,

@@ -12,7 +12,7 @@
 // TMEM, so no gradient goes through atomics at these head dims.
 //
 // ---------------------------------------------------------------------------
-// sqa_bwd_kernel<DH>: work item, one CTA each, a 128-key tile of one (batch,
+// sqa_bwd_kernel<DH, LO>: work item, one CTA each, a 128-key tile of one (batch,
 // KV head).  K and V stay in shared memory; the stacked Q tiles that see the
 // keys (the g query heads of the group, row r = t * g + head) stream through
 // two Q / dO stages.  Because a Q tile holds every head of the group, dV +=
@@ -21,8 +21,11 @@
 // tensor-core accumulation in TMEM (GQA summary, "The idea": the heads of a
 // group share one key and one value head).
 //
-//   TMEM  [0, 128)    S^T (fp32), rewritten in place as P^T (bf16 pairs)
-//         [128, 256)  dP^T (fp32), rewritten in place as dS^T (bf16 pairs)
+//   TMEM  [0, 128)    S^T (fp32), rewritten in place as P^T (bf16 pairs; for
+//                     groups of kBwdSplitGroup or more also the remainders,
+//                     in the columns the packed pairs leave)
+//         [128, 256)  dP^T (fp32), rewritten in place as dS^T (bf16 pairs, the
+//                     same way)
 //         [256, ...)  dV, then dK (fp32, dh columns each)
 //
 //   Per Q tile i, in the issuing thread's order (MMAs of one thread run in
@@ -50,6 +53,15 @@
 #include "sqa_tmem_wide.cuh"
 
 namespace sqa {
+
+// From this group size on, the dK / dV kernel carries P^T and dS^T as bf16
+// pairs hi + lo (split_bf16x2) and issues each dV / dK MMA twice.  Each dV or
+// dK element sums g rows of every Q tile, and under a causal mask the first
+// keys of a sequence take P near 1 from all g heads of the first tokens: with
+// P rounded once to bf16 (relative error up to 2^-9) a 16-head group puts
+// dV elements of magnitude 2-4 up to 0.03 off; the remainder brings that to
+// the 1e-5 range, for 1.5 times the tensor work of this kernel.
+constexpr int kBwdSplitGroup = 8;
 
 template <int DH>
 struct BwdBf16Traits {
@@ -84,7 +96,7 @@ struct BwdBf16Traits {
   static_assert(TM_DK + DH <= 512, "TMEM budget");
 };
 
-template <int DH>
+template <int DH, bool LO>
 __global__ void __launch_bounds__(384, 1)
     sqa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -242,7 +254,8 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t q_addr = sbase + Tr::OFF_Q + s * Tr::TILE, do_addr = sbase + Tr::OFF_DO + s * Tr::TILE;
       // dV += P^T dO: M = 128 keys, N = dh, K = the 64 query rows of one half in
       // steps of 16.  Warpgroup w packed the P^T of rows 64 hh + 32 w + [0, 32)
-      // into columns 64 hh + 32 w + [0, 16).
+      // into columns 64 hh + 32 w + [0, 16), with LO the remainders into
+      // 64 hh + 32 w + [16, 32): a second MMA on the same dO rows adds them.
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         if (!(ok = mbar_wait_warp(p_ready(hh), i & 1, abort_flag, kSiteMma))) break;
@@ -251,9 +264,9 @@ __global__ void __launch_bounds__(384, 1)
         for (int k4 = 0; k4 < 4; ++k4) {
           const uint32_t acol = 64u * hh + 32u * (k4 >> 1) + 8u * (k4 & 1);
           const uint32_t row0 = 64u * hh + 16u * k4;
-          mma_ts_w(tmem + Tr::TM_DV, tmem + Tr::TM_ST + acol,
-                   smem_desc(do_addr + row0 * ROWB, BM * ROWB, 8 * ROWB, Tr::LAYOUT), idesc_kv,
-                   (i > 0 || hh > 0 || k4 > 0) ? 1u : 0u);
+          const uint64_t bdesc = smem_desc(do_addr + row0 * ROWB, BM * ROWB, 8 * ROWB, Tr::LAYOUT);
+          mma_ts_w(tmem + Tr::TM_DV, tmem + Tr::TM_ST + acol, bdesc, idesc_kv, (i > 0 || hh > 0 || k4 > 0) ? 1u : 0u);
+          if constexpr (LO) mma_ts_w(tmem + Tr::TM_DV, tmem + Tr::TM_ST + acol + 16u, bdesc, idesc_kv, 1u);
         }
       }
       if (!ok) break;
@@ -270,9 +283,9 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int k8 = 0; k8 < 8; ++k8) {
         const uint32_t acol = 64u * (k8 >> 2) + 32u * ((k8 >> 1) & 1) + 8u * (k8 & 1);
-        mma_ts_w(tmem + Tr::TM_DK, tmem + Tr::TM_DPT + acol,
-                 smem_desc(q_addr + 16u * k8 * ROWB, BM * ROWB, 8 * ROWB, Tr::LAYOUT), idesc_kv,
-                 (i > 0 || k8 > 0) ? 1u : 0u);
+        const uint64_t bdesc = smem_desc(q_addr + 16u * k8 * ROWB, BM * ROWB, 8 * ROWB, Tr::LAYOUT);
+        mma_ts_w(tmem + Tr::TM_DK, tmem + Tr::TM_DPT + acol, bdesc, idesc_kv, (i > 0 || k8 > 0) ? 1u : 0u);
+        if constexpr (LO) mma_ts_w(tmem + Tr::TM_DK, tmem + Tr::TM_DPT + acol + 16u, bdesc, idesc_kv, 1u);
       }
       mma_commit_w(qd_empty(s));  // the last MMAs reading Q / dO of this stage
       // dP^T of the next tile, over the dS^T columns the dK MMAs just issued read first.
@@ -331,8 +344,15 @@ __global__ void __launch_bounds__(384, 1)
           pr[hh][e + 3] = lim > r4.w ? 0.f : ex2(x23.y);
         }
         uint32_t pk[16];
+        if constexpr (LO) {
+          uint32_t pl[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pr[hh][2 * e], pr[hh][2 * e + 1]);
+          for (int e = 0; e < 16; ++e) split_bf16x2(pr[hh][2 * e], pr[hh][2 * e + 1], pk[e], pl[e]);
+          tmem_st16(lane_addr + Tr::TM_ST + col0 + 16, pl);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(pr[hh][2 * e], pr[hh][2 * e + 1]);
+        }
         tmem_st16(lane_addr + Tr::TM_ST + col0, pk);
         tmem_wait_st();
         tc_fence_before();
@@ -349,7 +369,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int hh = 0; hh < 2; ++hh) {
         const int col0 = 64 * hh + 32 * w;
         const uint32_t* dr = dr2 + 32 * hh;
-        uint32_t dk[16];
+        uint32_t dk[16], dl[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           const float4 d4 = *reinterpret_cast<const float4*>(nd + col0 + e);
@@ -359,10 +379,16 @@ __global__ void __launch_bounds__(384, 1)
                                         make_float2(d4.z, d4.w));
           const float2 s01 = __fmul2_rn(make_float2(pr[hh][e], pr[hh][e + 1]), t01);
           const float2 s23 = __fmul2_rn(make_float2(pr[hh][e + 2], pr[hh][e + 3]), t23);
-          dk[e >> 1] = pack_bf16x2(s01.x, s01.y);
-          dk[(e >> 1) + 1] = pack_bf16x2(s23.x, s23.y);
+          if constexpr (LO) {
+            split_bf16x2(s01.x, s01.y, dk[e >> 1], dl[e >> 1]);
+            split_bf16x2(s23.x, s23.y, dk[(e >> 1) + 1], dl[(e >> 1) + 1]);
+          } else {
+            dk[e >> 1] = pack_bf16x2(s01.x, s01.y);
+            dk[(e >> 1) + 1] = pack_bf16x2(s23.x, s23.y);
+          }
         }
         tmem_st16(lane_addr + Tr::TM_DPT + col0, dk);
+        if constexpr (LO) tmem_st16(lane_addr + Tr::TM_DPT + col0 + 16, dl);
       }
       tmem_wait_st();
       tc_fence_before();

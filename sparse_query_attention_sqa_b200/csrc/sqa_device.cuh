@@ -297,6 +297,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+// A pair of values as two bf16 pairs whose sum carries 16 significant bits:
+// hi rounded to nearest, lo the rounded remainder (a - hi, b - hi').  A product
+// against a bf16 operand then loses only the rounding of lo, 2^-17 relative.
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16x2(a, b);
+  lo = pack_bf16x2(a - __uint_as_float(hi << 16), b - __uint_as_float(hi & 0xffff0000u));
+}
 
 
 // 2^x for a pair of values on the FMA pipe instead of the special-function

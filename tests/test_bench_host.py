@@ -98,7 +98,8 @@ def test_launched_kernel_names_the_decoding_path_that_runs():
     assert bench.launched_kernel(WORKLOADS["decode_sqatm"], 2) == "sqa_decode_split_kernel<16,2>"
     assert bench.launched_kernel(WORKLOADS["decode_dh128"], 2) == "sqa_decode_split_kernel<128,2>"
     assert bench.launched_kernel(WORKLOADS["decode_mqa"], 2) == "sqa_decode_mma_kernel<16>"
-    assert bench.launched_kernel(WORKLOADS["large_dh128"], 1) == "sqa_bwd_kernel<128>+sqa_bwd_q_kernel<128>"
+    assert bench.launched_kernel(WORKLOADS["large_dh128"], 1) == "sqa_bwd_kernel<128,false>+sqa_bwd_q_kernel<128>"
+    assert bench.launched_kernel(WORKLOADS["large_dh128_mqa"], 1) == "sqa_bwd_kernel<128,true>+sqa_bwd_q_kernel<128>"
     assert bench.launched_kernel(WORKLOADS["sqatm_train_sqa"], 1) == "sqa_bwd_tf32_kernel<16>"
 
 

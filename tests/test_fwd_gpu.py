@@ -25,10 +25,14 @@ SHAPES = [
     (1, 390, 8, 4, 64),
     (2, 300, 8, 4, 128),
     (1, 129, 4, 4, 128),
+    (1, 200, 16, 1, 128),  # MQA at dh 128: 8 tokens per Q tile
+    (2, 150, 12, 4, 128),  # g = 3: 126 of the 128 tile rows used
+    (1, 257, 12, 2, 64),
     # more work items than SMs, so every persistent CTA walks several items
     # (buffer and barrier phases carried across items), with ragged tails
     (6, 1000, 8, 4, 16),
     (26, 300, 8, 2, 32),
+    (4, 1216, 8, 4, 128),  # 160 forward items of 148 SMs: turns in CTAs that walk several items, one-tile items
 ]
 
 
