@@ -20,6 +20,11 @@ rotation, so every step reads its inputs from HBM.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--no-compare]
   python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
 
+Without --steps the number of timed steps follows from the warm-up's step time:
+about 20 s of timed work for the workload (at least 5 steps, at most 2000) and
+about 8 s for each comparison layout, so a run without flags ends within a few
+minutes; with --steps K exactly K steps are timed, comparisons included.
+
 Under torchrun every rank runs its own copy of the workload (independent
 batches, no collective on the data path): weak scaling.  One JSON line is
 printed by rank 0.
@@ -48,7 +53,8 @@ SFU_EXP2_PER_CLK_PER_SM = 16
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: about 20 s of the workload's warm-up step time)")
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="large_dh128")
@@ -466,25 +472,35 @@ def make_graphs(lib, w, sets, torch):
 
 def warm_up(lib, w, sets, warmup, torch):
     """Warm-up steps; each times its main kernels with the library's hook.
-    Returns ({kernel: [ms]}, the dominant kernel's name, its hook index)."""
+    Returns ({kernel: [ms]}, the dominant kernel's name, its hook index, the
+    median step time in ms)."""
     ev = lambda: torch.cuda.Event(enable_timing=True)
-    kern = {}
+    kern, steps_ms = {}, []
     hooks = (2,) if w.decode else ((0, 1) if w.backward else (0,))  # timing-hook indices: fwd, bwd, decode
     for i in range(max(warmup, 3)):
         s = sets[i % len(sets)]
         evs = {h: (ev(), ev()) for h in hooks}
         for h, (e0, e1) in evs.items():
             lib.set_timing_events(h, e0, e1)
+        a, b = ev(), ev()
+        a.record()
         step(lib, w, s)
+        b.record()
         for h in hooks:
             lib.set_timing_events(h)
         torch.cuda.synchronize()
+        steps_ms.append(a.elapsed_time(b))
         for h, (e0, e1) in evs.items():
             kern.setdefault(launched_kernel(w, h), []).append(e0.elapsed_time(e1))
     assert lib.device_status() == 0, "a kernel wait gave up during warm-up"
     dominant = max(kern, key=lambda n: statistics.median(kern[n]))
     dom_idx = next(h for h in hooks if launched_kernel(w, h) == dominant)
-    return kern, dominant, dom_idx
+    return kern, dominant, dom_idx, statistics.median(steps_ms)
+
+
+def auto_steps(step_ms: float, seconds: float) -> int:
+    """Timed steps that take about the given time at the warm-up's step time."""
+    return max(5, min(2000, int(seconds * 1e3 / max(step_ms, 1e-3))))
 
 
 def compare_variants(args, w):
@@ -512,14 +528,16 @@ def time_variant(args, lib, w, torch, world, rank, peaks, peak_kind):
     n_sets = max(2, math.ceil(2 * L2_BYTES / set_bytes(first)))
     sets = [first] + [alloc_set(w, q, k, v, dout, lib, torch) for _ in range(n_sets - 1)]
     del q, k, v, dout
-    kern, dominant, dom_idx = warm_up(lib, w, sets, args.warmup, torch)
+    kern, dominant, dom_idx, warm_ms = warm_up(lib, w, sets, args.warmup, torch)
     graphs = make_graphs(lib, w, sets, torch) if w.graph and not args.no_graph else None
-    starts = [ev() for _ in range(args.steps)]
-    stops = [ev() for _ in range(args.steps)]
+    n_steps = (auto_steps(max_over_ranks(warm_ms, world, "cuda"), 8.0) if getattr(args, "steps_auto", False)
+               else args.steps)
+    starts = [ev() for _ in range(n_steps)]
+    stops = [ev() for _ in range(n_steps)]
     t0, t1 = ev(), ev()
     torch.cuda.synchronize()
     t0.record()
-    for i in range(args.steps):
+    for i in range(n_steps):
         if graphs:
             graphs[i % n_sets].replay()
         else:
@@ -529,13 +547,13 @@ def time_variant(args, lib, w, torch, world, rank, peaks, peak_kind):
     lib.set_timing_events(dom_idx)
     torch.cuda.synchronize()
     assert lib.device_status() == 0, "a kernel wait gave up while timing a comparison layout"
-    ms_step = max_over_ranks(t0.elapsed_time(t1), world, "cuda") / args.steps
+    ms_step = max_over_ranks(t0.elapsed_time(t1), world, "cuda") / n_steps
     # with graphs the dominant kernel's time is the warm-up's (the hook records outside graphs)
     dom_ms = (statistics.fmean(kern[dominant]) if graphs else
               statistics.fmean(a.elapsed_time(b) for a, b in zip(starts, stops)))
     rl = roofline_for(w, dominant, dom_ms, peaks, peak_kind)
     rl.pop("traffic", None)
-    out = {"workload": w.name, "H_q": w.Hq, "H_kv": w.Hkv, "ms_per_step": ms_step,
+    out = {"workload": w.name, "H_q": w.Hq, "H_kv": w.Hkv, "steps": n_steps, "ms_per_step": ms_step,
            "value": job_tflops(w, world, ms_step), "unit": "TFLOP/s",
            "kernel_ms": {n: statistics.median(v) for n, v in kern.items()}, "roofline": rl}
     del sets
@@ -566,8 +584,11 @@ def run_ours(args, w):
     sets = [first] + [alloc_set(w, q, k, v, dout, lib, torch) for _ in range(n_sets - 1)]
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
-    kern, dominant, dom_idx = warm_up(lib, w, sets, args.warmup, torch)
+    kern, dominant, dom_idx, warm_ms = warm_up(lib, w, sets, args.warmup, torch)
     graphs = make_graphs(lib, w, sets, torch) if w.graph and not args.no_graph else None
+    if args.steps is None:  # every rank times the same number of steps
+        args.steps = auto_steps(max_over_ranks(warm_ms, world, "cuda"), 20.0)
+        args.steps_auto = True
 
     # Timed region: K steps, per-step events around the dominant kernel (graph
     # replays instead for launch-bound workloads; the dominant kernel's time is
@@ -722,7 +743,8 @@ def run_reference(args, w):
     one = time.perf_counter() - t
     budget = 150.0
     warm = min(args.warmup, max(0, int(0.1 * budget / one)))
-    steps = max(1, min(args.steps, int(0.9 * budget / one)))
+    requested = args.steps if args.steps is not None else 2000
+    steps = max(1, min(requested, int(0.9 * budget / one)))
     for _ in range(warm):
         run_oracle_step(sub, data)
     t0 = time.perf_counter()
@@ -732,7 +754,7 @@ def run_reference(args, w):
     ms = el / steps * 1e3
     value = counted_flops(sub) / (ms * 1e-3) / 1e12
     sample = (f"fp64 oracle {pass_name(w)} on batch entry 0, KV head 0 and its {sub.Hq} "
-              f"query heads (N={w.N}, dh={w.dh}); {steps} of the requested {args.steps} steps run")
+              f"query heads (N={w.N}, dh={w.dh}); {steps} of the requested {requested} steps run")
     return {"impl": "reference", "metric": f"{metric_name(w)} {pass_name(w)} TFLOP/s ({w.note})",
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",

@@ -360,9 +360,6 @@ sqa_status launch_bwd(const void* dout, const void* q, const void* k, const void
   pp.lse2 = lse2;
   pp.D = Dst;
   pp.dq_acc = dq_acc;
-  pp.q = static_cast<const __nv_bfloat16*>(q);
-  pp.q32 = DH <= 32 ? reinterpret_cast<float*>(ws + L.off_q32) : nullptr;
-  pp.do32 = DH <= 32 ? reinterpret_cast<float*>(ws + L.off_do32) : nullptr;
   pp.N = s.N;
   pp.Hq = s.H_q;
   pp.Hkv = s.H_kv;
@@ -390,8 +387,6 @@ sqa_status launch_bwd(const void* dout, const void* q, const void* k, const void
   p.lse2 = lse2;
   p.D = Dst;
   p.dq_acc = dq_acc;
-  p.q32 = pp.q32;
-  p.do32 = pp.do32;
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.N = s.N;

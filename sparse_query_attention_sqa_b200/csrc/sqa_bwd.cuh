@@ -6,8 +6,7 @@
 //   1. prep:  -D_i = -<dO_i, O_i> and -lse_i * log2(e) for every query row,
 //             written in the stacked-tile order the main kernel reads (slots of
 //             padding rows get lse = +inf and D = 0, which makes their P exactly
-//             0), the fp32 dQ accumulator zeroed, and for dh <= 32 transposed
-//             fp32 images of the Q and dO tiles (tf32 MMA operands).
+//             0), and for dh <= 32 the fp32 dQ accumulator zeroed.
 //   2. main:  work item = (128-key tile, batch, KV head).  K and V stay in
 //             shared memory while the Q tiles that see those keys stream by.  A
 //             Q tile stacks the g query heads of the group (row r = t * g +
@@ -40,8 +39,6 @@ struct BwdLayout {
   size_t n_slots;     // B * H_kv * n_qt * 128
   size_t off_D;       // byte offsets inside the workspace
   size_t off_dq;       // dh <= 32 only: the fp32 dQ accumulator
-  size_t off_q32;     // dh <= 32 only: fp32 transposed images of the stacked Q and dO tiles
-  size_t off_do32;
   size_t bytes;
 };
 
@@ -56,13 +53,8 @@ inline BwdLayout bwd_layout(int B, int N, int Hq, int Hkv, int dh) {
   L.off_D = align256(L.n_slots * sizeof(float));
   L.off_dq = L.off_D + align256(L.n_slots * sizeof(float));
   L.bytes = L.off_dq;
-  if (dh <= 32) {  // dh 64 / 128: dQ comes from its own kernel, with no accumulator
+  if (dh <= 32)  // dh 64 / 128: dQ comes from its own kernel, with no accumulator
     L.bytes += align256(static_cast<size_t>(B) * N * Hq * dh * sizeof(float));
-    const size_t img = align256(L.n_slots * dh * sizeof(float));
-    L.off_q32 = L.bytes;
-    L.off_do32 = L.bytes + img;
-    L.bytes += 2 * img;
-  }
   return L;
 }
 
@@ -75,27 +67,14 @@ inline size_t bwd_workspace_bytes(int B, int N, int Hq, int Hkv, int dh) {
 struct BwdPrepParams {
   const __nv_bfloat16* dout;
   const __nv_bfloat16* out;
-  const __nv_bfloat16* q;
   const float* lse;
   float* lse2;
   float* D;
   float* dq_acc;
-  float* q32;   // null, or the fp32 tile images (see below)
-  float* do32;
   int N, Hq, Hkv, g, T, rows, n_qt;
   long long n_slots;
   long long dq_vec4;  // dq accumulator length / 4
 };
-
-// Offset (in floats) of element (row r, column n) inside the fp32 image of one
-// stacked 128-row tile: the tile transposed to [dh][128] and cut into four
-// panels of 32 rows, each panel dh lines of 128 bytes with the 128-byte swizzle
-// (16-byte chunk c of line n stored at chunk c ^ (n % 8)).  This is the K-major
-// operand layout of a tf32 MMA whose contraction runs over the tile's rows, so
-// the image is copied to shared memory as is.
-__host__ __device__ __forceinline__ int tf32_image_index(int r, int n, int dh) {
-  return (r >> 5) * dh * 32 + n * 32 + ((((r & 31) >> 2) ^ (n & 7)) << 2) + (r & 3);
-}
 
 template <int DH>
 __global__ void __launch_bounds__(256) sqa_bwd_prep_kernel(const BwdPrepParams p) {
@@ -110,8 +89,6 @@ __global__ void __launch_bounds__(256) sqa_bwd_prep_kernel(const BwdPrepParams p
     const int tok = qt * p.T + r / p.g;
     float l2 = INFINITY, d = 0.f;
     const bool live = r < p.rows && tok < p.N;
-    float* qi = p.q32 ? p.q32 + (s - r) * DH : nullptr;
-    float* di = p.q32 ? p.do32 + (s - r) * DH : nullptr;
     if (live) {
       const int head = kvh * p.g + r % p.g;
       const size_t row = (static_cast<size_t>(b) * p.N + tok) * p.Hq + head;
@@ -127,30 +104,9 @@ __global__ void __launch_bounds__(256) sqa_bwd_prep_kernel(const BwdPrepParams p
           const float2 fa = __bfloat1622float2(a2[e]), fb = __bfloat1622float2(b2[e]);
           d = fmaf(fa.x, fb.x, d);
           d = fmaf(fa.y, fb.y, d);
-          if (DH <= 32 && di) {
-            di[tf32_image_index(r, 8 * c + 2 * e, DH)] = fb.x;
-            di[tf32_image_index(r, 8 * c + 2 * e + 1, DH)] = fb.y;
-          }
-        }
-      }
-      if (DH <= 32 && qi) {
-        const uint4* qr = reinterpret_cast<const uint4*>(p.q + row * DH);
-#pragma unroll
-        for (int c = 0; c < DH / 8; ++c) {
-          const uint4 a = qr[c];
-          const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 fa = __bfloat1622float2(a2[e]);
-            qi[tf32_image_index(r, 8 * c + 2 * e, DH)] = fa.x;
-            qi[tf32_image_index(r, 8 * c + 2 * e + 1, DH)] = fa.y;
-          }
         }
       }
       l2 = p.lse[(static_cast<size_t>(b) * p.Hq + head) * p.N + tok] * 1.4426950408889634f;
-    } else if (DH <= 32 && qi) {
-#pragma unroll
-      for (int n = 0; n < DH; ++n) qi[tf32_image_index(r, n, DH)] = di[tf32_image_index(r, n, DH)] = 0.f;
     }
     // Stored negated: the main kernels add them (x = S * scale * log2(e) - lse2, dP - D).
     p.lse2[s] = -l2;
@@ -183,8 +139,6 @@ struct BwdParams {
   const float* lse2;  // stacked [B*H_kv][n_qt][128], negated: -lse * log2(e) (-inf on padding rows)
   const float* D;     // negated: -<dO, O> (0 on padding rows)
   float* dq_acc;      // [B][N][H_q][dh] fp32
-  const float* q32;   // dh <= 32: fp32 images of the stacked Q and dO tiles
-  const float* do32;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int N, Hq, Hkv, g, T, rows, n_qt, n_bh, causal;

@@ -12,8 +12,10 @@
 //
 //  * dV += P^T dO and dK += dS^T Q run as tf32 MMAs with K-major operands (tf32
 //    operands stored MN-major produced zeros on this hardware).  P^T and dS^T
-//    stay in fp32 in TMEM, in place; the transposed fp32 copies of the Q and dO
-//    tiles come ready-made from the prep kernel and are bulk-copied.  dS is
+//    stay in fp32 in TMEM, in place; the transposed fp32 copies of the dO and Q
+//    tiles are built in shared memory from the bf16 tiles by the DV and DK
+//    issuing warps themselves, while the softmax warps work on the tile's
+//    first half (the issuers are otherwise waiting for them).  dS is
 //    rounded to tf32 (to nearest), P is passed as is.  tf32 keeps bf16's
 //    exponent range and three more mantissa bits, which matters when a large
 //    query group sums many terms into one dK or dV row.  dQ = dS K sums only
@@ -35,8 +37,9 @@
 // Roles (384 threads):
 //   warps 0-7   P^T / dS^T (warpgroup w: half w of each Q tile), the dQ
 //               epilogue (fp32 atomics) and the dK / dV epilogue
-//   warp 8      TMA producer (K, V once; Q, dO, their fp32 images, lse2, D per Q tile)
-//   warp 9      TMEM allocator and MMA issuer A; warp 10 issuer DV; warp 11 issuer DK
+//   warp 8      TMA producer (K, V once; Q, dO, lse2, D per Q tile)
+//   warp 9      TMEM allocator and MMA issuer A; warp 10 issuer DV (and the dO
+//               images); warp 11 issuer DK (and the Q images)
 // TMEM: buffer x (0..2): S^T at 128 x, dP^T at 128 x + 64 (64 columns each);
 // dV at 384, dK at 416, dQ of Q tile i at 448 + 32 (i % 2).
 // The softmax statistics arrive negated (-lse * log2 e and -D), so they are added.
@@ -74,6 +77,41 @@ __device__ __forceinline__ void mma_ts_tf32_w(uint32_t d_tmem, uint32_t a_tmem, 
       : "memory");
 }
 }  // namespace dev
+
+// Offset (in floats) of element (row r, column n) inside the fp32 image of one
+// stacked 128-row tile: the tile transposed to [dh][128] and cut into four
+// panels of 32 rows, each panel dh lines of 128 bytes with the 128-byte swizzle
+// (16-byte chunk c of line n stored at chunk c ^ (n % 8)).  This is the K-major
+// operand layout of a tf32 MMA whose contraction runs over the tile's rows.
+__host__ __device__ __forceinline__ int tf32_image_index(int r, int n, int dh) {
+  return (r >> 5) * dh * 32 + n * 32 + ((((r & 31) >> 2) ^ (n & 7)) << 2) + (r & 3);
+}
+
+// The fp32 image of a bf16 tile as the tensor map wrote it into shared memory
+// (row r at r * 2 dh bytes, its 16-byte chunks permuted by the 32-byte swizzle
+// at dh 16 and the 64-byte one at dh 32: byte offset o is stored at
+// o ^ (((o >> 7) & m) << 4), m = 1 or 3), by the 32 lanes of one warp: lane l
+// takes rows l, l + 32, l + 64, l + 96.  For a fixed column the 32 lanes write
+// the 32 words of one 128-byte line, so the stores are free of bank conflicts.
+template <int DH>
+__device__ __forceinline__ void to_tf32_image(const uint8_t* src, float* dst, int lane) {
+  constexpr uint32_t ROWB = DH * 2, M = DH == 16 ? 1u : 3u;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = 32 * k + lane;
+#pragma unroll
+    for (int c = 0; c < DH / 8; ++c) {
+      const uint32_t o = r * ROWB + 16u * c;
+      const uint4 v = *reinterpret_cast<const uint4*>(src + (o ^ (((o >> 7) & M) << 4)));
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {  // a bf16 is the upper half of its fp32 value
+        dst[tf32_image_index(r, 8 * c + 2 * e, DH)] = __uint_as_float(wv[e] << 16);
+        dst[tf32_image_index(r, 8 * c + 2 * e + 1, DH)] = __uint_as_float(wv[e] & 0xffff0000u);
+      }
+    }
+  }
+}
 
 template <int DH>
 struct BwdTf32Traits {
@@ -259,7 +297,7 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_map(&tmDO);
       tma_prefetch_map(&tmK);
       tma_prefetch_map(&tmV);
-      const uint32_t qd_bytes = 2u * p.rows * ROWB + 2u * 512u + 2u * Tr::TILE32;
+      const uint32_t qd_bytes = 2u * p.rows * ROWB + 2u * 512u;
       int gt = 0, items_issued = 0, tiles_issued = 0;
       bool ok = true;
       for (int r = 0, item; ok && (item = snake_item(r, p.n_items)) >= 0; ++r) {
@@ -282,8 +320,6 @@ __global__ void __launch_bounds__(384, 1)
           const size_t slot = (static_cast<size_t>(it.bh) * p.n_qt + qt) * kBwdTile;
           bulk_load(sbase + Tr::OFF_STAT + s * 1024, p.lse2 + slot, 512, qd_full(s));
           bulk_load(sbase + Tr::OFF_STAT + s * 1024 + 512, p.D + slot, 512, qd_full(s));
-          bulk_load(sbase + Tr::OFF_Q32 + s * Tr::TILE32, p.q32 + slot * DH, Tr::TILE32, qd_full(s));
-          bulk_load(sbase + Tr::OFF_DO32 + s * Tr::TILE32, p.do32 + slot * DH, Tr::TILE32, qd_full(s));
           tiles_issued = G + 1;
         }
         gt += it.nq;
@@ -374,11 +410,21 @@ __global__ void __launch_bounds__(384, 1)
       const BwdItem it = bwd_decode(p, item);
       for (int hl = 0; hl < 2 * it.nq; ++hl) {
         const int G = gt + (hl >> 1), H = 2 * gt + hl, s = G % QS, x = H % NBUF;
+        if ((hl & 1) == 0) {
+          // This warp's fp32 image of tile G (dO for DV, Q for DK), built while
+          // the softmax warps work on the tile.  The stage's previous image was
+          // last read by this warp's MMAs of tile G - QS, which completed before
+          // the producer could refill the stage (qd_empty), so before qd_full.
+          if (!(ok = mbar_wait_warp(qd_full(s), (G / QS) & 1, abort_flag, kSiteMma))) break;
+          to_tf32_image<DH>(smem + (is_dv ? Tr::OFF_DO : Tr::OFF_Q) + s * Tr::TILE,
+                            reinterpret_cast<float*>(smem + (is_dv ? Tr::OFF_DO32 : Tr::OFF_Q32) + s * Tr::TILE32),
+                            lane);
+          fence_async_smem();  // the image, to the tensor core's reads
+          __syncwarp();
+        }
         if (!(ok = mbar_wait_warp(ds_ready(x), (H / NBUF) & 1, abort_flag, kSiteMma))) break;
         // The accumulators still hold the previous item until its epilogue has read them.
         if (hl == 0 && r > 0 && !(ok = mbar_wait_warp(dkv_free, (r - 1) & 1, abort_flag, kSiteMma))) break;
-        // The image arrived with the Q tile (already complete: the warpgroups waited for it).
-        if ((hl & 1) == 0 && !(ok = mbar_wait_warp(qd_full(s), (G / QS) & 1, abort_flag, kSiteMma))) break;
         tc_fence_after();
         // K = 8 query rows per tf32 MMA: rows q0..q0+7 are 32 bytes at offset
         // (q0 % 32) * 4 of panel q0 / 32 of the image.

@@ -187,8 +187,7 @@ def test_plain_c_client_builds_links_and_runs(lib, tmp_path):
 def _bwd_ws_expected(B, N, Hq, Hkv, dh):
     """Workspace rule of sqa_bwd: -lse*log2(e) and -D per stacked-tile slot
     (B * H_kv * n_qtiles * 128 fp32 each); for dh <= 32 also the fp32 dQ
-    accumulator [B][N][H_q][dh] and fp32 images of every stacked Q and dO tile
-    (dh floats per slot each; at dh 64 and 128 dQ comes from its own kernel
+    accumulator [B][N][H_q][dh] (at dh 64 and 128 dQ comes from its own kernel
     with no accumulator); every part rounded up to 256 bytes."""
     def a256(x):
         return -(-x // 256) * 256
@@ -198,7 +197,7 @@ def _bwd_ws_expected(B, N, Hq, Hkv, dh):
     slots = B * Hkv * -(-N // T) * 128
     total = 2 * a256(slots * 4)
     if dh <= 32:
-        total += a256(B * N * Hq * dh * 4) + 2 * a256(slots * dh * 4)
+        total += a256(B * N * Hq * dh * 4)
     return total
 
 

@@ -117,3 +117,14 @@ def test_block_stack_counts_attention_and_matrix_products():
     # the MHA stack does the same matrix products as SQAT-m plus wider attention ones
     m = WORKLOADS["sqatm_block_mha"]
     assert bench.block_gemm_params(m) - params == 256 * (16 + 32 - 16) * 16 + 8 * 16 * 256
+
+
+def test_default_step_count_follows_the_warm_up_time():
+    """Without --steps the timed region lasts about the given time: 20 s of
+    68.5 ms steps is 291 steps; very short steps stop at 2000, very long ones
+    keep at least 5."""
+    import bench
+
+    assert bench.auto_steps(68.5, 20.0) == 291
+    assert bench.auto_steps(0.01, 20.0) == 2000
+    assert bench.auto_steps(10_000.0, 20.0) == 5

@@ -34,7 +34,11 @@ WARPS = 4 * NWG
 # Stages of every version of each buffer: (who, number of users).
 STAGES = {
     "kv": [("producer writes K, V", 1), ("issuer A reads", 1)],
-    "stage": [("producer writes Q, dO, images, stats", 1), ("issuer A, DV, DK and the warps read", 3 + WARPS)],
+    "stage": [("producer writes Q, dO, stats", 1), ("issuer A, DV, DK and the warps read", 3 + WARPS)],
+    # the fp32 image of a stage's dO (Q): built by the DV (DK) warp from the
+    # bf16 tile, read by that warp's MMAs
+    "img_acc_dv": [("DV converts dO", 1), ("DV MMAs read", 1)],
+    "img_acc_dk": [("DK converts Q", 1), ("DK MMAs read", 1)],
     "S": [("issuer A writes S^T, dP^T", 1), ("the half's warpgroup rewrites P^T, dS^T", 4), ("DV and DK read", 2)],
     "dsbuf": [("warps write dS", WARPS), ("issuer A reads (dQ)", 1)],
     "dqtm": [("issuer A writes dQ", 1), ("warps read dQ", WARPS)],
@@ -131,19 +135,23 @@ def _roles(nqs, QS):
     def kv_issuer(acc):  # DV and DK issuers: the same sequence on their own accumulator
         ops, gt = [], 0
         for r, nq in enumerate(nqs):
+            img = "img_" + acc
             for hl in range(2 * nq):
                 G, H = gt + (hl >> 1), 2 * gt + hl
                 s, x = G % QS, H % NBUF
+                if hl % 2 == 0:  # the tile's fp32 image, from the bf16 tile
+                    ops += [W(f"qd_full{s}", G // QS), B("stage", s, G, 1), B(img, s, G, 0), E(img, s, G, 0),
+                            E("stage", s, G, 1)]
                 ops.append(W(f"ds_ready{x}", H // NBUF))
                 if hl == 0 and r > 0:
                     ops.append(W("dkv_free", r - 1))
                 if hl == 0:
                     ops.append(B(acc, 0, r, 0))
                 if hl % 2 == 0:
-                    ops += [W(f"qd_full{s}", G // QS), B("stage", s, G, 1)]
+                    ops.append(B(img, s, G, 1))
                 ops += [B("S", x, H, 2), E("S", x, H, 2), A(f"kvmma_done{x}")]
                 if hl % 2 == 1:
-                    ops += [E("stage", s, G, 1), A(f"qd_empty{s}")]
+                    ops += [E(img, s, G, 1), A(f"qd_empty{s}")]
             ops += [E(acc, 0, r, 0), A("dkv_final")]
             gt += nq
         return ops
@@ -226,6 +234,10 @@ DROPS = {
     "warps: s_full": _drop_wait("warp", "s_full"),
     # issuer A's dQ MMA would read dS before every warp wrote it
     "issuer A: dsq_ready": _drop_wait("issuer_a", "dsq_ready"),
+    # DV / DK would build an fp32 image from a bf16 tile that has not landed,
+    # over the image their MMAs of tile G - QS may still read
+    "dv: qd_full": _drop_wait("dv", "qd_full"),
+    "dk: qd_full": _drop_wait("dk", "qd_full"),
 }
 
 
