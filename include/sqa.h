@@ -67,6 +67,34 @@ sqa_status sqa_fwd(const void *q, const void *k, const void *v, void *out, float
                    int causal, float scale, sqa_stream_t stream);
 
 /*
+ * Bytes of device scratch that sqa_fwd_with_workspace uses for shape s: 0 for
+ * every shape except small ones (dh <= 64, B * H_kv * ceil(N / T) Q tiles of
+ * T = floor(128 / g) tokens filling less than half the device's SMs), whose
+ * key tiles are then split into ranges run by separate CTAs: per range and
+ * stacked row, dh + 1 fp32 partial values, and one int counter per stacked row.
+ * The answer depends on the SM count of the current device (148 when none can
+ * be queried).
+ */
+size_t sqa_fwd_workspace_bytes(sqa_shape s, int causal);
+
+/*
+ * sqa_fwd with scratch (same definition, arguments and results).  With
+ * sqa_fwd_workspace_bytes(s, causal) > 0, workspace (256-byte aligned, at least
+ * that many bytes, contents arbitrary) takes the ranges' partial outputs and
+ * log-sum-exps; each row's ranges are merged by the CTA that finishes the last
+ * of them (its counter, cleared by an asynchronous memset on `stream` before the
+ * kernel, says which).  The partials are normalised within their range, so the
+ * merge is O = sum_c 2^(L_c - M) O_c / sum_c 2^(L_c - M) in fp32.  With 0 bytes
+ * needed, workspace may be NULL and the call is sqa_fwd.  Errors: those of
+ * sqa_fwd; SQA_ERR_INVALID_ARG for a null or too small workspace when one is
+ * needed, SQA_ERR_UNSUPPORTED for a misaligned one.  The workspace must not be
+ * used by another call until this one has completed on `stream`.
+ */
+sqa_status sqa_fwd_with_workspace(const void *q, const void *k, const void *v, void *out, float *lse,
+                                  void *workspace, size_t workspace_bytes, sqa_shape s, int causal,
+                                  float scale, sqa_stream_t stream);
+
+/*
  * Bytes of device scratch that sqa_bwd needs for shape s (fp32 dQ accumulator
  * plus per-row softmax statistics).  The caller allocates it; 256-byte aligned.
  */

@@ -56,6 +56,10 @@ def load_library():
     vp, fp, c_int, c_float, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.sqa_fwd.argtypes = [vp, vp, vp, vp, fp, Shape, c_int, c_float, vp]
     lib.sqa_fwd.restype = c_int
+    lib.sqa_fwd_workspace_bytes.argtypes = [Shape, c_int]
+    lib.sqa_fwd_workspace_bytes.restype = sz
+    lib.sqa_fwd_with_workspace.argtypes = [vp, vp, vp, vp, fp, vp, sz, Shape, c_int, c_float, vp]
+    lib.sqa_fwd_with_workspace.restype = c_int
     lib.sqa_bwd_workspace_bytes.argtypes = [Shape]
     lib.sqa_bwd_workspace_bytes.restype = sz
     lib.sqa_bwd.argtypes = [vp, vp, vp, vp, vp, fp, vp, vp, vp, vp, sz, Shape, c_int, c_float, vp]
@@ -122,9 +126,17 @@ def shape_of(q, k) -> Shape:
     return Shape(B, N, Hq, Hkv, dh)
 
 
-def sqa_fwd(q, k, v, out=None, lse=None, causal: bool = False, scale: float = 0.0, stream=None):
+def fwd_workspace_bytes(B: int, N: int, H_q: int, H_kv: int, dh: int, causal: bool) -> int:
+    return int(load_library().sqa_fwd_workspace_bytes(Shape(B, N, H_q, H_kv, dh), int(bool(causal))))
+
+
+def sqa_fwd(q, k, v, out=None, lse=None, causal: bool = False, scale: float = 0.0, stream=None, workspace=None,
+            key_ranges: bool = True):
     """Forward.  q [B,N,H_q,dh], k/v [B,N,H_kv,dh] bf16 CUDA tensors.
-    Returns (out [B,N,H_q,dh] bf16, lse [B,H_q,N] fp32).  scale <= 0 means 1/sqrt(dh)."""
+    Returns (out [B,N,H_q,dh] bf16, lse [B,H_q,N] fp32).  scale <= 0 means 1/sqrt(dh).
+    Small problems split each Q tile's keys into ranges over several CTAs when
+    key_ranges is true (sqa_fwd_with_workspace); workspace: a uint8 CUDA tensor
+    of at least fwd_workspace_bytes(...) bytes, or None to allocate one."""
     import torch
 
     lib = load_library()
@@ -140,8 +152,18 @@ def sqa_fwd(q, k, v, out=None, lse=None, causal: bool = False, scale: float = 0.
         lse = torch.empty((s.B, s.H_q, s.N), dtype=torch.float32, device=q.device)
     _need(out, "out", (s.B, s.N, s.H_q, s.dh), torch.bfloat16)
     _need(lse, "lse", (s.B, s.H_q, s.N), torch.float32)
-    _check(lib.sqa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), s,
-                       int(bool(causal)), float(scale), _stream(stream)))
+    need = int(lib.sqa_fwd_workspace_bytes(s, int(bool(causal)))) if key_ranges else 0
+    if need == 0:
+        _check(lib.sqa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), s,
+                           int(bool(causal)), float(scale), _stream(stream)))
+        return out, lse
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace.dtype != torch.uint8 or not workspace.is_cuda or workspace.numel() < need:
+        raise ValueError(f"workspace must be a uint8 CUDA tensor of at least {need} bytes")
+    _check(lib.sqa_fwd_with_workspace(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                      workspace.data_ptr(), workspace.numel(), s, int(bool(causal)),
+                                      float(scale), _stream(stream)))
     return out, lse
 
 

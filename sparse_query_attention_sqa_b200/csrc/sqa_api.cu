@@ -3,6 +3,7 @@
 // stream.  This is the only translation unit of libsqa.so.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdarg>
@@ -120,9 +121,74 @@ int sm_count() {
   return sms;
 }
 
+// SMs of the current device (148 on B200; also the answer when no device can
+// be queried, so that workspace sizes can be computed without a GPU).
+int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                cudaSuccess || sms <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return sms;
+}
+
+// How the forward splits its work.  Pairs of Q tiles per CTA; for problems
+// whose pairs would fill less than half the SMs, one Q tile per CTA with its
+// key tiles shared between the two tile slots (split mode, dh <= 64); and when
+// even single Q tiles fill less than half the SMs and the caller gives a
+// workspace, ranges of `chunk` key tiles of a Q tile as separate work items,
+// merged by the last range to finish.  chunk: the smallest even count whose
+// items do not outnumber the SMs (a second item on an SM costs more than
+// longer ranges).  Ranges are used only if they shorten the longest Q tile's
+// walk by at least kMinRangeSaving key tiles per slot: the memset (a second
+// node when a step is replayed as a graph), the partials and the merge cost
+// about as much as four to six key-tile steps.
+struct FwdPlan {
+  int g, T, n_qtiles, n_pairs, n_bh, split, chunk, nch_max;
+  long long items;
+  size_t part_off, part_l_off, cnt_off, ws_bytes;
+};
+
+FwdPlan fwd_plan(const sqa_shape& s, int causal, int sms, bool ranges_allowed) {
+  FwdPlan P{};
+  const int NK = s.dh == 128 ? 128 : 64;
+  P.g = s.H_q / s.H_kv;
+  P.T = 128 / P.g;
+  P.n_qtiles = (s.N + P.T - 1) / P.T;
+  P.n_pairs = (P.n_qtiles + 1) / 2;
+  P.n_bh = s.B * s.H_kv;
+  P.split = (s.dh <= 64 && static_cast<long long>(P.n_pairs) * P.n_bh < sms / 2) ? 1 : 0;
+  P.items = static_cast<long long>(P.split ? P.n_qtiles : P.n_pairs) * P.n_bh;
+  if (!P.split || !ranges_allowed || static_cast<long long>(P.n_qtiles) * P.n_bh >= sms / 2) return P;
+  auto nkv_of = [&](int qt) {
+    const long long end = causal ? std::min<long long>(s.N, static_cast<long long>(qt + 1) * P.T) : s.N;
+    return static_cast<int>((end + NK - 1) / NK);
+  };
+  constexpr int kMinRangeSaving = 6;
+  const int nkv_max = nkv_of(P.n_qtiles - 1);
+  auto items_of = [&](int chunk) {
+    long long n = 0;
+    for (int qt = 0; qt < P.n_qtiles; ++qt) n += (nkv_of(qt) + chunk - 1) / chunk;
+    return n * P.n_bh;
+  };
+  int chunk = 2;
+  while (chunk < nkv_max && items_of(chunk) > sms) chunk += 2;
+  if ((nkv_max + 1) / 2 - chunk / 2 < kMinRangeSaving) return P;
+  P.chunk = chunk;
+  P.nch_max = (nkv_max + chunk - 1) / chunk;
+  P.items = items_of(chunk);
+  const size_t slots = static_cast<size_t>(P.n_bh) * P.n_qtiles * P.nch_max * 128;
+  P.part_off = 0;
+  P.part_l_off = sqa::align256(slots * s.dh * sizeof(float));
+  P.cnt_off = P.part_l_off + sqa::align256(slots * sizeof(float));
+  P.ws_bytes = P.cnt_off + sqa::align256(static_cast<size_t>(P.n_bh) * P.n_qtiles * 128 * sizeof(int));
+  return P;
+}
+
 template <int DH>
 sqa_status launch_fwd(const void* q, const void* k, const void* v, void* out, float* lse, const sqa_shape& s,
-                      int causal, float scale, cudaStream_t stream) {
+                      int causal, float scale, cudaStream_t stream, void* workspace = nullptr) {
   using Tr = sqa::FwdTraits<DH>;
   sqa::FwdParams p{};
   p.out = static_cast<__nv_bfloat16*>(out);
@@ -142,13 +208,23 @@ sqa_status launch_fwd(const void* q, const void* k, const void* v, void* out, fl
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return cuda_fail(e, "querying the SM count");
-  // Small problems, whose pairs of Q tiles would fill less than half the SMs:
-  // one Q tile per CTA, its key tiles shared between the two tile slots
-  // (needs a K/V ring of at least four stages: dh <= 64).
-  p.split = (DH <= 64 && static_cast<long long>(p.n_pairs) * p.n_bh < sms / 2) ? 1 : 0;
-  const long long items = static_cast<long long>(p.split ? p.n_qtiles : p.n_pairs) * p.n_bh;
+  // Split mode (one Q tile per CTA, key tiles shared by the two slots) needs a
+  // K/V ring of at least four stages: dh <= 64.  Key ranges need the workspace.
+  const FwdPlan P = fwd_plan(s, causal, sms, workspace != nullptr);
+  p.split = P.split;
+  const long long items = P.items;
   if (items > 0x7fffffffLL) return fail(SQA_ERR_UNSUPPORTED, "problem too large for one launch");
   p.n_items = static_cast<int>(items);
+  if (P.chunk > 0) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.chunk = P.chunk;
+    p.nch_max = P.nch_max;
+    p.part = reinterpret_cast<float*>(ws + P.part_off);
+    p.part_l = reinterpret_cast<float*>(ws + P.part_l_off);
+    p.cnt = reinterpret_cast<int*>(ws + P.cnt_off);
+    e = cudaMemsetAsync(p.cnt, 0, P.ws_bytes - P.cnt_off, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the forward's range counters");
+  }
   // Persistent kernel: at most one CTA per SM, each walking several work items.
   const long long grid = items < sms ? items : sms;
 
@@ -800,6 +876,39 @@ sqa_status sqa_fwd(const void* q, const void* k, const void* v, void* out, float
     case 32: return launch_fwd<32>(q, k, v, out, lse, s, causal, sc, cs);
     case 64: return launch_fwd<64>(q, k, v, out, lse, s, causal, sc, cs);
     default: return launch_fwd<128>(q, k, v, out, lse, s, causal, sc, cs);
+  }
+}
+
+size_t sqa_fwd_workspace_bytes(sqa_shape s, int causal) {
+  if (check_shape(s) != SQA_OK) return 0;
+  return fwd_plan(s, causal, device_sms(), true).ws_bytes;
+}
+
+sqa_status sqa_fwd_with_workspace(const void* q, const void* k, const void* v, void* out, float* lse,
+                                  void* workspace, size_t workspace_bytes, sqa_shape s, int causal, float scale,
+                                  sqa_stream_t stream) {
+  g_last_error.clear();
+  if (!q || !k || !v || !out || !lse) return fail(SQA_ERR_INVALID_ARG, "null pointer argument");
+  sqa_status st = check_shape(s);
+  if (st != SQA_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4))
+    return fail(SQA_ERR_UNSUPPORTED, "q, k, v, out must be 16-byte aligned and lse 4-byte aligned");
+  const size_t need = fwd_plan(s, causal, device_sms(), true).ws_bytes;
+  if (need > 0) {
+    if (!workspace) return fail(SQA_ERR_INVALID_ARG, "null workspace (%zu bytes needed)", need);
+    if (!aligned(workspace, 256)) return fail(SQA_ERR_UNSUPPORTED, "workspace must be 256-byte aligned");
+    if (workspace_bytes < need)
+      return fail(SQA_ERR_INVALID_ARG, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
+  }
+  float sc;
+  if ((st = resolve_scale(scale, s.dh, &sc)) != SQA_OK) return st;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  void* ws = need > 0 ? workspace : nullptr;
+  switch (s.dh) {
+    case 16: return launch_fwd<16>(q, k, v, out, lse, s, causal, sc, cs, ws);
+    case 32: return launch_fwd<32>(q, k, v, out, lse, s, causal, sc, cs, ws);
+    case 64: return launch_fwd<64>(q, k, v, out, lse, s, causal, sc, cs, ws);
+    default: return launch_fwd<128>(q, k, v, out, lse, s, causal, sc, cs, ws);
   }
 }
 

@@ -58,6 +58,14 @@ struct FwdParams {
   int causal;
   int split;         // 1: both tile slots of a CTA work on one Q tile, even / odd key tiles
   float scale_log2;  // scale * log2(e)
+  // Split mode with a workspace (chunk > 0): a work item is a range of at most
+  // `chunk` key tiles of one Q tile; items of a Q tile with several ranges
+  // leave partial results, and the last of them to finish merges them.
+  int chunk;
+  int nch_max;    // ranges of the longest Q tile (layout of the partials)
+  float* part;    // [n_bh][n_qtiles][nch_max][128][dh] outputs normalised within their range
+  float* part_l;  // [n_bh][n_qtiles][nch_max][128] log2 of each range's sum of exponentials (log2 units)
+  int* cnt;       // [n_bh][n_qtiles][128] ranges finished per row (zero before the launch)
 };
 
 template <int DH>
@@ -110,7 +118,16 @@ __device__ __forceinline__ int fwd_item(int r, int n_items) { return dev::snake_
 struct FwdItem {
   int b, kvh, qt0, nkv0, nkv1, nkv;
   bool has1;
+  int kt0;  // first key tile (split mode with ranges; 0 otherwise)
+  int c;    // range index and number of ranges of the Q tile (1: no partials)
+  int nch;
 };
+
+// Key tiles a Q tile needs: all of them, or under a causal mask those up to its last token.
+__device__ __forceinline__ int fwd_nkv(const FwdParams& p, int qt, int NK) {
+  const int end = p.causal ? min(p.N, (qt + 1) * p.T) : p.N;
+  return (end + NK - 1) / NK;
+}
 
 template <bool SPLIT>
 __device__ __forceinline__ FwdItem fwd_decode(const FwdParams& p, int item, int NK) {
@@ -118,11 +135,33 @@ __device__ __forceinline__ FwdItem fwd_decode(const FwdParams& p, int item, int 
   const int bh = item % p.n_bh;
   it.b = bh / p.Hkv;
   it.kvh = bh % p.Hkv;
+  it.kt0 = 0;
+  it.c = 0;
+  it.nch = 1;
   if (SPLIT) {
-    // One Q tile; slot 0 takes its even key tiles, slot 1 the odd ones.
-    it.qt0 = p.n_qtiles - 1 - item / p.n_bh;  // latest tokens (heaviest under a causal mask) first
-    const int end = p.causal ? min(p.N, (it.qt0 + 1) * p.T) : p.N;
-    it.nkv = (end + NK - 1) / NK;
+    // One Q tile (or, with ranges, up to `chunk` of its key tiles); slot 0
+    // takes the even key tiles, slot 1 the odd ones.  Latest tokens (heaviest
+    // under a causal mask) first.
+    int k = item / p.n_bh;
+    int qt = p.n_qtiles - 1;
+    if (p.chunk > 0) {
+      // the k-th range of this (batch, KV head): Q tiles from the last, ranges in key order
+      int nkv = fwd_nkv(p, qt, NK), nch = (nkv + p.chunk - 1) / p.chunk;
+      while (k >= nch && qt > 0) {
+        k -= nch;
+        --qt;
+        nkv = fwd_nkv(p, qt, NK);
+        nch = (nkv + p.chunk - 1) / p.chunk;
+      }
+      it.c = k;
+      it.nch = nch;
+      it.kt0 = k * p.chunk;
+      it.nkv = max(0, min(nkv - it.kt0, p.chunk));
+    } else {
+      qt -= k;
+      it.nkv = fwd_nkv(p, qt, NK);
+    }
+    it.qt0 = qt;
     it.nkv0 = (it.nkv + 1) / 2;
     it.nkv1 = it.nkv / 2;
     it.has1 = false;  // one Q tile to load
@@ -137,6 +176,66 @@ __device__ __forceinline__ FwdItem fwd_decode(const FwdParams& p, int item, int 
   it.nkv1 = it.has1 ? (end1 + NK - 1) / NK : 0;
   it.nkv = max(it.nkv0, it.nkv1);
   return it;
+}
+
+// One row's result of a Q tile whose keys were split into nch ranges over
+// several CTAs.  Each range leaves its output normalised within the range and
+// its log2-sum-exp L_c; the row's counter in the workspace counts the ranges
+// written, and the thread that completes it (seeing every other range's
+// stores: each writer fences before its increment) merges them:
+//   O = sum_c 2^(L_c - M) O_c / W,  W = sum_c 2^(L_c - M),  M = max_c L_c,
+//   lse = ln 2 (M + log2 W),
+// in one pass with a running maximum (range 0 always holds key 0, so its L_0
+// is finite for every valid row), four ranges' loads in flight at a time.
+// No thread waits for another CTA, so there is nothing to time out.
+template <int DH>
+__device__ __noinline__ void fwd_merge_ranges(const FwdParams& p, size_t slot_base, int c, int nch, int row,
+                                              int* counter, float l2_own, __nv_bfloat16* dst, float* lse_dst) {
+  using namespace dev;
+  constexpr int BM = 128;
+  p.part_l[(slot_base + c) * BM + row] = l2_own;
+  __threadfence();
+  if (atomicAdd(counter, 1) + 1 != nch) return;
+  __threadfence();
+  float acc[DH];
+  const float* y0 = p.part + (slot_base * BM + row) * DH;
+#pragma unroll
+  for (int i = 0; i < DH; i += 4) {
+    const float4 a = __ldcg(reinterpret_cast<const float4*>(y0 + i));
+    acc[i] = a.x;
+    acc[i + 1] = a.y;
+    acc[i + 2] = a.z;
+    acc[i + 3] = a.w;
+  }
+  float M = __ldcg(p.part_l + slot_base * BM + row), W = 1.f;
+#pragma unroll 4
+  for (int cc = 1; cc < nch; ++cc) {
+    const float L = __ldcg(p.part_l + (slot_base + cc) * BM + row);
+    const float* y = p.part + ((slot_base + cc) * BM + row) * DH;
+    const float Mn = fmaxf(M, L);
+    const float a = ex2(M - Mn), b = ex2(L - Mn);  // L = -inf (no visible key in the range): b = 0
+    W = fmaf(W, a, b);
+#pragma unroll
+    for (int i = 0; i < DH; i += 4) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(y + i));
+      acc[i] = fmaf(acc[i], a, v.x * b);
+      acc[i + 1] = fmaf(acc[i + 1], a, v.y * b);
+      acc[i + 2] = fmaf(acc[i + 2], a, v.z * b);
+      acc[i + 3] = fmaf(acc[i + 3], a, v.w * b);
+    }
+    M = Mn;
+  }
+  const float inv_w = 1.f / W;
+#pragma unroll
+  for (int col = 0; col < DH; col += 8) {
+    uint4 o;
+    o.x = pack_bf16x2(acc[col] * inv_w, acc[col + 1] * inv_w);
+    o.y = pack_bf16x2(acc[col + 2] * inv_w, acc[col + 3] * inv_w);
+    o.z = pack_bf16x2(acc[col + 4] * inv_w, acc[col + 5] * inv_w);
+    o.w = pack_bf16x2(acc[col + 6] * inv_w, acc[col + 7] * inv_w);
+    *reinterpret_cast<uint4*>(dst + col) = o;
+  }
+  *lse_dst = (M + __log2f(W)) * 0.69314718055994531f;
 }
 
 // SPLIT: split mode (FwdParams::split), compiled separately so that the
@@ -257,9 +356,9 @@ __global__ void __launch_bounds__(384, 1)
           mbar_expect_tx(kv_full(s), 2u * Tr::KV_BYTES);
           for (int pn = 0; pn < Tr::NPANEL; ++pn) {
             tma_load_4d(sbase + Tr::OFF_K + s * Tr::KV_BYTES + pn * NK * ROWB, &tmK, kv_full(s), pn * PANEL,
-                        it.kvh, j * NK, it.b);
+                        it.kvh, (it.kt0 + j) * NK, it.b);
             tma_load_4d(sbase + Tr::OFF_V + s * Tr::KV_BYTES + pn * NK * ROWB, &tmV, kv_full(s), pn * PANEL,
-                        it.kvh, j * NK, it.b);
+                        it.kvh, (it.kt0 + j) * NK, it.b);
           }
         }
       }
@@ -419,7 +518,7 @@ __global__ void __launch_bounds__(384, 1)
         if (!ok) break;
         tc_fence_after();
         const uint32_t tS = lane_addr + Tr::tm_s(t, Gt % NSB);
-        const int k0 = (SPLIT ? 2 * j + t : j) * NK;
+        const int k0 = (it.kt0 + (SPLIT ? 2 * j + t : j)) * NK;
         const bool masked = (k0 + NK > p.N) || (p.causal && k0 + NK - 1 > qt * p.T);
         // The tile's scores are handled 64 columns (a half at NK = 128) at a time.
         // last visible key of this tile, relative to k0 (may be negative)
@@ -569,10 +668,17 @@ __global__ void __launch_bounds__(384, 1)
         l = l * a0 + l1 * a1;
         m = M;
       }
-      const float inv_l = row_valid ? 1.f / l : 0.f;
+      // (With key ranges a row may see no key of its range: l = 0, output 0.)
+      const float inv_l = (row_valid && l > 0.f) ? 1.f / l : 0.f;
       const float c0 = a0 * inv_l, c1 = a1 * inv_l;
       __nv_bfloat16* dst =
           p.out + ((static_cast<size_t>(it.b) * p.N + (row_valid ? tok : 0)) * p.Hq + head) * DH;
+      // One range of several: the fp32 result normalised within the range goes
+      // to the workspace instead, for the merge below.
+      const bool partial = SPLIT && it.nch > 1;
+      const size_t slot_base =
+          partial ? (static_cast<size_t>(it.b * p.Hkv + it.kvh) * p.n_qtiles + qt) * p.nch_max : 0;
+      float* pdst = partial ? p.part + ((slot_base + it.c) * BM + row) * DH : nullptr;
 #pragma unroll 1
       for (int c = 0; c < DH; c += 16) {
         uint32_t rr[16];
@@ -584,6 +690,14 @@ __global__ void __launch_bounds__(384, 1)
           tmem_ld16(tO1 + c, rr);
 #pragma unroll
           for (int i = 0; i < 16; ++i) y[i] = fmaf(__uint_as_float(rr[i]), c1, y[i]);
+        }
+        if (partial) {
+          if (row_valid) {
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+              *reinterpret_cast<float4*>(pdst + c + i) = make_float4(y[i], y[i + 1], y[i + 2], y[i + 3]);
+          }
+          continue;
         }
         uint4 lo, hi;
         lo.x = pack_bf16x2(y[0], y[1]);
@@ -607,8 +721,15 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive(split_done);
         ++nc;
       }
-      if (row_valid)
-        p.lse[(static_cast<size_t>(it.b) * p.Hq + head) * p.N + tok] = (m + __log2f(l)) * 0.69314718055994531f;
+      float* lse_dst = p.lse + (static_cast<size_t>(it.b) * p.Hq + head) * p.N + tok;
+      if (partial) {
+        if (row_valid)
+          fwd_merge_ranges<DH>(p, slot_base, it.c, it.nch, row,
+                               p.cnt + (static_cast<size_t>(it.b * p.Hkv + it.kvh) * p.n_qtiles + qt) * BM + row,
+                               l > 0.f ? m + __log2f(l) : -INFINITY, dst, lse_dst);
+      } else if (row_valid) {
+        *lse_dst = (m + __log2f(l)) * 0.69314718055994531f;
+      }
       G += nkv_t;
       ++nd;
     }

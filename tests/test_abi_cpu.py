@@ -266,3 +266,64 @@ def test_exp2_rate_probe_rejects_bad_arguments_before_launch(lib):
     assert f(0x100, 65536, 1, None) == 1
     assert f(0x100, 1, 0, None) == 1
     assert f(0x100, 1, (1 << 20) + 1, None) == 1
+
+
+def _fwd_ws_expected(B, N, Hq, Hkv, dh, causal, sms=148):
+    """Workspace rule of sqa_fwd_with_workspace: nothing unless the problem is
+    small (dh <= 64, pairs of Q tiles and single Q tiles both under half the
+    SMs) and ranges of `chunk` key tiles (the smallest even count, at least 2,
+    whose items do not outnumber the SMs) shorten the longest Q tile's walk
+    by at least 6 key tiles per slot; then fp32 partial outputs
+    [B*H_kv][n_qtiles][ranges of the longest tile][128][dh], their
+    log-sum-exps [..][128] and int counters [B*H_kv][n_qtiles][128], each
+    rounded up to 256 bytes."""
+    def a256(x):
+        return -(-x // 256) * 256
+
+    g = Hq // Hkv
+    T = 128 // g
+    n_qt = -(-N // T)
+    n_bh = B * Hkv
+    NK = 128 if dh == 128 else 64
+    if dh > 64 or -(-n_qt // 2) * n_bh >= sms // 2 or n_qt * n_bh >= sms // 2:
+        return 0
+    nkv = [-(-(min(N, (qt + 1) * T) if causal else N) // NK) for qt in range(n_qt)]
+    chunk = 2
+    while chunk < nkv[-1] and n_bh * sum(-(-n // chunk) for n in nkv) > sms:
+        chunk += 2
+    if -(-nkv[-1] // 2) - chunk // 2 < 6:
+        return 0
+    slots = n_bh * n_qt * -(-nkv[-1] // chunk) * 128
+    return a256(slots * dh * 4) + a256(slots * 4) + a256(n_bh * n_qt * 128 * 4)
+
+
+@pytest.mark.parametrize("shape", [(1, 1024, 8, 4, 16), (1, 333, 12, 4, 16), (1, 390, 8, 4, 64), (1, 2000, 2, 1, 32),
+                                   (32, 1024, 8, 4, 16), (2, 65536, 8, 4, 128), (1, 300, 8, 4, 128), (1, 64, 8, 4, 16),
+                                   (1, 200, 16, 1, 64), (1, 4096, 2, 1, 16), (1, 2500, 3, 1, 64), (1, 513, 6, 1, 16),
+                                   (1, 1500, 6, 1, 16), (1, 1000, 2, 2, 16)])
+@pytest.mark.parametrize("causal", [0, 1])
+def test_fwd_workspace_follows_its_rule(lib, shape, causal):
+    assert lib.sqa_fwd_workspace_bytes(sqa.Shape(*shape), causal) == _fwd_ws_expected(*shape, causal)
+
+
+def test_fwd_workspace_sizes_of_two_small_shapes(lib):
+    """B=1, N=4096, 2/1 heads, dh 16, causal: 64 Q tiles, ranges of 18 key
+    tiles (16 would make 160 items for 148 SMs), at most 4 per Q tile:
+    64 * 4 * 128 slots of 16 + 1 floats, 8192 counters.  The SQAT-m
+    layer-sized forward (B=1, N=1024, 8/4) would save 5 key tiles per slot
+    (8 -> 3): none."""
+    assert lib.sqa_fwd_workspace_bytes(sqa.Shape(1, 4096, 2, 1, 16), 1) == 32768 * 17 * 4 + 8192 * 4
+    assert lib.sqa_fwd_workspace_bytes(sqa.Shape(1, 1024, 8, 4, 16), 1) == 0
+
+
+def test_fwd_with_workspace_rejects_bad_arguments_before_launch(lib):
+    f = lib.sqa_fwd_with_workspace
+    s = sqa.Shape(1, 4096, 2, 1, 16)
+    need = lib.sqa_fwd_workspace_bytes(s, 1)
+    assert need > 0
+    ptrs = [0x1000, 0x2000, 0x3000, 0x4000, 0x5000]
+    assert f(*ptrs, None, need, s, 1, 0.0, None) == 1  # workspace needed
+    assert f(*ptrs, 0x6010, need, s, 1, 0.0, None) == 2  # workspace not 256-byte aligned
+    assert f(*ptrs, 0x6000, need - 1, s, 1, 0.0, None) == 1  # workspace too small
+    assert f(None, *ptrs[1:], 0x6000, need, s, 1, 0.0, None) == 1  # null q
+    assert f(*ptrs, 0x6000, need, sqa.Shape(1, 4096, 3, 2, 16), 1, 0.0, None) == 1  # H_q % H_kv

@@ -128,3 +128,15 @@ def test_default_step_count_follows_the_warm_up_time():
     assert bench.auto_steps(68.5, 20.0) == 291
     assert bench.auto_steps(0.01, 20.0) == 2000
     assert bench.auto_steps(10_000.0, 20.0) == 5
+
+
+def test_graph_replayed_single_launch_step_bounds_the_kernel_time():
+    """With CUDA-graph replay the hook's warm-up events include the host's
+    launch latency; for a one-launch step the replayed step time is the
+    tighter bound, for longer steps the warm-up's kernel time stands."""
+    import bench
+    from sparse_query_attention_sqa_b200.inputs import WORKLOADS
+
+    kern = {"k": [0.018, 0.018]}
+    assert bench.dominant_ms(kern, "k", [], [], True, WORKLOADS["sqatm_layer_fwd"], 0.0135) == 0.0135
+    assert bench.dominant_ms(kern, "k", [], [], True, WORKLOADS["sqatm_block_sqa"], 7.17) == 0.018

@@ -115,3 +115,40 @@ def test_errors_launch_nothing(cuda_lib):
     with pytest.raises(SqaError) as e:
         cuda_lib.sqa_fwd(q.cuda(), k.cuda(), v.cuda())
     assert e.value.status == 2
+
+
+# Small problems whose Q tiles fill less than half the SMs: the key tiles of
+# each Q tile are split into ranges computed by separate CTAs and merged by the
+# last range to finish (sqa_fwd_with_workspace).  g = 3 and g = 6 leave rows
+# with no visible key in a later range (tokens of a tile before that range's
+# first key).
+RANGE_SHAPES = [
+    (1, 2000, 2, 1, 32),  # eight ranges per Q tile at the end of the causal sequence
+    (1, 4096, 2, 1, 16),  # 148 items of up to 18 key tiles
+    (1, 2500, 3, 1, 64),
+    (1, 1500, 6, 1, 16),
+    (2, 1500, 2, 1, 32),
+    (1, 1000, 2, 2, 16),  # MHA layout: 128 tokens per Q tile
+]
+
+
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("shape", RANGE_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_fwd_key_ranges_match_oracle_and_one_cta_per_tile(cuda_lib, shape, causal):
+    """The ranges path (workspace filled with 0xff bytes first: the call clears
+    its counters itself) and the one-CTA-per-Q-tile path both match the oracle;
+    a second call with the same workspace gives the same bits."""
+    assert cuda_lib.fwd_workspace_bytes(*shape, causal) > 0, "shape does not take the ranges path"
+    q, k, v, _ = make_inputs(*shape, seed=6)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    ws = torch.full((cuda_lib.fwd_workspace_bytes(*shape, causal),), 255, dtype=torch.uint8, device="cuda")
+    out_r, lse_r = cuda_lib.sqa_fwd(qd, kd, vd, causal=causal, workspace=ws)
+    out_r2, lse_r2 = cuda_lib.sqa_fwd(qd, kd, vd, causal=causal, workspace=ws)
+    out_1, lse_1 = cuda_lib.sqa_fwd(qd, kd, vd, causal=causal, key_ranges=False)
+    torch.cuda.synchronize()
+    assert cuda_lib.device_status() == 0
+    ref_out, ref_lse = oracle.sqa_fwd(q, k, v, causal, None)
+    for out, lse in ((out_r, lse_r), (out_1, lse_1)):
+        assert_lse_close("lse", to_np(lse), ref_lse)
+        assert_close("out", to_np(out), ref_out)
+    assert torch.equal(out_r, out_r2) and torch.equal(lse_r, lse_r2)

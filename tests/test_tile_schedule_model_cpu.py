@@ -211,3 +211,102 @@ def test_forward_split_mode_visits_exactly_the_needed_key_tiles(B, N, Hkv, g, ca
     for b, kvh in itertools.product(range(B), range(Hkv)):
         for qt, kt in need:
             assert seen.get((b, kvh, qt, kt)) == 1
+
+
+def fwd_range_plan(B, N, Hkv, g, causal, sms=148):
+    """The host's choice of key ranges for small problems (split mode with a
+    workspace): None when every Q tile stays one item, else (chunk, number of
+    items).  Chunk: the smallest even number of key tiles (at least 2) whose
+    items do not outnumber the SMs; ranges only if they shorten the longest Q
+    tile's walk by at least 6 key tiles per slot."""
+    T = BM // g
+    n_qt = -(-N // T)
+    n_bh = B * Hkv
+    if not (-(-n_qt // 2) * n_bh < sms // 2 and n_qt * n_bh < sms // 2):
+        return None
+    nkv = [-(-(min(N, (qt + 1) * T) if causal else N) // NK_FWD) for qt in range(n_qt)]
+    chunk = 2
+    while chunk < nkv[-1] and n_bh * sum(-(-n // chunk) for n in nkv) > sms:
+        chunk += 2
+    if -(-nkv[-1] // 2) - chunk // 2 < 6:
+        return None
+    return chunk, n_bh * sum(-(-n // chunk) for n in nkv)
+
+
+def fwd_range_items(B, N, Hkv, g, causal, chunk, n_items):
+    """The items as the kernel decodes them: the k-th range of a (batch, KV
+    head), Q tiles from the last, ranges in key order: (b, kvh, qt, c, nch,
+    [key tiles of slot 0], [key tiles of slot 1])."""
+    T = BM // g
+    n_qt = -(-N // T)
+    n_bh = B * Hkv
+
+    def nkv_of(qt):
+        return -(-(min(N, (qt + 1) * T) if causal else N) // NK_FWD)
+
+    out = []
+    for item in range(n_items):
+        k, bh = item // n_bh, item % n_bh
+        qt = n_qt - 1
+        nkv = nkv_of(qt)
+        nch = -(-nkv // chunk)
+        while k >= nch and qt > 0:
+            k -= nch
+            qt -= 1
+            nkv = nkv_of(qt)
+            nch = -(-nkv // chunk)
+        kt0 = k * chunk
+        n = max(0, min(nkv - kt0, chunk))
+        n0, n1 = (n + 1) // 2, n // 2
+        out.append((bh // Hkv, bh % Hkv, qt, k, nch, [kt0 + 2 * j for j in range(n0)],
+                    [kt0 + 2 * j + 1 for j in range(n1)]))
+    return out
+
+
+RANGE_SHAPES = [(1, 2000, 1, 2), (1, 4096, 1, 2), (1, 2500, 1, 3), (1, 1500, 1, 6), (1, 2300, 1, 4), (1, 3000, 1, 1),
+                (1, 1000, 2, 1), (2, 1500, 1, 2)]
+
+
+@pytest.mark.parametrize("B,N,Hkv,g", RANGE_SHAPES)
+@pytest.mark.parametrize("causal", [True, False])
+def test_forward_key_ranges_visit_exactly_the_needed_key_tiles(B, N, Hkv, g, causal):
+    """Split mode with key ranges over several CTAs: every needed (Q tile, key
+    tile) pair is computed by exactly one slot of one range, the ranges of a Q
+    tile are consecutive and disjoint and their count is the one the merge
+    waits for, and tiles holding hidden pairs are flagged for masking."""
+    plan = fwd_range_plan(B, N, Hkv, g, causal)
+    if plan is None:
+        pytest.skip("no key ranges for this shape")
+    chunk, n_items = plan
+    T = BM // g
+    need = _tile_pairs_needed(N, T, NK_FWD, causal)
+    seen, ranges = {}, {}
+    for b, kvh, qt, c, nch, tiles0, tiles1 in fwd_range_items(B, N, Hkv, g, causal, chunk, n_items):
+        assert 0 <= c < nch and tiles0, "empty range"
+        assert len(tiles0) >= len(tiles1) and not set(tiles0) & set(tiles1)
+        assert all(c * chunk <= kt < (c + 1) * chunk for kt in tiles0 + tiles1)
+        ranges.setdefault((b, kvh, qt), []).append((c, nch))
+        for kt in tiles0 + tiles1:
+            seen[(b, kvh, qt, kt)] = seen.get((b, kvh, qt, kt), 0) + 1
+            assert (qt, kt) in need, f"fully masked tile pair visited: q tile {qt}, k tile {kt}"
+            if _hidden(qt, kt, T, NK_FWD, N, causal):
+                assert fwd_masked(kt * NK_FWD, qt, T, N, causal), f"unflagged tile pair {qt}, {kt}"
+    for b, kvh in itertools.product(range(B), range(Hkv)):
+        for qt, kt in need:
+            assert seen.get((b, kvh, qt, kt)) == 1
+    for key, rs in ranges.items():
+        nch = rs[0][1]
+        assert sorted(c for c, _ in rs) == list(range(nch)) and all(n == nch for _, n in rs), key
+
+
+def test_forward_key_ranges_choice():
+    """One long sequence with a single KV head (B=1, N=4096, 2/1, causal): 64
+    Q tiles, ranges of 16 key tiles would make 160 items for 148 SMs, so 18:
+    148 items (one Q tile per CTA walked up to 32 key tiles per slot, now 9).
+    The SQAT-m layer-sized forward (B=1, N=1024, 8/4) would go from 8 key
+    tiles per slot to 3, too little to pay for the merge: no ranges."""
+    assert fwd_range_plan(1, 4096, 1, 2, True) == (18, 148)
+    assert fwd_range_plan(1, 4096, 1, 2, False) == (32, 128)
+    assert fwd_range_plan(1, 1024, 4, 2, True) is None
+    assert fwd_range_plan(32, 1024, 4, 2, True) is None
+    assert fwd_range_plan(1, 256, 4, 2, True) is None
