@@ -115,15 +115,9 @@ sqa_status set_smem(Kernel k, int bytes) {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-int sm_count() {
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return sms;
-}
-
 // SMs of the current device (148 on B200; also the answer when no device can
 // be queried, so that workspace sizes can be computed without a GPU).
-int device_sms() {
+int sm_count() {
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
                                                 cudaSuccess || sms <= 0) {
@@ -881,7 +875,7 @@ sqa_status sqa_fwd(const void* q, const void* k, const void* v, void* out, float
 
 size_t sqa_fwd_workspace_bytes(sqa_shape s, int causal) {
   if (check_shape(s) != SQA_OK) return 0;
-  return fwd_plan(s, causal, device_sms(), true).ws_bytes;
+  return fwd_plan(s, causal, sm_count(), true).ws_bytes;
 }
 
 sqa_status sqa_fwd_with_workspace(const void* q, const void* k, const void* v, void* out, float* lse,
@@ -893,7 +887,7 @@ sqa_status sqa_fwd_with_workspace(const void* q, const void* k, const void* v, v
   if (st != SQA_OK) return st;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4))
     return fail(SQA_ERR_UNSUPPORTED, "q, k, v, out must be 16-byte aligned and lse 4-byte aligned");
-  const size_t need = fwd_plan(s, causal, device_sms(), true).ws_bytes;
+  const size_t need = fwd_plan(s, causal, sm_count(), true).ws_bytes;
   if (need > 0) {
     if (!workspace) return fail(SQA_ERR_INVALID_ARG, "null workspace (%zu bytes needed)", need);
     if (!aligned(workspace, 256)) return fail(SQA_ERR_UNSUPPORTED, "workspace must be 256-byte aligned");
