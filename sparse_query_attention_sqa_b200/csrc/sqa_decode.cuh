@@ -76,8 +76,10 @@ __host__ __device__ constexpr bool rows_path(int g, int hkv, int dh) {
 __host__ __device__ constexpr int rows_min_span(int dh, int hkv) { return kRowsMinSteps * rows_step(dh) / hkv; }
 // Rows in flight per thread of the register-resident path, and its ring of
 // shared-memory slots (one more than that, so a refill never targets the slot
-// being read).
-constexpr int kRowsDepth = 10, kRowsSlots = kRowsDepth + 1;
+// being read).  Three rows ahead keep the ring at 32 KB, so that registers,
+// not shared memory, bound the resident CTAs (three per SM for a group of
+// two); more CTAs hide the arithmetic's latencies better than deeper rings.
+constexpr int kRowsDepth = 3, kRowsSlots = kRowsDepth + 1;
 // Shared memory of the register-resident path: the per-thread ring of K and V
 // row pieces (16 bytes each) during the run, then one (o, m, l) record per
 // thread slot for the end-of-range merge.

@@ -100,6 +100,22 @@ def test_fwd_bwd_write_only_their_outputs(cuda_lib, shape):
     assert cuda_lib.device_status() == 0
 
 
+@pytest.mark.parametrize("shape", [(1, 1500, 6, 1, 16), (1, 2500, 3, 1, 64)], ids=lambda s: "x".join(map(str, s)))
+def test_fwd_key_ranges_write_only_their_outputs_and_workspace(cuda_lib, shape):
+    """The key-range forward (partials, counters) stays inside its workspace."""
+    B, N, Hq, Hkv, dh = shape
+    nbytes = cuda_lib.fwd_workspace_bytes(B, N, Hq, Hkv, dh, True)
+    assert nbytes > 0
+    q, k, v, _ = (t.cuda() if t is not None else None for t in make_inputs(B, N, Hq, Hkv, dh, seed=4))
+    out, lse = Guarded((B, N, Hq, dh), torch.bfloat16), Guarded((B, Hq, N), torch.float32)
+    ws = Guarded((nbytes,), torch.uint8)
+    cuda_lib.sqa_fwd(q, k, v, out=out.t, lse=lse.t, causal=True, workspace=ws.t)
+    out.check("out")
+    lse.check("lse")
+    assert bool((ws.raw[:GUARD] == PATTERN).all()) and bool((ws.raw[-GUARD:] == PATTERN).all()), "workspace"
+    assert cuda_lib.device_status() == 0
+
+
 def test_decode_writes_only_its_outputs(cuda_lib):
     B, N, Hq, Hkv, dh = 3, 1000, 16, 1, 16
     q, k, v = (t.cuda() for t in make_decode_inputs(B, N, Hq, Hkv, dh, seed=3))
