@@ -457,21 +457,50 @@ def traffic_for(kernel_name, w):
     return None
 
 
-def make_graphs(lib, w, sets, torch):
-    """One CUDA graph per buffer set holding a whole step (launch-bound
-    workloads: the step's launches cost the host more than the device's work).
-    The timing hooks are off while capturing."""
-    graphs = []
-    for s in sets:
-        gph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gph, capture_error_mode="thread_local"):
-            step(lib, w, s)
-        graphs.append(gph)
-    for gph in graphs:
-        gph.replay()
-    torch.cuda.synchronize()
-    assert lib.device_status() == 0, "a kernel wait gave up in a graph's first replay"
-    return graphs
+class GraphSteps:
+    """CUDA graphs holding whole steps, for launch-bound workloads (the step's
+    launches cost the host more than the device's work).  A step of a single
+    launch takes about as long on the device as the host needs to replay a
+    graph, so such steps are captured `per_graph` at a time over consecutive
+    buffer sets; run(k) replays exactly k steps.  The timing hooks are off
+    while capturing."""
+
+    def __init__(self, lib, w, sets, torch, per_graph):
+        self.lib, self.w, self.sets, self.torch, self.per = lib, w, sets, torch, per_graph
+        self.graphs = [self._capture(start, per_graph) for start in range(0, len(sets), per_graph)]
+        self.tails = {}
+        for gph in self.graphs:
+            gph.replay()
+        torch.cuda.synchronize()
+        assert lib.device_status() == 0, "a kernel wait gave up in a graph's first replay"
+
+    def _capture(self, start, count):
+        gph = self.torch.cuda.CUDAGraph()
+        with self.torch.cuda.graph(gph, capture_error_mode="thread_local"):
+            for i in range(count):
+                step(self.lib, self.w, self.sets[(start + i) % len(self.sets)])
+        return gph
+
+    def prepare(self, k):
+        """Capture the graph of the last k % per_graph steps before timing."""
+        rem = k % self.per
+        if rem and rem not in self.tails:
+            self.tails[rem] = self._capture(0, rem)
+            self.tails[rem].replay()
+            self.torch.cuda.synchronize()
+
+    def run(self, k):
+        full, rem = divmod(k, self.per)
+        for i in range(full):
+            self.graphs[i % len(self.graphs)].replay()
+        if rem:
+            self.tails[rem].replay()
+
+
+def graph_steps(lib, w, sets, torch, args):
+    if not w.graph or args.no_graph:
+        return None
+    return GraphSteps(lib, w, sets, torch, 16 if launches_per_step(w) == 1 else 1)
 
 
 def warm_up(lib, w, sets, warmup, torch):
@@ -545,18 +574,20 @@ def time_variant(args, lib, w, torch, world, rank, peaks, peak_kind):
     sets = [first] + [alloc_set(w, q, k, v, dout, lib, torch) for _ in range(n_sets - 1)]
     del q, k, v, dout
     kern, dominant, dom_idx, warm_ms = warm_up(lib, w, sets, args.warmup, torch)
-    graphs = make_graphs(lib, w, sets, torch) if w.graph and not args.no_graph else None
+    graphs = graph_steps(lib, w, sets, torch, args)
     n_steps = (auto_steps(max_over_ranks(warm_ms, world, "cuda"), 8.0) if getattr(args, "steps_auto", False)
                else args.steps)
+    if graphs:
+        graphs.prepare(n_steps)
     starts = [ev() for _ in range(n_steps)]
     stops = [ev() for _ in range(n_steps)]
     t0, t1 = ev(), ev()
     torch.cuda.synchronize()
     t0.record()
-    for i in range(n_steps):
-        if graphs:
-            graphs[i % n_sets].replay()
-        else:
+    if graphs:
+        graphs.run(n_steps)
+    else:
+        for i in range(n_steps):
             lib.set_timing_events(dom_idx, starts[i], stops[i])
             step(lib, w, sets[i % n_sets])
     t1.record()
@@ -599,10 +630,12 @@ def run_ours(args, w):
 
     ev = lambda: torch.cuda.Event(enable_timing=True)
     kern, dominant, dom_idx, warm_ms = warm_up(lib, w, sets, args.warmup, torch)
-    graphs = make_graphs(lib, w, sets, torch) if w.graph and not args.no_graph else None
+    graphs = graph_steps(lib, w, sets, torch, args)
     if args.steps is None:  # every rank times the same number of steps
         args.steps = auto_steps(max_over_ranks(warm_ms, world, "cuda"), 20.0)
         args.steps_auto = True
+    if graphs:
+        graphs.prepare(args.steps)
 
     # Timed region: K steps, per-step events around the dominant kernel (graph
     # replays instead for launch-bound workloads; the dominant kernel's time is
@@ -617,10 +650,10 @@ def run_ours(args, w):
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
     t0.record()
-    for i in range(args.steps):
-        if graphs:
-            graphs[i % n_sets].replay()
-        else:
+    if graphs:
+        graphs.run(args.steps)
+    else:
+        for i in range(args.steps):
             lib.set_timing_events(dom_idx, starts[i], stops[i])
             step(lib, w, sets[i % n_sets])
     t1.record()
@@ -697,7 +730,8 @@ def run_ours(args, w):
                        "parallelism": f"{world} independent replicas" if world > 1 else "single GPU",
                        "l2": f"{n_sets} rotating buffer sets of {set_bytes(first) / 2**20:.0f} MiB "
                              f"(> L2 in total), no flush",
-                       "launch": "CUDA-graph replay of each step" if graphs else "host launches",
+                       "launch": (f"CUDA-graph replay, {graphs.per} step(s) per graph" if graphs
+                                  else "host launches"),
                        **({"d": w.d, "hidden": w.hidden, "layers": w.layers,
                            "weights": "random, one set shared by every block"} if w.block else {})},
             "tokens_per_s": (w.B if w.decode else w.B * w.N) * world / (ms_step * 1e-3),

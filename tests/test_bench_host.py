@@ -140,3 +140,42 @@ def test_graph_replayed_single_launch_step_bounds_the_kernel_time():
     kern = {"k": [0.018, 0.018]}
     assert bench.dominant_ms(kern, "k", [], [], True, WORKLOADS["sqatm_layer_fwd"], 0.0135) == 0.0135
     assert bench.dominant_ms(kern, "k", [], [], True, WORKLOADS["sqatm_block_sqa"], 7.17) == 0.018
+
+
+def test_graph_steps_replay_exactly_k_steps(monkeypatch):
+    """Graphs of several one-launch steps: run(k) replays exactly k steps, the
+    last k % per_graph of them from a graph captured before timing; each graph
+    walks consecutive buffer sets."""
+    import contextlib
+    import types
+
+    import bench
+
+    log = {"captured": [], "replayed": 0, "current": None}
+
+    class FakeGraph:
+        def __init__(self):
+            self.steps = []
+
+        def replay(self):
+            log["replayed"] += len(self.steps)
+
+    @contextlib.contextmanager
+    def graph(g, capture_error_mode=None):
+        log["current"] = g
+        yield
+        log["current"] = None
+
+    cuda = types.SimpleNamespace(CUDAGraph=FakeGraph, graph=graph, synchronize=lambda: None)
+    fake_torch = types.SimpleNamespace(cuda=cuda)
+    lib = types.SimpleNamespace(device_status=lambda: 0)
+    monkeypatch.setattr(bench, "step", lambda lib_, w, s: log["current"].steps.append(s))
+    sets = list(range(37))
+    gs = bench.GraphSteps(lib, None, sets, fake_torch, 16)
+    assert [g.steps for g in gs.graphs][:2] == [list(range(16)), list(range(16, 32))]
+    assert gs.graphs[2].steps == [32, 33, 34, 35, 36] + list(range(11))
+    for k in (1, 16, 2000, 2001, 37 * 16 + 5):
+        gs.prepare(k)
+        log["replayed"] = 0
+        gs.run(k)
+        assert log["replayed"] == k
