@@ -63,6 +63,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="time budget of the CPU-baseline sample")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--shard", action="store_true",
+                    help="under torchrun: split one problem over the ranks by (batch entry, KV head) "
+                         "(strong scaling) instead of a replica per rank")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every step from the host even where the workload asks for CUDA-graph replay")
     return ap.parse_args()
@@ -606,6 +609,27 @@ def time_variant(args, lib, w, torch, world, rank, peaks, peak_kind):
     return out
 
 
+def shard_inputs(w, world, rank):
+    """This rank's part of one problem split by (batch entry, KV head): the
+    workload of its block and the block of the problem's inputs (drawn whole
+    with seed 0 on every rank, then sliced, so the blocks together are the
+    problem)."""
+    import dataclasses
+
+    from sparse_query_attention_sqa_b200 import shard
+    from sparse_query_attention_sqa_b200.inputs import workload_inputs
+
+    if w.decode or w.block:
+        raise SystemExit("--shard splits attention forward / backward workloads only")
+    blk = shard.shard_block(w.B, w.Hkv, world, rank)
+    g = w.Hq // w.Hkv
+    part = dataclasses.replace(w, B=blk.b1 - blk.b0, Hq=g * (blk.k1 - blk.k0), Hkv=blk.k1 - blk.k0)
+    q, k, v, dout = workload_inputs(w, seed=0)
+    qh, kh = shard.q_heads(blk, g), shard.kv_heads(blk)
+    return part, (shard.take(q, blk, qh), shard.take(k, blk, kh), shard.take(v, blk, kh),
+                  shard.take(dout, blk, qh) if dout is not None else None)
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -623,7 +647,12 @@ def run_ours(args, w):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
     lib.load_library()
 
-    q, k, v, dout = workload_inputs(w, seed=rank)
+    w_job = w
+    if args.shard and world > 1:
+        # One problem over the ranks: this rank's (batch entry, KV head) block of it.
+        w, (q, k, v, dout) = shard_inputs(w_job, world, rank)
+    else:
+        q, k, v, dout = workload_inputs(w, seed=rank)
     first = alloc_set(w, q, k, v, dout, lib, torch)
     n_sets = max(2, math.ceil(2 * L2_BYTES / set_bytes(first)))
     sets = [first] + [alloc_set(w, q, k, v, dout, lib, torch) for _ in range(n_sets - 1)]
@@ -667,7 +696,8 @@ def run_ours(args, w):
     assert lib.device_status() == 0, "a kernel wait gave up during the timed region"
     ms_step = ms_total / args.steps
     dom_ms = dominant_ms(kern, dominant, starts, stops, graphs, w, ms_step)
-    value = job_tflops(w, world, ms_step)
+    sharded = w_job is not w
+    value = counted_flops(w_job) / (ms_step * 1e-3) / 1e12 if sharded else job_tflops(w, world, ms_step)
     peaks, peak_kind = load_peaks()
 
     # End to end through the public API with host buffers: every step copies its
@@ -720,25 +750,30 @@ def run_ours(args, w):
 
     line = None
     if rank == 0:
+        wj = w_job
+        parallelism = (f"{world} ranks, each a (batch entry, KV head) block of one problem, no exchange" if sharded
+                       else f"{world} independent replicas" if world > 1 else "single GPU")
         line = {
-            "metric": f"{metric_name(w)} {pass_name(w)} TFLOP/s ({w.note})",
+            "metric": f"{metric_name(wj)} {pass_name(wj)} TFLOP/s ({wj.note})",
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16", "data": "synthetic (seeded Gaussian bf16 inputs)",
-            "config": {"workload": w.name, "B": w.B, "N": w.N, "H_q": w.Hq, "H_kv": w.Hkv, "dh": w.dh,
-                       "causal": w.causal, "pass": pass_name(w),
-                       "parallelism": f"{world} independent replicas" if world > 1 else "single GPU",
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong" if sharded else "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Gaussian bf16 inputs)",
+            "config": {"workload": wj.name, "B": wj.B, "N": wj.N, "H_q": wj.Hq, "H_kv": wj.Hkv, "dh": wj.dh,
+                       "causal": wj.causal, "pass": pass_name(wj),
+                       "parallelism": parallelism,
                        "l2": f"{n_sets} rotating buffer sets of {set_bytes(first) / 2**20:.0f} MiB "
                              f"(> L2 in total), no flush",
                        "launch": (f"CUDA-graph replay, {graphs.per} step(s) per graph" if graphs
                                   else "host launches"),
                        **({"d": w.d, "hidden": w.hidden, "layers": w.layers,
                            "weights": "random, one set shared by every block"} if w.block else {})},
-            "tokens_per_s": (w.B if w.decode else w.B * w.N) * world / (ms_step * 1e-3),
+            "tokens_per_s": (w_job.B * w_job.N if sharded else (w.B if w.decode else w.B * w.N) * world)
+                            / (ms_step * 1e-3),
             "tensor_frac_of_bf16_peak": value / peaks["bf16_tflops"],
             "roofline": roofline_for(w, dominant, dom_ms, peaks, peak_kind),
             "kernel_ms": {n: statistics.median(v) for n, v in kern.items()},
-            "e2e": {"value": job_tflops(w, world, e2e_ms), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "e2e": {"value": (counted_flops(w_job) / (e2e_ms * 1e-3) / 1e12 if sharded
+                              else job_tflops(w, world, e2e_ms)), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "streams": n_pipe,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": args.steps * launches_per_step(w),
@@ -748,7 +783,7 @@ def run_ours(args, w):
             "source_sha256": kernel_source_sha256(),
         }
     # The same kernels on the MHA / GQA / MQA head layouts of the same model.
-    variants = compare_variants(args, w)
+    variants = [] if sharded else compare_variants(args, w)
     if variants:
         sets.clear()
         first = host_in = host_out = None

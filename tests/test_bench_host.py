@@ -179,3 +179,22 @@ def test_graph_steps_replay_exactly_k_steps(monkeypatch):
         log["replayed"] = 0
         gs.run(k)
         assert log["replayed"] == k
+
+
+def test_shard_inputs_split_one_problem_by_kv_head():
+    """--shard: the two ranks' parts of the SQAT-m layer forward (B=1, 8/4)
+    are query heads 0-3 with KV heads 0-1 and query heads 4-7 with KV heads
+    2-3 of the same inputs; together they are the whole problem."""
+    import torch
+
+    import bench
+    from sparse_query_attention_sqa_b200.inputs import WORKLOADS, workload_inputs
+
+    w = WORKLOADS["sqatm_layer_fwd"]
+    q, k, v, _ = workload_inputs(w, seed=0)
+    parts = [bench.shard_inputs(w, 2, r) for r in range(2)]
+    assert [(p.B, p.Hq, p.Hkv) for p, _ in parts] == [(1, 4, 2), (1, 4, 2)]
+    assert torch.equal(torch.cat([t[0] for _, t in parts], dim=2), q)
+    assert torch.equal(torch.cat([t[1] for _, t in parts], dim=2), k)
+    assert torch.equal(torch.cat([t[2] for _, t in parts], dim=2), v)
+    assert sum(bench.counted_flops(p) for p, _ in parts) == bench.counted_flops(w)
