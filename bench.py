@@ -368,7 +368,7 @@ def launched_kernel(w, hook: int) -> str:
     if hook == 1:  # at dh 64 / 128 the hook brackets the dK/dV and the dQ kernels
         if w.dh <= 32:
             return f"sqa_bwd_tf32_kernel<{w.dh}>"
-        lo = "true" if g >= 8 else "false"  # groups of 8+ carry P and dS as bf16 hi + lo
+        lo = "true" if g >= 6 else "false"  # groups of 6+ carry P and dS as bf16 hi + lo
         return f"sqa_bwd_kernel<{w.dh},{lo}>+sqa_bwd_q_kernel<{w.dh}>"
     if g <= 4 and (w.Hkv & (w.Hkv - 1)) == 0 and w.Hkv <= 2048 // w.dh:  # register-resident path
         return f"sqa_decode_split_kernel<{w.dh},{g}>"

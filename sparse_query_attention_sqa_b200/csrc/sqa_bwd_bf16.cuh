@@ -58,10 +58,11 @@ namespace sqa {
 // pairs hi + lo (split_bf16x2) and issues each dV / dK MMA twice.  Each dV or
 // dK element sums g rows of every Q tile, and under a causal mask the first
 // keys of a sequence take P near 1 from all g heads of the first tokens: with
-// P rounded once to bf16 (relative error up to 2^-9) a 16-head group puts
-// dV elements of magnitude 2-4 up to 0.03 off; the remainder brings that to
-// the 1e-5 range, for 1.5 times the tensor work of this kernel.
-constexpr int kBwdSplitGroup = 8;
+// P rounded once to bf16 (relative error up to 2^-9) the largest dV errors
+// below magnitude 4 grow with g, 0.014 at g = 6 and 0.020 at g = 7 (dh 64)
+// and 0.032 at g = 16 (dh 128); the remainder brings them to the 1e-5 range,
+// for 1.5 times the tensor work of this kernel.
+constexpr int kBwdSplitGroup = 6;
 
 template <int DH>
 struct BwdBf16Traits {
