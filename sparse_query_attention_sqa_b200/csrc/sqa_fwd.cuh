@@ -95,9 +95,12 @@ struct FwdTraits {
   // The softmax warpgroups take turns for the exponentials (one S buffer per tile).
   static constexpr bool TOKEN = NSBUF == 1;
   // With one Q buffer a slot cannot start the next item before the other slot
-  // has finished this one, so a slot that skips the other's turns (an item with
-  // one Q tile) stays within one phase of the turn barriers; with two Q buffers
-  // it could run a whole item ahead and alias their phases.
+  // has passed its last turn of this one (each thread arrives on turn(t) before
+  // p_full, and the Q buffer is released after the last P V), so a slot that
+  // skips the other's last turns of an item (an item with one Q tile, or the
+  // other tile's extra causal step) finds those phases completed: a parity wait
+  // neither passes on a phase still open nor on one two ahead.  With two Q
+  // buffers a slot could run a whole item ahead and alias their phases.
   static_assert(!TOKEN || QBUF == 1, "turns need one Q buffer");
   // split mode: slot 1's running maximum and sum per row, for slot 0's combine
   static constexpr int OFF_ML = OFF_BAR + N_BARS * 8 + 16;
@@ -630,8 +633,11 @@ __global__ void __launch_bounds__(384, 1)
         l += ((sum0[0] + sum1[0]) + (sum0[1] + sum1[1])) + ((sum0[2] + sum1[2]) + (sum0[3] + sum1[3]));
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(p_full(t, Gt % NSB));
+        // The turn goes before P: the MMA issuer releases the Q buffer only after
+        // the last P of the item, so every turn of an item has completed before
+        // either slot starts the next one.
         if constexpr (Tr::TOKEN) mbar_arrive(turn(t));
+        mbar_arrive(p_full(t, Gt % NSB));
       }
       if (!ok) break;
       ok = __all_sync(0xffffffffu, mbar_wait(o_final(t), nd & 1, abort_flag, kSiteEpilogue));

@@ -16,7 +16,8 @@ A model is a dict role -> list of operations, in the role's program order:
 
 ``run`` executes one random interleaving and raises AssertionError on phase
 aliasing (a wait finds the barrier k + 2 completions ahead, so a parity wait
-would pass on the wrong phase), over-arrival, deadlock, or a buffer hazard (a
+would pass on the wrong phase, or only k - 1 completions in, so a parity wait
+would pass before phase k has completed), over-arrival, deadlock, or a buffer hazard (a
 use starts before every user of the previous stage or version has finished).
 """
 import random
@@ -74,6 +75,8 @@ def run(roles, counts, stages, seed, custom=None, skewed=False):
             else:
                 _, b, k = op
                 assert done[b] < k + 2, f"phase aliasing: {r} waits on {b} phase {k} after {done[b]} completions"
+                assert done[b] != k - 1, f"parity wait passes early: {r} waits on {b} phase {k} " \
+                    f"after {done[b]} completions (phase {k - 1}, same parity, still open)"
                 if done[b] == k + 1:
                     ready.append(r)
         if not ready:

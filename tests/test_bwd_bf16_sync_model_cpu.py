@@ -163,6 +163,35 @@ def test_model_detects_a_dropped_wait(name):
     assert failures > 0, name
 
 
+def test_p_ready_is_needed_per_half():
+    """p_ready exists per half of 64 query rows, each completing once per tile.
+    With one barrier completing twice per tile the producer, which waits only
+    for the second half (phase 2 i + 1), finds phase 2 i - 1 of the same parity
+    completed as soon as tile i - 1 is done and would refill the statistics
+    while tile i still reads them, and the issuer can find the barrier two
+    phases ahead of its wait; the checker must report one or the other."""
+    def merge(op):
+        if op[0] in ("wait", "arrive") and op[1] in ("p_ready0", "p_ready1"):
+            if op[0] == "arrive":
+                return ("arrive", "p_ready", op[2])
+            return ("wait", "p_ready", 2 * op[2] + (op[1] == "p_ready1"))
+        return op
+
+    rnd = random.Random(5)
+    failures = 0
+    for trial in range(300):
+        roles, cnt = _roles(rnd.randint(2, 8))
+        roles = {r: [merge(op) for op in ops] for r, ops in roles.items()}
+        cnt["p_ready"] = cnt.pop("p_ready0")
+        del cnt["p_ready1"]
+        try:
+            sync_model.run(roles, cnt, _stages(), trial, skewed=trial % 2 == 1)
+        except AssertionError as e:
+            assert any(w in str(e) for w in ("passes early", "aliasing", "hazard")), e
+            failures += 1
+    assert failures > 0
+
+
 # --------------------------------------------------------------------------- sqa_bwd_q_kernel
 
 

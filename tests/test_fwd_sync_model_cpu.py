@@ -217,9 +217,10 @@ def _roles(items, QB, ST, rnd, NSB=2, split=False):
                     if 0 <= k_other < nkv_o:
                         ops.append(W(f"tok{1 - t}", G_o + k_other))
                 ops += [B("X", t, ("exp", r)), E("X", t, ("exp", r))]
-                ops += [E(S, step % NSB, step, 1), A(f"p_full{t}{step % NSB}", 32)]
-                if token:
+                ops.append(E(S, step % NSB, step, 1))
+                if token:  # the turn before P (the Q buffer is released after the last P V)
                     ops.append(A(f"tok{t}", 32))
+                ops.append(A(f"p_full{t}{step % NSB}", 32))
             ops.append(W(f"o_final{t}", nd))
             if combine and t == 1:
                 # hand m, l to slot 0; O_1 stays until slot 0 has read it
@@ -340,6 +341,29 @@ DROPS = {
 # P V MMA in the issuer's order, so the warps' s_full wait also implies the
 # P V of the previous step completed: there the o_done wait is implied.
 IMPLIED = {("warps: o_done", 1), ("warps: tok", 2)}  # no token with two S buffers
+
+
+def test_turn_after_p_would_let_a_wait_pass_early():
+    # why each slot arrives on its turn barrier before p_full: with the turn
+    # last, the Q buffer can be released (and the next item started) while a
+    # thread of the other slot has not yet passed its last turn of this item, so
+    # a slot that skipped those turns finds a phase of the same parity open
+    rnd = random.Random(7)
+    failures = 0
+    for trial in range(200):
+        items = _items(rnd)
+        roles, cnt = _roles(items, 1, 2, random.Random(trial), 1)
+        for r, ops in roles.items():
+            for n in range(len(ops) - 1):  # swap each (turn, p_full) arrival pair back
+                if ops[n][0] == ops[n + 1][0] == "arrive" and ops[n][1].startswith("tok") \
+                        and ops[n + 1][1].startswith("p_full"):
+                    ops[n], ops[n + 1] = ops[n + 1], ops[n]
+        try:
+            sync_model.run(roles, cnt, STAGES, trial, custom={"O": _OCheck(), "X": _ExpCheck(True)},
+                           skewed=trial % 2 == 1)
+        except AssertionError as e:
+            failures += "passes early" in str(e)
+    assert failures > 0
 
 
 def test_turns_with_two_q_buffers_would_alias_their_phases():
